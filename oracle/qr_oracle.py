@@ -1,0 +1,376 @@
+"""Plain, slow CPU restatement of the online W4A4 rotated linear layer.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` leg of ``bench.py`` may import or run this module.  It shares
+no code with the CUDA library (``w4a4_rotation_quantized_b200``) and imports
+nothing from it; both sides draw their inputs from ``workloads`` only.
+
+Everything here is numpy in float64, written for a reader to check against the
+pages by eye: rotations are dense matrix products (never a fast transform),
+quantization is division then round-half-to-even, and the integer GEMM is an
+exact dot product.  The pages cited, by title:
+
+* [QS]  "QuaRot & SpinQuant" reading notes (chenghuawang.github.io, papers/
+        quant_quarot_spinquant): §1 Computational Invariance, §2 Quarot,
+        §3 SpinQuant.
+* [FQ]  "LLM量化新篇章：4-bit权重激活量化几乎无损！FlatQuant的平坦之道":
+        §2.3 方法概述 (affine transform, Kronecker decomposition, per-channel
+        scaling, clipping), 模型架构, §3 实验结果 (量化设置).
+* [GSR] "Grouped Sequency-arranged Rotation: Optimizing Rotation
+        Transformation for Quantization for Free": 方法详解, 摘要（原文）.
+* [QK]  "QUIK：LLM上的一种4-bit推理方法": QUIK量化 §1 (workflow), §3
+        (outlier selection), §4 (efficient inference).
+* [SR]  "SpinQuant: LLM Quantization with Learned Rotations" (review
+        discussion): Q1/A1 (min-max quantizer), reviewer Jf43 W1/A1 (QuIP#
+        incoherence bound), W2/A2 (R1/R2 absorbed into the weights).
+
+Readings taken where the pages are silent or garbled:
+
+R1  Codes are symmetric in [-(2^(b-1)-1), 2^(b-1)-1] = [-7, 7] for 4 bits;
+    the range printed in [SR] Q1/A1 is garbled, -8 is never produced.
+R2  Scale s = alpha * absmax / 7 (min-max, [SR] Q1/A1), alpha the clip ratio
+    ([FQ] §2.3 clipping, applied to both sides); codes are clamped to +-7.
+R3  Rounding is round-half-to-even; the code decision is taken in float32,
+    the precision the CUDA kernels take it in.
+R4  An all-zero row gets s = 0 and all-zero codes.
+R5  Hadamard matrices are Sylvester-ordered, scaled by 1/sqrt(n).
+R6  X' = X R and W' = W R^{-T} with W stored [N out x K in], so that
+    X' W'^T = X W^T ([QS] §1; [QK] §1 writes the linear layer as X W^T).
+R7  A GSR block is the sequency-ordered Walsh matrix: the rows of the
+    Sylvester Hadamard matrix sorted by their number of sign changes,
+    scaled by 1/sqrt(b); blocks are contiguous along K ([GSR]).
+R8  The Kronecker transform acts on a row x as x (P1 (x) P2), i.e.
+    vec(P1^T mat(x) P2) with mat(x)[a, b] = x[a*n2 + b]; the per-channel
+    scale divides X and multiplies W before the transform ([FQ] §2.3).
+R9  QUIK: the outlier columns stay fp16 and unrotated; the remaining columns,
+    in ascending order, are zero-padded to a multiple of the block size and
+    rotated; activations are quantized symmetrically (not asymmetrically as
+    [QK] §1 says of the original), weights by RTN instead of GPTQ.
+R10 Outlier columns are the top-k columns by infinity-norm over a calibration
+    batch, ties to the lower index, returned in ascending order ([QK] §3).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+QMAX = 7                      # R1: 4-bit symmetric range [-7, 7]
+NONE, HADAMARD, GSR, KRON = "none", "hadamard", "gsr", "kron"
+
+
+# --------------------------------------------------------------------------
+# Rotation matrices
+# --------------------------------------------------------------------------
+
+def hadamard(n: int) -> np.ndarray:
+    """Sylvester Hadamard matrix H_n (entries +-1, unscaled), n a power of 2.
+
+    [QS] §2: QuaRot rotates with Hadamard matrices; the pages do not name a
+    construction, so the Sylvester doubling H_2n = [[H, H], [H, -H]] (R5).
+    """
+    if n < 1 or n & (n - 1):
+        raise ValueError(f"Hadamard size must be a power of two, got {n}")
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def sign_changes(row: np.ndarray) -> int:
+    """Number of sign changes along a +-1 row (its sequency)."""
+    return int(np.count_nonzero(row[1:] != row[:-1]))
+
+
+def walsh_sequency(n: int) -> np.ndarray:
+    """Sequency-ordered Walsh matrix: Hadamard rows sorted by sign changes.
+
+    [GSR] 摘要（原文）/方法详解: the Walsh-Hadamard transform with sequency
+    ordering, which clusters similar frequency components (R7).
+    """
+    h = hadamard(n)
+    seq = np.array([sign_changes(r) for r in h])
+    return h[np.argsort(seq, kind="stable")]
+
+
+@dataclass
+class Rotation:
+    """What the layer does to a row before quantizing it."""
+    kind: str = NONE
+    block: int = 1                       # HADAMARD / GSR block size
+    P1: Optional[np.ndarray] = None      # KRON factors, [n1 x n1], [n2 x n2]
+    P2: Optional[np.ndarray] = None
+    chan_scale: Optional[np.ndarray] = None   # KRON per-channel scale c [K]
+    clip_ratio: float = 1.0
+
+
+def packed_width(rot: Rotation, K: int, n_out: int = 0) -> int:
+    """Width K_p of the rotated, quantized part of a row.
+
+    The K - n_out non-outlier columns are zero-padded to a multiple of the
+    block size and of 128 (R9; 128 keeps every row a whole number of the
+    GEMM's K steps).  A Kronecker transform needs exactly n1*n2 columns.
+    """
+    kr = K - n_out
+    if rot.kind == KRON:
+        n = rot.P1.shape[0] * rot.P2.shape[0]
+        if kr != n:
+            raise ValueError("Kronecker transform needs K - n_out == n1*n2")
+        return n
+    unit = 128
+    if rot.kind in (HADAMARD, GSR):
+        unit = max(unit, rot.block)
+    return -(-kr // unit) * unit
+
+
+def block_rotation(kind: str, block: int) -> np.ndarray:
+    """One diagonal block of R: H_b/sqrt(b) (HADAMARD) or Wal_b/sqrt(b) (GSR)."""
+    base = hadamard(block) if kind == HADAMARD else walsh_sequency(block)
+    return base / np.sqrt(block)
+
+
+def dense_rotation(rot: Rotation, k_p: int) -> np.ndarray:
+    """The full K_p x K_p rotation R as a dense matrix (small sizes only)."""
+    if rot.kind == NONE:
+        return np.eye(k_p)
+    if rot.kind == KRON:
+        return np.kron(rot.P1.astype(np.float64), rot.P2.astype(np.float64))
+    blk = block_rotation(rot.kind, rot.block)
+    return np.kron(np.eye(k_p // rot.block), blk)
+
+
+def _apply_blocks(x: np.ndarray, blk: np.ndarray) -> np.ndarray:
+    b = blk.shape[0]
+    rows, k = x.shape
+    return (x.reshape(rows, k // b, b) @ blk).reshape(rows, k)
+
+
+def _apply_kron(x: np.ndarray, p1: np.ndarray, p2: np.ndarray) -> np.ndarray:
+    """x (P1 (x) P2) row by row, as the two small products P1^T mat(x) P2.
+
+    [FQ] §2.3 Kronecker Decomposition / 模型架构: the transform is stored as
+    two small matrices and applied as two small matmuls per token (R8).
+    """
+    n1, n2 = p1.shape[0], p2.shape[0]
+    xm = x.reshape(x.shape[0], n1, n2)
+    return np.einsum("ac,mab,bd->mcd", p1, xm, p2, optimize=True).reshape(x.shape[0], n1 * n2)
+
+
+def rotate_activations(x: np.ndarray, rot: Rotation) -> np.ndarray:
+    """X' = X R (fp64).  [QS] §2 (online Hadamard on activations), [GSR],
+    [FQ] §2.3 (per-channel scale divides X, then the affine transform)."""
+    x = np.asarray(x, dtype=np.float64)
+    if rot.kind == NONE:
+        return x.copy()
+    if rot.kind in (HADAMARD, GSR):
+        return _apply_blocks(x, block_rotation(rot.kind, rot.block))
+    if rot.chan_scale is not None:
+        x = x / rot.chan_scale.astype(np.float64)[None, :]
+    return _apply_kron(x, rot.P1.astype(np.float64), rot.P2.astype(np.float64))
+
+
+def rotate_weights(w: np.ndarray, rot: Rotation) -> np.ndarray:
+    """W' = W R^{-T} (fp64), so that X' W'^T = X W^T (R6).
+
+    For the orthogonal rotations R^{-T} = R ([QS] §1, §2; [SR] W2/A2: R1/R2
+    are merged into the weights offline).  For the Kronecker transform
+    (P1 (x) P2)^{-T} = P1^{-T} (x) P2^{-T}, and the per-channel scale
+    multiplies W ([FQ] §2.3).
+    """
+    w = np.asarray(w, dtype=np.float64)
+    if rot.kind == NONE:
+        return w.copy()
+    if rot.kind in (HADAMARD, GSR):
+        return _apply_blocks(w, block_rotation(rot.kind, rot.block))
+    if rot.chan_scale is not None:
+        w = w * rot.chan_scale.astype(np.float64)[None, :]
+    q1 = np.linalg.inv(rot.P1.astype(np.float64)).T
+    q2 = np.linalg.inv(rot.P2.astype(np.float64)).T
+    return _apply_kron(w, q1, q2)
+
+
+# --------------------------------------------------------------------------
+# Quantization, packing, GEMM, epilogue
+# --------------------------------------------------------------------------
+
+@dataclass
+class Quantized:
+    codes: np.ndarray        # int8 [rows x K_p], values in [-7, 7]
+    scales: np.ndarray       # float32 [rows]
+    quotient: np.ndarray     # float32 x/s before rounding (for the tie window)
+
+
+def quantize_rows(xr: np.ndarray, clip_ratio: float = 1.0) -> Quantized:
+    """Symmetric per-row min-max quantization to 4-bit codes.
+
+    [SR] Q1/A1: min-max quantization scales each row into the symmetric
+    range (R1, R2); [FQ] §3 量化设置: activations per token, weights per
+    output channel, both symmetric.  The decision q = round(x/s) is taken in
+    float32 with round-half-to-even (R3); zero rows give s = 0 (R4).
+    """
+    x32 = np.asarray(xr, dtype=np.float64).astype(np.float32)
+    absmax = np.max(np.abs(x32), axis=1) if x32.shape[1] else np.zeros(x32.shape[0], np.float32)
+    s = (np.float32(clip_ratio) * absmax) / np.float32(QMAX)
+    s = s.astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    v = (x32 / safe[:, None]).astype(np.float32)
+    v[s == 0] = 0.0
+    q = np.clip(np.rint(v), -QMAX, QMAX).astype(np.int8)
+    return Quantized(codes=q, scales=s, quotient=v)
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """Two's-complement nibbles, two per byte, element 2j in the low nibble."""
+    q = np.asarray(q, dtype=np.int64)
+    if q.shape[-1] % 2:
+        raise ValueError("packed rows need an even width")
+    lo = q[..., 0::2] & 0xF
+    hi = q[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_int4(b: np.ndarray) -> np.ndarray:
+    """Inverse of pack_int4."""
+    b = np.asarray(b, dtype=np.int64)
+    lo = b & 0xF
+    hi = (b >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def int_gemm(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k qa[m, k] qw[n, k], exact, as int64.
+
+    [QK] §4: the INT4 x INT4 product accumulates in INT32.  The products are
+    formed in float64: every product and partial sum is an integer below
+    49 * K < 2^53, so each float64 operation is exact whatever the order.
+    """
+    a = np.asarray(qa, dtype=np.float64)
+    w = np.asarray(qw, dtype=np.float64)
+    if a.shape[1] * QMAX * QMAX >= 2 ** 53:
+        raise ValueError("K too large for an exact float64 dot product")
+    return np.rint(a @ w.T).astype(np.int64)
+
+
+def dequant_epilogue(acc: np.ndarray, sa: np.ndarray, sw: np.ndarray,
+                     x_out: Optional[np.ndarray] = None,
+                     w_out: Optional[np.ndarray] = None) -> np.ndarray:
+    """Y = fp16( acc * s_a[m] * s_w[n] + X_out W_out^T ).
+
+    [QK] §1: the INT4 product is dequantized to FP16 and added to the FP16
+    product of the outlier columns.  The sum is formed in float64 and rounded
+    once to fp16 (round-to-nearest-even).
+    """
+    y = acc.astype(np.float64) * np.asarray(sa, np.float64)[:, None] \
+        * np.asarray(sw, np.float64)[None, :]
+    if x_out is not None and w_out is not None and x_out.shape[1]:
+        y = y + np.asarray(x_out, np.float64) @ np.asarray(w_out, np.float64).T
+    return y.astype(np.float16)
+
+
+# --------------------------------------------------------------------------
+# QUIK outlier columns
+# --------------------------------------------------------------------------
+
+def select_outliers(x_calib: np.ndarray, k: int) -> np.ndarray:
+    """Top-k columns by infinity-norm over the calibration batch (R10).
+
+    [QK] §3: outliers are chosen by the column infinity-norm (the largest
+    absolute entry) and kept in FP16; §1: they are found from calibration
+    activations.
+    """
+    norms = np.max(np.abs(np.asarray(x_calib, np.float64)), axis=0)
+    order = np.lexsort((np.arange(norms.size), -norms))   # by -norm, then index
+    return np.sort(order[:k]).astype(np.int32)
+
+
+def split_outliers(x: np.ndarray, idx: Optional[np.ndarray]):
+    """(X_in, X_out): the kept columns in ascending order, and X[:, idx].
+
+    [QK] §1: outlier columns are moved to the end; the permutation has no
+    numerical effect, so the kept columns simply keep their order (R9).
+    """
+    x = np.asarray(x)
+    if idx is None or len(idx) == 0:
+        return x, x[:, :0]
+    keep = np.ones(x.shape[1], dtype=bool)
+    keep[np.asarray(idx)] = False
+    return x[:, keep], x[:, np.asarray(idx)]
+
+
+def pad_columns(x: np.ndarray, k_p: int) -> np.ndarray:
+    out = np.zeros((x.shape[0], k_p), dtype=np.float64)
+    out[:, : x.shape[1]] = x
+    return out
+
+
+# --------------------------------------------------------------------------
+# The layer, end to end
+# --------------------------------------------------------------------------
+
+@dataclass
+class Side:
+    """One operand after rotation and quantization."""
+    rotated: np.ndarray      # fp64 [rows x K_p]
+    q: Quantized
+    packed: np.ndarray       # uint8 [rows x K_p/2]
+    fp16_part: np.ndarray    # the outlier columns, fp16 [rows x n_out]
+
+
+def quantize_activations(x: np.ndarray, rot: Rotation,
+                         outlier_idx: Optional[np.ndarray] = None) -> Side:
+    """Online activation path: outlier split, rotation, per-token quantization."""
+    x_in, x_out = split_outliers(x, outlier_idx)
+    n_out = 0 if outlier_idx is None else len(outlier_idx)
+    k_p = packed_width(rot, np.asarray(x).shape[1], n_out)
+    xr = rotate_activations(pad_columns(np.asarray(x_in, np.float64), k_p), rot)
+    q = quantize_rows(xr, rot.clip_ratio)
+    return Side(xr, q, pack_int4(q.codes), np.asarray(x_out, np.float16))
+
+
+def quantize_weights(w: np.ndarray, rot: Rotation,
+                     outlier_idx: Optional[np.ndarray] = None) -> Side:
+    """Offline weight path: the same split, W R^{-T}, per-channel RTN ([QS] §2)."""
+    w_in, w_out = split_outliers(w, outlier_idx)
+    n_out = 0 if outlier_idx is None else len(outlier_idx)
+    k_p = packed_width(rot, np.asarray(w).shape[1], n_out)
+    wr = rotate_weights(pad_columns(np.asarray(w_in, np.float64), k_p), rot)
+    q = quantize_rows(wr, rot.clip_ratio)
+    return Side(wr, q, pack_int4(q.codes), np.asarray(w_out, np.float16))
+
+
+def linear(a: Side, w: Side):
+    """(acc, Y) of the quantized layer for prepared operands."""
+    acc = int_gemm(a.q.codes, w.q.codes)
+    y = dequant_epilogue(acc, a.q.scales, w.q.scales, a.fp16_part, w.fp16_part)
+    return acc, y
+
+
+def linear_forward(x, w, rot: Rotation, outlier_idx=None):
+    """The whole layer: Y ~= X W^T through rotated 4-bit codes."""
+    a = quantize_activations(x, rot, outlier_idx)
+    ws = quantize_weights(w, rot, outlier_idx)
+    acc, y = linear(a, ws)
+    return a, ws, acc, y
+
+
+# --------------------------------------------------------------------------
+# Diagnostics used by the pins
+# --------------------------------------------------------------------------
+
+def rmsnorm(x: np.ndarray) -> np.ndarray:
+    """x_i <- x_i / ||x_i|| per row, the no-rescale RMSNorm of [QS] §1."""
+    x = np.asarray(x, np.float64)
+    return x / np.linalg.norm(x, axis=1, keepdims=True)
+
+
+def incoherence_bound(w: np.ndarray, delta: float) -> float:
+    """mu ||W||_F / sqrt(mn) with mu = 2 log(4mn/delta) ([SR] Jf43 W1/A1)."""
+    m, n = w.shape
+    mu = 2.0 * np.log(4.0 * m * n / delta)
+    return mu * np.linalg.norm(w) / np.sqrt(m * n)

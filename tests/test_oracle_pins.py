@@ -1,0 +1,372 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test fixes one part of the oracle against a hand-worked fixture
+(tests/golden), a closed form, an invariant from the pages, or an
+independent algorithm (a butterfly transform, brute-force loops), chosen so
+that a dropped term, a wrong sign or index, or a transposed operand fails.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads
+from tests.conftest import read_golden_rows
+
+
+def _golden_matrix(name):
+    return np.array([[float(v) for v in r] for r in read_golden_rows(name)])
+
+
+# ---------------------------------------------------------------- Hadamard
+
+def test_hadamard_matches_textbook_h4():
+    assert np.array_equal(O.hadamard(4), _golden_matrix("hadamard4.txt"))
+
+
+@pytest.mark.parametrize("n", [1, 2, 8, 64, 1024])
+def test_hadamard_closed_form_entries(n):
+    # Sylvester order has H[i, j] = (-1)^popcount(i & j).
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    pc = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    assert np.array_equal(O.hadamard(n), np.where(pc % 2 == 0, 1.0, -1.0))
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 16, 128, 2048])
+def test_hadamard_orthogonal(n):
+    h = O.hadamard(n)
+    assert np.array_equal(h @ h.T, n * np.eye(n))
+
+
+def _fwht(x):
+    """Independent radix-2 butterfly transform along the last axis (unscaled)."""
+    x = np.array(x, dtype=np.float64)
+    n = x.shape[-1]
+    hlen = 1
+    while hlen < n:
+        y = x.reshape(x.shape[:-1] + (n // (2 * hlen), 2, hlen))
+        a, b = y[..., 0, :].copy(), y[..., 1, :].copy()
+        y[..., 0, :], y[..., 1, :] = a + b, a - b
+        x = y.reshape(x.shape)
+        hlen *= 2
+    return x
+
+
+@pytest.mark.parametrize("n", [2, 8, 32, 64, 4096])
+def test_dense_hadamard_rotation_equals_butterfly(n):
+    rng = np.random.default_rng(n)
+    x = rng.standard_normal((3, n))
+    rot = O.Rotation(O.HADAMARD, block=n)
+    np.testing.assert_allclose(O.rotate_activations(x, rot), _fwht(x) / np.sqrt(n),
+                               rtol=0, atol=1e-12 * np.sqrt(n))
+
+
+def test_block_diagonal_hadamard_acts_per_block():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((2, 8192))
+    rot = O.Rotation(O.HADAMARD, block=4096)
+    y = O.rotate_activations(x, rot)
+    np.testing.assert_allclose(y[:, :4096], _fwht(x[:, :4096]) / 64, atol=1e-11)
+    np.testing.assert_allclose(y[:, 4096:], _fwht(x[:, 4096:]) / 64, atol=1e-11)
+
+
+# ---------------------------------------------------------------- Walsh / GSR
+
+def test_walsh_matches_textbook_order8():
+    assert np.array_equal(O.walsh_sequency(8), _golden_matrix("walsh8_sequency.txt"))
+
+
+@pytest.mark.parametrize("n", [2, 4, 16, 128, 1024])
+def test_walsh_row_i_has_i_sign_changes(n):
+    w = O.walsh_sequency(n)
+    assert [O.sign_changes(r) for r in w] == list(range(n))
+
+
+def _bitrev(v, bits):
+    return int(format(v, f"0{bits}b")[::-1], 2) if bits else 0
+
+
+@pytest.mark.parametrize("n", [2, 8, 128, 512])
+def test_walsh_is_gray_bitreversed_hadamard_and_symmetric(n):
+    # Textbook: sequency index i corresponds to natural index bitrev(gray(i)).
+    bits = n.bit_length() - 1
+    h = O.hadamard(n)
+    w = O.walsh_sequency(n)
+    perm = [_bitrev(i ^ (i >> 1), bits) for i in range(n)]
+    assert np.array_equal(w, h[perm])
+    assert np.array_equal(w, w.T)
+    assert np.array_equal(w @ w.T, n * np.eye(n))
+
+
+def test_gsr_rotation_is_blockwise_permuted_fwht():
+    rng = np.random.default_rng(2)
+    b, nb = 128, 86
+    x = rng.standard_normal((2, b * nb))
+    y = O.rotate_activations(x, O.Rotation(O.GSR, block=b))
+    perm = [_bitrev(i ^ (i >> 1), 7) for i in range(b)]
+    for blk in (0, 41, 85):
+        z = _fwht(x[:, blk * b:(blk + 1) * b]) / np.sqrt(b)
+        np.testing.assert_allclose(y[:, blk * b:(blk + 1) * b], z[:, perm], atol=1e-12)
+
+
+# ---------------------------------------------------------------- Kronecker
+
+def test_kron_of_hadamards_is_the_8192_hadamard():
+    # H_128 (x) H_64 = H_8192 in Sylvester order: pins the x (P1 (x) P2)
+    # index convention mat(x)[a, b] = x[a*n2 + b].
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((2, 8192))
+    kron = O.Rotation(O.KRON, P1=O.hadamard(128) / np.sqrt(128), P2=O.hadamard(64) / 8.0)
+    had = O.Rotation(O.HADAMARD, block=8192)
+    np.testing.assert_allclose(O.rotate_activations(x, kron), O.rotate_activations(x, had),
+                               atol=1e-11)
+
+
+def test_kron_factored_form_equals_dense_kron_product():
+    rng = np.random.default_rng(4)
+    p1, p2 = rng.standard_normal((4, 4)), rng.standard_normal((8, 8))
+    x = rng.standard_normal((5, 32))
+    rot = O.Rotation(O.KRON, P1=p1, P2=p2)
+    np.testing.assert_allclose(O.rotate_activations(x, rot), x @ np.kron(p1, p2), rtol=1e-12,
+                               atol=1e-12)
+
+
+def test_kron_identity_factors_are_no_rotation():
+    x = np.random.default_rng(5).standard_normal((3, 64))
+    rot = O.Rotation(O.KRON, P1=np.eye(8), P2=np.eye(8))
+    np.testing.assert_array_equal(O.rotate_activations(x, rot), x)
+
+
+def test_kron_affine_pair_preserves_the_product():
+    # X' = (X / c)(P1 (x) P2), W' = (W c)(P1 (x) P2)^{-T}  =>  X' W'^T = X W^T.
+    wl = workloads.make_workload("flatquant_gate_up_8192", M=4, N=6)
+    rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale, clip_ratio=0.9)
+    x, w = wl.X.astype(np.float64), wl.W.astype(np.float64)
+    xr, wr = O.rotate_activations(x, rot), O.rotate_weights(w, rot)
+    ref = x @ w.T
+    np.testing.assert_allclose(xr @ wr.T, ref, rtol=0, atol=1e-9 * np.abs(ref).max())
+
+
+# ---------------------------------------------------------------- invariance
+
+@pytest.mark.parametrize("kind,block,k", [(O.HADAMARD, 256, 256), (O.HADAMARD, 64, 512),
+                                          (O.GSR, 128, 1024)])
+def test_computational_invariance(kind, block, k):
+    rng = np.random.default_rng(6)
+    x, w = rng.standard_normal((8, k)), rng.standard_normal((16, k))
+    rot = O.Rotation(kind, block=block)
+    xr, wr = O.rotate_activations(x, rot), O.rotate_weights(w, rot)
+    np.testing.assert_allclose(xr @ wr.T, x @ w.T, rtol=1e-12, atol=1e-12 * np.abs(x @ w.T).max())
+    np.testing.assert_allclose(np.linalg.norm(xr, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+
+
+def test_rmsnorm_commutes_with_rotation():
+    # RMSNorm(X) = RMSNorm(X Q^T) Q for orthogonal Q (the QuaRot/SpinQuant notes, §1).
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((4, 128))
+    q = O.dense_rotation(O.Rotation(O.GSR, block=64), 128)
+    np.testing.assert_allclose(O.rmsnorm(x @ q.T) @ q, O.rmsnorm(x), atol=1e-13)
+
+
+def test_zero_padding_is_exact():
+    rng = np.random.default_rng(8)
+    x, w = rng.standard_normal((3, 7936)), rng.standard_normal((5, 7936))
+    rot = O.Rotation(O.HADAMARD, block=4096)
+    xp, wp = O.pad_columns(x, 8192), O.pad_columns(w, 8192)
+    got = O.rotate_activations(xp, rot) @ O.rotate_weights(wp, rot).T
+    np.testing.assert_allclose(got, x @ w.T, rtol=1e-12, atol=1e-10)
+
+
+# ---------------------------------------------------------------- quantizer
+
+def test_quantizer_hand_example():
+    rows = read_golden_rows("quantizer_1x8.txt")
+    x = np.array([[float(v) for v in rows[0][1:]]])
+    for r in rows[1:]:
+        alpha, scale = float(r[1]), float(r[3])
+        codes = [int(v) for v in r[5:]]
+        q = O.quantize_rows(x, alpha)
+        assert q.scales[0] == np.float32(scale)
+        assert q.codes[0].tolist() == codes
+
+
+def test_quantizer_properties():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((64, 256)) * rng.uniform(0.01, 100, size=(64, 1))
+    x[3] = 0.0
+    q = O.quantize_rows(x, 1.0)
+    assert q.codes.min() >= -7 and q.codes.max() <= 7
+    assert q.scales[3] == 0 and not q.codes[3].any()
+    nz = np.arange(64) != 3
+    assert np.all(np.abs(q.codes[nz]).max(axis=1) == 7)
+    err = np.abs(x[nz] - q.scales[nz, None].astype(np.float64) * q.codes[nz])
+    assert np.all(err <= 0.5 * q.scales[nz, None] * (1 + 1e-6))
+
+
+def test_quantizer_clips_beyond_alpha():
+    x = np.array([[10.0, -10.0, 1.0, 0.0]])
+    q = O.quantize_rows(x, 0.5)        # s = 0.5 * 10 / 7
+    assert q.codes[0].tolist() == [7, -7, 1, 0]
+    assert np.isclose(q.scales[0], 5.0 / 7.0)
+
+
+def test_pack_hand_example_and_roundtrip():
+    rows = read_golden_rows("pack_int4.txt")
+    codes = np.array([[int(v) for v in rows[0][1:]]])
+    expect = np.array([[int(v, 16) for v in rows[1][1:]]], dtype=np.uint8)
+    assert np.array_equal(O.pack_int4(codes), expect)
+    assert np.array_equal(O.unpack_int4(expect), codes)
+    q = np.random.default_rng(10).integers(-7, 8, size=(5, 64))
+    assert np.array_equal(O.unpack_int4(O.pack_int4(q)), q)
+
+
+# ---------------------------------------------------------------- GEMM, epilogue
+
+def test_int_gemm_equals_brute_force():
+    rng = np.random.default_rng(11)
+    for m, n, k in [(1, 1, 2), (3, 5, 7), (7, 4, 33)]:
+        a = rng.integers(-7, 8, size=(m, k))
+        w = rng.integers(-7, 8, size=(n, k))
+        brute = [[sum(int(a[i, t]) * int(w[j, t]) for t in range(k)) for j in range(n)]
+                 for i in range(m)]
+        assert O.int_gemm(a, w).tolist() == brute
+
+
+def test_int_gemm_extremes_exact():
+    k = 11008
+    a = np.full((2, k), 7)
+    a[1] = -7
+    w = np.full((3, k), -7)
+    w[2, ::2] = 7
+    acc = O.int_gemm(a, w)
+    assert acc[0, 0] == -49 * k and acc[1, 0] == 49 * k and acc[0, 2] == 0
+
+
+def test_epilogue_hand_example():
+    acc = np.array([[10, -3], [0, 2048]])
+    sa = np.array([0.5, 2.0 ** -11], np.float32)
+    sw = np.array([0.25, 1.0], np.float32)
+    y = O.dequant_epilogue(acc, sa, sw)
+    # 10*.5*.25 = 1.25 ; -3*.5 = -1.5 ; 0 ; 2048*2^-11 = 1
+    assert y.tolist() == [[1.25, -1.5], [0.0, 1.0]]
+    # fp16 round-half-even: 1 + 2^-11 is a tie between 1 and 1 + 2^-10
+    y = O.dequant_epilogue(np.array([[2049]]), np.array([2.0 ** -11]), np.array([1.0]))
+    assert y[0, 0] == np.float16(1.0)
+    # outlier product is added: 1*2 + 3*4 = 14
+    y = O.dequant_epilogue(np.array([[4]]), np.array([1.0]), np.array([1.0]),
+                           np.array([[1.0, 3.0]]), np.array([[2.0, 4.0]]))
+    assert y[0, 0] == 18.0
+
+
+# ---------------------------------------------------------------- QUIK outliers
+
+def test_select_outliers_hand_example_ties_to_lower_index():
+    x = np.array([[3.0, -5.0, 5.0, 1.0], [0.0, 1.0, -2.0, 0.5]])
+    assert O.select_outliers(x, 2).tolist() == [1, 2]
+    assert O.select_outliers(x, 1).tolist() == [1]
+    assert O.select_outliers(x, 3).tolist() == [0, 1, 2]
+
+
+def test_select_outliers_recovers_injected_columns():
+    wl = workloads.make_workload("quik_decode_8192", with_weights=False)
+    idx = O.select_outliers(wl.X_calib, 256)
+    assert np.array_equal(idx, np.sort(wl.outlier_channels))
+
+
+def test_outlier_split_partitions_the_product():
+    rng = np.random.default_rng(12)
+    x, w = rng.standard_normal((4, 40)), rng.standard_normal((6, 40))
+    idx = np.array([3, 17, 18, 39])
+    xi, xo = O.split_outliers(x, idx)
+    wi, wo = O.split_outliers(w, idx)
+    assert xi.shape == (4, 36) and xo.shape == (4, 4)
+    np.testing.assert_allclose(xi @ wi.T + xo @ wo.T, x @ w.T, atol=1e-12)
+    assert np.array_equal(xo, x[:, idx])
+
+
+# ---------------------------------------------------------------- end to end
+
+def _exact_case(kind, k, rng, clip=1.0, n_out=0):
+    """X, W built so that the rotated rows are integer codes with absmax 7."""
+    m, n = 6, 10
+    qa = workloads.random_codes_rows(rng, m, k)
+    qw = workloads.random_codes_rows(rng, n, k)
+    if kind == O.KRON:
+        n1, n2 = 8, k // 8
+        p1 = rng.standard_normal((n1, n1)) + 3 * np.eye(n1)
+        p2 = rng.standard_normal((n2, n2)) + 3 * np.eye(n2)
+        c = rng.uniform(0.5, 2.0, size=k)
+        rot = O.Rotation(O.KRON, P1=p1, P2=p2, chan_scale=c, clip_ratio=clip)
+        p = np.kron(p1, p2)
+        x = (qa @ np.linalg.inv(p)) * c[None, :]          # (x / c) P = qa
+        w = (qw @ p.T) / c[None, :]                        # (w c) P^{-T} = qw
+    else:
+        rot = O.Rotation(kind, block=32 if kind == O.GSR else 64, clip_ratio=clip)
+        r = O.dense_rotation(rot, k)
+        x, w = qa @ r.T, qw @ r.T                          # x R = qa, w R = qw
+    xo = wo = None
+    idx = None
+    if n_out:
+        idx = np.sort(rng.choice(k + n_out, size=n_out, replace=False))
+        keep = np.setdiff1d(np.arange(k + n_out), idx)
+        xf = np.zeros((m, k + n_out)); xf[:, keep] = x
+        wf = np.zeros((n, k + n_out)); wf[:, keep] = w
+        xo = rng.integers(-4, 5, size=(m, n_out)).astype(np.float64)
+        wo = rng.integers(-4, 5, size=(n, n_out)).astype(np.float64)
+        xf[:, idx] = xo; wf[:, idx] = wo
+        x, w = xf, wf
+    return rot, x, w, qa, qw, idx, xo, wo
+
+
+@pytest.mark.parametrize("kind", [O.NONE, O.HADAMARD, O.GSR, O.KRON])
+def test_end_to_end_on_exactly_representable_rows(kind):
+    rng = np.random.default_rng(13)
+    rot, x, w, qa, qw, _, _, _ = _exact_case(kind, 128, rng)
+    a, ws, acc, y = O.linear_forward(x, w, rot)
+    assert np.array_equal(a.q.codes, qa) and np.array_equal(ws.q.codes, qw)
+    np.testing.assert_allclose(a.q.scales, 1.0, rtol=1e-6)
+    assert np.array_equal(acc, qa @ qw.T)
+    np.testing.assert_array_equal(y, (qa @ qw.T).astype(np.float16))
+
+
+def test_end_to_end_with_outliers_and_padding():
+    rng = np.random.default_rng(14)
+    # 128 rotated columns + 8 fp16 outlier columns; hadamard blocks of 64
+    rot, x, w, qa, qw, idx, xo, wo = _exact_case(O.HADAMARD, 128, rng, n_out=8)
+    a, ws, acc, y = O.linear_forward(x, w, rot, idx)
+    assert np.array_equal(a.q.codes, qa) and np.array_equal(ws.q.codes, qw)
+    np.testing.assert_array_equal(y, (qa @ qw.T + xo @ wo.T).astype(np.float16))
+
+
+def test_end_to_end_clip_ratio_maps_codes():
+    # alpha = 0.9: s = 0.9, codes = clamp(rne(q / 0.9), -7, 7) -> 0..7 map to 0,1,2,3,4,6,7,7
+    rng = np.random.default_rng(15)
+    rot, x, w, qa, qw, _, _, _ = _exact_case(O.KRON, 128, rng, clip=0.9)
+    a, ws, acc, y = O.linear_forward(x, w, rot)
+    lut = np.array([0, 1, 2, 3, 4, 6, 7, 7])
+    expect_a = np.sign(qa) * lut[np.abs(qa)]
+    expect_w = np.sign(qw) * lut[np.abs(qw)]
+    assert np.array_equal(a.q.codes, expect_a) and np.array_equal(ws.q.codes, expect_w)
+    np.testing.assert_allclose(a.q.scales, 0.9, rtol=1e-6)
+
+
+def test_rotation_reduces_error_on_outlier_inputs():
+    # The pages' claim (QuaRot §2, FlatQuant §2, GSR): rotating spreads the
+    # outlier channels, so the 4-bit layer is closer to X W^T than without.
+    wl = workloads.make_workload("tiny_256")
+    x, w = wl.X.astype(np.float64), wl.W.astype(np.float64)
+    exact = x @ w.T
+    errs, act = {}, {}
+    for name, rot in [("none", O.Rotation(O.NONE)), ("had", O.Rotation(O.HADAMARD, block=256))]:
+        a, _, _, y = O.linear_forward(x, w, rot)
+        errs[name] = np.linalg.norm(y.astype(np.float64) - exact) / np.linalg.norm(exact)
+        deq = a.q.codes * a.q.scales[:, None].astype(np.float64)
+        act[name] = np.linalg.norm(deq - a.rotated) / np.linalg.norm(a.rotated)
+    assert errs["had"] < errs["none"], errs
+    assert act["had"] < 0.6 * act["none"], act
+
+
+def test_hadamard_bounds_weight_entries_incoherence():
+    wl = workloads.make_workload("tiny_256")
+    wr = O.rotate_weights(wl.W.astype(np.float64), O.Rotation(O.HADAMARD, block=256))
+    assert np.abs(wr).max() <= O.incoherence_bound(wr, 0.01)
