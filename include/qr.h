@@ -1,0 +1,212 @@
+/*
+ * qr.h -- C ABI of the B200 online W4A4 rotated linear layer.
+ *
+ * The layer computes, for activations X [M x K] and weights W [N x K]
+ * (fp16, row-major, W stored output-major as in Y = X W^T):
+ *
+ *     Y = fp16( dequant( Q(X R) . Q(W R^{-T})^T ) + X_out W_out^T )
+ *
+ * where R is a rotation (full or block-diagonal Walsh-Hadamard, the
+ * grouped sequency-ordered Walsh rotation, or a Kronecker affine transform
+ * with per-channel scaling), Q is symmetric per-row 4-bit quantization and
+ * X_out, W_out are the QUIK fp16 outlier columns.
+ *
+ * Sources, by page title and section:
+ *   - "QuaRot & SpinQuant" reading notes, §1 Computational Invariance and
+ *     §2 Quarot: weights are rotated offline, activations online, so that
+ *     the rotated product equals the original one.
+ *   - "QUIK：LLM上的一种4-bit推理方法", QUIK量化 §1 (workflow: outlier
+ *     columns kept fp16, per-token quantization of the rest, INT4 GEMM with
+ *     INT32 accumulation, dequant to fp16, outlier product added) and §3
+ *     (outliers chosen by column infinity-norm).
+ *   - "LLM量化新篇章：4-bit权重激活量化几乎无损！FlatQuant的平坦之道",
+ *     §2.3 方法概述 (Kronecker-decomposed affine transform, per-channel
+ *     scaling, clipping) and §3 量化设置 (per-token / per-channel symmetric).
+ *   - "Grouped Sequency-arranged Rotation: Optimizing Rotation
+ *     Transformation for Quantization for Free", abstract and 方法详解
+ *     (block-diagonal sequency-ordered Walsh blocks).
+ *   - "SpinQuant: LLM Quantization with Learned Rotations" review
+ *     discussion, Q1/A1 (min-max quantizer onto +-(2^(N-1)-1)).
+ *
+ * Conventions shared by every call:
+ *   - Every array pointer is a DEVICE pointer unless stated otherwise; the
+ *     caller allocates and owns every buffer.  No call allocates memory.
+ *   - fp16 arrays are passed as uint16_t (IEEE binary16 bit patterns).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and operate on the device that is current.
+ *   - Argument errors return before any launch and write nothing.  A failed
+ *     launch returns QR_ERR_CUDA.  Faults inside a kernel surface as usual
+ *     CUDA errors at the next synchronization.
+ *   - Kernels that wait on barriers bound every wait; if a wait ever runs out
+ *     (a library bug, not a user error) the kernel records a code in a
+ *     per-device status word, abandons its work and returns; read it with
+ *     qr_device_status().
+ *   - 4-bit codes are two's-complement nibbles, two per byte, element 2j in
+ *     the low nibble, rows of K_p/2 bytes (K_p from qr_packed_k).  Codes lie
+ *     in [-7, 7].  Scales are fp32, one per row.
+ */
+#ifndef QR_H_
+#define QR_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QR_API __attribute__((visibility("default")))
+#else
+#define QR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                      /* cudaStream_t is struct CUstream_st* */
+typedef struct CUstream_st* qr_stream;
+
+typedef enum {
+  QR_OK = 0,
+  QR_ERR_INVALID_ARG = 1,    /* null pointer, negative or inconsistent size */
+  QR_ERR_UNSUPPORTED = 2,    /* a size or kind outside what the kernels handle */
+  QR_ERR_ALIGNMENT = 3,      /* a pointer or leading dimension is misaligned */
+  QR_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  QR_ERR_DEVICE = 5          /* a kernel recorded an error (qr_device_status) */
+} qr_status;
+
+typedef enum {
+  QR_ROT_NONE = 0,           /* quantize the (outlier-free, padded) row as is */
+  QR_ROT_HADAMARD = 1,       /* block-diagonal Sylvester Hadamard, H_b/sqrt(b) */
+  QR_ROT_GSR = 2,            /* block-diagonal sequency-ordered Walsh, Wal_b/sqrt(b) */
+  QR_ROT_KRON = 3            /* x -> (x op c) (P1 kron P2): vec(P1^T mat(x) P2) */
+} qr_rot_kind;
+
+typedef enum {
+  QR_CHAN_DIVIDE = 0,        /* activation side: x_k / c_k  */
+  QR_CHAN_MULTIPLY = 1       /* weight side:     w_k * c_k  */
+} qr_chan_mode;
+
+/* What is done to a row before it is quantized.  Host struct; the arrays it
+ * points to are device arrays that must stay valid until the call's work on
+ * the stream has finished. */
+typedef struct {
+  int32_t kind;              /* qr_rot_kind */
+  int32_t block;             /* HADAMARD, GSR: block size b, a power of two,
+                                1 <= b <= 16384 (GSR: 2 <= b <= 256);
+                                ignored otherwise */
+  const float* p1;           /* KRON: row-major n1 x n1 */
+  int32_t n1;
+  const float* p2;           /* KRON: row-major n2 x n2 */
+  int32_t n2;                /* KRON: n1, n2 multiples of 4, n1 + n2 <= 192,
+                                n1*n2 % 128 == 0 */
+  const float* chan_scale;   /* KRON: per-channel scale c [n1*n2], or NULL */
+  int32_t chan_mode;         /* qr_chan_mode: how chan_scale is applied */
+  float clip_ratio;          /* alpha in (0, 1]: s = alpha*absmax/7, codes
+                                clamped to +-7 (1.0 = plain min-max) */
+} qr_rotation;
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define QR_ABI_VERSION 1
+QR_API int32_t qr_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+QR_API const char* qr_status_string(qr_status status);
+
+/* Width K_p of the rotated, quantized part of a row of K columns of which
+ * n_out are fp16 outliers: the other K - n_out columns, zero-padded to a
+ * multiple of max(b, 128) (HADAMARD, GSR) or of 128 (NONE); for KRON,
+ * K - n_out must equal n1*n2.  The zero padding changes neither the scale
+ * nor any dot product (the QUIK page's split plus the orthogonality of R).
+ * Returns -1 if the descriptor or sizes are invalid.  Host-only. */
+QR_API int64_t qr_packed_k(const qr_rotation* rot, int64_t K, int32_t n_out);
+
+/* Online activation path (QuaRot §2 online rotation; QUIK §1 per-token
+ * quantization of the non-outlier columns; FlatQuant §2.3 fused transform
+ * and quantization).  For each row m of X:
+ *   x_out[m, j] = X[m, outlier_idx[j]]                       (fp16 copy)
+ *   x = X[m, kept columns] zero-padded to K_p, x' = rotate(x)
+ *   scales[m] = alpha * max|x'| / 7   (0 for an all-zero row)
+ *   codes[m, k] = clamp(round_half_even(x'[k] / scales[m]), -7, 7), packed
+ *
+ *  rot          host descriptor (activation side: chan_mode DIVIDE)
+ *  X            fp16 [M x ldx], ldx >= K
+ *  outlier_idx  int32 [n_out], strictly ascending in [0, K); may be NULL
+ *               when n_out == 0.  Out-of-range entries are skipped by the
+ *               kernel (their x_out column reads as zero), never read
+ *               out of bounds.
+ *  codes        uint8 [M x K_p/2] (row stride K_p/2 bytes), 16-byte aligned
+ *  scales       fp32 [M]
+ *  x_out        fp16 [M x n_out] (row stride n_out), NULL iff n_out == 0
+ *  x_rot_debug  fp32 [M x K_p] rotated rows before quantization, or NULL
+ * Errors: INVALID_ARG (null/negative/inconsistent, clip_ratio outside (0,1]),
+ * UNSUPPORTED (block, n1/n2 outside the limits above, K_p > 32768, or with
+ * outliers K > 32768 or n_out > 8192), ALIGNMENT (codes not 16-byte
+ * aligned). */
+QR_API qr_status qr_rotate_quant(const qr_rotation* rot, const uint16_t* X, int64_t M,
+                          int64_t K, int64_t ldx, const int32_t* outlier_idx,
+                          int32_t n_out, uint8_t* codes, float* scales,
+                          uint16_t* x_out, float* x_rot_debug, qr_stream stream);
+
+/* Offline weight path (QuaRot §2 stage 1: rotate the weights in full
+ * precision, then quantize them; SpinQuant review W2/A2: R1/R2 merged into
+ * the weights; QUIK §1: weight columns permuted to match the outliers).
+ * Same as qr_rotate_quant applied to the rows of W with the weight-side
+ * descriptor rot_w: for HADAMARD/GSR it equals the activation descriptor;
+ * for KRON it holds P1^{-T}, P2^{-T} (see qr_invert_transpose) and the same
+ * c with chan_mode MULTIPLY, so that X' W'^T = X W^T.
+ *  W            fp16 [N x ldw], ldw >= K
+ *  w_codes      uint8 [N x K_p/2], 16-byte aligned;  w_scales fp32 [N]
+ *  w_out        fp16 [N x n_out], NULL iff n_out == 0
+ *  w_rot_debug  fp32 [N x K_p] or NULL
+ * Errors as qr_rotate_quant. */
+QR_API qr_status qr_pack_weights(const qr_rotation* rot_w, const uint16_t* W, int64_t N,
+                          int64_t K, int64_t ldw, const int32_t* outlier_idx,
+                          int32_t n_out, uint8_t* w_codes, float* w_scales,
+                          uint16_t* w_out, float* w_rot_debug, qr_stream stream);
+
+/* The W4A4 linear (QUIK §4: the INT4 x INT4 product on integer tensor cores
+ * with INT32 accumulation, dequantized to fp16, plus the fp16 outlier
+ * product; FlatQuant §3: per-token x per-channel symmetric scales):
+ *   acc[m, n] = sum_k qa[m, k] qw[n, k]                      (exact int32)
+ *   Y[m, n]   = fp16( acc * a_scales[m] * w_scales[n]
+ *                     + sum_j x_out[m, j] w_out[n, j] )      (fp32 math)
+ *  a_codes   uint8 [M x K_p/2], w_codes uint8 [N x K_p/2], both 16-byte
+ *            aligned; K_p % 128 == 0, K_p <= 65536
+ *  x_out     fp16 [M x n_out], w_out fp16 [N x n_out] (NULL iff n_out == 0),
+ *            16-byte aligned, n_out % 8 == 0
+ *  Y         fp16 [M x ldy], ldy >= N
+ *  acc_debug int32 [M x N] (row stride N), or NULL
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT as above. */
+QR_API qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales,
+                         const uint8_t* w_codes, const float* w_scales,
+                         int64_t M, int64_t N, int64_t K_p,
+                         const uint16_t* x_out, const uint16_t* w_out, int32_t n_out,
+                         uint16_t* Y, int64_t ldy, int32_t* acc_debug,
+                         qr_stream stream);
+
+/* QUIK calibration (QUIK §3: outliers are the columns with the largest
+ * infinity-norm over a calibration batch).  Writes the k selected column
+ * indices of X_calib [T x ldx] (fp16, ldx >= K) to idx_out[k] in ascending
+ * order; ties in the norm go to the lower column index.
+ * Limits: 1 <= K <= 16384, 0 <= k <= K.  One CTA; offline. */
+QR_API qr_status qr_select_outliers(const uint16_t* X_calib, int64_t T, int64_t K,
+                             int64_t ldx, int32_t k, int32_t* idx_out,
+                             qr_stream stream);
+
+/* Weight-side Kronecker factor (FlatQuant §2.3: W is multiplied by the
+ * inverse of the affine transform): out = (P^{-1})^T for a row-major
+ * n x n matrix P, by Gauss-Jordan elimination with partial pivoting in
+ * fp64, rounded to fp32.  info (int32 [1]) receives 0, or j+1 if column j
+ * had no usable pivot (P singular to working precision; out is then
+ * undefined).  1 <= n <= 256.  One CTA; offline. */
+QR_API qr_status qr_invert_transpose(const float* P, int32_t n, float* out,
+                              int32_t* info, qr_stream stream);
+
+/* Reads, and clears, the current device's status word that kernels set when
+ * a bounded wait ran out.  Synchronizes the device.  *code_out = 0 when no
+ * kernel reported anything. */
+QR_API qr_status qr_device_status(int32_t* code_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* QR_H_ */

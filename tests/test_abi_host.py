@@ -1,0 +1,143 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+include/qr.h declares, and rejects bad arguments before launching anything.
+No test here runs a kernel (this file runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from tests.conftest import ROOT
+from w4a4_rotation_quantized_b200 import _lib as L
+from w4a4_rotation_quantized_b200 import build as B
+
+HEADER = os.path.join(ROOT, "include", "qr.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qr_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(L.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {L.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (qr_[a-z0-9_]+)", out))
+    assert exported == set(declared_functions())
+
+
+def test_abi_version_and_status_strings(lib):
+    assert L.qr_abi_version() == 1
+    for s in range(6):
+        assert L.status_string(s) and L.status_string(s) != "unknown status"
+    assert L.status_string(99) == "unknown status"
+
+
+FAKE = 0x10000          # never dereferenced: every call below fails validation first
+
+
+def _rot(kind, block=0, n1=0, n2=0, clip=1.0, p=FAKE):
+    return L.make_rotation(kind, block, p if n1 else 0, n1, p if n2 else 0, n2, 0,
+                           L.QR_CHAN_DIVIDE, clip)
+
+
+@pytest.mark.parametrize("kind,block,n1,n2,K,n_out", [
+    (L.QR_ROT_HADAMARD, 4096, 0, 0, 4096, 0),
+    (L.QR_ROT_HADAMARD, 4096, 0, 0, 8192, 256),
+    (L.QR_ROT_HADAMARD, 256, 0, 0, 256, 0),
+    (L.QR_ROT_HADAMARD, 2, 0, 0, 300, 4),
+    (L.QR_ROT_GSR, 128, 0, 0, 11008, 0),
+    (L.QR_ROT_GSR, 256, 0, 0, 1000, 0),
+    (L.QR_ROT_NONE, 0, 0, 0, 33, 0),
+    (L.QR_ROT_NONE, 0, 0, 0, 0, 0),
+    (L.QR_ROT_KRON, 0, 128, 64, 8192, 0),
+    (L.QR_ROT_KRON, 0, 16, 8, 136, 8),
+])
+def test_packed_k_matches_the_oracle(lib, kind, block, n1, n2, K, n_out):
+    names = {L.QR_ROT_NONE: O.NONE, L.QR_ROT_HADAMARD: O.HADAMARD, L.QR_ROT_GSR: O.GSR,
+             L.QR_ROT_KRON: O.KRON}
+    orot = O.Rotation(names[kind], block=block,
+                      P1=np.eye(n1) if n1 else None, P2=np.eye(n2) if n2 else None)
+    assert L.qr_packed_k(_rot(kind, block, n1, n2), K, n_out) == O.packed_width(orot, K, n_out)
+
+
+@pytest.mark.parametrize("rot,K,n_out", [
+    (_rot(L.QR_ROT_HADAMARD, 96), 96, 0),          # block not a power of two
+    (_rot(L.QR_ROT_HADAMARD, 32768), 32768, 0),    # block too large
+    (_rot(L.QR_ROT_GSR, 512), 512, 0),             # GSR block too large
+    (_rot(L.QR_ROT_KRON, 0, 128, 64), 8000, 0),    # K != n1*n2
+    (_rot(L.QR_ROT_KRON, 0, 128, 128), 16384, 0),  # factors too large
+    (_rot(L.QR_ROT_KRON, 0, 6, 8), 48, 0),         # n1 not a multiple of 4
+    (_rot(L.QR_ROT_HADAMARD, 64, clip=0.0), 64, 0),
+    (_rot(L.QR_ROT_HADAMARD, 64, clip=1.5), 64, 0),
+    (_rot(7, 64), 64, 0),                           # unknown kind
+    (_rot(L.QR_ROT_NONE), 10, 11),                 # n_out > K
+])
+def test_packed_k_rejects_bad_descriptors(lib, rot, K, n_out):
+    assert L.qr_packed_k(rot, K, n_out) == -1
+
+
+def _rq(rot, X=FAKE, M=4, K=256, ldx=256, idx=None, n_out=0, codes=FAKE, scales=FAKE, xo=None,
+        dbg=None):
+    return L.qr_rotate_quant(rot, X, M, K, ldx, idx, n_out, codes, scales, xo, dbg, None,
+                             check=False)
+
+
+def test_rotate_quant_argument_errors(lib):
+    h = _rot(L.QR_ROT_HADAMARD, 256)
+    assert _rq(h, M=-1) == L.QR_ERR_INVALID_ARG
+    assert _rq(h, ldx=100) == L.QR_ERR_INVALID_ARG              # ldx < K
+    assert _rq(h, X=None) == L.QR_ERR_INVALID_ARG
+    assert _rq(h, codes=None) == L.QR_ERR_INVALID_ARG
+    assert _rq(h, n_out=4, idx=None, xo=FAKE) == L.QR_ERR_INVALID_ARG
+    assert _rq(h, n_out=4, idx=FAKE, xo=None) == L.QR_ERR_INVALID_ARG
+    assert _rq(h, codes=FAKE + 8) == L.QR_ERR_ALIGNMENT
+    assert _rq(_rot(L.QR_ROT_HADAMARD, 96)) == L.QR_ERR_UNSUPPORTED
+    assert _rq(_rot(L.QR_ROT_HADAMARD, 64, clip=2.0)) == L.QR_ERR_INVALID_ARG
+    assert _rq(_rot(L.QR_ROT_NONE), K=40000, ldx=40000) == L.QR_ERR_UNSUPPORTED
+    assert _rq(h, M=0) == L.QR_OK                                 # empty: nothing to do
+
+
+def _lin(M=16, N=16, Kp=256, a=FAKE, sa=FAKE, w=FAKE, sw=FAKE, xo=None, wo=None, n_out=0,
+         Y=FAKE, ldy=None, acc=None):
+    return L.qr_w4a4_linear(a, sa, w, sw, M, N, Kp, xo, wo, n_out, Y, N if ldy is None else ldy,
+                            acc, None, check=False)
+
+
+def test_linear_argument_errors(lib):
+    assert _lin(Kp=200) == L.QR_ERR_INVALID_ARG                   # K_p % 128
+    assert _lin(M=-1) == L.QR_ERR_INVALID_ARG
+    assert _lin(ldy=8) == L.QR_ERR_INVALID_ARG
+    assert _lin(Y=None) == L.QR_ERR_INVALID_ARG
+    assert _lin(a=None) == L.QR_ERR_INVALID_ARG
+    assert _lin(n_out=8, xo=None, wo=FAKE) == L.QR_ERR_INVALID_ARG
+    assert _lin(n_out=12, xo=FAKE, wo=FAKE) == L.QR_ERR_UNSUPPORTED   # n_out % 8
+    assert _lin(Kp=65536 + 128) == L.QR_ERR_UNSUPPORTED
+    assert _lin(a=FAKE + 4) == L.QR_ERR_ALIGNMENT
+    assert _lin(n_out=8, xo=FAKE + 2, wo=FAKE) == L.QR_ERR_ALIGNMENT
+    assert _lin(M=0) == L.QR_OK and _lin(N=0) == L.QR_OK
+
+
+def test_calibration_argument_errors(lib):
+    assert L.qr_select_outliers(FAKE, 8, 0, 8, 1, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG
+    assert L.qr_select_outliers(FAKE, 8, 16, 8, 1, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG
+    assert L.qr_select_outliers(FAKE, 8, 16, 16, 17, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG
+    assert L.qr_select_outliers(FAKE, 8, 20000, 20000, 4, FAKE, None,
+                                check=False) == L.QR_ERR_UNSUPPORTED
+    assert L.qr_invert_transpose(FAKE, 0, FAKE, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG
+    assert L.qr_invert_transpose(FAKE, 200, FAKE, FAKE, None, check=False) == L.QR_ERR_UNSUPPORTED
+    assert L.qr_invert_transpose(None, 4, FAKE, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG

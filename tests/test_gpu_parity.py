@@ -1,0 +1,257 @@
+"""GPU parity of the CUDA path against the oracle on small seeded cases that
+span several tiles and ragged tails, plus edge cases.  All calls go through
+the C ABI (libqr.so)."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import w4a4_rotation_quantized_b200 as Q
+import workloads
+from tests.gpu_helpers import (Y_TOL, check_side, dev, gpu_rotation, host,
+                               oracle_rows_from_gpu_codes, rel_fro, require_gpu, unpack)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+    yield
+    assert Q._lib.qr_device_status() == 0
+
+
+def _rows(rng, m, k, scale=1.0, outl=()):
+    x = rng.standard_normal((m, k)).astype(np.float32) * scale
+    for c in outl:
+        x[:, c] *= 40
+    return x.astype(np.float16)
+
+
+def _run_rows(x16, orot, idx=None, weights=False):
+    xg = dev(x16)
+    ig = None if idx is None else dev(np.asarray(idx, np.int32))
+    grot = gpu_rotation(orot)
+    if weights:
+        gpu = Q.pack_weights(xg, Q.weight_rotation(grot), ig, debug=True)
+        ref = O.quantize_weights(x16.astype(np.float64), orot, idx)
+    else:
+        gpu = Q.rotate_quant(xg, grot, ig, debug=True)
+        ref = O.quantize_activations(x16.astype(np.float64), orot, idx)
+    torch.cuda.synchronize()
+    return gpu, ref
+
+
+# ---------------------------------------------------------------- rotate + quantize
+
+ROW_CASES = [
+    # (name, K, rows, rotation)
+    ("had256", 256, 16, O.Rotation(O.HADAMARD, block=256)),
+    ("had4096", 4096, 19, O.Rotation(O.HADAMARD, block=4096)),
+    ("had8192_cross_warp", 8192, 5, O.Rotation(O.HADAMARD, block=8192)),
+    ("had16384_cross_warp", 16384, 3, O.Rotation(O.HADAMARD, block=16384)),
+    ("had_blocks2", 384, 9, O.Rotation(O.HADAMARD, block=2)),
+    ("had_blocks8", 640, 9, O.Rotation(O.HADAMARD, block=8)),
+    ("had_blocks64", 640, 9, O.Rotation(O.HADAMARD, block=64)),
+    ("had_blocks512", 1536, 9, O.Rotation(O.HADAMARD, block=512)),
+    ("had_blocks4096_two", 8192, 4, O.Rotation(O.HADAMARD, block=4096)),
+    ("gsr128", 11008, 7, O.Rotation(O.GSR, block=128)),
+    ("gsr2", 256, 5, O.Rotation(O.GSR, block=2)),
+    ("gsr16", 384, 5, O.Rotation(O.GSR, block=16)),
+    ("gsr256", 768, 5, O.Rotation(O.GSR, block=256)),
+    ("none_ragged", 200, 11, O.Rotation(O.NONE)),
+    ("none_long", 8192, 3, O.Rotation(O.NONE)),
+    ("had_clip", 1024, 9, O.Rotation(O.HADAMARD, block=1024, clip_ratio=0.5)),
+    ("gsr_clip", 1024, 9, O.Rotation(O.GSR, block=128, clip_ratio=0.9)),
+]
+
+
+@pytest.mark.parametrize("name,K,rows,rot", ROW_CASES, ids=[c[0] for c in ROW_CASES])
+@pytest.mark.parametrize("weights", [False, True], ids=["act", "wgt"])
+def test_rotate_quant_matches_oracle(name, K, rows, rot, weights):
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    x = _rows(rng, rows, K, outl=(3, K // 2))
+    x[rows // 2] = 0                                 # an all-zero row
+    gpu, ref = _run_rows(x, rot, weights=weights)
+    check_side(gpu, ref, name, clip=rot.clip_ratio)
+    assert host(gpu[1])[rows // 2] == 0 and not host(gpu[0])[rows // 2].any()
+
+
+def test_rotate_quant_unaligned_leading_dimension():
+    rng = np.random.default_rng(1)
+    full = _rows(rng, 6, 203)
+    x = dev(full)[:, :200]                           # ldx = 203: scalar loads
+    rot = O.Rotation(O.HADAMARD, block=128)
+    gpu = Q.rotate_quant(x, gpu_rotation(rot), debug=True)
+    ref = O.quantize_activations(full[:, :200].astype(np.float64), rot)
+    check_side(gpu, ref, "ldx203")
+
+
+@pytest.mark.parametrize("K,n_out,block", [(300, 5, 64), (8192, 256, 4096), (1000, 40, 128),
+                                           (256, 256, 128)])
+def test_rotate_quant_with_outlier_columns(K, n_out, block):
+    rng = np.random.default_rng(K + n_out)
+    idx = np.sort(rng.choice(K, size=n_out, replace=False)).astype(np.int32)
+    x = _rows(rng, 7, K, outl=idx[:3])
+    rot = O.Rotation(O.HADAMARD, block=block)
+    for weights in (False, True):
+        gpu, ref = _run_rows(x, rot, idx, weights=weights)
+        check_side(gpu, ref, f"outliers K={K} n_out={n_out}")
+
+
+def test_kron_rotate_quant_small_factors():
+    rng = np.random.default_rng(3)
+    n1, n2 = 16, 8
+    p1 = (np.eye(n1) + 0.3 * rng.standard_normal((n1, n1))).astype(np.float32)
+    p2 = (np.eye(n2) + 0.3 * rng.standard_normal((n2, n2))).astype(np.float32)
+    c = rng.uniform(0.5, 2.0, n1 * n2).astype(np.float32)
+    rot = O.Rotation(O.KRON, P1=p1, P2=p2, chan_scale=c, clip_ratio=0.9)
+    x = _rows(rng, 9, n1 * n2, outl=(5,))
+    for weights in (False, True):
+        gpu, ref = _run_rows(x, rot, weights=weights)
+        check_side(gpu, ref, "kron16x8", clip=0.9)
+
+
+def test_kron_flatquant_factors_with_outliers():
+    wl = workloads.make_workload("flatquant_gate_up_8192", M=8, N=8)
+    rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale, clip_ratio=0.9)
+    for x in (wl.X, wl.W):
+        gpu, ref = _run_rows(x, rot, weights=x is wl.W)
+        check_side(gpu, ref, "flatquant", clip=0.9)
+    # Kronecker transform together with an outlier split: 8 fp16 columns + 8192 rotated
+    rng = np.random.default_rng(4)
+    idx = np.sort(rng.choice(8200, 8, replace=False)).astype(np.int32)
+    x = _rows(rng, 5, 8200)
+    gpu, ref = _run_rows(x, rot, idx)
+    check_side(gpu, ref, "flatquant+outliers", clip=0.9)
+
+
+def test_invert_transpose_matches_numpy():
+    wl = workloads.make_workload("flatquant_gate_up_8192", M=1, N=1)
+    for p in (wl.P1, wl.P2):
+        q = host(Q.invert_transpose(dev(p)))
+        want = np.linalg.inv(p.astype(np.float64)).T
+        np.testing.assert_allclose(q, want, rtol=0, atol=1e-6 * np.abs(want).max())
+    with pytest.raises(ValueError):
+        Q.invert_transpose(dev(np.zeros((4, 4), np.float32)))
+
+
+def test_select_outliers_matches_oracle():
+    wl = workloads.make_workload("quik_decode_8192", with_weights=False)
+    idx = host(Q.select_outliers(dev(wl.X_calib), 256))
+    assert np.array_equal(idx, O.select_outliers(wl.X_calib, 256))
+    rng = np.random.default_rng(5)
+    x = rng.integers(-3, 4, size=(16, 1000)).astype(np.float16)   # many exact ties
+    for k in (1, 7, 100, 1000):
+        assert np.array_equal(host(Q.select_outliers(dev(x), k)), O.select_outliers(x, k))
+
+
+# ---------------------------------------------------------------- W4A4 linear
+
+LINEAR_CASES = [
+    # (M, N, K, n_out)
+    (1, 16, 128, 0), (7, 100, 256, 0), (16, 256, 640, 0), (33, 300, 384, 0), (64, 512, 256, 0),
+    (65, 129, 128, 0), (128, 256, 512, 0), (200, 520, 384, 0), (300, 1000, 1024, 0),
+    (4, 64, 256, 8), (16, 200, 512, 40), (64, 256, 256, 256), (100, 300, 384, 64),
+    (256, 384, 256, 32), (3, 40, 0, 16), (130, 70, 0, 24),
+]
+
+
+@pytest.mark.parametrize("M,N,K,n_out", LINEAR_CASES)
+def test_linear_matches_oracle(M, N, K, n_out):
+    rng = np.random.default_rng(M * 1000 + N + K)
+    qa = rng.integers(-7, 8, size=(M, K)).astype(np.int8)
+    qw = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+    sa = rng.uniform(0.01, 0.2, M).astype(np.float32)
+    sw = rng.uniform(0.001, 0.01, N).astype(np.float32)
+    xo = (rng.standard_normal((M, n_out)) * 3).astype(np.float16) if n_out else None
+    wo = (rng.standard_normal((N, n_out)) * 0.02).astype(np.float16) if n_out else None
+    a_codes = dev(O.pack_int4(qa) if K else np.zeros((M, 0), np.uint8))
+    w_codes = dev(O.pack_int4(qw) if K else np.zeros((N, 0), np.uint8))
+    y, acc = Q.w4a4_linear(a_codes, dev(sa), w_codes, dev(sw),
+                           None if xo is None else dev(xo), None if wo is None else dev(wo),
+                           acc_debug=True)
+    torch.cuda.synchronize()
+    want_acc = O.int_gemm(qa, qw)
+    assert np.array_equal(host(acc).astype(np.int64), want_acc)
+    want_y = O.dequant_epilogue(want_acc, sa, sw, xo, wo).astype(np.float64)
+    got_y = host(y).astype(np.float64)
+    # fp32 epilogue vs float64: at most one fp16 rounding step apart
+    ulp = np.maximum(np.abs(want_y), 2.0 ** -14) * 2.0 ** -10
+    assert np.all(np.abs(got_y - want_y) <= ulp + 1e-3 * np.abs(want_y).max() * (n_out > 0))
+    assert rel_fro(got_y, want_y) < 1e-3
+
+
+def test_linear_extreme_codes_are_exact():
+    # all +-7 at the largest K: |acc| = 49*K, the int32 headroom case
+    K = 65536
+    a = np.full((2, K), 7, np.int8); a[1] = -7
+    w = np.full((32, K), 7, np.int8); w[1::2, ::2] = -7
+    y, acc = Q.w4a4_linear(dev(O.pack_int4(a)), dev(np.ones(2, np.float32)),
+                           dev(O.pack_int4(w)), dev(np.ones(32, np.float32)), acc_debug=True)
+    assert np.array_equal(host(acc).astype(np.int64), O.int_gemm(a, w))
+
+
+def test_linear_writes_into_strided_output():
+    rng = np.random.default_rng(9)
+    M, N, K = 40, 96, 256
+    qa = rng.integers(-7, 8, size=(M, K)); qw = rng.integers(-7, 8, size=(N, K))
+    big = torch.full((M, N + 13), 7.0, dtype=torch.float16, device="cuda")
+    out = big[:, 5:5 + N]                                   # ldy = N + 13, unaligned base
+    Q.w4a4_linear(dev(O.pack_int4(qa)), dev(np.ones(M, np.float32)),
+                  dev(O.pack_int4(qw)), dev(np.full(N, 0.5, np.float32)), out=out)
+    torch.cuda.synchronize()
+    want = O.dequant_epilogue(O.int_gemm(qa, qw), np.ones(M), np.full(N, 0.5))
+    np.testing.assert_array_equal(host(out), want)
+    assert np.all(host(big[:, :5]) == 7) and np.all(host(big[:, 5 + N:]) == 7)
+
+
+# ---------------------------------------------------------------- end to end
+
+E2E_CASES = [
+    ("tiny_256", None, None),
+    ("qkv_prefill_4096", 96, 512),
+    ("down_proj_gsr_11008", 40, 384),
+    ("flatquant_gate_up_8192", 24, 256),
+]
+
+
+def _oracle_rotation(wl):
+    s = wl.spec
+    if s.rotation == workloads.KRON:
+        return O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale,
+                          clip_ratio=s.clip_ratio)
+    kind = {workloads.HADAMARD: O.HADAMARD, workloads.GSR: O.GSR, workloads.NONE: O.NONE}
+    return O.Rotation(kind[s.rotation], block=s.block, clip_ratio=s.clip_ratio)
+
+
+@pytest.mark.parametrize("name,M,N", E2E_CASES, ids=[c[0] for c in E2E_CASES])
+def test_layer_end_to_end(name, M, N):
+    wl = workloads.make_workload(name, M=M, N=N)
+    rot = _oracle_rotation(wl)
+    layer = Q.QuantizedLinear(dev(wl.W), gpu_rotation(rot))
+    y = layer(dev(wl.X))
+    torch.cuda.synchronize()
+    a, ws, acc, y_ref = O.linear_forward(wl.X.astype(np.float64), wl.W.astype(np.float64), rot)
+    assert rel_fro(host(y), y_ref) < Y_TOL
+    # and the accumulators from the GPU's own codes are exact
+    codes, scales, _, _ = Q.rotate_quant(dev(wl.X), gpu_rotation(rot))
+    y2, acc2 = Q.w4a4_linear(codes, scales, layer.w_codes, layer.w_scales, acc_debug=True)
+    acc_ref, y2_ref = oracle_rows_from_gpu_codes(codes, scales, layer.w_codes, layer.w_scales)
+    assert np.array_equal(host(acc2).astype(np.int64), acc_ref)
+    assert rel_fro(host(y2), y2_ref) < 1e-3
+
+
+@pytest.mark.parametrize("M", workloads.DECODE_TOKENS)
+def test_quik_decode_end_to_end(M):
+    wl = workloads.make_workload("quik_decode_8192", M=M, N=1024)
+    rot = _oracle_rotation(wl)
+    idx = O.select_outliers(wl.X_calib, wl.spec.n_keep_fp16)
+    idx_g = Q.select_outliers(dev(wl.X_calib), wl.spec.n_keep_fp16)
+    layer = Q.QuantizedLinear(dev(wl.W), gpu_rotation(rot), idx_g)
+    y = layer(dev(wl.X))
+    torch.cuda.synchronize()
+    _, _, _, y_ref = O.linear_forward(wl.X.astype(np.float64), wl.W.astype(np.float64), rot, idx)
+    assert rel_fro(host(y), y_ref) < Y_TOL

@@ -1,0 +1,13 @@
+"""B200-native online W4A4 rotated linear layer.
+
+The layer rotates fp16 activations per token (Walsh-Hadamard, grouped
+sequency-ordered Walsh, or a Kronecker affine transform), quantizes them to
+symmetric 4-bit codes, multiplies the codes with pre-rotated 4-bit weights on
+tcgen05 integer tensor cores and dequantizes to fp16, adding the QUIK fp16
+outlier product.  The compute lives in libqr.so (include/qr.h); this package
+is its ctypes binding plus torch-facing helpers.
+"""
+from . import _lib  # noqa: F401
+from .layer import (GSR, HADAMARD, KRON, NONE, QuantizedLinear, Rotation,  # noqa: F401
+                    invert_transpose, pack_weights, packed_k, rotate_quant, select_outliers,
+                    w4a4_linear, weight_rotation)

@@ -1,0 +1,238 @@
+// qr_api.cu -- the extern "C" entry points: argument validation on the host,
+// then one launch on the caller's stream.  Nothing here allocates memory.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "qr_internal.h"
+
+namespace qr {
+
+namespace {
+
+__device__ int32_t g_status_word;   // see qr_device_status()
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int32_t* g_status_ptr[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+int g_smem[kMaxDevices] = {};
+
+int current_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
+  return d;
+}
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int32_t* device_status_word() {
+  const int d = current_device();
+  if (d < 0) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_status_ptr[d] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[d] = static_cast<int32_t*>(p);
+  }
+  return g_status_ptr[d];
+}
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0) return 1;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_sms[d] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d);
+    g_sms[d] = v > 0 ? v : 1;
+  }
+  return g_sms[d];
+}
+
+int max_smem_optin() {
+  const int d = current_device();
+  if (d < 0) return 48 * 1024;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_smem[d] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, d);
+    g_smem[d] = v > 0 ? v : 48 * 1024;
+  }
+  return g_smem[d];
+}
+
+// K_p for a descriptor, or -1.  Shared by qr_packed_k and the row calls.
+static int64_t packed_k(const qr_rotation* rot, int64_t K, int32_t n_out) {
+  if (rot == nullptr || K < 0 || n_out < 0 || n_out > K) return -1;
+  if (!(rot->clip_ratio > 0.0f && rot->clip_ratio <= 1.0f)) return -1;
+  const int64_t kr = K - n_out;
+  switch (rot->kind) {
+    case QR_ROT_NONE:
+      return (kr + 127) / 128 * 128;
+    case QR_ROT_HADAMARD:
+    case QR_ROT_GSR: {
+      const int64_t b = rot->block;
+      if (!is_pow2(b) || b > 16384) return -1;
+      if (rot->kind == QR_ROT_GSR && (b < 2 || b > 256)) return -1;
+      const int64_t unit = b > 128 ? b : 128;
+      return (kr + unit - 1) / unit * unit;
+    }
+    case QR_ROT_KRON: {
+      const int64_t n1 = rot->n1, n2 = rot->n2;
+      if (n1 < 4 || n2 < 4 || n1 % 4 || n2 % 4 || n1 + n2 > 192) return -1;
+      if ((n1 * n2) % 128 || kr != n1 * n2) return -1;
+      if (rot->p1 == nullptr || rot->p2 == nullptr) return -1;
+      if (rot->chan_scale != nullptr && rot->chan_mode != QR_CHAN_DIVIDE &&
+          rot->chan_mode != QR_CHAN_MULTIPLY)
+        return -1;
+      return kr;
+    }
+    default:
+      return -1;
+  }
+}
+
+static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t rows, int64_t K,
+                           int64_t ld, const int32_t* outlier_idx, int32_t n_out, uint8_t* codes,
+                           float* scales, uint16_t* out16, float* rot_debug, qr_stream stream) {
+  if (rot == nullptr || rows < 0 || K < 0 || n_out < 0 || n_out > K) return QR_ERR_INVALID_ARG;
+  const int64_t kp = packed_k(rot, K, n_out);
+  if (kp < 0) {
+    // distinguish malformed from merely unsupported where it is cheap to
+    if (rot->kind < QR_ROT_NONE || rot->kind > QR_ROT_KRON) return QR_ERR_INVALID_ARG;
+    return (rot->clip_ratio > 0.0f && rot->clip_ratio <= 1.0f) ? QR_ERR_UNSUPPORTED
+                                                               : QR_ERR_INVALID_ARG;
+  }
+  if (rows == 0) return QR_OK;
+  if (ld < K || src == nullptr || scales == nullptr) return QR_ERR_INVALID_ARG;
+  if (kp > 0 && codes == nullptr) return QR_ERR_INVALID_ARG;
+  if (n_out > 0 && (outlier_idx == nullptr || out16 == nullptr)) return QR_ERR_INVALID_ARG;
+  if (kp > 32768 || K > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
+  if (n_out > 0 && (K > 32768 || n_out > 8192)) return QR_ERR_UNSUPPORTED;
+  if (kp > 0 && !aligned16(codes)) return QR_ERR_ALIGNMENT;
+  RowJob job{};
+  job.src = src;
+  job.rows = rows;
+  job.K = K;
+  job.ld = ld;
+  job.outlier_idx = n_out > 0 ? outlier_idx : nullptr;
+  job.n_out = n_out;
+  job.Kp = static_cast<int32_t>(kp);
+  job.Kr = static_cast<int32_t>(K - n_out);
+  job.rot = rot;
+  job.codes = codes;
+  job.scales = scales;
+  job.out16 = n_out > 0 ? out16 : nullptr;
+  job.rot_debug = rot_debug;
+  return launch_rotate_quant(job, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace qr
+
+using namespace qr;
+
+extern "C" {
+
+int32_t qr_abi_version(void) { return QR_ABI_VERSION; }
+
+const char* qr_status_string(qr_status s) {
+  switch (s) {
+    case QR_OK: return "ok";
+    case QR_ERR_INVALID_ARG: return "invalid argument";
+    case QR_ERR_UNSUPPORTED: return "unsupported size or kind";
+    case QR_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case QR_ERR_CUDA: return "CUDA runtime error";
+    case QR_ERR_DEVICE: return "a kernel reported an error";
+  }
+  return "unknown status";
+}
+
+int64_t qr_packed_k(const qr_rotation* rot, int64_t K, int32_t n_out) {
+  return packed_k(rot, K, n_out);
+}
+
+qr_status qr_rotate_quant(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                          int64_t ldx, const int32_t* outlier_idx, int32_t n_out, uint8_t* codes,
+                          float* scales, uint16_t* x_out, float* x_rot_debug, qr_stream stream) {
+  return rows_call(rot, X, M, K, ldx, outlier_idx, n_out, codes, scales, x_out, x_rot_debug,
+                   stream);
+}
+
+qr_status qr_pack_weights(const qr_rotation* rot_w, const uint16_t* W, int64_t N, int64_t K,
+                          int64_t ldw, const int32_t* outlier_idx, int32_t n_out, uint8_t* w_codes,
+                          float* w_scales, uint16_t* w_out, float* w_rot_debug, qr_stream stream) {
+  return rows_call(rot_w, W, N, K, ldw, outlier_idx, n_out, w_codes, w_scales, w_out, w_rot_debug,
+                   stream);
+}
+
+qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales, const uint8_t* w_codes,
+                         const float* w_scales, int64_t M, int64_t N, int64_t K_p,
+                         const uint16_t* x_out, const uint16_t* w_out, int32_t n_out, uint16_t* Y,
+                         int64_t ldy, int32_t* acc_debug, qr_stream stream) {
+  if (M < 0 || N < 0 || K_p < 0 || n_out < 0) return QR_ERR_INVALID_ARG;
+  if (K_p % 128 != 0) return QR_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return QR_OK;
+  if (Y == nullptr || ldy < N || a_scales == nullptr || w_scales == nullptr)
+    return QR_ERR_INVALID_ARG;
+  if (K_p > 0 && (a_codes == nullptr || w_codes == nullptr)) return QR_ERR_INVALID_ARG;
+  if (n_out > 0 && (x_out == nullptr || w_out == nullptr)) return QR_ERR_INVALID_ARG;
+  if (K_p > 65536 || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
+  if (n_out % 8 != 0) return QR_ERR_UNSUPPORTED;
+  if (K_p > 0 && (!aligned16(a_codes) || !aligned16(w_codes))) return QR_ERR_ALIGNMENT;
+  if (n_out > 0 && (!aligned16(x_out) || !aligned16(w_out))) return QR_ERR_ALIGNMENT;
+  GemmJob j{};
+  j.a_codes = a_codes;
+  j.a_scales = a_scales;
+  j.w_codes = w_codes;
+  j.w_scales = w_scales;
+  j.M = M;
+  j.N = N;
+  j.Kp = K_p;
+  j.x_out = n_out > 0 ? x_out : nullptr;
+  j.w_out = n_out > 0 ? w_out : nullptr;
+  j.n_out = n_out;
+  j.Y = Y;
+  j.ldy = ldy;
+  j.acc_debug = acc_debug;
+  return launch_w4a4_gemm(j, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qr_status qr_select_outliers(const uint16_t* X_calib, int64_t T, int64_t K, int64_t ldx,
+                             int32_t k, int32_t* idx_out, qr_stream stream) {
+  if (T < 0 || K < 1 || k < 0 || k > K || ldx < K) return QR_ERR_INVALID_ARG;
+  if (k > 0 && (idx_out == nullptr || (T > 0 && X_calib == nullptr))) return QR_ERR_INVALID_ARG;
+  if (K > 16384) return QR_ERR_UNSUPPORTED;
+  return launch_select_outliers(X_calib, T, K, ldx, k, idx_out,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+qr_status qr_invert_transpose(const float* P, int32_t n, float* out, int32_t* info,
+                              qr_stream stream) {
+  if (P == nullptr || out == nullptr || info == nullptr || n < 1) return QR_ERR_INVALID_ARG;
+  if (n > 128) return QR_ERR_UNSUPPORTED;
+  return launch_invert_transpose(P, n, out, info, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qr_status qr_device_status(int32_t* code_out) {
+  if (code_out == nullptr) return QR_ERR_INVALID_ARG;
+  *code_out = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QR_ERR_CUDA;
+  int32_t* p = device_status_word();
+  if (p == nullptr) return QR_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return QR_ERR_CUDA;
+  if (v != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return QR_ERR_CUDA;
+  }
+  *code_out = v;
+  return QR_OK;
+}
+
+}  // extern "C"

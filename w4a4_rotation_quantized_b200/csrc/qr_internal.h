@@ -1,0 +1,55 @@
+// qr_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qr.h"
+
+namespace qr {
+
+// Device address of this device's status word (see qr_device_status).
+int32_t* device_status_word();
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+// Maximum opt-in dynamic shared memory per block of the current device.
+int max_smem_optin();
+
+// Parameters of the row kernels (rotate + quantize one matrix row by row);
+// used for activations (kernel a) and weights (kernel c) alike.
+struct RowJob {
+  const uint16_t* src;        // fp16 [rows x ld]
+  int64_t rows, K, ld;
+  const int32_t* outlier_idx; // [n_out] or null
+  int32_t n_out;
+  int32_t Kp;                 // packed width
+  int32_t Kr;                 // K - n_out, the rotated columns
+  const qr_rotation* rot;
+  uint8_t* codes;             // [rows x Kp/2]
+  float* scales;              // [rows]
+  uint16_t* out16;            // [rows x n_out] or null
+  float* rot_debug;           // [rows x Kp] or null
+};
+
+qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream);
+
+struct GemmJob {
+  const uint8_t* a_codes; const float* a_scales;
+  const uint8_t* w_codes; const float* w_scales;
+  int64_t M, N, Kp;
+  const uint16_t* x_out; const uint16_t* w_out; int32_t n_out;
+  uint16_t* Y; int64_t ldy;
+  int32_t* acc_debug;
+};
+
+qr_status launch_w4a4_gemm(const GemmJob& job, cudaStream_t stream);
+
+qr_status launch_select_outliers(const uint16_t* x, int64_t T, int64_t K, int64_t ld,
+                                 int32_t k, int32_t* idx_out, cudaStream_t stream);
+
+qr_status launch_invert_transpose(const float* P, int32_t n, float* out, int32_t* info,
+                                  cudaStream_t stream);
+
+}  // namespace qr

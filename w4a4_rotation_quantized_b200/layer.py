@@ -1,0 +1,158 @@
+"""Torch-facing helpers over the C ABI: allocate outputs as torch CUDA tensors,
+pass their pointers and the current stream, nothing else.  All arithmetic
+runs in libqr.so's kernels."""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+NONE, HADAMARD, GSR, KRON = L.QR_ROT_NONE, L.QR_ROT_HADAMARD, L.QR_ROT_GSR, L.QR_ROT_KRON
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _need_cuda(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+@dataclass
+class Rotation:
+    """Python-side rotation descriptor; keeps its device tensors alive."""
+    kind: int = NONE
+    block: int = 1
+    p1: Optional[torch.Tensor] = None       # fp32 [n1, n1] (KRON)
+    p2: Optional[torch.Tensor] = None       # fp32 [n2, n2]
+    chan_scale: Optional[torch.Tensor] = None   # fp32 [n1*n2]
+    chan_mode: int = L.QR_CHAN_DIVIDE
+    clip_ratio: float = 1.0
+    _c: Optional[L.QrRotation] = field(default=None, repr=False)
+
+    def c(self) -> L.QrRotation:
+        for t in (self.p1, self.p2, self.chan_scale):
+            if t is not None:
+                _need_cuda(t, torch.float32, "rotation tensor")
+                if not t.is_contiguous():
+                    raise ValueError("rotation tensors must be contiguous")
+        n1 = 0 if self.p1 is None else self.p1.shape[0]
+        n2 = 0 if self.p2 is None else self.p2.shape[0]
+        self._c = L.make_rotation(self.kind, self.block, _ptr(self.p1) or 0, n1,
+                                  _ptr(self.p2) or 0, n2, _ptr(self.chan_scale) or 0,
+                                  self.chan_mode, self.clip_ratio)
+        return self._c
+
+
+def invert_transpose(p: torch.Tensor) -> torch.Tensor:
+    """(P^{-1})^T on the GPU (fp64 Gauss-Jordan); raises if P is singular."""
+    _need_cuda(p, torch.float32, "P")
+    p = p.contiguous()
+    n = p.shape[0]
+    out = torch.empty_like(p)
+    info = torch.zeros(1, dtype=torch.int32, device=p.device)
+    L.qr_invert_transpose(p.data_ptr(), n, out.data_ptr(), info.data_ptr(), _stream())
+    if int(info.item()) != 0:
+        raise ValueError(f"P is singular (no pivot in column {int(info.item()) - 1})")
+    return out
+
+
+def weight_rotation(rot: Rotation) -> Rotation:
+    """The weight-side descriptor matching an activation-side one."""
+    if rot.kind != KRON:
+        return rot
+    return Rotation(KRON, p1=invert_transpose(rot.p1), p2=invert_transpose(rot.p2),
+                    chan_scale=rot.chan_scale, chan_mode=L.QR_CHAN_MULTIPLY,
+                    clip_ratio=rot.clip_ratio)
+
+
+def packed_k(rot: Rotation, K: int, n_out: int = 0) -> int:
+    kp = L.qr_packed_k(rot.c(), K, n_out)
+    if kp < 0:
+        raise ValueError("invalid rotation descriptor or sizes")
+    return kp
+
+
+def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool):
+    _need_cuda(x, torch.float16, "input")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("input must be a 2-D row-major tensor")
+    rows, K = x.shape
+    n_out = 0 if outlier_idx is None else int(outlier_idx.numel())
+    if n_out:
+        _need_cuda(outlier_idx, torch.int32, "outlier_idx")
+    crot = rot.c()
+    kp = L.qr_packed_k(crot, K, n_out)
+    if kp < 0:
+        raise ValueError("invalid rotation descriptor or sizes")
+    dev = x.device
+    codes = torch.empty((rows, kp // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(rows, dtype=torch.float32, device=dev)
+    out16 = torch.empty((rows, n_out), dtype=torch.float16, device=dev) if n_out else None
+    dbg = torch.empty((rows, kp), dtype=torch.float32, device=dev) if debug else None
+    fn(crot, x.data_ptr(), rows, K, x.stride(0), _ptr(outlier_idx) if n_out else None, n_out,
+       codes.data_ptr(), scales.data_ptr(), _ptr(out16), _ptr(dbg), _stream())
+    return codes, scales, out16, dbg
+
+
+def rotate_quant(x, rot: Rotation, outlier_idx=None, debug: bool = False):
+    """Online activation path: (codes, scales, x_out, x_rot or None)."""
+    return _rows(L.qr_rotate_quant, rot, x, outlier_idx, debug)
+
+
+def pack_weights(w, rot_w: Rotation, outlier_idx=None, debug: bool = False):
+    """Offline weight path: (codes, scales, w_out, w_rot or None)."""
+    return _rows(L.qr_pack_weights, rot_w, w, outlier_idx, debug)
+
+
+def w4a4_linear(a_codes, a_scales, w_codes, w_scales, x_out=None, w_out=None,
+                out: Optional[torch.Tensor] = None, acc_debug: bool = False):
+    """Y = fp16(acc * sa * sw + x_out w_out^T); returns (Y, acc or None)."""
+    M, kp2 = a_codes.shape
+    N = w_codes.shape[0]
+    n_out = 0 if x_out is None else x_out.shape[1]
+    dev = a_codes.device
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev) if acc_debug else None
+    L.qr_w4a4_linear(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(),
+                     w_scales.data_ptr(), M, N, 2 * kp2, _ptr(x_out), _ptr(w_out), n_out,
+                     y.data_ptr(), y.stride(0), _ptr(acc), _stream())
+    return y, acc
+
+
+def select_outliers(x_calib: torch.Tensor, k: int) -> torch.Tensor:
+    """QUIK calibration: the k columns of largest infinity-norm, ascending."""
+    _need_cuda(x_calib, torch.float16, "x_calib")
+    T, K = x_calib.shape
+    idx = torch.empty(k, dtype=torch.int32, device=x_calib.device)
+    L.qr_select_outliers(x_calib.data_ptr(), T, K, x_calib.stride(0), k, idx.data_ptr(),
+                         _stream())
+    return idx
+
+
+class QuantizedLinear:
+    """A linear layer held as rotated 4-bit weights; forward() is the online path."""
+
+    def __init__(self, weight: torch.Tensor, rot: Rotation, outlier_idx=None):
+        self.rot = rot
+        self.rot_w = weight_rotation(rot)
+        self.outlier_idx = outlier_idx
+        self.w_codes, self.w_scales, self.w_out, _ = pack_weights(weight, self.rot_w, outlier_idx)
+        self.out_features, self.in_features = weight.shape
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        codes, scales, x_out, _ = rotate_quant(x, self.rot, self.outlier_idx)
+        y, _ = w4a4_linear(codes, scales, self.w_codes, self.w_scales, x_out, self.w_out)
+        return y
+
+    __call__ = forward
