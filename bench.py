@@ -1,0 +1,475 @@
+"""Benchmark of the online W4A4 rotated linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--tokens M] [--no-cpu-baseline]
+
+One step is one pass of the layer's online hot path over one batch: rotate +
+quantize the activations (one kernel) and the W4A4 GEMM with its fused
+dequant/outlier epilogue (one kernel).  The weights are rotated and packed
+once, offline, before timing (their time is reported separately).  Default
+workload: the LLaMA-2-7B-shaped fused QKV prefill, X[2048 x 4096] through a
+full 4096-point Hadamard into W[12288 x 4096].
+
+Timing: W warm-up steps, then exactly K steps bracketed by a barrier and a
+device synchronize on both sides, CUDA events on the launching stream, max
+over ranks.  Inputs rotate over several copies whose total exceeds the
+126 MB L2, so no step reads inputs left in L2 by the previous one.  Under
+torchrun each rank runs an independent replica (tokens are independent; no
+collective on the data path): weak scaling.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "W4A4 linear TOPS & rotate+quant GB/s at 1 B200, % of INT8/HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 4.5 / 2.25          # nominal dense INT8 : dense BF16 on B200
+DATASHEET_INT8_TOPS = 4500.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = [("gpu_idle", "nvmlClocksEventReasonGpuIdle"),
+               ("applications_clocks", "nvmlClocksEventReasonApplicationsClocksSetting"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("sync_boost", "nvmlClocksEventReasonSyncBoost"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []          # (t, sm_mhz, reasons bitmask)
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.err = repr(e)
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self.thread.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": getattr(self, "err", "nvml unavailable")}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if len(win) < 3:       # very short timed region: widen to the samples around it
+            win = [s for s in self.samples if t0 - 0.5 <= s[0] <= t1 + 0.05]
+            window = "timed+0.5s before"
+        mhz = [s[1] for s in win]
+        mask = 0
+        for s in win:
+            mask |= s[2]
+        reasons = [name for name, attr in self.REASONS
+                   if getattr(self.nv, attr, 0) and (mask & getattr(self.nv, attr))
+                   and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win), "window": window}
+
+
+# --------------------------------------------------------------------------- workload
+
+def rotation_for(wl, Q):
+    s = wl.spec
+    import torch
+    if s.rotation == "kron":
+        return Q.Rotation(Q.KRON, p1=torch.from_numpy(wl.P1).cuda(),
+                          p2=torch.from_numpy(wl.P2).cuda(),
+                          chan_scale=torch.from_numpy(wl.chan_scale).cuda(),
+                          clip_ratio=s.clip_ratio)
+    kind = {"hadamard": Q.HADAMARD, "gsr": Q.GSR, "none": Q.NONE}[s.rotation]
+    return Q.Rotation(kind, block=s.block, clip_ratio=s.clip_ratio)
+
+
+def algorithmic_counts(wl, M, kp):
+    """Algorithmic work of one step (padding excluded)."""
+    s = wl.spec
+    K, N = s.K, s.N
+    n_out = s.n_keep_fp16
+    k_int = K - n_out
+    gemm_ops = 2.0 * M * N * k_int + 2.0 * M * N * n_out
+    # rotate+quant: read X, write packed codes, scales (and the fp16 outlier copy)
+    rq_bytes = M * K * 2 + M * k_int / 2 + M * 4 + M * n_out * 2
+    # GEMM: read codes, scales and outlier columns, write Y
+    gemm_bytes = (M + N) * k_int / 2 + (M + N) * 4 + (M + N) * n_out * 2 + M * N * 2
+    return gemm_ops, rq_bytes, gemm_bytes
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import w4a4_rotation_quantized_b200 as Q
+    import workloads
+    from w4a4_rotation_quantized_b200 import build as B
+
+    torch.cuda.set_device(local_rank)
+    if rank == 0:
+        B.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    Q._lib.load()
+
+    wl = workloads.make_workload(args.workload, M=args.tokens)
+    s = wl.spec
+    M = wl.X.shape[0]
+    rot = rotation_for(wl, Q)
+    idx = None
+    if s.n_keep_fp16:
+        idx = Q.select_outliers(torch.from_numpy(wl.X_calib).cuda(), s.n_keep_fp16)
+    kp = Q.packed_k(rot, s.K, s.n_keep_fp16)
+    gemm_ops, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp)
+
+    # input sets: enough copies that one pass over them exceeds L2 twice
+    x0 = torch.from_numpy(wl.X).cuda()
+    w0 = torch.from_numpy(wl.W).cuda()
+    t_pack0 = torch.cuda.Event(enable_timing=True)
+    t_pack1 = torch.cuda.Event(enable_timing=True)
+    t_pack0.record()
+    layer0 = Q.QuantizedLinear(w0, rot, idx)
+    t_pack1.record()
+    torch.cuda.synchronize()
+    pack_ms = t_pack0.elapsed_time(t_pack1)
+    set_bytes = x0.numel() * 2 + layer0.w_codes.numel() + 4 * s.N + \
+        (0 if layer0.w_out is None else layer0.w_out.numel() * 2)
+    nsets = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    xs = [x0] + [x0.clone() for _ in range(nsets - 1)]
+    wsets = [(layer0.w_codes, layer0.w_scales, layer0.w_out)]
+    for _ in range(nsets - 1):
+        wsets.append((layer0.w_codes.clone(), layer0.w_scales.clone(),
+                      None if layer0.w_out is None else layer0.w_out.clone()))
+    del w0
+    y = torch.empty((M, s.N), dtype=torch.float16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i, evs=None):
+        x = xs[i % nsets]
+        wc, wsc, wo = wsets[i % nsets]
+        if evs is not None:
+            evs[0].record(stream)
+        codes, scales, x_out, _ = Q.rotate_quant(x, rot, idx)
+        if evs is not None:
+            evs[1].record(stream)
+        Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
+        if evs is not None:
+            evs[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    status = Q._lib.qr_device_status()
+    if status != 0:
+        raise RuntimeError(f"a kernel reported device status {status:#x}")
+
+    elapsed_ms = start.elapsed_time(end)
+    rq_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    elapsed_ms = aggregate_max(elapsed_ms, world)
+
+    # end to end through the public API with host buffers
+    e2e_steps = min(args.steps, 50)
+    x_host = torch.from_numpy(wl.X).pin_memory()
+    y_host = torch.empty((M, s.N), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty_like(x0)
+    layer0_call = Q.QuantizedLinear.__call__
+    for _ in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        y_host.copy_(layer0_call(layer0, x_dev), non_blocking=True)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        y_host.copy_(layer0_call(layer0, x_dev), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = aggregate_max(e0.elapsed_time(e1), world) / e2e_steps
+
+    peaks, peak_src = load_peaks()
+    ms_per_step = elapsed_ms / args.steps
+    value = world * gemm_ops / (ms_per_step * 1e-3) / 1e12
+    gemm_avg = sum(gemm_ms) / len(gemm_ms)
+    rq_avg = sum(rq_ms) / len(rq_ms)
+    gemm_tops = gemm_ops / (gemm_avg * 1e-3) / 1e12
+    rq_gbs = rq_bytes / (rq_avg * 1e-3) / 1e9
+    int8_sust = peaks["bf16_tflops_sustained"] * INT8_PER_BF16
+    int8_burst = peaks["bf16_tflops"] * INT8_PER_BF16
+    hbm = peaks["hbm_gbs"]
+    clocks = sampler.summary(t0, t1)
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8",
+        "precision": "int4 codes on s8 tensor-core MMA, s32 accumulate; fp32 rotation; "
+                     "fp16 in/out",
+        "data": "synthetic",
+        "config": {"workload": s.name, "M": M, "K": s.K, "N": s.N, "K_p": kp,
+                   "rotation": f"{s.rotation}-{s.block}" if s.rotation != "kron"
+                   else f"kron-{s.n1}x{s.n2}", "n_out": s.n_keep_fp16,
+                   "clip_ratio": s.clip_ratio, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
+                         f"> 126 MB L2)"},
+        "roofline": {"bound": "tensor", "kernel": "w4a4_gemm_kernel",
+                     "achieved": round(gemm_tops, 1), "peak": round(int8_sust, 1),
+                     "unit": "TOP/s", "frac": round(gemm_tops / int8_sust, 4),
+                     "peak_source": f"{peak_src} bf16 sustained x {INT8_PER_BF16:g} (nominal "
+                                    f"INT8:BF16)",
+                     "frac_of_burst": round(gemm_tops / int8_burst, 4),
+                     "frac_of_datasheet_4500": round(gemm_tops / DATASHEET_INT8_TOPS, 4),
+                     "ops_per_launch": gemm_ops, "ms_per_launch": round(gemm_avg, 5),
+                     "traffic": None},
+        "rotate_quant": {"bound": "hbm", "kernel": "wht_rotate_quant_kernel",
+                         "achieved": round(rq_gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(rq_gbs / hbm, 4), "bytes_per_launch": rq_bytes,
+                         "ms_per_launch": round(rq_avg, 5)},
+        "gemm_hbm_bytes_per_launch": gemm_bytes,
+        "offline_weight_pack_ms": round(pack_ms, 3),
+        "e2e": {"value": round(world * gemm_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2), "steps": e2e_steps},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    return result
+
+
+def aggregate_max(value_ms: float, world: int) -> float:
+    """Max over ranks of a per-rank duration (device-timed)."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value_ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle
+
+def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None):
+    """Times the CPU oracle's online path on `tokens` tokens of the workload."""
+    import oracle as O
+    import workloads
+    from threadpoolctl import threadpool_info
+
+    wl = workloads.make_workload(workload, M=M_total)
+    s = wl.spec
+    if s.rotation == "kron":
+        rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale,
+                         clip_ratio=s.clip_ratio)
+    else:
+        rot = O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR, "none": O.NONE}[s.rotation],
+                         block=s.block, clip_ratio=s.clip_ratio)
+    idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
+    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)     # offline, untimed
+    x = wl.X[:tokens].astype(np.float64)
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        a = O.quantize_activations(x, rot, idx)
+        O.linear(a, wside)
+        times.append(time.perf_counter() - t0)
+    gemm_ops, _, _ = algorithmic_counts(wl, tokens, 0)
+    sec = statistics.median(times)
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    return {"value": round(gemm_ops / sec / 1e12, 6), "unit": "TOPS", "cores": threads,
+            "kind": "oracle", "seconds_per_sample": round(sec, 3),
+            "sample": f"{tokens} of {wl.X.shape[0]} tokens of {workload} through the oracle's "
+                      f"online path (rotate+quantize+integer GEMM+epilogue), median of {repeats}; "
+                      f"weights prepared untimed"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm, on the host cores."""
+    if rank != 0:
+        return None
+    import oracle as O
+    import workloads
+
+    wl = workloads.make_workload(args.workload, M=args.tokens)
+    s = wl.spec
+    tokens = min(wl.X.shape[0], args.reference_tokens)
+    if s.rotation == "kron":
+        rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale,
+                         clip_ratio=s.clip_ratio)
+    else:
+        rot = O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR, "none": O.NONE}[s.rotation],
+                         block=s.block, clip_ratio=s.clip_ratio)
+    idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
+    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)
+    x = wl.X[:tokens].astype(np.float64)
+
+    def step():
+        a = O.quantize_activations(x, rot, idx)
+        O.linear(a, wside)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    sec = (time.perf_counter() - t0) / args.steps
+    gemm_ops, _, _ = algorithmic_counts(wl, tokens, 0)
+    from threadpoolctl import threadpool_info
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    value = gemm_ops / sec / 1e12
+    sample = (f"{tokens} of {wl.X.shape[0]} tokens of {s.name} per step through the oracle's "
+              f"online path; weights prepared untimed")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": s.name, "M": tokens, "K": s.K, "N": s.N,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# --------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qkv_prefill_4096")
+    ap.add_argument("--tokens", type=int, default=None, help="override the token count M")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=256)
+    ap.add_argument("--reference-tokens", type=int, default=64)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                tokens = min(args.cpu_baseline_tokens, res["config"]["M"])
+                res["cpu_baseline"] = oracle_baseline(args.workload, tokens, repeats=3,
+                                                      M_total=args.tokens)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

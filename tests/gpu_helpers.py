@@ -55,7 +55,7 @@ def check_side(gpu, ref: O.Side, what: str, clip: float = 1.0, check_rot: bool =
     """Compares (codes, scales, fp16 part, rotated) from the GPU with an oracle Side."""
     codes, scales, out16, rot = gpu
     scales = host(scales)
-    if check_rot and rot is not None:
+    if check_rot and rot is not None and ref.rotated.shape[1]:
         r = host(rot).astype(np.float64)
         norm = np.linalg.norm(ref.rotated, axis=1)
         err = np.abs(r - ref.rotated).max(axis=1)

@@ -1,0 +1,67 @@
+"""The N>1 host logic of bench.py on CPU: two gloo ranks, max-over-ranks
+timing, and the launcher checks.  No GPU is touched."""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, values, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out[rank] = bench.aggregate_max(values[rank], world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    values = [3.25, 7.5]
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, values, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    assert out[0] == 7.5 and out[1] == 7.5
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.aggregate_max(1.5, 1) == 1.5
+
+
+def test_gpus_must_match_world_size(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "2"])
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "1"])
+
+
+def test_reference_arm_is_silent_on_other_ranks(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    assert bench.main(["--gpus", "2", "--impl", "reference", "--steps", "1"]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_counts_of_the_qkv_workload():
+    import workloads
+    wl = workloads.make_workload("qkv_prefill_4096", M=4, N=8, with_weights=False)
+    ops, rq, gm = bench.algorithmic_counts(wl, 2048, 4096)
+    assert ops == 2.0 * 2048 * 12288 * 4096
+    assert rq == 2048 * 4096 * 2 + 2048 * 4096 / 2 + 2048 * 4
