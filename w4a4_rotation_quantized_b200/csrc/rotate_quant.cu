@@ -69,24 +69,6 @@ __device__ __forceinline__ int gray_inverse(int g) {
   return g;
 }
 
-struct WhtParams {
-  const __half* src;
-  int64_t rows, ld;
-  int32_t K, Kr, Kp, n_out;
-  const int32_t* outlier_idx;
-  int32_t log_block;          // butterflies on index bits [0, log_block)
-  int32_t gsr;                // sequency order within blocks (log_block <= 8)
-  int32_t vec_ok;             // 16-byte loads allowed (aligned, no gather)
-  int32_t warps_per_row, rows_per_cta;
-  float clip_ratio, inv_sqrt_block;
-  uint8_t* codes;
-  float* scales;
-  __half* out16;
-  float* rot_debug;
-  // shared memory carve-up (byte offsets)
-  int32_t off_red, off_xbuf, off_gsr, off_kept, off_idx;
-};
-
 // Builds, in shared memory, kept[e] = the source column of rotated column e
 // (0xFFFF = none), from the strictly ascending outlier index list.  Malformed
 // lists never write outside [0, Kr).
@@ -108,209 +90,394 @@ __device__ void build_kept_table(const int32_t* __restrict__ outlier_idx, int n_
   __syncthreads();
 }
 
-template <int CPW, bool CLIP>
-__global__ void __launch_bounds__(256) wht_rotate_quant_kernel(const WhtParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int W = p.warps_per_row;
-  const int rg = warp / W;
-  const int wr = warp - rg * W;
-  const bool gather = p.n_out > 0;
+struct WhtParams {
+  const __half* src;
+  int64_t rows, ld;
+  int32_t K, Kr, Kp, n_out;
+  const int32_t* outlier_idx;
+  int32_t lb;                 // butterflies on in-block index bits [0, lb)
+  int32_t nb;                 // blocks per row, Kp >> lb
+  int32_t gsr;                // sequency order within blocks
+  int32_t vec_ok;             // 16-byte loads allowed (aligned rows, no gather)
+  int32_t nt;                 // threads per row group (multiple of 32)
+  int32_t rows_per_cta;       // row groups per CTA
+  int32_t items;              // items per thread in the register-held phase
+  float clip_ratio, inv_sqrt_block;
+  uint8_t* codes;
+  float* scales;
+  __half* out16;
+  float* rot_debug;
+  int32_t off_buf, buf_bytes, off_red, off_kept, off_idx;   // shared-memory carve-up
+};
 
-  uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
-  if (gather) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
-                               reinterpret_cast<int32_t*>(smem + p.off_idx));
+// Loads 8 consecutive rotated-domain elements [e, e+8) of a row as fp32:
+// gathered through the kept-column table when outliers are split off,
+// zero beyond the Kr real columns.
+__device__ __forceinline__ void load8(const WhtParams& p, const __half* srow, const uint16_t* kept,
+                                      int e, float (&x)[8]) {
+  if (p.n_out == 0 && p.vec_ok && e + 8 <= p.Kr) {
+    const uint4 u = ld_stream_v4(srow + e);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __half22float2(h[q]);
+      x[2 * q] = f.x;
+      x[2 * q + 1] = f.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ei = e + i;
+      float v = 0.0f;
+      if (ei < p.Kr) {
+        const int c = p.n_out ? static_cast<int>(kept[ei]) : ei;
+        if (c < p.K) v = __half2float(srow[c]);
+      }
+      x[i] = v;
+    }
+  }
+}
 
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * p.rows_per_cta + rg;
-  if (rg >= p.rows_per_cta || row >= p.rows) return;
-  const __half* srow = p.src + row * p.ld;
-  const int nthr_row = W * 32;
-
-  // QUIK outlier columns, copied through unchanged.
-  if (gather && p.out16 != nullptr) {
-    for (int j = wr * 32 + lane; j < p.n_out; j += nthr_row) {
+// The QUIK outlier columns of a row, copied through unchanged.
+__device__ __forceinline__ void copy_outliers(const WhtParams& p, const __half* srow, int64_t row,
+                                              int t, int nt) {
+  if (p.n_out > 0 && p.out16 != nullptr)
+    for (int j = t; j < p.n_out; j += nt) {
       const int c = __ldg(p.outlier_idx + j);
       p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? srow[c] : __float2half(0.0f);
     }
-  }
+}
 
-  // ---- load (gather + zero padding), fp16 -> fp32
-  float v[CPW][8];
-#pragma unroll
-  for (int j = 0; j < CPW; ++j) {
-    const int e0 = (wr * CPW + j) * 256 + lane * 8;
-    if (!gather && p.vec_ok && e0 + 8 <= p.Kr) {
-      const uint4 u = ld_stream_v4(srow + e0);
-      const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __half22float2(h[q]);
-        v[j][2 * q] = f.x;
-        v[j][2 * q + 1] = f.y;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int e = e0 + i;
-        float x = 0.0f;
-        if (e < p.Kr) {
-          const int c = gather ? static_cast<int>(kept[e]) : e;
-          if (c < p.K) x = __half2float(srow[c]);
-        }
-        v[j][i] = x;
-      }
-    }
-  }
+// Shared-memory position of rotated element e: bits 3-4 are XORed with the
+// two bits above the layout-B in-register bits, so that the 8-float groups a
+// warp reads in layout B fall in distinct banks.
+template <int SH>
+__device__ __forceinline__ int swz(int e) {
+  return e ^ (((e >> SH) & 3) << 3);
+}
 
-  const int lb = p.log_block;
-  // ---- butterflies on bits 0..2 (inside a thread)
-#pragma unroll
-  for (int s = 0; s < 3; ++s) {
-    if (s < lb) {
-#pragma unroll
-      for (int j = 0; j < CPW; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (!(i & (1 << s))) {
-            const float a = v[j][i], b = v[j][i | (1 << s)];
-            v[j][i] = a + b;
-            v[j][i | (1 << s)] = a - b;
-          }
-    }
-  }
-  // ---- bits 3..7 (across lanes): lower half keeps a+b, upper half a-b
-#pragma unroll
-  for (int s = 3; s < 8; ++s) {
-    if (s < lb) {
-      const int m = 1 << (s - 3);
-      const float sg = (lane & m) ? -1.0f : 1.0f;
-#pragma unroll
-      for (int j = 0; j < CPW; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float o = __shfl_xor_sync(0xffffffffu, v[j][i], m);
-          v[j][i] = fmaf(sg, v[j][i], o);
-        }
-    }
-  }
-  // ---- bits 8 .. 8+log2(CPW)-1 (across this thread's chunks)
-#pragma unroll
-  for (int t = 0; (1 << t) < CPW; ++t) {
-    if (8 + t < lb) {
-#pragma unroll
-      for (int j = 0; j < CPW; ++j)
-        if (!(j & (1 << t))) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a = v[j][i], b = v[j | (1 << t)][i];
-            v[j][i] = a + b;
-            v[j | (1 << t)][i] = a - b;
-          }
-        }
-    }
-  }
-  // ---- remaining bits: across the warps of the row, through shared memory
-  {
-    constexpr int LC = (CPW >= 16) ? 4 : (CPW >= 8) ? 3 : (CPW >= 4) ? 2 : (CPW >= 2) ? 1 : 0;
-    float* xb = reinterpret_cast<float*>(smem + p.off_xbuf) + static_cast<size_t>(rg) * W * CPW * 256;
-    for (int t = 0; 8 + LC + t < lb; ++t) {
-      float* mine = xb + static_cast<size_t>(wr) * CPW * 256;
-      float* peer = xb + static_cast<size_t>(wr ^ (1 << t)) * CPW * 256;
-#pragma unroll
-      for (int j = 0; j < CPW; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mine[(j * 8 + i) * 32 + lane] = v[j][i];
-      row_barrier(rg, nthr_row);
-      const bool upper = (wr >> t) & 1;
-#pragma unroll
-      for (int j = 0; j < CPW; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float o = peer[(j * 8 + i) * 32 + lane];
-          v[j][i] = upper ? (o - v[j][i]) : (v[j][i] + o);
-        }
-      row_barrier(rg, nthr_row);
-    }
-  }
-
-  // ---- row absmax
-  float am = 0.0f;
-#pragma unroll
-  for (int j = 0; j < CPW; ++j)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[j][i]));
+// Reduce a row's absmax over its row group; returns the maximum.
+__device__ __forceinline__ float row_absmax(float am, float* red, int rg, int t, int nt) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  if (W > 1) {
-    float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * W;
-    if (lane == 0) red[wr] = am;
-    row_barrier(rg, nthr_row);
+  const int nw = nt >> 5;
+  if (nw > 1) {
+    if ((t & 31) == 0) red[t >> 5] = am;
+    row_barrier(rg, nt);
     am = 0.0f;
-    for (int w = 0; w < W; ++w) am = fmaxf(am, red[w]);
+    for (int w = 0; w < nw; ++w) am = fmaxf(am, red[w]);
   }
+  return am;
+}
 
-  // s = alpha * max|x'| / 7 with x' = (unscaled butterfly output) / sqrt(b);
-  // the codes use the unscaled values times r = 7 / (alpha * max).
-  const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
-  const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
-  if (wr == 0 && lane == 0) p.scales[row] = s;
+// Sequency output of a block of 2^LB (6 <= LB <= 8) held by a layout-B
+// thread (natural in-block index tb_low + 8 j, j < 2^(LB-3)): output word k
+// (positions 8k..8k+7) takes Hadamard outputs perm(8k+t) = bitrev(gray(8k+t)),
+// whose three low bits do not depend on t, so one thread owns each word.  For
+// p_m the bits of a position, the low three bits of perm are
+// (p_{LB-1}, p_{LB-2}^p_{LB-1}, p_{LB-3}^p_{LB-2}); the in-register index j
+// of perm(8k+t) is a constant of (t, k's free bits) XOR p_{LB-3}.
+template <int LB>
+__host__ __device__ constexpr int gsr_j_static(int t, int f) {
+  // position with p_{LB-3..LB-1} = 0: pos = 8 f + t
+  int pos = 8 * f + t;
+  int j = 0;
+  for (int m = 3; m < LB; ++m) {
+    const int i = LB - 1 - m;                       // j bit (m-3) = g_i
+    const int gi = ((pos >> i) & 1) ^ ((i + 1 < LB) ? ((pos >> (i + 1)) & 1) : 0);
+    j |= gi << (m - 3);
+  }
+  return j;
+}
 
-  uint8_t* crow = p.codes + row * (p.Kp / 2);
-  if (!p.gsr) {
+// Kernel for blocks of 2^LB with LB = 3 + MB + HA >= 4.
+//   layout A: a thread holds in-block bits {0,1,2} and the top HA bits
+//             (2^(3+HA) values, loaded as 16-byte rows of 8), T_A = 2^MB
+//             threads per block;
+//   layout B: a thread holds the MB middle bits {3..2+MB} (2^MB values),
+//             T_B = 2^(3+HA) threads per block.
+// Butterflies run in registers in each layout; one pass through shared
+// memory (fp32, swizzled) moves the row from A to B.  OUT: 0 = natural order
+// via 8x8 nibble transposes across lanes, 1 = sequency order assembled in a
+// thread (HA = 0, 3 <= MB <= 5), 2 = codes scattered through shared memory.
+template <int MB, int HA, int ITEMS>
+struct AbBounds {
+  static constexpr int value = ((8 << HA) <= 64 && (1 << MB) * ITEMS <= 64) ? 512 : 256;
+};
+
+template <int MB, int HA, int ITEMS, bool CLIP, int OUT>
+__global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(const WhtParams p) {
+  constexpr int LB = 3 + MB + HA;
+  constexpr int EA = 8 << HA, TA = 1 << MB;
+  constexpr int EB = 1 << MB, TB = 8 << HA;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int nt = p.nt;
+  const int rg = threadIdx.x / nt;
+  const int t = threadIdx.x - rg * nt;
+  const int lane = threadIdx.x & 31;
+  uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
+  if (p.n_out > 0) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
+                                    reinterpret_cast<int32_t*>(smem + p.off_idx));
+  float* buf = reinterpret_cast<float*>(smem + p.off_buf + static_cast<size_t>(rg) * p.buf_bytes);
+  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 16;
+  const int items_a = p.nb * TA, items_b = p.nb * TB;
+  const int64_t row_step = static_cast<int64_t>(gridDim.x) * p.rows_per_cta;
+
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * p.rows_per_cta + rg; row < p.rows;
+       row += row_step) {
+    const __half* srow = p.src + row * p.ld;
+    copy_outliers(p, srow, row, t, nt);
+
+    // ---- phase A: load, butterflies on bits {0,1,2} and the top HA bits
+#pragma unroll 1
+    for (int w = t; w < items_a; w += nt) {
+      const int blk = w >> MB, ta = w & (TA - 1);
+      const int e0 = (blk << LB) + 8 * ta;
+      float v[EA];
 #pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int e0 = (wr * CPW + j) * 256 + lane * 8;
-      if (e0 < p.Kp) {
-        uint32_t word = 0;
+      for (int h = 0; h < (1 << HA); ++h) {
+        float x[8];
+        load8(p, srow, kept, e0 + (h << (3 + MB)), x);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word |= quant_nibble<CLIP>(v[j][i], r) << (4 * i);
-        *reinterpret_cast<uint32_t*>(crow + e0 / 2) = word;
-        if (p.rot_debug != nullptr) {
-          float* d = p.rot_debug + row * p.Kp + e0;
+        for (int i = 0; i < 8; ++i) v[8 * h + i] = x[i];
+      }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) d[i] = v[j][i] * p.inv_sqrt_block;
+      for (int s = 0; s < 3; ++s)
+#pragma unroll
+        for (int i = 0; i < EA; ++i)
+          if (!(i & (1 << s))) {
+            const float a = v[i], b = v[i | (1 << s)];
+            v[i] = a + b;
+            v[i | (1 << s)] = a - b;
+          }
+#pragma unroll
+      for (int s = 3; s < 3 + HA; ++s)
+#pragma unroll
+        for (int i = 0; i < EA; ++i)
+          if (!(i & (1 << s))) {
+            const float a = v[i], b = v[i | (1 << s)];
+            v[i] = a + b;
+            v[i | (1 << s)] = a - b;
+          }
+#pragma unroll
+      for (int h = 0; h < (1 << HA); ++h) {
+        const int e = e0 + (h << (3 + MB));
+        float4* d = reinterpret_cast<float4*>(buf + swz<3 + MB>(e));
+        d[0] = make_float4(v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3]);
+        d[1] = make_float4(v[8 * h + 4], v[8 * h + 5], v[8 * h + 6], v[8 * h + 7]);
+      }
+    }
+    row_barrier(rg, nt);
+
+    // ---- phase B: butterflies on the middle bits, absmax
+    float v[ITEMS][EB];
+    float am = 0.0f;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+      const int w = t + k * nt;
+      const bool ok = w < items_b;
+      const int blk = w >> (3 + HA), tb = w & (TB - 1);
+      const int e0 = (blk << LB) + (tb & 7) + ((tb >> 3) << (3 + MB));
+#pragma unroll
+      for (int j = 0; j < EB; ++j) v[k][j] = ok ? buf[swz<3 + MB>(e0 + 8 * j)] : 0.0f;
+#pragma unroll
+      for (int s = 0; s < MB; ++s)
+#pragma unroll
+        for (int j = 0; j < EB; ++j)
+          if (!(j & (1 << s))) {
+            const float a = v[k][j], b = v[k][j | (1 << s)];
+            v[k][j] = a + b;
+            v[k][j | (1 << s)] = a - b;
+          }
+#pragma unroll
+      for (int j = 0; j < EB; ++j) am = fmaxf(am, fabsf(v[k][j]));
+    }
+    am = row_absmax(am, red, rg, t, nt);
+    const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
+    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
+    if (t == 0) p.scales[row] = s;
+    uint8_t* crow = p.codes + row * (p.Kp >> 1);
+
+    if (p.rot_debug != nullptr) {
+#pragma unroll
+      for (int k = 0; k < ITEMS; ++k) {
+        const int w = t + k * nt;
+        if (w < items_b) {
+          const int blk = w >> (3 + HA), tb = w & (TB - 1);
+          const int e0 = (blk << LB) + (tb & 7) + ((tb >> 3) << (3 + MB));
+#pragma unroll
+          for (int j = 0; j < EB; ++j) {
+            int n = (e0 & ((1 << LB) - 1)) + 8 * j;
+            if (p.gsr) {
+              const int rev = static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - LB));
+              n = gray_inverse(rev);
+            }
+            p.rot_debug[row * p.Kp + (blk << LB) + n] = v[k][j] * p.inv_sqrt_block;
+          }
         }
       }
     }
-  } else {
-    // Natural Hadamard position q of a chunk -> sequency output position.
-    const int bmask = (1 << lb) - 1;
-    int pos[8];
+
+    if constexpr (OUT == 0) {
+      static_assert(MB >= 3, "nibble transposes need 8 values per lane");
+      const int l = lane & 7;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int q = lane * 8 + i;
-      const int n = q & bmask;
-      const int rev = lb ? static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - lb)) : 0;
-      pos[i] = (q & ~bmask) + gray_inverse(rev);
-    }
-    uint8_t* g = smem + p.off_gsr + static_cast<size_t>(rg) * p.Kp;
+      for (int k = 0; k < ITEMS; ++k) {
+        const int w = t + k * nt;
+        const int blk = w >> (3 + HA), tb = w & (TB - 1);
 #pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int c0 = (wr * CPW + j) * 256;
-      if (c0 + lane * 8 < p.Kp) {
+        for (int wb = 0; wb < EB / 8; ++wb) {
+          uint32_t W = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          g[c0 + pos[i]] = static_cast<uint8_t>(quant_nibble<CLIP>(v[j][i], r));
-          if (p.rot_debug != nullptr)
-            p.rot_debug[row * p.Kp + c0 + pos[i]] = v[j][i] * p.inv_sqrt_block;
+          for (int jj = 0; jj < 8; ++jj) W |= quant_nibble<CLIP>(v[k][8 * wb + jj], r) << (4 * jj);
+          // transpose the 8x8 nibble block held by lanes with tb_low = 0..7
+#pragma unroll
+          for (int m = 4; m >= 1; m >>= 1) {
+            const uint32_t mk = (m == 4) ? 0x0000FFFFu : (m == 2) ? 0x00FF00FFu : 0x0F0F0F0Fu;
+            const int sh = 4 * m;
+            const uint32_t P = __shfl_xor_sync(0xffffffffu, W, m);
+            W = (l & m) ? (((P >> sh) & mk) | (W & ~mk)) : ((W & mk) | ((P & mk) << sh));
+          }
+          if (w < items_b) {
+            const int e = (blk << LB) + 8 * (8 * wb + l) + ((tb >> 3) << (3 + MB));
+            *reinterpret_cast<uint32_t*>(crow + (e >> 1)) = W;
+          }
         }
       }
-    }
-    row_barrier(rg, nthr_row);
+    } else if constexpr (OUT == 1) {
+      static_assert(HA == 0 && MB >= 3 && MB <= 5, "in-thread sequency words");
 #pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int e0 = (wr * CPW + j) * 256 + lane * 8;
-      if (e0 < p.Kp) {
-        const uint32_t lo = *reinterpret_cast<const uint32_t*>(g + e0);
-        const uint32_t hi = *reinterpret_cast<const uint32_t*>(g + e0 + 4);
+      for (int k = 0; k < ITEMS; ++k) {
+        const int w = t + k * nt;
+        if (w < items_b) {
+          const int blk = w >> 3, tbl = w & 7;
+          const int a0 = tbl & 1, a1 = (tbl >> 1) & 1, a2 = (tbl >> 2) & 1;
+          const int p1 = a0, p2 = a1 ^ a0, p3 = a2 ^ p2;   // p_{LB-1}, p_{LB-2}, p_{LB-3}
+          uint32_t nib[EB];
+#pragma unroll
+          for (int j = 0; j < EB; ++j) nib[j] = quant_nibble<CLIP>(v[k][j], r);
+#pragma unroll
+          for (int f = 0; f < (1 << (MB - 3)); ++f) {
+            const int kw = f | (p3 << (MB - 3)) | (p2 << (MB - 2)) | (p1 << (MB - 1));
+            uint32_t W = 0;
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt) {
+              const int js = gsr_j_static<LB>(tt, f);
+              const uint32_t nv = p3 ? nib[js ^ 1] : nib[js];
+              W |= nv << (4 * tt);
+            }
+            *reinterpret_cast<uint32_t*>(crow + (((blk << LB) + 8 * kw) >> 1)) = W;
+          }
+        }
+      }
+    } else {
+      // codes through shared memory (one byte each), then packed
+      row_barrier(rg, nt);                 // every thread is done reading buf
+      uint8_t* cb = reinterpret_cast<uint8_t*>(buf);
+#pragma unroll
+      for (int k = 0; k < ITEMS; ++k) {
+        const int w = t + k * nt;
+        if (w < items_b) {
+          const int blk = w >> (3 + HA), tb = w & (TB - 1);
+          const int e0 = (blk << LB) + (tb & 7) + ((tb >> 3) << (3 + MB));
+#pragma unroll
+          for (int j = 0; j < EB; ++j) {
+            int n = (e0 & ((1 << LB) - 1)) + 8 * j;
+            if (p.gsr) {
+              const int rev = static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - LB));
+              n = gray_inverse(rev);
+            }
+            cb[(blk << LB) + n] = static_cast<uint8_t>(quant_nibble<CLIP>(v[k][j], r));
+          }
+        }
+      }
+      row_barrier(rg, nt);
+      for (int e = 8 * t; e < p.Kp; e += 8 * nt) {
+        const uint32_t lo = *reinterpret_cast<const uint32_t*>(cb + e);
+        const uint32_t hi = *reinterpret_cast<const uint32_t*>(cb + e + 4);
         const uint32_t plo = (lo & 0xFu) | ((lo >> 4) & 0xF0u) | ((lo >> 8) & 0xF00u) |
                              ((lo >> 12) & 0xF000u);
         const uint32_t phi = (hi & 0xFu) | ((hi >> 4) & 0xF0u) | ((hi >> 8) & 0xF00u) |
                              ((hi >> 12) & 0xF000u);
-        *reinterpret_cast<uint32_t*>(crow + e0 / 2) = plo | (phi << 16);
+        *reinterpret_cast<uint32_t*>(crow + (e >> 1)) = plo | (phi << 16);
       }
     }
+    row_barrier(rg, nt);                   // buf and red are reused by the next row
+  }
+}
+
+// Blocks of at most 8 (and no rotation): a thread holds ITEMS groups of 8
+// consecutive elements, all block bits are inside a thread.
+template <int ITEMS, bool CLIP>
+__global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int nt = p.nt;
+  const int rg = threadIdx.x / nt;
+  const int t = threadIdx.x - rg * nt;
+  uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
+  if (p.n_out > 0) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
+                                    reinterpret_cast<int32_t*>(smem + p.off_idx));
+  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 16;
+  const int lb = p.lb;
+  const int ngroups = p.Kp >> 3;
+  const int64_t row_step = static_cast<int64_t>(gridDim.x) * p.rows_per_cta;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * p.rows_per_cta + rg; row < p.rows;
+       row += row_step) {
+    const __half* srow = p.src + row * p.ld;
+    copy_outliers(p, srow, row, t, nt);
+    float v[ITEMS][8];
+    float am = 0.0f;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+      const int g = t + k * nt;
+      float x[8];
+      if (g < ngroups) {
+        load8(p, srow, kept, 8 * g, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+      }
+#pragma unroll
+      for (int s = 0; s < 3; ++s)
+        if (s < lb)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (!(i & (1 << s))) {
+              const float a = x[i], b = x[i | (1 << s)];
+              x[i] = a + b;
+              x[i | (1 << s)] = a - b;
+            }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[k][i] = x[i];
+        am = fmaxf(am, fabsf(x[i]));
+      }
+    }
+    am = row_absmax(am, red, rg, t, nt);
+    const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
+    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
+    if (t == 0) p.scales[row] = s;
+    uint8_t* crow = p.codes + row * (p.Kp >> 1);
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+      const int g = t + k * nt;
+      if (g < ngroups) {
+        uint32_t W = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          int pos = i;
+          if (p.gsr && lb > 0) {
+            const int bm = (1 << lb) - 1;
+            const int rev = static_cast<int>(__brev(static_cast<unsigned>(i & bm)) >> (32 - lb));
+            pos = (i & ~bm) + gray_inverse(rev);
+          }
+          W |= quant_nibble<CLIP>(v[k][i], r) << (4 * pos);
+          if (p.rot_debug != nullptr) p.rot_debug[row * p.Kp + 8 * g + pos] = v[k][i] * p.inv_sqrt_block;
+        }
+        *reinterpret_cast<uint32_t*>(crow + 4 * g) = W;
+      }
+    }
+    row_barrier(rg, nt);                   // red is reused by the next row
   }
 }
 
@@ -474,25 +641,83 @@ cudaError_t set_smem(Kernel k, size_t bytes) {
                               static_cast<int>(bytes));
 }
 
-template <int CPW, bool CLIP>
-cudaError_t launch_wht(const WhtParams& p, int grid, int threads, size_t smem, cudaStream_t s) {
-  auto k = wht_rotate_quant_kernel<CPW, CLIP>;
+template <typename Kernel>
+cudaError_t launch_rows_kernel(Kernel k, const WhtParams& p, int threads, size_t smem,
+                               cudaStream_t s) {
   cudaError_t e = set_smem(k, smem);
   if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t want = (p.rows + p.rows_per_cta - 1) / p.rows_per_cta;
+  const int64_t cap = static_cast<int64_t>(std::max(per_sm, 1)) * sm_count();
+  const int grid = static_cast<int>(std::min(want, cap));
   k<<<grid, threads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-template <bool CLIP>
-cudaError_t dispatch_cpw(int cpw, const WhtParams& p, int grid, int threads, size_t smem,
-                         cudaStream_t s) {
-  switch (cpw) {
-    case 1: return launch_wht<1, CLIP>(p, grid, threads, smem, s);
-    case 2: return launch_wht<2, CLIP>(p, grid, threads, smem, s);
-    case 4: return launch_wht<4, CLIP>(p, grid, threads, smem, s);
-    case 8: return launch_wht<8, CLIP>(p, grid, threads, smem, s);
-    default: return launch_wht<16, CLIP>(p, grid, threads, smem, s);
+template <int MB, int HA, int OUT, bool CLIP>
+cudaError_t dispatch_items(int items, const WhtParams& p, int threads, size_t smem,
+                           cudaStream_t s) {
+  constexpr int EB = 1 << MB;
+  constexpr int IMAX = (64 / EB) >= 8 ? 8 : ((64 / EB) < 1 ? 1 : 64 / EB);
+  switch (items) {
+    case 1: return launch_rows_kernel(wht_ab_kernel<MB, HA, 1, CLIP, OUT>, p, threads, smem, s);
+    case 2:
+      if constexpr (IMAX >= 2)
+        return launch_rows_kernel(wht_ab_kernel<MB, HA, 2, CLIP, OUT>, p, threads, smem, s);
+      break;
+    case 4:
+      if constexpr (IMAX >= 4)
+        return launch_rows_kernel(wht_ab_kernel<MB, HA, 4, CLIP, OUT>, p, threads, smem, s);
+      break;
+    case 8:
+      if constexpr (IMAX >= 8)
+        return launch_rows_kernel(wht_ab_kernel<MB, HA, 8, CLIP, OUT>, p, threads, smem, s);
+      break;
+    default: break;
   }
+  return cudaErrorInvalidValue;
+}
+
+template <bool CLIP>
+cudaError_t dispatch_ab(int lb, int out, int items, const WhtParams& p, int threads, size_t smem,
+                        cudaStream_t s) {
+  switch (lb) {
+    case 4: return dispatch_items<1, 0, 2, CLIP>(items, p, threads, smem, s);
+    case 5: return dispatch_items<2, 0, 2, CLIP>(items, p, threads, smem, s);
+    case 6: return out == 1 ? dispatch_items<3, 0, 1, CLIP>(items, p, threads, smem, s)
+                            : dispatch_items<3, 0, 0, CLIP>(items, p, threads, smem, s);
+    case 7: return out == 1 ? dispatch_items<4, 0, 1, CLIP>(items, p, threads, smem, s)
+                            : dispatch_items<4, 0, 0, CLIP>(items, p, threads, smem, s);
+    case 8: return out == 1 ? dispatch_items<5, 0, 1, CLIP>(items, p, threads, smem, s)
+                            : dispatch_items<5, 0, 0, CLIP>(items, p, threads, smem, s);
+    case 9: return dispatch_items<5, 1, 0, CLIP>(items, p, threads, smem, s);
+    case 10: return dispatch_items<5, 2, 0, CLIP>(items, p, threads, smem, s);
+    case 11: return dispatch_items<5, 3, 0, CLIP>(items, p, threads, smem, s);
+    case 12: return dispatch_items<6, 3, 0, CLIP>(items, p, threads, smem, s);
+    case 13: return dispatch_items<6, 4, 0, CLIP>(items, p, threads, smem, s);
+    case 14: return dispatch_items<7, 4, 0, CLIP>(items, p, threads, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <bool CLIP>
+cudaError_t dispatch_small(int items, const WhtParams& p, int threads, size_t smem,
+                           cudaStream_t s) {
+  switch (items) {
+    case 1: return launch_rows_kernel(wht_small_kernel<1, CLIP>, p, threads, smem, s);
+    case 2: return launch_rows_kernel(wht_small_kernel<2, CLIP>, p, threads, smem, s);
+    case 4: return launch_rows_kernel(wht_small_kernel<4, CLIP>, p, threads, smem, s);
+    case 8: return launch_rows_kernel(wht_small_kernel<8, CLIP>, p, threads, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int pow2_at_least(int v) {
+  int r = 1;
+  while (r < v) r <<= 1;
+  return r;
 }
 
 qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
@@ -507,7 +732,9 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.n_out = job.n_out;
   p.outlier_idx = job.outlier_idx;
   const int block = (rot.kind == QR_ROT_NONE) ? 1 : rot.block;
-  p.log_block = ilog2(block);
+  const int lb = ilog2(block);
+  p.lb = lb;
+  p.nb = job.Kp >> lb;
   p.gsr = rot.kind == QR_ROT_GSR;
   p.vec_ok = job.n_out == 0 && (reinterpret_cast<uintptr_t>(job.src) % 16 == 0) && (job.ld % 8 == 0);
   p.clip_ratio = rot.clip_ratio;
@@ -516,40 +743,53 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.scales = job.scales;
   p.out16 = reinterpret_cast<__half*>(job.out16);
   p.rot_debug = job.rot_debug;
+  if (job.Kp > 32768) return QR_ERR_UNSUPPORTED;
 
-  // Chunks per warp: enough registers to hold a whole block up to 4096
-  // elements, and no more than 8 warps per row unless the row is long.
-  const int chunks = (job.Kp + 255) / 256;
-  int cpw = 1;
-  if (p.log_block > 8) cpw = std::min(16, 1 << (p.log_block - 8));
-  while (cpw < 16 && (chunks + cpw - 1) / cpw > 8) cpw *= 2;
-  const int W = std::max(1, (chunks + cpw - 1) / cpw);
-  if (W > 8 || job.Kp > 32768) return QR_ERR_UNSUPPORTED;
-  const bool cross = p.log_block > 8 + ilog2(cpw);
-  int R = cross ? 1 : std::max(1, 8 / W);
+  const bool small = lb <= 3;
+  int items_total, imax;
+  int out = 0;
+  if (small) {
+    items_total = std::max(1, job.Kp / 8);
+    imax = 8;
+  } else {
+    const int mb = (lb <= 8) ? lb - 3 : (lb == 9 || lb == 10 || lb == 11) ? 5 : (lb == 14 ? 7 : 6);
+    const int ha = lb - 3 - mb;
+    items_total = p.nb * (8 << ha);
+    const int eb = 1 << mb;
+    imax = std::min(8, std::max(1, 64 / eb));
+    out = (lb <= 5) ? 2 : (p.gsr ? 1 : 0);
+  }
+  int nt = std::max(32, (((items_total + imax - 1) / imax) + 31) / 32 * 32);
+  if (nt > 512) return QR_ERR_UNSUPPORTED;
+  int items = pow2_at_least((items_total + nt - 1) / nt);
+  if (items > imax) return QR_ERR_UNSUPPORTED;
+  int R = std::max(1, std::min(8, 256 / nt));
   if (job.rows < R) R = static_cast<int>(std::max<int64_t>(job.rows, 1));
-  p.warps_per_row = W;
+  p.nt = nt;
+  p.items = items;
   p.rows_per_cta = R;
 
   size_t off = 0;
   p.off_red = static_cast<int32_t>(off);
-  off = align_up(off + sizeof(float) * R * W, 16);
-  p.off_xbuf = static_cast<int32_t>(off);
-  if (cross) off = align_up(off + sizeof(float) * static_cast<size_t>(R) * W * cpw * 256, 16);
-  p.off_gsr = static_cast<int32_t>(off);
-  if (p.gsr) off = align_up(off + static_cast<size_t>(R) * job.Kp, 16);
+  off = align_up(off + sizeof(float) * 16 * R, 16);
+  p.off_buf = static_cast<int32_t>(off);
+  p.buf_bytes = small ? 0 : static_cast<int32_t>(align_up(sizeof(float) * job.Kp, 16));
+  off += static_cast<size_t>(p.buf_bytes) * R;
   p.off_kept = static_cast<int32_t>(off);
   if (job.n_out > 0) off = align_up(off + sizeof(uint16_t) * job.Kr, 16);
   p.off_idx = static_cast<int32_t>(off);
   if (job.n_out > 0) off = align_up(off + sizeof(int32_t) * job.n_out, 16);
   if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
 
-  const int64_t grid64 = (job.rows + R - 1) / R;
-  if (grid64 > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
-  const int threads = R * W * 32;
+  const int threads = R * nt;
   const bool clip = rot.clip_ratio < 1.0f;
-  cudaError_t e = clip ? dispatch_cpw<true>(cpw, p, static_cast<int>(grid64), threads, off, stream)
-                       : dispatch_cpw<false>(cpw, p, static_cast<int>(grid64), threads, off, stream);
+  cudaError_t e;
+  if (small)
+    e = clip ? dispatch_small<true>(items, p, threads, off, stream)
+             : dispatch_small<false>(items, p, threads, off, stream);
+  else
+    e = clip ? dispatch_ab<true>(lb, out, items, p, threads, off, stream)
+             : dispatch_ab<false>(lb, out, items, p, threads, off, stream);
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
 
