@@ -156,6 +156,9 @@ LINEAR_CASES = [
     (65, 129, 128, 0), (128, 256, 512, 0), (200, 520, 384, 0), (300, 1000, 1024, 0),
     (4, 64, 256, 8), (16, 200, 512, 40), (64, 256, 256, 256), (100, 300, 384, 64),
     (256, 384, 256, 32), (3, 40, 0, 16), (130, 70, 0, 24),
+    # two-SM tiles: 256-row pairs, widths 128..224, ragged edges, long K
+    (257, 225, 384, 0), (512, 448, 1280, 0), (300, 1000, 11008, 0), (1000, 700, 256, 0),
+    (100, 4096, 128, 0), (65, 33, 0, 0),
 ]
 
 
@@ -184,19 +187,21 @@ def test_linear_matches_oracle(M, N, K, n_out):
     assert rel_fro(got_y, want_y) < 1e-3
 
 
-def test_linear_extreme_codes_are_exact():
+@pytest.mark.parametrize("M", [2, 100])
+def test_linear_extreme_codes_are_exact(M):
     # all +-7 at the largest K: |acc| = 49*K, the int32 headroom case
     K = 65536
-    a = np.full((2, K), 7, np.int8); a[1] = -7
+    a = np.full((M, K), 7, np.int8); a[1::2] = -7
     w = np.full((32, K), 7, np.int8); w[1::2, ::2] = -7
-    y, acc = Q.w4a4_linear(dev(O.pack_int4(a)), dev(np.ones(2, np.float32)),
+    y, acc = Q.w4a4_linear(dev(O.pack_int4(a)), dev(np.ones(M, np.float32)),
                            dev(O.pack_int4(w)), dev(np.ones(32, np.float32)), acc_debug=True)
     assert np.array_equal(host(acc).astype(np.int64), O.int_gemm(a, w))
 
 
-def test_linear_writes_into_strided_output():
+@pytest.mark.parametrize("M", [40, 100])
+def test_linear_writes_into_strided_output(M):
     rng = np.random.default_rng(9)
-    M, N, K = 40, 96, 256
+    N, K = 96, 256
     qa = rng.integers(-7, 8, size=(M, K)); qw = rng.integers(-7, 8, size=(N, K))
     big = torch.full((M, N + 13), 7.0, dtype=torch.float16, device="cuda")
     out = big[:, 5:5 + N]                                   # ldy = N + 13, unaligned base

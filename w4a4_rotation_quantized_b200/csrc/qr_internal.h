@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/qr.h"
@@ -45,6 +46,17 @@ struct GemmJob {
 };
 
 qr_status launch_w4a4_gemm(const GemmJob& job, cudaStream_t stream);
+
+// Prefill path: 2-SM tcgen05 MMA with the activation operand in TMEM
+// (M > 64, no fp16 outlier columns).
+qr_status launch_w4a4_gemm_pair(const GemmJob& job, cudaStream_t stream);
+int pair_tile_width(int64_t M, int64_t N, int sms);
+
+// Row-major 2-D tensor map: `rows` rows of `cols` elements, row pitch
+// `pitch_bytes`, box of box_cols x box_rows elements.
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr,
+                        uint64_t cols, uint64_t rows, uint64_t pitch_bytes, uint32_t box_cols,
+                        uint32_t box_rows, CUtensorMapSwizzle swz);
 
 qr_status launch_select_outliers(const uint16_t* x, int64_t T, int64_t K, int64_t ld,
                                  int32_t k, int32_t* idx_out, cudaStream_t stream);

@@ -353,9 +353,11 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -371,7 +373,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Row-major 2-D tensor of `rows` rows, `cols` elements per row, row pitch
 // `pitch_bytes`; box of box_cols x box_rows elements.
-bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* ptr,
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr,
               uint64_t cols, uint64_t rows, uint64_t pitch_bytes, uint32_t box_cols,
               uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
@@ -380,11 +382,12 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  (void)elem_bytes;
   return fn(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int BN, bool SWAP, bool OUT>
 cudaError_t run(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& moa,
@@ -415,6 +418,7 @@ qr_status launch_w4a4_gemm(const GemmJob& j, cudaStream_t stream) {
   if (j.M == 0 || j.N == 0) return QR_OK;
   const bool swap = j.M <= 64;
   const bool out = j.n_out > 0;
+  if (!swap && !out) return launch_w4a4_gemm_pair(j, stream);
   const int64_t rows_a = swap ? j.N : j.M;      // MMA-M side
   const int64_t rows_b = swap ? j.M : j.N;      // MMA-N side
   int bn;
@@ -450,16 +454,16 @@ qr_status launch_w4a4_gemm(const GemmJob& j, cudaStream_t stream) {
   CUtensorMap ma{}, mb{}, moa{}, mob{};
   const uint64_t kb = static_cast<uint64_t>(j.Kp) / 2;   // packed bytes per row
   if (p.kt > 0 &&
-      (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ca, kb, rows_a, kb, kStepBytes, kBM,
+      (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, ca, kb, rows_a, kb, kStepBytes, kBM,
                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-       !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cb, kb, rows_b, kb, kStepBytes, bn,
+       !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, cb, kb, rows_b, kb, kStepBytes, bn,
                  CU_TENSOR_MAP_SWIZZLE_NONE)))
     return QR_ERR_CUDA;
   if (out) {
     const uint64_t no = static_cast<uint64_t>(j.n_out);
-    if (!make_map(&moa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, oa, no, rows_a, no * 2, kOutStep, kBM,
+    if (!make_tensor_map_2d(&moa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, oa, no, rows_a, no * 2, kOutStep, kBM,
                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map(&mob, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ob, no, rows_b, no * 2, kOutStep, bn,
+        !make_tensor_map_2d(&mob, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ob, no, rows_b, no * 2, kOutStep, bn,
                   CU_TENSOR_MAP_SWIZZLE_64B))
       return QR_ERR_CUDA;
   } else {
