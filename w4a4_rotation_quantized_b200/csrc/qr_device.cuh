@@ -372,3 +372,76 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_add
 }
 
 }  // namespace qr
+
+namespace qr {
+
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completion counted on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Radix-2 Walsh-Hadamard stage on register-index bit S of v[E]: v[i], v[i|2^S]
+// -> sum, difference.  Bit 0 pairs adjacent registers and runs as scalar
+// adds; higher bits run two butterflies per f32x2 add/sub.
+template <int S, int E>
+__device__ __forceinline__ void wht_stage(float (&v)[E]) {
+  static_assert(S >= 0 && (1 << S) < E, "stage bit");
+  if constexpr (S == 0) {
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      const float a = v[i], b = v[i + 1];
+      v[i] = a + b;
+      v[i + 1] = a - b;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      if (i & (1 << S)) continue;
+      const uint64_t a = f2_pack(v[i], v[i + 1]);
+      const uint64_t b = f2_pack(v[i + (1 << S)], v[i + 1 + (1 << S)]);
+      f2_unpack(f2_add(a, b), v[i], v[i + 1]);
+      f2_unpack(f2_sub(a, b), v[i + (1 << S)], v[i + 1 + (1 << S)]);
+    }
+  }
+}
+
+template <int S0, int S1, int E>
+__device__ __forceinline__ void wht_stages(float (&v)[E]) {
+  if constexpr (S0 < S1) {
+    wht_stage<S0>(v);
+    wht_stages<S0 + 1, S1>(v);
+  }
+}
+
+}  // namespace qr

@@ -108,6 +108,9 @@ struct WhtParams {
   __half* out16;
   float* rot_debug;
   int32_t off_buf, buf_bytes, off_red, off_kept, off_idx;   // shared-memory carve-up
+  // ring mode: rows stream into shared memory by bulk copies
+  int32_t ring_slots, ring_row_bytes, off_ring, off_bars, rows_per_block;
+  int32_t* status;
 };
 
 // Loads 8 consecutive rotated-domain elements [e, e+8) of a row as fp32:
@@ -148,12 +151,13 @@ __device__ __forceinline__ void copy_outliers(const WhtParams& p, const __half* 
     }
 }
 
-// Shared-memory position of rotated element e: bits 3-4 are XORed with the
-// two bits above the layout-B in-register bits, so that the 8-float groups a
-// warp reads in layout B fall in distinct banks.
+// Shared-memory position of rotated element e: 8 floats of padding after
+// every 2^SH elements (SH = the layout-B stride bits), so that the 8-float
+// groups a warp reads in layout B fall in distinct banks while each thread's
+// layout-B values stay at constant offsets from one base.
 template <int SH>
 __device__ __forceinline__ int swz(int e) {
-  return e ^ (((e >> SH) & 3) << 3);
+  return e + ((e >> SH) << 3);
 }
 
 // Reduce a row's absmax over its row group; returns the maximum.
@@ -205,7 +209,7 @@ struct AbBounds {
   static constexpr int value = ((8 << HA) <= 64 && (1 << MB) * ITEMS <= 64) ? 512 : 256;
 };
 
-template <int MB, int HA, int ITEMS, bool CLIP, int OUT>
+template <int MB, int HA, int ITEMS, bool CLIP, int OUT, bool RING>
 __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(const WhtParams p) {
   constexpr int LB = 3 + MB + HA;
   constexpr int EA = 8 << HA, TA = 1 << MB;
@@ -221,12 +225,68 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
   float* buf = reinterpret_cast<float*>(smem + p.off_buf + static_cast<size_t>(rg) * p.buf_bytes);
   float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 16;
   const int items_a = p.nb * TA, items_b = p.nb * TB;
-  const int64_t row_step = static_cast<int64_t>(gridDim.x) * p.rows_per_cta;
 
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * p.rows_per_cta + rg; row < p.rows;
-       row += row_step) {
+  // Ring mode: the CTA owns rows [row0, row1); a producer warp (after the
+  // row groups) streams them into ring slots with bulk copies; row group g
+  // takes the CTA's rows g, g+R, ...
+  uint64_t* ring_full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
+  uint64_t* ring_empty = ring_full + p.ring_slots;
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(ring_empty + p.ring_slots);
+  int64_t row0 = 0, row1 = 0;
+  if constexpr (RING) {
+    row0 = static_cast<int64_t>(blockIdx.x) * p.rows_per_block;
+    row1 = row0 + p.rows_per_block < p.rows ? row0 + p.rows_per_block : p.rows;
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < p.ring_slots; ++i) {
+        mbar_init(&ring_full[i], 1);
+        mbar_init(&ring_empty[i], nt / 32);
+      }
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+    __syncthreads();
+    if (rg == p.rows_per_cta) {            // the producer warp
+      if (lane == 0) {
+        const int n = static_cast<int>(row1 - row0);
+        int i = 0;
+        bool ok = true;
+        for (; i < n; ++i) {
+          const int s = i % p.ring_slots;
+          const uint32_t ph = (i / p.ring_slots) & 1;
+          if (!(ok = mbar_wait_bounded(&ring_empty[s], ph ^ 1, abort_flag, p.status,
+                                       kDevTimeoutProducer)))
+            break;
+          mbar_arrive_expect_tx(&ring_full[s], p.ring_row_bytes);
+          bulk_load(smem + p.off_ring + static_cast<size_t>(s) * p.ring_row_bytes,
+                    p.src + (row0 + i) * p.ld, p.ring_row_bytes, &ring_full[s]);
+        }
+        // every copy issued lands before the CTA may exit
+        for (int j = (i > p.ring_slots ? i - p.ring_slots : 0); j < i; ++j)
+          mbar_wait_bounded(&ring_full[j % p.ring_slots], (j / p.ring_slots) & 1, abort_flag,
+                            nullptr, 0, kDrainLimitNs);
+      }
+      return;
+    }
+  }
+  const int64_t row_first = RING ? row0 + rg : static_cast<int64_t>(blockIdx.x) * p.rows_per_cta + rg;
+  const int64_t row_end = RING ? row1 : p.rows;
+  const int64_t row_step = RING ? p.rows_per_cta : static_cast<int64_t>(gridDim.x) * p.rows_per_cta;
+
+  for (int64_t row = row_first; row < row_end; row += row_step) {
     const __half* srow = p.src + row * p.ld;
-    copy_outliers(p, srow, row, t, nt);
+    const __half* ring_row = nullptr;
+    int slot = 0;
+    if constexpr (RING) {
+      const int i = static_cast<int>(row - row0);
+      slot = i % p.ring_slots;
+      if (!mbar_wait_bounded(&ring_full[slot], (i / p.ring_slots) & 1, abort_flag, p.status,
+                             kDevTimeoutWiden))
+        break;
+      ring_row = reinterpret_cast<const __half*>(smem + p.off_ring +
+                                                 static_cast<size_t>(slot) * p.ring_row_bytes);
+    } else {
+      copy_outliers(p, srow, row, t, nt);
+    }
 
     // ---- phase A: load, butterflies on bits {0,1,2} and the top HA bits
 #pragma unroll 1
@@ -237,28 +297,28 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
 #pragma unroll
       for (int h = 0; h < (1 << HA); ++h) {
         float x[8];
-        load8(p, srow, kept, e0 + (h << (3 + MB)), x);
+        const int e = e0 + (h << (3 + MB));
+        if constexpr (RING) {
+          if (e + 8 <= p.Kr) {
+            const uint4 u = *reinterpret_cast<const uint4*>(ring_row + e);
+            const __half2* hh = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 f = __half22float2(hh[q]);
+              x[2 * q] = f.x;
+              x[2 * q + 1] = f.y;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+          }
+        } else {
+          load8(p, srow, kept, e, x);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[8 * h + i] = x[i];
       }
-#pragma unroll
-      for (int s = 0; s < 3; ++s)
-#pragma unroll
-        for (int i = 0; i < EA; ++i)
-          if (!(i & (1 << s))) {
-            const float a = v[i], b = v[i | (1 << s)];
-            v[i] = a + b;
-            v[i | (1 << s)] = a - b;
-          }
-#pragma unroll
-      for (int s = 3; s < 3 + HA; ++s)
-#pragma unroll
-        for (int i = 0; i < EA; ++i)
-          if (!(i & (1 << s))) {
-            const float a = v[i], b = v[i | (1 << s)];
-            v[i] = a + b;
-            v[i | (1 << s)] = a - b;
-          }
+      wht_stages<0, 3 + HA>(v);
 #pragma unroll
       for (int h = 0; h < (1 << HA); ++h) {
         const int e = e0 + (h << (3 + MB));
@@ -266,6 +326,10 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
         d[0] = make_float4(v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3]);
         d[1] = make_float4(v[8 * h + 4], v[8 * h + 5], v[8 * h + 6], v[8 * h + 7]);
       }
+    }
+    if constexpr (RING) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring_empty[slot]);
     }
     row_barrier(rg, nt);
 
@@ -278,17 +342,10 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
       const bool ok = w < items_b;
       const int blk = w >> (3 + HA), tb = w & (TB - 1);
       const int e0 = (blk << LB) + (tb & 7) + ((tb >> 3) << (3 + MB));
+      const float* bp = buf + swz<3 + MB>(e0);          // e0 + 8j never crosses 2^(3+MB)
 #pragma unroll
-      for (int j = 0; j < EB; ++j) v[k][j] = ok ? buf[swz<3 + MB>(e0 + 8 * j)] : 0.0f;
-#pragma unroll
-      for (int s = 0; s < MB; ++s)
-#pragma unroll
-        for (int j = 0; j < EB; ++j)
-          if (!(j & (1 << s))) {
-            const float a = v[k][j], b = v[k][j | (1 << s)];
-            v[k][j] = a + b;
-            v[k][j | (1 << s)] = a - b;
-          }
+      for (int j = 0; j < EB; ++j) v[k][j] = ok ? bp[8 * j] : 0.0f;
+      wht_stages<0, MB>(v[k]);
 #pragma unroll
       for (int j = 0; j < EB; ++j) am = fmaxf(am, fabsf(v[k][j]));
     }
@@ -656,48 +713,60 @@ cudaError_t launch_rows_kernel(Kernel k, const WhtParams& p, int threads, size_t
   return cudaGetLastError();
 }
 
-template <int MB, int HA, int OUT, bool CLIP>
-cudaError_t dispatch_items(int items, const WhtParams& p, int threads, size_t smem,
+// Ring-mode launch: one CTA per SM (at most one per row), contiguous rows.
+template <typename Kernel>
+cudaError_t launch_ring_kernel(Kernel k, const WhtParams& p, int threads, size_t smem,
+                               int grid, cudaStream_t s) {
+  cudaError_t e = set_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, threads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int MB, int HA, int OUT, bool CLIP, bool RING>
+cudaError_t dispatch_items(int items, const WhtParams& p, int threads, size_t smem, int grid,
                            cudaStream_t s) {
   constexpr int EB = 1 << MB;
   constexpr int IMAX = (64 / EB) >= 8 ? 8 : ((64 / EB) < 1 ? 1 : 64 / EB);
+#define QR_LAUNCH(I)                                                                      \
+  return RING ? launch_ring_kernel(wht_ab_kernel<MB, HA, I, CLIP, OUT, RING>, p, threads, \
+                                   smem, grid, s)                                         \
+              : launch_rows_kernel(wht_ab_kernel<MB, HA, I, CLIP, OUT, RING>, p, threads, smem, s)
   switch (items) {
-    case 1: return launch_rows_kernel(wht_ab_kernel<MB, HA, 1, CLIP, OUT>, p, threads, smem, s);
+    case 1: QR_LAUNCH(1);
     case 2:
-      if constexpr (IMAX >= 2)
-        return launch_rows_kernel(wht_ab_kernel<MB, HA, 2, CLIP, OUT>, p, threads, smem, s);
+      if constexpr (IMAX >= 2) { QR_LAUNCH(2); }
       break;
     case 4:
-      if constexpr (IMAX >= 4)
-        return launch_rows_kernel(wht_ab_kernel<MB, HA, 4, CLIP, OUT>, p, threads, smem, s);
+      if constexpr (IMAX >= 4) { QR_LAUNCH(4); }
       break;
     case 8:
-      if constexpr (IMAX >= 8)
-        return launch_rows_kernel(wht_ab_kernel<MB, HA, 8, CLIP, OUT>, p, threads, smem, s);
+      if constexpr (IMAX >= 8) { QR_LAUNCH(8); }
       break;
     default: break;
   }
+#undef QR_LAUNCH
   return cudaErrorInvalidValue;
 }
 
-template <bool CLIP>
+template <bool CLIP, bool RING>
 cudaError_t dispatch_ab(int lb, int out, int items, const WhtParams& p, int threads, size_t smem,
-                        cudaStream_t s) {
+                        int grid, cudaStream_t s) {
   switch (lb) {
-    case 4: return dispatch_items<1, 0, 2, CLIP>(items, p, threads, smem, s);
-    case 5: return dispatch_items<2, 0, 2, CLIP>(items, p, threads, smem, s);
-    case 6: return out == 1 ? dispatch_items<3, 0, 1, CLIP>(items, p, threads, smem, s)
-                            : dispatch_items<3, 0, 0, CLIP>(items, p, threads, smem, s);
-    case 7: return out == 1 ? dispatch_items<4, 0, 1, CLIP>(items, p, threads, smem, s)
-                            : dispatch_items<4, 0, 0, CLIP>(items, p, threads, smem, s);
-    case 8: return out == 1 ? dispatch_items<5, 0, 1, CLIP>(items, p, threads, smem, s)
-                            : dispatch_items<5, 0, 0, CLIP>(items, p, threads, smem, s);
-    case 9: return dispatch_items<5, 1, 0, CLIP>(items, p, threads, smem, s);
-    case 10: return dispatch_items<5, 2, 0, CLIP>(items, p, threads, smem, s);
-    case 11: return dispatch_items<5, 3, 0, CLIP>(items, p, threads, smem, s);
-    case 12: return dispatch_items<6, 3, 0, CLIP>(items, p, threads, smem, s);
-    case 13: return dispatch_items<6, 4, 0, CLIP>(items, p, threads, smem, s);
-    case 14: return dispatch_items<7, 4, 0, CLIP>(items, p, threads, smem, s);
+    case 4: return dispatch_items<1, 0, 2, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 5: return dispatch_items<2, 0, 2, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 6: return out == 1 ? dispatch_items<3, 0, 1, CLIP, RING>(items, p, threads, smem, grid, s)
+                            : dispatch_items<3, 0, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 7: return out == 1 ? dispatch_items<4, 0, 1, CLIP, RING>(items, p, threads, smem, grid, s)
+                            : dispatch_items<4, 0, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 8: return out == 1 ? dispatch_items<5, 0, 1, CLIP, RING>(items, p, threads, smem, grid, s)
+                            : dispatch_items<5, 0, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 9: return dispatch_items<5, 1, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 10: return dispatch_items<5, 2, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 11: return dispatch_items<5, 3, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 12: return dispatch_items<6, 3, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 13: return dispatch_items<6, 4, 0, CLIP, RING>(items, p, threads, smem, grid, s);
+    case 14: return dispatch_items<7, 4, 0, CLIP, RING>(items, p, threads, smem, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -748,6 +817,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   const bool small = lb <= 3;
   int items_total, imax;
   int out = 0;
+  int ea = 8, eb = 1;
   if (small) {
     items_total = std::max(1, job.Kp / 8);
     imax = 8;
@@ -755,7 +825,8 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
     const int mb = (lb <= 8) ? lb - 3 : (lb == 9 || lb == 10 || lb == 11) ? 5 : (lb == 14 ? 7 : 6);
     const int ha = lb - 3 - mb;
     items_total = p.nb * (8 << ha);
-    const int eb = 1 << mb;
+    ea = 8 << ha;
+    eb = 1 << mb;
     imax = std::min(8, std::max(1, 64 / eb));
     out = (lb <= 5) ? 2 : (p.gsr ? 1 : 0);
   }
@@ -773,7 +844,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.off_red = static_cast<int32_t>(off);
   off = align_up(off + sizeof(float) * 16 * R, 16);
   p.off_buf = static_cast<int32_t>(off);
-  p.buf_bytes = small ? 0 : static_cast<int32_t>(align_up(sizeof(float) * job.Kp, 16));
+  p.buf_bytes = small ? 0 : static_cast<int32_t>(align_up(sizeof(float) * (job.Kp + job.Kp / 8 + 8), 16));
   off += static_cast<size_t>(p.buf_bytes) * R;
   p.off_kept = static_cast<int32_t>(off);
   if (job.n_out > 0) off = align_up(off + sizeof(uint16_t) * job.Kr, 16);
@@ -781,15 +852,55 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   if (job.n_out > 0) off = align_up(off + sizeof(int32_t) * job.n_out, 16);
   if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
 
-  const int threads = R * nt;
+  p.status = device_status_word();
+  // Ring mode: aligned rows without an outlier gather stream into shared
+  // memory by bulk copies, all of a CTA's rows in flight at once when they fit.
+  bool ring = !small && job.n_out == 0 && p.vec_ok && (job.K % 8 == 0) && job.K > 0 &&
+              p.status != nullptr;
+  int grid = 0;
+  if (ring) {
+    const int64_t blocks = std::min<int64_t>(job.rows, sm_count());
+    const int64_t per_block = (job.rows + blocks - 1) / blocks;
+    const int row_bytes = static_cast<int>(job.K * 2);
+    const int max_groups = std::max(1, std::min(8, (512 - 32) / nt));
+    const int bound = (ea <= 64 && eb * items <= 64) ? 512 : 256;   // the kernel's launch bound
+    int groups = static_cast<int>(std::min<int64_t>(max_groups, per_block));
+    while (groups > 1 && groups * nt + 32 > bound) --groups;
+    // layout: red | row-group buffers | ring slots | barriers
+    size_t roff = align_up(sizeof(float) * 16 * groups, 16);
+    const size_t buf_off = roff;
+    roff = align_up(roff + static_cast<size_t>(p.buf_bytes) * groups, 128);
+    const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - static_cast<int64_t>(roff) -
+                         16 * per_block - 16 - 1024) / row_bytes;
+    const int slots = static_cast<int>(std::min<int64_t>(per_block, fit));
+    if (slots >= 1 && groups * nt + 32 <= bound) {
+      p.off_red = 0;
+      p.off_buf = static_cast<int32_t>(buf_off);
+      p.off_kept = p.off_idx = 0;                                // no outlier gather here
+      p.ring_slots = slots;
+      p.ring_row_bytes = row_bytes;
+      p.off_ring = static_cast<int32_t>(roff);
+      p.off_bars = static_cast<int32_t>(align_up(roff + static_cast<size_t>(slots) * row_bytes, 16));
+      p.rows_per_block = static_cast<int32_t>(per_block);
+      p.rows_per_cta = groups;                                   // row groups
+      off = p.off_bars + 16 * static_cast<size_t>(slots) + 16;
+      grid = static_cast<int>((job.rows + per_block - 1) / per_block);
+    } else {
+      ring = false;
+    }
+  }
+  const int threads = ring ? p.rows_per_cta * nt + 32 : R * nt;
   const bool clip = rot.clip_ratio < 1.0f;
   cudaError_t e;
   if (small)
     e = clip ? dispatch_small<true>(items, p, threads, off, stream)
              : dispatch_small<false>(items, p, threads, off, stream);
+  else if (ring)
+    e = clip ? dispatch_ab<true, true>(lb, out, items, p, threads, off, grid, stream)
+             : dispatch_ab<false, true>(lb, out, items, p, threads, off, grid, stream);
   else
-    e = clip ? dispatch_ab<true>(lb, out, items, p, threads, off, stream)
-             : dispatch_ab<false>(lb, out, items, p, threads, off, stream);
+    e = clip ? dispatch_ab<true, false>(lb, out, items, p, threads, off, 0, stream)
+             : dispatch_ab<false, false>(lb, out, items, p, threads, off, 0, stream);
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
 
