@@ -49,6 +49,40 @@ __device__ __forceinline__ uint32_t quant_nibble(float v, float r) {
   return __float_as_uint(t) & 0xFu;
 }
 
+// Byte-permute (PTX prmt): byte i of the result is byte sel[i] of {b, a}.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Eight consecutive codes round_half_even(v[i] * r) (clamped to +-7 when
+// CLIP) packed two per byte, v[0] in the low nibble.  Each fused multiply-add
+// with 1.5*2^23 leaves the integer's two's-complement byte in the low byte;
+// byte permutes gather the even and the odd codes, and one shift and one
+// 3-input logic op interleave their nibbles.
+template <bool CLIP>
+__device__ __forceinline__ uint32_t quant_word(const float (&v)[8], float r) {
+  uint32_t b[8];
+  const uint64_t r2 = f2_pack(r, r), c2 = f2_pack(kRoundMagic, kRoundMagic);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float t0, t1;
+    f2_unpack(f2_fma(f2_pack(v[i], v[i + 1]), r2, c2), t0, t1);
+    if (CLIP) {
+      t0 = fminf(fmaxf(t0, kRoundMagic - 7.0f), kRoundMagic + 7.0f);
+      t1 = fminf(fmaxf(t1, kRoundMagic - 7.0f), kRoundMagic + 7.0f);
+    }
+    b[i] = __float_as_uint(t0);
+    b[i + 1] = __float_as_uint(t1);
+  }
+  const uint32_t even = prmt(prmt(b[0], b[2], 0x0040u), prmt(b[4], b[6], 0x4000u), 0x7610u);
+  const uint32_t odd = prmt(prmt(b[1], b[3], 0x0040u), prmt(b[5], b[7], 0x4000u), 0x7610u);
+  uint32_t w;
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(w) : "r"(even), "r"(odd << 4), "r"(0x0F0F0F0Fu));
+  return w;   // (even & 0x0F0F0F0F) | ((odd << 4) & ~0x0F0F0F0F)
+}
+
 __device__ __forceinline__ void row_barrier(int group, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(group + 1), "r"(nthreads) : "memory");
 }
@@ -378,22 +412,31 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
     if constexpr (OUT == 0) {
       static_assert(MB >= 3, "nibble transposes need 8 values per lane");
       const int l = lane & 7;
+      const uint32_t sel4 = (l & 4) ? 0x3276u : 0x5410u;
+      const uint32_t sel2 = (l & 2) ? 0x3715u : 0x6240u;
+      const uint32_t rot1 = (l & 1) ? 28u : 4u;
+      const uint32_t msk1 = (l & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
 #pragma unroll
       for (int k = 0; k < ITEMS; ++k) {
         const int w = t + k * nt;
         const int blk = w >> (3 + HA), tb = w & (TB - 1);
 #pragma unroll
         for (int wb = 0; wb < EB / 8; ++wb) {
-          uint32_t W = 0;
+          float q8[8];
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) W |= quant_nibble<CLIP>(v[k][8 * wb + jj], r) << (4 * jj);
-          // transpose the 8x8 nibble block held by lanes with tb_low = 0..7
-#pragma unroll
-          for (int m = 4; m >= 1; m >>= 1) {
-            const uint32_t mk = (m == 4) ? 0x0000FFFFu : (m == 2) ? 0x00FF00FFu : 0x0F0F0F0Fu;
-            const int sh = 4 * m;
-            const uint32_t P = __shfl_xor_sync(0xffffffffu, W, m);
-            W = (l & m) ? (((P >> sh) & mk) | (W & ~mk)) : ((W & mk) | ((P & mk) << sh));
+          for (int jj = 0; jj < 8; ++jj) q8[jj] = v[k][8 * wb + jj];
+          uint32_t W = quant_word<CLIP>(q8, r);
+          // Transpose the 8x8 nibble block held by the lanes with tb_low =
+          // 0..7: swap 16-bit halves with lane^4, bytes with lane^2 (byte
+          // permutes), nibbles with lane^1 (rotate + 3-input logic op).
+          W = prmt(W, __shfl_xor_sync(0xffffffffu, W, 4), sel4);
+          W = prmt(W, __shfl_xor_sync(0xffffffffu, W, 2), sel2);
+          {
+            const uint32_t P = __shfl_xor_sync(0xffffffffu, W, 1);
+            const uint32_t s4 = __funnelshift_l(P, P, rot1);
+            uint32_t nw;
+            asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(nw) : "r"(W), "r"(s4), "r"(msk1));
+            W = nw;   // (W & msk1) | (s4 & ~msk1)
           }
           if (w < items_b) {
             const int e = (blk << LB) + 8 * (8 * wb + l) + ((tb >> 3) << (3 + MB));
