@@ -36,6 +36,11 @@ struct RowJob {
 
 qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream);
 
+// FlatQuant Kronecker transform on tensor cores (n1 = 128, n2 = 64, no
+// outlier split, aligned rows); other Kronecker shapes run on CUDA cores.
+bool kron_tc_supported(const RowJob& job);
+qr_status launch_kron_tc(const RowJob& job, cudaStream_t stream);
+
 struct GemmJob {
   const uint8_t* a_codes; const float* a_scales;
   const uint8_t* w_codes; const float* w_scales;

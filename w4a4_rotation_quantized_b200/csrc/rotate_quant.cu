@@ -998,7 +998,8 @@ qr_status launch_kron_rows(const RowJob& job, cudaStream_t stream) {
 
 qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream) {
   if (job.rows == 0) return QR_OK;
-  if (job.rot->kind == QR_ROT_KRON) return launch_kron_rows(job, stream);
+  if (job.rot->kind == QR_ROT_KRON)
+    return kron_tc_supported(job) ? launch_kron_tc(job, stream) : launch_kron_rows(job, stream);
   return launch_wht_rows(job, stream);
 }
 
