@@ -416,9 +416,13 @@ cudaError_t run_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, const C
 
 qr_status launch_w4a4_gemm(const GemmJob& j, cudaStream_t stream) {
   if (j.M == 0 || j.N == 0) return QR_OK;
+  return launch_w4a4_gemm_pair(j, stream);
+}
+
+qr_status launch_w4a4_gemm_single(const GemmJob& j, cudaStream_t stream) {
+  if (j.M == 0 || j.N == 0) return QR_OK;
   const bool swap = j.M <= 64;
   const bool out = j.n_out > 0;
-  if (!swap && !out) return launch_w4a4_gemm_pair(j, stream);
   const int64_t rows_a = swap ? j.N : j.M;      // MMA-M side
   const int64_t rows_b = swap ? j.M : j.N;      // MMA-N side
   int bn;

@@ -1,37 +1,40 @@
-// w4a4_gemm_pair.cu -- the W4A4 linear on a pair of SMs (prefill shapes).
+// w4a4_gemm_pair.cu -- the W4A4 linear on pairs of SMs.
 //
-// Same computation as w4a4_gemm.cu (QUIK §4: INT4 codes multiplied on
-// integer tensor cores with INT32 accumulation, dequantized per token and
-// per channel in the epilogue), arranged to move fewer bytes through shared
-// memory per MMA:
+// Same computation as w4a4_gemm.cu (QUIK §1 and §4: INT4 codes multiplied on
+// integer tensor cores with INT32 accumulation, dequantized per token and per
+// channel in the epilogue, plus the fp16 product of the outlier columns),
+// arranged to move fewer bytes through shared memory per MMA:
 //
 //  * tcgen05.mma.cta_group::2: the two CTAs of a cluster compute a 256 x BN
-//    tile; each CTA holds its own 128 activation rows and half of the BN
-//    weight rows, and the pair's MMA reads both halves.
-//  * The activation operand is widened by the CTA's widen warps straight
-//    into tensor memory (tcgen05.st): one thread owns one activation row, so
-//    shared memory carries only the packed activation tile once.
-//  * The weight operand is widened in shared memory into the canonical
-//    128-byte-swizzled K-major layout, as in the one-SM kernel.
+//    tile; each CTA holds its own 128 rows of the "A" operand and half of the
+//    BN rows of the "B" operand, and the pair's MMA reads both halves.
+//  * The A operand is widened by the CTA's widen warps straight into tensor
+//    memory (tcgen05.st): one thread owns one row, so shared memory carries
+//    only the packed A tile once.
+//  * The B operand is widened in shared memory into the canonical
+//    128-byte-swizzled K-major layout.
+//  * Prefill (M > 64): A = activations, B = weights.  Decode (SWAP, M <= 64):
+//    A = weights, B = tokens, and the epilogue writes Y transposed.
+//  * OUT: the fp16 outlier columns run as a second cta_group::2 MMA of
+//    kind::f16 into an fp32 accumulator in TMEM, added in the epilogue.
 //
 // Widening writes each nibble in the high half of a byte (the byte is 16*q)
 // and the 32 codes of a 16-byte packed chunk as (even elements, odd
 // elements); both operands use that K order, so acc = 256 * sum qa*qw.
 //
-// Tensor memory per CTA: two BN-column int32 accumulators (the epilogue of
-// one tile overlaps the MMAs of the next) and up to four 32-column
-// activation stages: 2*BN + 32*stages <= 512.
+// Tensor memory per CTA: two accumulator buffers (the epilogue of one tile
+// overlaps the MMAs of the next) of BN int32 columns, plus BN fp32 outlier
+// columns when OUT, and up to four 32-column A stages.
 //
 // Warp roles, per CTA (448 threads):
-//   warps 0-3   epilogue  (TMEM lanes = the CTA's 128 rows of the tile)
+//   warps 0-3   epilogue  (TMEM lanes = the CTA's 128 A rows of the tile)
 //   warps 4-11  widen     (two groups of four warps taking alternate K
-//                          steps: one activation row per thread -> TMEM,
-//                          weight chunks -> smem)
-//   warp  12    producer  (TMA of the packed tiles; no multicast)
+//                          steps: one A row per thread -> TMEM, B chunks ->
+//                          smem)
+//   warp  12    producer  (TMA of the packed and outlier tiles; no multicast)
 //   warp  13    TMEM allocation; in the even CTA one thread issues the MMAs,
-//               in the odd CTA one thread relays "stage widened" to the even
-//               CTA (one cluster-scope arrive per stage instead of one per
-//               widen warp)
+//               in the odd CTA one thread relays "stage ready" to the even
+//               CTA (one relaxed cluster-scope arrive per stage)
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -47,56 +50,71 @@ namespace {
 
 constexpr int kStep = 64;          // packed bytes per row per K step (128 codes)
 constexpr int kNP = 8;             // packed ring depth
-constexpr int kWidenWarps = 8;                 // two groups of four
+constexpr int kNO = 2;             // outlier ring depth
+constexpr int kOutCols = 32;       // fp16 outlier columns per step (64-byte rows)
+constexpr int kWidenWarps = 8;     // two groups of four
 constexpr int kGroupThreads = 128;
 constexpr int kProducerWarp = 4 + kWidenWarps;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
-// Widened stages: as many 32-column activation stages as tensor memory holds
-// next to two BN-column accumulators, at most 4.
-template <int BN>
+// A stages: as many 32-column stages as tensor memory holds next to the two
+// accumulator buffers, at most 4.
+template <int BN, bool OUT>
 constexpr int widened_stages() {
-  return (512 - 2 * BN) / 32 < 4 ? (512 - 2 * BN) / 32 : 4;
+  return (512 - (OUT ? 4 : 2) * BN) / 32 < 4 ? (512 - (OUT ? 4 : 2) * BN) / 32 : 4;
 }
 
 struct PairParams {
-  const float* scale_a;            // [M]
-  const float* scale_b;            // [N]
+  const float* scale_a;            // per A-side row
+  const float* scale_b;            // per B-side row
   __half* Y;
   int64_t ldy;
   int32_t* acc_debug;              // [M x N] or null
-  int32_t M, N;
-  int32_t kt;                      // K steps
-  int32_t tiles_a, tiles_b;        // 256-row tiles, BN-column tiles
+  int32_t rows_a, rows_b;          // A-side and B-side row counts
+  int32_t M, N;                    // output shape
+  int32_t kt, ot;                  // int4 K steps, outlier steps
+  int32_t tiles_a, tiles_b;        // 256-row A tiles, BN-row B tiles
   int32_t y_vec_ok;
   int32_t* status;
 };
 
-template <int BN>
+template <int BN, bool OUT>
 struct PairSmem {
-  static constexpr int kNW = widened_stages<BN>();
-  static constexpr int kHalf = BN / 2;                     // weight rows per CTA
+  static constexpr int kNW = widened_stages<BN, OUT>();
+  static constexpr int kHalf = BN / 2;                     // B rows per CTA
   static constexpr int kPackA = 128 * kStep;               // 8 KB, 64-byte swizzle
   static constexpr int kPackB = kHalf * kStep;
   static constexpr int kWideB = kHalf * 2 * kStep;         // SW128 K-major
+  static constexpr int kOutA = OUT ? 128 * kOutCols * 2 : 0;     // SW64 K-major
+  static constexpr int kOutB = OUT ? kHalf * kOutCols * 2 : 0;
   static constexpr int off_wide_b = 0;                     // 1024-aligned
-  static constexpr int off_pack_a = off_wide_b + kNW * kWideB;
+  static constexpr int off_out_a = off_wide_b + kNW * kWideB;
+  static constexpr int off_out_b = off_out_a + kNO * kOutA;
+  static constexpr int off_pack_a = off_out_b + kNO * kOutB;
   static constexpr int off_pack_b = off_pack_a + kNP * kPackA;
   static constexpr int off_bar = off_pack_b + kNP * kPackB;
-  static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 + 2 + 1;
+  // full_p, empty_p, full_w, empty_w, full_o, full_o2, empty_o,
+  // tmem_full[2], tmem_empty[2], drain
+  static constexpr int kNumBars = 2 * kNP + 2 * kNW + 3 * kNO + 5;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
   static constexpr int kBytes = off_misc + 16 + 1024;
+  static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
 };
 
-template <int BN>
+template <int BN, bool SWAP, bool OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
-                      const __grid_constant__ CUtensorMap map_b, const PairParams p) {
-  using S = PairSmem<BN>;
+                      const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_oa,
+                      const __grid_constant__ CUtensorMap map_ob, const PairParams p) {
+  using S = PairSmem<BN, OUT>;
   constexpr int kNW = S::kNW;
-  static_assert(BN % 32 == 0 && BN >= 64 && kNW >= 2, "tile width");
-  constexpr uint32_t kAcol = 2 * BN;                       // activation stages in TMEM
+  static_assert(BN % 32 == 0 && BN >= 32 && kNW >= 2, "tile width");
+  constexpr uint32_t kColsAcc = OUT ? 2 * BN : BN;         // per accumulator buffer
+  constexpr uint32_t kAcol = 2 * kColsAcc;                 // A stages in TMEM
+  static_assert(kAcol + 32 * kNW <= 512, "tensor memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -105,7 +123,10 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   uint64_t* empty_p = full_p + kNP;          // local: widen done reading
   uint64_t* full_w = empty_p + kNP;          // widened: 4 local warps (+ the odd CTA's relay)
   uint64_t* empty_w = full_w + kNW;          // each CTA: the pair's MMAs done with the stage
-  uint64_t* tmem_full = empty_w + kNW;       // each CTA: accumulator ready
+  uint64_t* full_o = empty_w + kNW;          // local: outlier TMA landed
+  uint64_t* full_o2 = full_o + kNO;          // even CTA: the odd CTA's outlier TMA landed
+  uint64_t* empty_o = full_o2 + kNO;         // each CTA: the pair's MMAs done with the stage
+  uint64_t* tmem_full = empty_o + kNO;       // each CTA: accumulator ready
   uint64_t* tmem_empty = tmem_full + 2;      // even CTA: both epilogues drained (8 warps)
   uint64_t* drain = tmem_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::off_misc);
@@ -122,14 +143,19 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
       mbar_init(&full_w[i], leader ? 5 : 4);
       mbar_init(&empty_w[i], 1);
     }
+    for (int i = 0; i < kNO; ++i) {
+      mbar_init(&full_o[i], 1);
+      mbar_init(&full_o2[i], 1);
+      mbar_init(&empty_o[i], 1);
+    }
     for (int i = 0; i < 2; ++i) { mbar_init(&tmem_full[i], 1); mbar_init(&tmem_empty[i], 8); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0 && p.kt > 0) {
-    tma_prefetch_desc(&map_a);
-    tma_prefetch_desc(&map_b);
+  if (warp == kProducerWarp && lane == 0) {
+    if (p.kt > 0) { tma_prefetch_desc(&map_a); tma_prefetch_desc(&map_b); }
+    if (OUT && p.ot > 0) { tma_prefetch_desc(&map_oa); tma_prefetch_desc(&map_ob); }
   }
   if (warp == kMmaWarp) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -147,7 +173,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0, ot = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
         const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
@@ -160,38 +186,58 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
           tma_load_2d(smem + S::off_pack_a + s * S::kPackA, &map_a, &full_p[s], ks * kStep, ya);
           tma_load_2d(smem + S::off_pack_b + s * S::kPackB, &map_b, &full_p[s], ks * kStep, yb);
         }
+        if (OUT)
+          for (int os = 0; os < p.ot && ok; ++os, ++ot) {
+            const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
+            if (!(ok = mbar_wait_cluster_bounded(&empty_o[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
+            mbar_arrive_expect_tx(&full_o[s], S::kOutA + S::kOutB);
+            tma_load_2d(smem + S::off_out_a + s * S::kOutA, &map_oa, &full_o[s], os * kOutCols, ya);
+            tma_load_2d(smem + S::off_out_b + s * S::kOutB, &map_ob, &full_o[s], os * kOutCols, yb);
+          }
       }
-      if (!ok)
+      if (!ok) {
         for (uint32_t i = (it > kNP ? it - kNP : 0); i < it; ++i)
           mbar_wait_bounded(&full_p[i % kNP], (i / kNP) & 1, abort_flag, nullptr, 0, kDrainLimitNs);
+        for (uint32_t i = (ot > kNO ? ot - kNO : 0); i < ot; ++i)
+          mbar_wait_bounded(&full_o[i % kNO], (i / kNO) & 1, abort_flag, nullptr, 0, kDrainLimitNs);
+      }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA (even CTA)
     if (!leader && lane == 0) {
-      // relay: this CTA's stage is widened -> the even CTA's full_w
+      // ------------------------------------------------------------ relay (odd CTA)
+      // This CTA's stages are ready -> the even CTA's barriers.  The local
+      // waits acquire the widen warps' fenced writes and the TMA's
+      // completion; a release at cluster scope here would also wait for the
+      // epilogue's outstanding global stores (~0.7 us per stage).
       const uint32_t full_w0 = mapa_shared(smem_u32(&full_w[0]), 0);
-      uint32_t wi = 0;
+      const uint32_t full_o20 = mapa_shared(smem_u32(&full_o2[0]), 0);
+      uint32_t wi = 0, oi = 0;
       bool ok = true;
-      for (int tile = cid; tile < num_tiles && ok; tile += ncl)
+      for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
         for (int ks = 0; ks < p.kt; ++ks, ++wi) {
           const uint32_t s = wi % kNW, ph = (wi / kNW) & 1;
           if (!(ok = mbar_wait_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
-          // The widen warps fenced their shared-memory and tensor-memory
-          // writes and released them on this CTA's barrier, which the wait
-          // above acquired; a release at cluster scope here would also wait
-          // for the epilogue's outstanding global stores (~0.7 us per stage).
           mbar_arrive_cluster_relaxed(full_w0 + s * 8);
         }
+        if (OUT)
+          for (int os = 0; os < p.ot && ok; ++os, ++oi) {
+            const uint32_t s = oi % kNO, ph = (oi / kNO) & 1;
+            if (!(ok = mbar_wait_bounded(&full_o[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
+            mbar_arrive_cluster_relaxed(full_o20 + s * 8);
+          }
+      }
     }
     if (leader && lane == 0) {
+      // ------------------------------------------------------------ MMA (even CTA)
       constexpr uint32_t idesc = idesc_i8_m256(BN);
-      uint32_t wi = 0, tcount = 0;
+      constexpr uint32_t idesc_o = idesc_f16_m256(BN);
+      uint32_t wi = 0, oi = 0, tcount = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++tcount) {
         const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
         if (!(ok = mbar_wait_cluster_bounded(&tmem_empty[buf], tph ^ 1, abort_flag, p.status, kDevTimeoutMma))) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + buf * BN;
+        const uint32_t d = tmem_base + buf * kColsAcc;
         for (int ks = 0; ks < p.kt; ++ks, ++wi) {
           const uint32_t s = wi % kNW, ph = (wi / kNW) & 1;
           if (!(ok = mbar_wait_cluster_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
@@ -202,6 +248,18 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
           for (int k = 0; k < 4; ++k) mma_i8_pair_ts(d, a + 8 * k, db + 2 * k, idesc, (ks | k) != 0);
           mma_commit_pair(&empty_w[s], 0x3);
         }
+        if (OUT && ok)
+          for (int os = 0; os < p.ot; ++os, ++oi) {
+            const uint32_t s = oi % kNO, ph = (oi / kNO) & 1;
+            if (!(ok = mbar_wait_cluster_bounded(&full_o[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
+            if (!(ok = mbar_wait_cluster_bounded(&full_o2[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
+            tc_fence_after();
+            const uint64_t da = smem_desc_kmajor(smem_u32(smem + S::off_out_a + s * S::kOutA), 64);
+            const uint64_t db = smem_desc_kmajor(smem_u32(smem + S::off_out_b + s * S::kOutB), 64);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) mma_f16_pair(d + BN, da + 2 * k, db + 2 * k, idesc_o, (os | k) != 0);
+            mma_commit_pair(&empty_o[s], 0x3);
+          }
         if (ok) mma_commit_pair(&tmem_full[buf], 0x3);
       }
       mma_commit_pair_local(drain);
@@ -212,7 +270,6 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
     const int wt = threadIdx.x - 128;
     const int group = wt >> 7;                     // takes K steps with it % 2 == group
     const int arow = wt & 127;                     // = TMEM lane (warp % 4 quadrant)
-    const int gt = arow;                           // thread index within the group
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t it = 0;
     bool ok = true;
@@ -223,7 +280,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
         const uint32_t sw = it % kNW, phw = (it / kNW) & 1;
         if (!(ok = mbar_wait_bounded(&full_p[s], ph, abort_flag, p.status, kDevTimeoutWiden))) break;
         if (!(ok = mbar_wait_cluster_bounded(&empty_w[sw], phw ^ 1, abort_flag, p.status, kDevTimeoutWiden))) break;
-        // activation row: 64 packed bytes (64-byte swizzled rows) -> 128 s8 in TMEM
+        // A row: 64 packed bytes (64-byte swizzled rows) -> 128 s8 in TMEM
         {
           const uint8_t* pa = smem + S::off_pack_a + s * S::kPackA + arow * kStep;
           uint32_t r[32];
@@ -241,13 +298,13 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
           }
           tmem_st_32x32b_x32(tmem_base + lane_off + kAcol + sw * 32, r);
         }
-        // weight rows: 16-byte packed chunks -> two 16-byte s8 chunks, SW128
+        // B rows: 16-byte packed chunks -> two 16-byte s8 chunks, SW128
         {
           const uint8_t* pb = smem + S::off_pack_b + s * S::kPackB;
           uint8_t* wb = smem + S::off_wide_b + sw * S::kWideB;
           constexpr int kTasks = S::kHalf * 4;
 #pragma unroll 2
-          for (int task = gt; task < kTasks; task += kGroupThreads) {
+          for (int task = arow; task < kTasks; task += kGroupThreads) {
             const int row = task >> 2, c = task & 3;
             const uint4 u = *reinterpret_cast<const uint4*>(pb + row * kStep + c * 16);
             uint4 ev, od;
@@ -282,48 +339,74 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
       const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
       if (!(ok = mbar_wait_cluster_bounded(&tmem_full[buf], tph, abort_flag, p.status, kDevTimeoutEpilogue))) break;
       tc_fence_after();
-      const int m = ta * 256 + static_cast<int>(rank) * 128 + lrow;
-      const bool m_ok = m < p.M;
-      const float s_row = m_ok ? __ldg(p.scale_a + m) * (1.0f / 256.0f) : 0.0f;
-      const uint32_t t_acc = tmem_base + lane_off + buf * BN;
-      __half* yrow = p.Y + static_cast<int64_t>(m) * p.ldy;
+      const int ra = ta * 256 + static_cast<int>(rank) * 128 + lrow;   // A-side row
+      const bool ra_ok = ra < p.rows_a;
+      const float s_row = ra_ok ? __ldg(p.scale_a + ra) * (1.0f / 256.0f) : 0.0f;
+      const uint32_t t_acc = tmem_base + lane_off + buf * kColsAcc;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t acc[32];
+        uint32_t oacc[32];
         tmem_ld_32x32b_x32(t_acc + c * 32, acc);
+        if (OUT) tmem_ld_32x32b_x32(t_acc + BN + c * 32, oacc);
         tmem_ld_wait();
         if (p.kt == 0) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) acc[j] = 0;
         }
-        const int n0 = tb * BN + c * 32;
-        if (!m_ok) continue;
-        uint32_t hp[16];
+        if (OUT && p.ot == 0) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float s0 = (n0 + j < p.N) ? __ldg(p.scale_b + n0 + j) : 0.0f;
-          const float s1 = (n0 + j + 1 < p.N) ? __ldg(p.scale_b + n0 + j + 1) : 0.0f;
-          const __half2 h2 = __floats2half2_rn(
-              static_cast<float>(static_cast<int32_t>(acc[j])) * s_row * s0,
-              static_cast<float>(static_cast<int32_t>(acc[j + 1])) * s_row * s1);
-          hp[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int j = 0; j < 32; ++j) oacc[j] = 0;
         }
-        if (p.y_vec_ok && n0 + 32 <= p.N) {
+        const int cb0 = tb * BN + c * 32;          // first B-side row of this chunk
+        if (!ra_ok) continue;
+        if (!SWAP) {
+          // lane owns output row m = ra; columns n = cb0 + j
+          __half* yrow = p.Y + static_cast<int64_t>(ra) * p.ldy;
+          uint32_t hp[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(yrow + n0 + 8 * q) =
-                make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
+          for (int j = 0; j < 32; j += 2) {
+            float y2[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int n = cb0 + j + t;
+              const float sb = (n < p.rows_b) ? __ldg(p.scale_b + n) : 0.0f;
+              y2[t] = static_cast<float>(static_cast<int32_t>(acc[j + t])) * s_row * sb;
+              if (OUT) y2[t] += __uint_as_float(oacc[j + t]);
+            }
+            const __half2 h2 = __floats2half2_rn(y2[0], y2[1]);
+            hp[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          if (p.y_vec_ok && cb0 + 32 <= p.rows_b) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(yrow + cb0 + 8 * q) =
+                  make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (cb0 + j < p.rows_b)
+                reinterpret_cast<uint16_t*>(yrow)[cb0 + j] =
+                    static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
+          }
+          if (p.acc_debug != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (cb0 + j < p.rows_b)
+                p.acc_debug[static_cast<int64_t>(ra) * p.N + cb0 + j] = static_cast<int32_t>(acc[j]) >> 8;
+          }
         } else {
+          // lane owns output column n = ra; rows m = cb0 + j (tokens)
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (n0 + j < p.N)
-              reinterpret_cast<uint16_t*>(yrow)[n0 + j] = static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
-        }
-        if (p.acc_debug != nullptr) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (n0 + j < p.N)
-              p.acc_debug[static_cast<int64_t>(m) * p.N + n0 + j] = static_cast<int32_t>(acc[j]) >> 8;
+          for (int j = 0; j < 32; ++j) {
+            const int m = cb0 + j;
+            if (m >= p.rows_b) continue;
+            float y = static_cast<float>(static_cast<int32_t>(acc[j])) * s_row * __ldg(p.scale_b + m);
+            if (OUT) y += __uint_as_float(oacc[j]);
+            p.Y[static_cast<int64_t>(m) * p.ldy + ra] = __float2half_rn(y);
+            if (p.acc_debug != nullptr)
+              p.acc_debug[static_cast<int64_t>(m) * p.N + ra] = static_cast<int32_t>(acc[j]) >> 8;
+          }
         }
       }
       tc_fence_before();
@@ -341,22 +424,23 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   }
 }
 
-template <int BN>
-cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const PairParams& p,
-                     cudaStream_t stream) {
-  auto k = w4a4_gemm_pair_kernel<BN>;
-  const int smem = PairSmem<BN>::kBytes;
+template <int BN, bool SWAP, bool OUT>
+cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& moa,
+                     const CUtensorMap& mob, const PairParams& p, cudaStream_t stream) {
+  auto k = w4a4_gemm_pair_kernel<BN, SWAP, OUT>;
+  const int smem = PairSmem<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int clusters = std::min(p.tiles_a * p.tiles_b, sm_count() / 2);
-  k<<<2 * clusters, kThreads, smem, stream>>>(ma, mb, p);
+  k<<<2 * clusters, kThreads, smem, stream>>>(ma, mb, moa, mob, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// Tile width for the pair kernel: the fewest tile rounds over the SM pairs,
-// weighted by the width (one round of a BN-wide tile costs about BN).
+// Tile width for prefill without outlier columns: the fewest tile rounds over
+// the SM pairs, weighted by the width (one round of a BN-wide tile costs
+// about BN).
 int pair_tile_width(int64_t M, int64_t N, int sms) {
   const int64_t ta = (M + 255) / 256;
   const int cands[] = {192, 160, 128};
@@ -376,34 +460,64 @@ int pair_tile_width(int64_t M, int64_t N, int sms) {
 }
 
 qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
-  const int bn = pair_tile_width(j.M, j.N, sm_count());
+  const bool swap = j.M <= 64;
+  const bool out = j.n_out > 0;
+  int bn;
+  if (swap) bn = j.M <= 32 ? 32 : 64;
+  else bn = out ? 96 : pair_tile_width(j.M, j.N, sm_count());
+  const int64_t rows_a = swap ? j.N : j.M;
+  const int64_t rows_b = swap ? j.M : j.N;
   PairParams p{};
-  p.scale_a = j.a_scales;
-  p.scale_b = j.w_scales;
+  p.scale_a = swap ? j.w_scales : j.a_scales;
+  p.scale_b = swap ? j.a_scales : j.w_scales;
   p.Y = reinterpret_cast<__half*>(j.Y);
   p.ldy = j.ldy;
   p.acc_debug = j.acc_debug;
+  p.rows_a = static_cast<int32_t>(rows_a);
+  p.rows_b = static_cast<int32_t>(rows_b);
   p.M = static_cast<int32_t>(j.M);
   p.N = static_cast<int32_t>(j.N);
   p.kt = static_cast<int32_t>(j.Kp / 128);
-  p.tiles_a = static_cast<int32_t>((j.M + 255) / 256);
-  p.tiles_b = static_cast<int32_t>((j.N + bn - 1) / bn);
+  p.ot = out ? (j.n_out + kOutCols - 1) / kOutCols : 0;
+  p.tiles_a = static_cast<int32_t>((rows_a + 255) / 256);
+  p.tiles_b = static_cast<int32_t>((rows_b + bn - 1) / bn);
   p.y_vec_ok = (reinterpret_cast<uintptr_t>(j.Y) % 16 == 0) && (j.ldy % 8 == 0);
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
-  CUtensorMap ma{}, mb{};
-  const uint64_t kb = static_cast<uint64_t>(j.Kp) / 2;
+  const uint8_t* ca = swap ? j.w_codes : j.a_codes;
+  const uint8_t* cb = swap ? j.a_codes : j.w_codes;
+  CUtensorMap ma{}, mb{}, moa{}, mob{};
+  const uint64_t kb = static_cast<uint64_t>(j.Kp) / 2;   // packed bytes per row
   if (p.kt > 0 &&
-      (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.a_codes, kb, j.M, kb, kStep, 128,
+      (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, ca, kb, rows_a, kb, kStep, 128,
                            CU_TENSOR_MAP_SWIZZLE_64B) ||
-       !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.w_codes, kb, j.N, kb, kStep,
+       !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, cb, kb, rows_b, kb, kStep,
                            bn / 2, CU_TENSOR_MAP_SWIZZLE_NONE)))
     return QR_ERR_CUDA;
+  if (out) {
+    const uint16_t* oa = swap ? j.w_out : j.x_out;
+    const uint16_t* ob = swap ? j.x_out : j.w_out;
+    const uint64_t no = static_cast<uint64_t>(j.n_out);
+    if (!make_tensor_map_2d(&moa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, oa, no, rows_a, no * 2,
+                            kOutCols, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tensor_map_2d(&mob, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ob, no, rows_b, no * 2,
+                            kOutCols, bn / 2, CU_TENSOR_MAP_SWIZZLE_64B))
+      return QR_ERR_CUDA;
+  }
   cudaError_t e;
-  switch (bn) {
-    case 192: e = run_pair<192>(ma, mb, p, stream); break;
-    case 160: e = run_pair<160>(ma, mb, p, stream); break;
-    default: e = run_pair<128>(ma, mb, p, stream); break;
+  if (swap) {
+    if (bn == 32) e = out ? run_pair<32, true, true>(ma, mb, moa, mob, p, stream)
+                          : run_pair<32, true, false>(ma, mb, moa, mob, p, stream);
+    else e = out ? run_pair<64, true, true>(ma, mb, moa, mob, p, stream)
+                 : run_pair<64, true, false>(ma, mb, moa, mob, p, stream);
+  } else if (out) {
+    e = run_pair<96, false, true>(ma, mb, moa, mob, p, stream);
+  } else {
+    switch (bn) {
+      case 192: e = run_pair<192, false, false>(ma, mb, moa, mob, p, stream); break;
+      case 160: e = run_pair<160, false, false>(ma, mb, moa, mob, p, stream); break;
+      default: e = run_pair<128, false, false>(ma, mb, moa, mob, p, stream); break;
+    }
   }
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
