@@ -85,6 +85,25 @@ def check_side(gpu, ref: O.Side, what: str, clip: float = 1.0, check_rot: bool =
     return int(diff.sum())
 
 
+# Rotate + quantize calls with at most this many rows run one CTA per row;
+# more rows run the row-group kernels.  Tests tile their rows past it to
+# cover both.
+FEW_ROWS = 148
+
+
+def tile_rows(x: np.ndarray, min_rows: int = FEW_ROWS + 52) -> tuple[np.ndarray, int]:
+    """x repeated row-wise to at least `min_rows` rows, and the repeat count."""
+    reps = -(-min_rows // max(1, x.shape[0]))
+    return np.tile(x, (reps, 1)), reps
+
+
+def tile_side(ref: O.Side, reps: int) -> O.Side:
+    """The oracle Side of rows repeated `reps` times."""
+    t = lambda a: np.tile(a, (reps, 1)) if a.ndim == 2 else np.tile(a, reps)
+    q = O.Quantized(codes=t(ref.q.codes), scales=t(ref.q.scales), quotient=t(ref.q.quotient))
+    return O.Side(rotated=t(ref.rotated), q=q, packed=t(ref.packed), fp16_part=t(ref.fp16_part))
+
+
 def rel_fro(a, b) -> float:
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)

@@ -11,7 +11,8 @@ import oracle as O
 import w4a4_rotation_quantized_b200 as Q
 import workloads
 from tests.gpu_helpers import (Y_TOL, check_side, dev, gpu_rotation, host,
-                               oracle_rows_from_gpu_codes, rel_fro, require_gpu, unpack)
+                               oracle_rows_from_gpu_codes, rel_fro, require_gpu, tile_rows,
+                               tile_side, unpack)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,8 +31,14 @@ def _rows(rng, m, k, scale=1.0, outl=()):
     return x.astype(np.float16)
 
 
-def _run_rows(x16, orot, idx=None, weights=False):
-    xg = dev(x16)
+def _run_rows(x16, orot, idx=None, weights=False, many=False):
+    """GPU and oracle results for the rows of x16; with `many`, the GPU call
+    gets the rows repeated past the few-rows kernel's limit."""
+    reps = 1
+    x_run = x16
+    if many:
+        x_run, reps = tile_rows(x16)
+    xg = dev(x_run)
     ig = None if idx is None else dev(np.asarray(idx, np.int32))
     grot = gpu_rotation(orot)
     if weights:
@@ -41,7 +48,7 @@ def _run_rows(x16, orot, idx=None, weights=False):
         gpu = Q.rotate_quant(xg, grot, ig, debug=True)
         ref = O.quantize_activations(x16.astype(np.float64), orot, idx)
     torch.cuda.synchronize()
-    return gpu, ref
+    return gpu, (tile_side(ref, reps) if reps > 1 else ref)
 
 
 # ---------------------------------------------------------------- rotate + quantize
@@ -70,23 +77,28 @@ ROW_CASES = [
 
 @pytest.mark.parametrize("name,K,rows,rot", ROW_CASES, ids=[c[0] for c in ROW_CASES])
 @pytest.mark.parametrize("weights", [False, True], ids=["act", "wgt"])
-def test_rotate_quant_matches_oracle(name, K, rows, rot, weights):
+@pytest.mark.parametrize("many", [False, True], ids=["few", "many"])
+def test_rotate_quant_matches_oracle(name, K, rows, rot, weights, many):
     rng = np.random.default_rng(zlib.crc32(name.encode()))
     x = _rows(rng, rows, K, outl=(3, K // 2))
     x[rows // 2] = 0                                 # an all-zero row
-    gpu, ref = _run_rows(x, rot, weights=weights)
+    gpu, ref = _run_rows(x, rot, weights=weights, many=many)
     check_side(gpu, ref, name, clip=rot.clip_ratio)
     assert host(gpu[1])[rows // 2] == 0 and not host(gpu[0])[rows // 2].any()
 
 
-def test_rotate_quant_unaligned_leading_dimension():
+@pytest.mark.parametrize("many", [False, True], ids=["few", "many"])
+def test_rotate_quant_unaligned_leading_dimension(many):
     rng = np.random.default_rng(1)
     full = _rows(rng, 6, 203)
+    reps = 1
+    if many:
+        full, reps = tile_rows(full)
     x = dev(full)[:, :200]                           # ldx = 203: scalar loads
     rot = O.Rotation(O.HADAMARD, block=128)
     gpu = Q.rotate_quant(x, gpu_rotation(rot), debug=True)
-    ref = O.quantize_activations(full[:, :200].astype(np.float64), rot)
-    check_side(gpu, ref, "ldx203")
+    ref = O.quantize_activations(full[:6, :200].astype(np.float64), rot)
+    check_side(gpu, tile_side(ref, reps) if reps > 1 else ref, "ldx203")
 
 
 @pytest.mark.parametrize("K,n_out,block", [(300, 5, 64), (8192, 256, 4096), (1000, 40, 128),
@@ -97,8 +109,9 @@ def test_rotate_quant_with_outlier_columns(K, n_out, block):
     x = _rows(rng, 7, K, outl=idx[:3])
     rot = O.Rotation(O.HADAMARD, block=block)
     for weights in (False, True):
-        gpu, ref = _run_rows(x, rot, idx, weights=weights)
-        check_side(gpu, ref, f"outliers K={K} n_out={n_out}")
+        for many in (False, True):
+            gpu, ref = _run_rows(x, rot, idx, weights=weights, many=many)
+            check_side(gpu, ref, f"outliers K={K} n_out={n_out} many={many}")
 
 
 def test_kron_rotate_quant_small_factors():
@@ -159,6 +172,9 @@ LINEAR_CASES = [
     # two-SM tiles: 256-row pairs, widths 128..224, ragged edges, long K
     (257, 225, 384, 0), (512, 448, 1280, 0), (300, 1000, 11008, 0), (1000, 700, 256, 0),
     (100, 4096, 128, 0), (65, 33, 0, 0),
+    # decode: K split over 1, 2 or 4 CTAs; outlier steps only on the first
+    (5, 12288, 256, 0), (33, 8192, 512, 0), (64, 384, 128, 256), (2, 1000, 2048, 32),
+    (17, 130, 8192, 0),
 ]
 
 
@@ -260,3 +276,22 @@ def test_quik_decode_end_to_end(M):
     torch.cuda.synchronize()
     _, _, _, y_ref = O.linear_forward(wl.X.astype(np.float64), wl.W.astype(np.float64), rot, idx)
     assert rel_fro(host(y), y_ref) < Y_TOL
+
+
+@pytest.mark.parametrize("M", [1, 64])
+def test_graphed_layer_matches_eager(M):
+    # the CUDA-graph replay computes what the eager calls compute, bit for bit,
+    # on fresh inputs copied in from pinned host memory
+    wl = workloads.make_workload("quik_decode_8192", M=M, N=512)
+    rot = _oracle_rotation(wl)
+    idx_g = Q.select_outliers(dev(wl.X_calib), wl.spec.n_keep_fp16)
+    layer = Q.QuantizedLinear(dev(wl.W), gpu_rotation(rot), idx_g)
+    glin = Q.GraphedLinear(layer, M)
+    rng = np.random.default_rng(M)
+    for _ in range(2):
+        x = (rng.standard_normal(wl.X.shape) * 0.5).astype(np.float16)
+        y_graph = host(glin(torch.from_numpy(x).pin_memory())).copy()
+        y_eager = host(layer(dev(x)))
+        assert np.array_equal(y_graph.view(np.uint16), y_eager.view(np.uint16))
+    with pytest.raises(ValueError):
+        glin(dev(np.zeros((M + 1, wl.spec.K), np.float16)))

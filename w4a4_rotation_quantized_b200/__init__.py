@@ -8,6 +8,7 @@ outlier product.  The compute lives in libqr.so (include/qr.h); this package
 is its ctypes binding plus torch-facing helpers.
 """
 from . import _lib  # noqa: F401
-from .layer import (GSR, HADAMARD, KRON, NONE, QuantizedLinear, Rotation,  # noqa: F401
+from .layer import (GSR, HADAMARD, KRON, NONE, GraphedLinear, QuantizedLinear,  # noqa: F401
+                    Rotation,
                     invert_transpose, pack_weights, packed_k, rotate_quant, select_outliers,
                     w4a4_linear, weight_rotation)

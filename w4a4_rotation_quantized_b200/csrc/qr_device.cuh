@@ -466,3 +466,25 @@ __host__ __device__ constexpr uint32_t idesc_f16_m256(uint32_t n) {
 }
 
 }  // namespace qr
+
+namespace qr {
+
+// D(tmem, int32) (+)= A(tmem) x B(smem)^T, 8-bit integer operands, M = 128
+// (one CTA).
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Atomic add into another CTA's shared memory (address from mapa_shared).
+__device__ __forceinline__ void red_add_cluster(uint32_t cluster_addr, int32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v)
+               : "memory");
+}
+
+}  // namespace qr

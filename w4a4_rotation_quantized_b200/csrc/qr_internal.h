@@ -52,11 +52,12 @@ struct GemmJob {
 
 qr_status launch_w4a4_gemm(const GemmJob& job, cudaStream_t stream);
 
-// 2-SM tcgen05 MMA with the "A" operand in TMEM (activations for M > 64,
-// weights for M <= 64), fp16 outlier columns as a second MMA.
+// M > 64: 2-SM tcgen05 MMA with the activation operand in TMEM, fp16
+// outlier columns as a second MMA.
 qr_status launch_w4a4_gemm_pair(const GemmJob& job, cudaStream_t stream);
-// One-SM kernel (128-row tiles, both operands widened in shared memory).
-qr_status launch_w4a4_gemm_single(const GemmJob& job, cudaStream_t stream);
+// M <= 64: weights in TMEM, K split over a cluster.
+qr_status launch_w4a4_gemm_decode(const GemmJob& job, cudaStream_t stream);
+int decode_k_split(int64_t tiles, int64_t steps, int sms);
 int pair_tile_width(int64_t M, int64_t N, int sms);
 
 // Row-major 2-D tensor map: `rows` rows of `cols` elements, row pitch

@@ -581,6 +581,207 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
   }
 }
 
+// ------------------------------------------------------------------ few rows
+
+// Few rows (decode): one CTA per row, the whole row in shared memory.  The
+// kernels above give each row one group of threads and keep it in
+// registers, which fills the GPU only with many rows; with a handful of
+// tokens a row's latency is the whole cost, so here up to 1024 threads share
+// one row.  Steps: load the row with vector loads (the outlier columns of
+// QUIK §1 removed by a block-wide prefix count over an outlier bitmap, the
+// kept columns compacted to their rotated positions), the Walsh-Hadamard
+// butterflies in passes of up to three stages through shared memory, the
+// row absmax, then quantize + pack as the other kernels do.
+struct FewRowsParams {
+  const __half* src;
+  int64_t rows, ld;
+  int32_t K, Kr, Kp, n_out;
+  const int32_t* outlier_idx;
+  int32_t lb, gsr, aligned;
+  int32_t off_bits, off_scan;
+  float clip_ratio, inv_sqrt_block;
+  uint8_t* codes;
+  float* scales;
+  __half* out16;
+  float* rot_debug;
+};
+
+// Exclusive prefix sum over the block (blockDim a multiple of 32); `sh`
+// holds 32 ints.  Contains two __syncthreads.
+__device__ __forceinline__ int block_exclusive_sum(int v, int* sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int s = lane < nw ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;
+  }
+  __syncthreads();
+  return (w > 0 ? sh[w - 1] : 0) + x - v;
+}
+
+// Maximum over the block; `sh` holds 32 floats.  Contains two __syncthreads.
+__device__ __forceinline__ float block_max(float v, float* sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  float m = 0.0f;
+  for (int i = 0; i < nw; ++i) m = fmaxf(m, sh[i]);
+  __syncthreads();
+  return m;
+}
+
+// R butterfly stages on index bits [s, s+R) of the row in shared memory.
+template <int R>
+__device__ __forceinline__ void wht_smem_pass(float* buf, int Kp, int s) {
+  constexpr int G = 1 << R;
+  const int ngroups = Kp >> R;
+  const int lowmask = (1 << s) - 1;
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+    const int base = (g & lowmask) | ((g >> s) << (s + R));
+    float x[G];
+#pragma unroll
+    for (int k = 0; k < G; ++k) x[k] = buf[base + (k << s)];
+#pragma unroll
+    for (int st = 0; st < R; ++st)
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+        if (!(k & (1 << st))) {
+          const float a = x[k], b = x[k | (1 << st)];
+          x[k] = a + b;
+          x[k | (1 << st)] = a - b;
+        }
+#pragma unroll
+    for (int k = 0; k < G; ++k) buf[base + (k << s)] = x[k];
+  }
+}
+
+template <bool CLIP>
+__global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* buf = reinterpret_cast<float*>(smem);                       // [Kp]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);   // outlier bitmap
+  int* scan = reinterpret_cast<int*>(smem + p.off_scan);             // 32 ints
+  float* red = reinterpret_cast<float*>(smem + p.off_scan + 128);    // 32 floats
+  const int t = threadIdx.x, nthr = blockDim.x;
+  const int nchunks = (p.K + 7) >> 3;                                // 8 source columns each
+  const int cpt = (nchunks + nthr - 1) / nthr;                       // chunks per thread
+  const int nwords = (p.K + 31) >> 5;
+  for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+    const __half* srow = p.src + row * p.ld;
+    if (p.n_out > 0) {
+      for (int w = t; w < nwords; w += nthr) bits[w] = 0u;
+      __syncthreads();
+      for (int j = t; j < p.n_out; j += nthr) {
+        const int c = __ldg(p.outlier_idx + j);
+        if (c >= 0 && c < p.K) atomicOr(&bits[c >> 5], 1u << (c & 31));
+        if (p.out16 != nullptr)
+          p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? srow[c] : __float2half(0.0f);
+      }
+      __syncthreads();
+    }
+    for (int e = p.Kr + t; e < p.Kp; e += nthr) buf[e] = 0.0f;
+    // this thread's chunks [c0, c0 + cpt): outliers before them, then scatter
+    const int c0 = t * cpt;
+    int before = 0;
+    if (p.n_out > 0) {
+      int cnt = 0;
+      for (int q = 0; q < cpt; ++q) {
+        const int c = c0 + q;
+        if (c < nchunks) cnt += __popc((bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu);
+      }
+      before = block_exclusive_sum(cnt, scan);
+    }
+    for (int q = 0; q < cpt; ++q) {
+      const int c = c0 + q;
+      if (c >= nchunks) break;
+      const int col0 = 8 * c;
+      float x[8];
+      if (p.aligned && col0 + 8 <= p.K) {
+        const uint4 u = ld_stream_v4(srow + col0);
+        const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(h[i]);
+          x[2 * i] = f.x;
+          x[2 * i + 1] = f.y;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = (col0 + i < p.K) ? __half2float(srow[col0 + i]) : 0.0f;
+      }
+      const uint32_t m8 = p.n_out > 0 ? (bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = col0 + i - before;
+        if ((m8 >> i) & 1u) {
+          ++before;
+        } else if (col0 + i < p.K && e < p.Kr) {
+          buf[e] = x[i];
+        }
+      }
+    }
+    __syncthreads();
+    for (int s = 0; s < p.lb; s += 3) {
+      const int r = min(3, p.lb - s);
+      if (r == 3) wht_smem_pass<3>(buf, p.Kp, s);
+      else if (r == 2) wht_smem_pass<2>(buf, p.Kp, s);
+      else wht_smem_pass<1>(buf, p.Kp, s);
+      __syncthreads();
+    }
+    const int ngroups = p.Kp >> 3;
+    float am = 0.0f;
+    for (int g = t; g < ngroups; g += nthr) {
+      const float4 a = *reinterpret_cast<const float4*>(buf + 8 * g);
+      const float4 b = *reinterpret_cast<const float4*>(buf + 8 * g + 4);
+      am = fmaxf(am, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+      am = fmaxf(am, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+    }
+    am = block_max(am, red);
+    const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
+    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
+    if (t == 0) p.scales[row] = s;
+    uint8_t* crow = p.codes + row * (p.Kp >> 1);
+    const int bm = (1 << p.lb) - 1;
+    for (int g = t; g < ngroups; g += nthr) {
+      float v[8];
+      if (p.gsr) {
+        // sequency position j of a block takes Hadamard output bitrev(gray(j))
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = 8 * g + i;
+          const int j = e & bm;
+          const int nat = static_cast<int>(__brev(static_cast<unsigned>(j ^ (j >> 1))) >> (32 - p.lb));
+          v[i] = buf[(e & ~bm) + nat];
+        }
+      } else {
+        const float4 a = *reinterpret_cast<const float4*>(buf + 8 * g);
+        const float4 b = *reinterpret_cast<const float4*>(buf + 8 * g + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      }
+      *reinterpret_cast<uint32_t*>(crow + 4 * g) = quant_word<CLIP>(v, r);
+      if (p.rot_debug != nullptr)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) p.rot_debug[row * p.Kp + 8 * g + i] = v[i] * p.inv_sqrt_block;
+    }
+    __syncthreads();                       // buf, bits and the scratch words are reused
+  }
+}
+
 // ------------------------------------------------------------------ Kronecker
 
 struct KronParams {
@@ -832,6 +1033,52 @@ int pow2_at_least(int v) {
   return r;
 }
 
+// One CTA per row while the rows do not fill the SMs.
+bool few_rows(const RowJob& job) {
+  return job.rows <= sm_count() && job.Kp <= 32768 && job.Kp > 0;
+}
+
+qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
+  const qr_rotation& rot = *job.rot;
+  FewRowsParams p{};
+  p.src = reinterpret_cast<const __half*>(job.src);
+  p.rows = job.rows;
+  p.ld = job.ld;
+  p.K = static_cast<int32_t>(job.K);
+  p.Kr = job.Kr;
+  p.Kp = job.Kp;
+  p.n_out = job.n_out;
+  p.outlier_idx = job.outlier_idx;
+  const int block = (rot.kind == QR_ROT_NONE) ? 1 : rot.block;
+  p.lb = ilog2(block);
+  p.gsr = rot.kind == QR_ROT_GSR;
+  p.aligned = (reinterpret_cast<uintptr_t>(job.src) % 16 == 0) && (job.ld % 8 == 0);
+  p.clip_ratio = rot.clip_ratio;
+  p.inv_sqrt_block = static_cast<float>(1.0 / std::sqrt(static_cast<double>(block)));
+  p.codes = job.codes;
+  p.scales = job.scales;
+  p.out16 = reinterpret_cast<__half*>(job.out16);
+  p.rot_debug = job.rot_debug;
+  size_t off = align_up(sizeof(float) * static_cast<size_t>(job.Kp), 16);
+  p.off_bits = static_cast<int32_t>(off);
+  off = align_up(off + sizeof(uint32_t) * static_cast<size_t>((job.K + 31) / 32), 16);
+  p.off_scan = static_cast<int32_t>(off);
+  off += 256;
+  if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
+  const int threads = std::min(1024, std::max(128, (job.Kp / 8 + 31) / 32 * 32));
+  const int grid = static_cast<int>(job.rows);
+  cudaError_t e;
+  if (rot.clip_ratio < 1.0f) {
+    e = set_smem(wht_few_rows_kernel<true>, off);
+    if (e == cudaSuccess) wht_few_rows_kernel<true><<<grid, threads, off, stream>>>(p);
+  } else {
+    e = set_smem(wht_few_rows_kernel<false>, off);
+    if (e == cudaSuccess) wht_few_rows_kernel<false><<<grid, threads, off, stream>>>(p);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+}
+
 qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   const qr_rotation& rot = *job.rot;
   WhtParams p{};
@@ -887,7 +1134,9 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.off_red = static_cast<int32_t>(off);
   off = align_up(off + sizeof(float) * 16 * R, 16);
   p.off_buf = static_cast<int32_t>(off);
-  p.buf_bytes = small ? 0 : static_cast<int32_t>(align_up(sizeof(float) * (job.Kp + job.Kp / 8 + 8), 16));
+  // fp32 row buffer with the layout-B padding: 8 floats after every 8*eb
+  // elements (swz<3 + MB>), plus 8 spare
+  p.buf_bytes = small ? 0 : static_cast<int32_t>(align_up(sizeof(float) * (job.Kp + job.Kp / eb + 8), 16));
   off += static_cast<size_t>(p.buf_bytes) * R;
   p.off_kept = static_cast<int32_t>(off);
   if (job.n_out > 0) off = align_up(off + sizeof(uint16_t) * job.Kr, 16);
@@ -1000,7 +1249,7 @@ qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream) {
   if (job.rows == 0) return QR_OK;
   if (job.rot->kind == QR_ROT_KRON)
     return kron_tc_supported(job) ? launch_kron_tc(job, stream) : launch_kron_rows(job, stream);
-  return launch_wht_rows(job, stream);
+  return few_rows(job) ? launch_wht_few_rows(job, stream) : launch_wht_rows(job, stream);
 }
 
 }  // namespace qr

@@ -1,0 +1,430 @@
+// w4a4_gemm_decode.cu -- the W4A4 linear for a few tokens (M <= 64).
+//
+// Same computation as the prefill kernels (QUIK §1 and §4: INT4 codes
+// multiplied on integer tensor cores with INT32 accumulation, dequantized
+// per token and per channel, plus the fp16 product of the outlier columns),
+// shaped for decode, where the packed weights are nearly all of the bytes:
+//
+//  * Operands swapped: the MMA's M side is 128 weight rows, widened by the
+//    widen warps straight into tensor memory; the tokens (BN = 32 or 64
+//    rows, zero-filled beyond M) are the shared-memory B operand.
+//  * One 128-row weight tile per cluster and K split over the cluster's KS
+//    CTAs (KS = 1, 2 or 4, chosen so that tiles x KS fills the SMs): CTA r
+//    runs a contiguous range of the K steps; CTAs r > 0 add their int32
+//    accumulators into CTA 0's shared memory (integer adds, so the sum does
+//    not depend on their order) and CTA 0 runs the epilogue.  The fp16
+//    outlier steps all run in CTA 0, so the fp32 outlier sum has one order.
+//  * One CTA per SM runs a deep ring of widened stages (the chain widen ->
+//    MMA -> stage free is local to the SM).
+//
+// Warp roles (448 threads):
+//   warps 0-3   epilogue (TMEM lane = weight row of the tile)
+//   warps 4-11  widen (two groups of four warps taking alternate K steps)
+//   warp  12    producer (TMA; no multicast)
+//   warp  13    TMEM allocation and the MMA-issuing thread
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "qr_device.cuh"
+#include "qr_internal.h"
+
+namespace qr {
+
+namespace {
+
+constexpr int kStep = 64;          // packed bytes per row per K step (128 codes)
+constexpr int kSlot = 2 * kStep;   // packed bytes per row per ring slot (two K steps)
+constexpr int kNP = 4;             // packed ring depth (slots)
+constexpr int kNO = 2;             // outlier ring depth
+constexpr int kOutCols = 32;       // fp16 outlier columns per step (64-byte rows)
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kThreads = 32 * 14;
+constexpr int kSmemBudget = 227 * 1024;
+
+struct DecodeParams {
+  const float* w_scales;           // [N]
+  const float* a_scales;           // [M]
+  __half* Y;
+  int64_t ldy;
+  int32_t* acc_debug;              // [M x N] or null
+  int32_t N, M;
+  int32_t kt, ot;                  // int4 K steps, outlier steps
+  int32_t ks;                      // CTAs splitting K in a cluster
+  int32_t* status;
+};
+
+template <int BN, bool OUT>
+struct DecodeLayout {
+  static constexpr int kPackA = 128 * kSlot;               // 16 KB, 128-byte swizzle
+  static constexpr int kPackB = BN * kSlot;
+  static constexpr int kWideB = BN * 2 * kStep;            // SW128 K-major
+  static constexpr int kOutA = OUT ? 128 * kOutCols * 2 : 0;     // SW64 K-major
+  static constexpr int kOutB = OUT ? BN * kOutCols * 2 : 0;
+  static constexpr int kRed = BN * 128 * 4;                // int32 [BN][128]
+  static constexpr int kFixed = kNP * (kPackA + kPackB) + kNO * (kOutA + kOutB) + kRed + 2048;
+  // tensor memory: int32 accumulator, fp32 outlier accumulator, A stages
+  static constexpr int kAcol = OUT ? 2 * BN : BN;
+  static constexpr int kNWtmem = (512 - kAcol) / 32;
+  static constexpr int kNWsmem = (kSmemBudget - kFixed) / kWideB;
+  static constexpr int kNW = kNWtmem < kNWsmem ? (kNWtmem < 12 ? kNWtmem : 12)
+                                               : (kNWsmem < 12 ? kNWsmem : 12);
+  static constexpr int off_wide_b = 0;                     // 1024-aligned
+  static constexpr int off_out_a = off_wide_b + kNW * kWideB;
+  static constexpr int off_out_b = off_out_a + kNO * kOutA;
+  static constexpr int off_pack_a = off_out_b + kNO * kOutB;
+  static constexpr int off_pack_b = off_pack_a + kNP * kPackA;
+  static constexpr int off_red = off_pack_b + kNP * kPackB;
+  static constexpr int off_bar = off_red + kRed;
+  // full_p, empty_p, full_w, empty_w, full_o, empty_o, tmem_full, red_done, drain
+  static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 * kNO + 3;
+  static constexpr int off_misc = off_bar + 8 * kNumBars;
+  static constexpr int kBytes = off_misc + 16 + 1024;
+  static_assert(kNW >= 4, "stage ring");
+  static_assert(kBytes <= kSmemBudget, "shared memory");
+  static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+};
+
+// K steps of CTA `r` of a cluster of `ks`: int steps [i0, i1), outlier steps
+// [o0, o1).  CTA 0 takes every outlier step and a share of the int steps
+// that evens out the totals; the other CTAs split the rest of the int steps.
+// Int ranges start at even steps (a ring slot holds two).
+struct StepRange { int i0, i1, o0, o1; };
+
+__device__ __forceinline__ StepRange step_range(int r, int ks, int kt, int ot) {
+  StepRange s{0, kt, 0, ot};
+  if (ks == 1) return s;
+  const int per = (kt + ot + ks - 1) / ks;
+  const int first = min(kt, (max(0, per - ot) + 1) & ~1);
+  if (r == 0) return StepRange{0, first, 0, ot};
+  const int q = (((kt - first + ks - 2) / (ks - 1)) + 1) & ~1;
+  const int i0 = min(kt, first + (r - 1) * q);
+  return StepRange{i0, min(kt, i0 + q), 0, 0};
+}
+
+template <int BN, bool OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
+                        const __grid_constant__ CUtensorMap map_x,
+                        const __grid_constant__ CUtensorMap map_wo,
+                        const __grid_constant__ CUtensorMap map_xo, const DecodeParams p) {
+  using L = DecodeLayout<BN, OUT>;
+  constexpr int kNW = L::kNW;
+  constexpr uint32_t kAcol = L::kAcol;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+  uint64_t* full_p = bars;                   // TMA landed
+  uint64_t* empty_p = full_p + kNP;          // widen done reading (both groups: 8 warps)
+  uint64_t* full_w = empty_p + kNP;          // stage widened (4 warps)
+  uint64_t* empty_w = full_w + kNW;          // MMAs done with the stage
+  uint64_t* full_o = empty_w + kNW;          // outlier TMA landed
+  uint64_t* empty_o = full_o + kNO;          // MMAs done with the outlier stage
+  uint64_t* tmem_full = empty_o + kNO;       // accumulators final
+  uint64_t* red_done = tmem_full + 1;        // CTA 0: the other CTAs' sums landed
+  uint64_t* drain = red_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_misc);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + L::off_misc + 4);
+  int32_t* red = reinterpret_cast<int32_t*>(smem + L::off_red);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = p.ks > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int tile = blockIdx.x / p.ks;
+  const StepRange sr = step_range(rank, p.ks, p.kt, p.ot);
+  const int n_int = sr.i1 - sr.i0, n_out = OUT ? sr.o1 - sr.o0 : 0;
+  const int n_slots = (n_int + 1) >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 8); }
+    for (int i = 0; i < kNW; ++i) { mbar_init(&full_w[i], 4); mbar_init(&empty_w[i], 1); }
+    for (int i = 0; i < kNO; ++i) { mbar_init(&full_o[i], 1); mbar_init(&empty_o[i], 1); }
+    mbar_init(tmem_full, 1);
+    mbar_init(red_done, 128 * (p.ks - 1) > 0 ? 128 * (p.ks - 1) : 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (rank == 0 && p.ks > 1)
+    for (int i = threadIdx.x; i < BN * 128; i += kThreads) red[i] = 0;
+  if (warp == kProducerWarp && lane == 0) {
+    if (n_int > 0) { tma_prefetch_desc(&map_w); tma_prefetch_desc(&map_x); }
+    if (n_out > 0) { tma_prefetch_desc(&map_wo); tma_prefetch_desc(&map_xo); }
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (p.ks > 1) cluster_sync();              // CTA 0's sum buffer zeroed, barriers initialized
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int y_w = tile * 128;                // first weight row of the tile
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0;
+      for (; static_cast<int>(it) < n_slots; ++it) {
+        const uint32_t s = it % kNP, ph = (it / kNP) & 1;
+        const int x = (sr.i0 + 2 * static_cast<int>(it)) * kStep;
+        if (!(ok = mbar_wait_bounded(&empty_p[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
+        mbar_arrive_expect_tx(&full_p[s], L::kPackA + L::kPackB);
+        tma_load_2d(smem + L::off_pack_a + s * L::kPackA, &map_w, &full_p[s], x, y_w);
+        tma_load_2d(smem + L::off_pack_b + s * L::kPackB, &map_x, &full_p[s], x, 0);
+      }
+      uint32_t ot = 0;
+      if (OUT && ok)
+        for (int os = sr.o0; os < sr.o1; ++os, ++ot) {
+          const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
+          if (!(ok = mbar_wait_bounded(&empty_o[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
+          mbar_arrive_expect_tx(&full_o[s], L::kOutA + L::kOutB);
+          tma_load_2d(smem + L::off_out_a + s * L::kOutA, &map_wo, &full_o[s], os * kOutCols, y_w);
+          tma_load_2d(smem + L::off_out_b + s * L::kOutB, &map_xo, &full_o[s], os * kOutCols, 0);
+        }
+      if (!ok) {
+        for (uint32_t i = (it > kNP ? it - kNP : 0); i < it; ++i)
+          mbar_wait_bounded(&full_p[i % kNP], (i / kNP) & 1, abort_flag, nullptr, 0, kDrainLimitNs);
+        for (uint32_t i = (ot > kNO ? ot - kNO : 0); i < ot; ++i)
+          mbar_wait_bounded(&full_o[i % kNO], (i / kNO) & 1, abort_flag, nullptr, 0, kDrainLimitNs);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(BN);
+      constexpr uint32_t idesc_o = idesc_f16(BN);
+      bool ok = true;
+      for (int it = 0; it < n_int; ++it) {
+        const uint32_t s = it % kNW, ph = (it / kNW) & 1;
+        if (!(ok = mbar_wait_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
+        tc_fence_after();
+        const uint32_t a = tmem_base + kAcol + s * 32;
+        const uint64_t db = smem_desc_kmajor(smem_u32(smem + L::off_wide_b + s * L::kWideB), 128);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mma_i8_ts(tmem_base, a + 8 * k, db + 2 * k, idesc, (it | k) != 0);
+        mma_commit(&empty_w[s]);
+      }
+      if (OUT && ok)
+        for (int ot = 0; ot < n_out; ++ot) {
+          const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
+          if (!(ok = mbar_wait_bounded(&full_o[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
+          tc_fence_after();
+          const uint64_t da = smem_desc_kmajor(smem_u32(smem + L::off_out_a + s * L::kOutA), 64);
+          const uint64_t db = smem_desc_kmajor(smem_u32(smem + L::off_out_b + s * L::kOutB), 64);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) mma_f16(tmem_base + BN, da + 2 * k, db + 2 * k, idesc_o, (ot | k) != 0);
+          mma_commit(&empty_o[s]);
+        }
+      if (ok) mma_commit(tmem_full);
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0, abort_flag, p.status, kDevTimeoutDrain, kDrainLimitNs);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ widen
+    const int wt = threadIdx.x - 128;
+    const int group = wt >> 7;                     // takes the steps with it % 2 == group,
+    const int row = wt & 127;                      // i.e. half `group` of every ring slot;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;   // row = TMEM lane
+    bool ok = true;
+    for (int it = group; it < 2 * n_slots && ok; it += 2) {
+      const uint32_t s = (it >> 1) % kNP, ph = ((it >> 1) / kNP) & 1;
+      const uint32_t sw = it % kNW, phw = (it / kNW) & 1;
+      if (!(ok = mbar_wait_bounded(&full_p[s], ph, abort_flag, p.status, kDevTimeoutWiden))) break;
+      if (it >= n_int) {                           // the unused half of the last slot
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_p[s]);
+        break;
+      }
+      if (!(ok = mbar_wait_bounded(&empty_w[sw], phw ^ 1, abort_flag, p.status, kDevTimeoutWiden))) break;
+      {
+        // weight row: 64 packed bytes of this half (128-byte swizzled rows)
+        // -> 128 s8 in TMEM
+        const uint8_t* pa = smem + L::off_pack_a + s * L::kPackA + row * kSlot;
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(pa + (((4 * group + c) ^ (row & 7)) << 4));
+          r[8 * c + 0] = (u.x << 4) & 0xF0F0F0F0u;
+          r[8 * c + 1] = (u.y << 4) & 0xF0F0F0F0u;
+          r[8 * c + 2] = (u.z << 4) & 0xF0F0F0F0u;
+          r[8 * c + 3] = (u.w << 4) & 0xF0F0F0F0u;
+          r[8 * c + 4] = u.x & 0xF0F0F0F0u;
+          r[8 * c + 5] = u.y & 0xF0F0F0F0u;
+          r[8 * c + 6] = u.z & 0xF0F0F0F0u;
+          r[8 * c + 7] = u.w & 0xF0F0F0F0u;
+        }
+        tmem_st_32x32b_x32(tmem_base + lane_off + kAcol + sw * 32, r);
+      }
+      {
+        // token rows: 16-byte packed chunks -> two 16-byte s8 chunks, SW128
+        const uint8_t* pb = smem + L::off_pack_b + s * L::kPackB;
+        uint8_t* wb = smem + L::off_wide_b + sw * L::kWideB;
+        for (int task = row; task < BN * 4; task += 128) {
+          const int br = task >> 2, c = task & 3;
+          const uint4 u = *reinterpret_cast<const uint4*>(pb + br * kSlot + (4 * group + c) * 16);
+          uint4 ev, od;
+          ev.x = (u.x << 4) & 0xF0F0F0F0u; od.x = u.x & 0xF0F0F0F0u;
+          ev.y = (u.y << 4) & 0xF0F0F0F0u; od.y = u.y & 0xF0F0F0F0u;
+          ev.z = (u.z << 4) & 0xF0F0F0F0u; od.z = u.z & 0xF0F0F0F0u;
+          ev.w = (u.w << 4) & 0xF0F0F0F0u; od.w = u.w & 0xF0F0F0F0u;
+          uint8_t* base = wb + (br >> 3) * 1024 + (br & 7) * 128;
+          *reinterpret_cast<uint4*>(base + (((2 * c) ^ (br & 7)) << 4)) = ev;
+          *reinterpret_cast<uint4*>(base + (((2 * c + 1) ^ (br & 7)) << 4)) = od;
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full_w[sw]);
+        mbar_arrive(&empty_p[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int lrow = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int n = y_w + lrow;                      // output column = weight row
+    bool ok = mbar_wait_bounded(tmem_full, 0, abort_flag, p.status, kDevTimeoutEpilogue);
+    tc_fence_after();
+    if (rank > 0) {
+      // add this CTA's partial sums into CTA 0's buffer, then signal it
+      const uint32_t red0 = mapa_shared(smem_u32(red), 0);
+      if (ok && n_int > 0) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t acc[32];
+          tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < p.M)
+              red_add_cluster(red0 + 4u * static_cast<uint32_t>((c * 32 + j) * 128 + lrow),
+                              static_cast<int32_t>(acc[j]));
+        }
+      }
+      mbar_arrive_cluster(mapa_shared(smem_u32(red_done), 0));
+    } else {
+      if (ok && p.ks > 1)
+        ok = mbar_wait_cluster_bounded(red_done, 0, abort_flag, p.status, kDevTimeoutEpilogue);
+      const bool n_ok = ok && n < p.N;
+      const float s_row = n_ok ? __ldg(p.w_scales + n) * (1.0f / 256.0f) : 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t acc[32];
+        uint32_t oacc[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
+        if (OUT) tmem_ld_32x32b_x32(tmem_base + lane_off + BN + c * 32, oacc);
+        tmem_ld_wait();
+        if (!n_ok) continue;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int m = c * 32 + j;
+          if (m >= p.M) continue;
+          int32_t a = n_int > 0 ? static_cast<int32_t>(acc[j]) : 0;
+          if (p.ks > 1) a += red[m * 128 + lrow];
+          float y = static_cast<float>(a) * s_row * __ldg(p.a_scales + m);
+          if (OUT && n_out > 0) y += __uint_as_float(oacc[j]);
+          p.Y[static_cast<int64_t>(m) * p.ldy + n] = __float2half_rn(y);
+          if (p.acc_debug != nullptr) p.acc_debug[static_cast<int64_t>(m) * p.N + n] = a >> 8;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (p.ks > 1) cluster_sync();              // no CTA leaves while another may still signal it
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int BN, bool OUT>
+cudaError_t run_decode(const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& mwo,
+                       const CUtensorMap& mxo, const DecodeParams& p, int tiles,
+                       cudaStream_t stream) {
+  auto k = w4a4_gemm_decode_kernel<BN, OUT>;
+  const int smem = DecodeLayout<BN, OUT>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * p.ks), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.ks);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, mw, mx, mwo, mxo, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// CTAs per cluster splitting K: the largest of 1, 2, 4 with tiles x KS <= SMs
+// and at least one K step per CTA.
+int decode_k_split(int64_t tiles, int64_t steps, int sms) {
+  int ks = 1;
+  while (ks < 4 && tiles * ks * 2 <= sms && steps >= ks * 2) ks *= 2;
+  return ks;
+}
+
+qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
+  const bool out = j.n_out > 0;
+  const int bn = j.M <= 32 ? 32 : 64;
+  const int64_t tiles = (j.N + 127) / 128;
+  DecodeParams p{};
+  p.w_scales = j.w_scales;
+  p.a_scales = j.a_scales;
+  p.Y = reinterpret_cast<__half*>(j.Y);
+  p.ldy = j.ldy;
+  p.acc_debug = j.acc_debug;
+  p.N = static_cast<int32_t>(j.N);
+  p.M = static_cast<int32_t>(j.M);
+  p.kt = static_cast<int32_t>(j.Kp / 128);
+  p.ot = out ? (j.n_out + kOutCols - 1) / kOutCols : 0;
+  p.ks = decode_k_split(tiles, p.kt + p.ot, sm_count());
+  p.status = device_status_word();
+  if (p.status == nullptr) return QR_ERR_CUDA;
+  CUtensorMap mw{}, mx{}, mwo{}, mxo{};
+  const uint64_t kb = static_cast<uint64_t>(j.Kp) / 2;   // packed bytes per row
+  if (p.kt > 0 &&
+      (!make_tensor_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.w_codes, kb, j.N, kb, kSlot, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+       !make_tensor_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.a_codes, kb, j.M, kb, kSlot, bn,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)))
+    return QR_ERR_CUDA;
+  if (out) {
+    const uint64_t no = static_cast<uint64_t>(j.n_out);
+    if (!make_tensor_map_2d(&mwo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.w_out, no, j.N, no * 2,
+                            kOutCols, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tensor_map_2d(&mxo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.x_out, no, j.M, no * 2,
+                            kOutCols, bn, CU_TENSOR_MAP_SWIZZLE_64B))
+      return QR_ERR_CUDA;
+  }
+  const int t = static_cast<int>(tiles);
+  cudaError_t e;
+  if (bn == 32) e = out ? run_decode<32, true>(mw, mx, mwo, mxo, p, t, stream)
+                        : run_decode<32, false>(mw, mx, mwo, mxo, p, t, stream);
+  else e = out ? run_decode<64, true>(mw, mx, mwo, mxo, p, t, stream)
+               : run_decode<64, false>(mw, mx, mwo, mxo, p, t, stream);
+  return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+}
+
+}  // namespace qr

@@ -13,8 +13,10 @@
 //    only the packed A tile once.
 //  * The B operand is widened in shared memory into the canonical
 //    128-byte-swizzled K-major layout.
-//  * Prefill (M > 64): A = activations, B = weights.  Decode (SWAP, M <= 64):
-//    A = weights, B = tokens, and the epilogue writes Y transposed.
+//  * A = activations (M > 64), B = weights.
+//  * The packed tiles arrive by TMA in 128-byte rows, two K steps per ring
+//    slot: the TMA unit moves a tile row by row, and at 64-byte rows its row
+//    rate, not HBM, limited the feed.
 //  * OUT: the fp16 outlier columns run as a second cta_group::2 MMA of
 //    kind::f16 into an fp32 accumulator in TMEM, added in the epilogue.
 //
@@ -49,7 +51,8 @@ namespace qr {
 namespace {
 
 constexpr int kStep = 64;          // packed bytes per row per K step (128 codes)
-constexpr int kNP = 8;             // packed ring depth
+constexpr int kSlot = 2 * kStep;   // packed bytes per row per ring slot (two K steps)
+constexpr int kNP = 4;             // packed ring depth (slots)
 constexpr int kNO = 2;             // outlier ring depth
 constexpr int kOutCols = 32;       // fp16 outlier columns per step (64-byte rows)
 constexpr int kWidenWarps = 8;     // two groups of four
@@ -83,8 +86,8 @@ template <int BN, bool OUT>
 struct PairSmem {
   static constexpr int kNW = widened_stages<BN, OUT>();
   static constexpr int kHalf = BN / 2;                     // B rows per CTA
-  static constexpr int kPackA = 128 * kStep;               // 8 KB, 64-byte swizzle
-  static constexpr int kPackB = kHalf * kStep;
+  static constexpr int kPackA = 128 * kSlot;               // 16 KB, 128-byte swizzle
+  static constexpr int kPackB = kHalf * kSlot;
   static constexpr int kWideB = kHalf * 2 * kStep;         // SW128 K-major
   static constexpr int kOutA = OUT ? 128 * kOutCols * 2 : 0;     // SW64 K-major
   static constexpr int kOutB = OUT ? kHalf * kOutCols * 2 : 0;
@@ -103,7 +106,7 @@ struct PairSmem {
                 "swizzled tiles need 1024-byte alignment");
 };
 
-template <int BN, bool SWAP, bool OUT>
+template <int BN, bool OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                       const __grid_constant__ CUtensorMap map_b,
@@ -120,7 +123,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::off_bar);
   uint64_t* full_p = bars;                   // local: TMA landed
-  uint64_t* empty_p = full_p + kNP;          // local: widen done reading
+  uint64_t* empty_p = full_p + kNP;          // local: both widen groups done reading
   uint64_t* full_w = empty_p + kNP;          // widened: 4 local warps (+ the odd CTA's relay)
   uint64_t* empty_w = full_w + kNW;          // each CTA: the pair's MMAs done with the stage
   uint64_t* full_o = empty_w + kNW;          // local: outlier TMA landed
@@ -138,7 +141,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 4); }
+    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 8); }
     for (int i = 0; i < kNW; ++i) {
       mbar_init(&full_w[i], leader ? 5 : 4);
       mbar_init(&empty_w[i], 1);
@@ -169,6 +172,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
 
   const int num_tiles = p.tiles_a * p.tiles_b;
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int slots = (p.kt + 1) >> 1;         // ring slots per tile
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -179,12 +183,12 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
         const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
         const int ya = ta * 256 + static_cast<int>(rank) * 128;
         const int yb = tb * BN + static_cast<int>(rank) * S::kHalf;
-        for (int ks = 0; ks < p.kt; ++ks, ++it) {
+        for (int ps = 0; ps < slots; ++ps, ++it) {
           const uint32_t s = it % kNP, ph = (it / kNP) & 1;
           if (!(ok = mbar_wait_bounded(&empty_p[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
           mbar_arrive_expect_tx(&full_p[s], S::kPackA + S::kPackB);
-          tma_load_2d(smem + S::off_pack_a + s * S::kPackA, &map_a, &full_p[s], ks * kStep, ya);
-          tma_load_2d(smem + S::off_pack_b + s * S::kPackB, &map_b, &full_p[s], ks * kStep, yb);
+          tma_load_2d(smem + S::off_pack_a + s * S::kPackA, &map_a, &full_p[s], ps * kSlot, ya);
+          tma_load_2d(smem + S::off_pack_b + s * S::kPackB, &map_b, &full_p[s], ps * kSlot, yb);
         }
         if (OUT)
           for (int os = 0; os < p.ot && ok; ++os, ++ot) {
@@ -268,25 +272,30 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   } else if (warp >= 4) {
     // ------------------------------------------------------------ widen
     const int wt = threadIdx.x - 128;
-    const int group = wt >> 7;                     // takes K steps with it % 2 == group
-    const int arow = wt & 127;                     // = TMEM lane (warp % 4 quadrant)
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t it = 0;
+    const int group = wt >> 7;                     // takes the K steps ks with ks % 2 == group,
+    const int arow = wt & 127;                     // i.e. half `group` of every ring slot
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;   // arow = TMEM lane
+    uint32_t it = 0, pi = 0;                       // steps and slots of the earlier tiles
     bool ok = true;
-    for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
-      for (int ks = 0; ks < p.kt; ++ks, ++it) {
-        if ((it & 1) != static_cast<uint32_t>(group)) continue;
-        const uint32_t s = it % kNP, ph = (it / kNP) & 1;
-        const uint32_t sw = it % kNW, phw = (it / kNW) & 1;
+    for (int tile = cid; tile < num_tiles && ok; tile += ncl, it += p.kt, pi += slots) {
+      for (int ks = group; ks < 2 * slots; ks += 2) {
+        const uint32_t s = (pi + (ks >> 1)) % kNP, ph = ((pi + (ks >> 1)) / kNP) & 1;
         if (!(ok = mbar_wait_bounded(&full_p[s], ph, abort_flag, p.status, kDevTimeoutWiden))) break;
+        if (ks >= p.kt) {                          // the unused half of the last slot
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty_p[s]);
+          break;
+        }
+        const uint32_t wi = it + ks;
+        const uint32_t sw = wi % kNW, phw = (wi / kNW) & 1;
         if (!(ok = mbar_wait_cluster_bounded(&empty_w[sw], phw ^ 1, abort_flag, p.status, kDevTimeoutWiden))) break;
-        // A row: 64 packed bytes (64-byte swizzled rows) -> 128 s8 in TMEM
+        // A row: the 64 packed bytes of this half (128-byte swizzled rows) -> 128 s8 in TMEM
         {
-          const uint8_t* pa = smem + S::off_pack_a + s * S::kPackA + arow * kStep;
+          const uint8_t* pa = smem + S::off_pack_a + s * S::kPackA + arow * kSlot;
           uint32_t r[32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const uint4 u = *reinterpret_cast<const uint4*>(pa + ((c ^ ((arow >> 1) & 3)) << 4));
+            const uint4 u = *reinterpret_cast<const uint4*>(pa + (((4 * group + c) ^ (arow & 7)) << 4));
             r[8 * c + 0] = (u.x << 4) & 0xF0F0F0F0u;
             r[8 * c + 1] = (u.y << 4) & 0xF0F0F0F0u;
             r[8 * c + 2] = (u.z << 4) & 0xF0F0F0F0u;
@@ -306,7 +315,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
 #pragma unroll 2
           for (int task = arow; task < kTasks; task += kGroupThreads) {
             const int row = task >> 2, c = task & 3;
-            const uint4 u = *reinterpret_cast<const uint4*>(pb + row * kStep + c * 16);
+            const uint4 u = *reinterpret_cast<const uint4*>(pb + row * kSlot + (4 * group + c) * 16);
             uint4 ev, od;
             ev.x = (u.x << 4) & 0xF0F0F0F0u; od.x = u.x & 0xF0F0F0F0u;
             ev.y = (u.y << 4) & 0xF0F0F0F0u; od.y = u.y & 0xF0F0F0F0u;
@@ -360,53 +369,39 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
         }
         const int cb0 = tb * BN + c * 32;          // first B-side row of this chunk
         if (!ra_ok) continue;
-        if (!SWAP) {
-          // lane owns output row m = ra; columns n = cb0 + j
-          __half* yrow = p.Y + static_cast<int64_t>(ra) * p.ldy;
-          uint32_t hp[16];
+        // lane owns output row m = ra; columns n = cb0 + j
+        __half* yrow = p.Y + static_cast<int64_t>(ra) * p.ldy;
+        uint32_t hp[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float y2[2];
+        for (int j = 0; j < 32; j += 2) {
+          float y2[2];
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const int n = cb0 + j + t;
-              const float sb = (n < p.rows_b) ? __ldg(p.scale_b + n) : 0.0f;
-              y2[t] = static_cast<float>(static_cast<int32_t>(acc[j + t])) * s_row * sb;
-              if (OUT) y2[t] += __uint_as_float(oacc[j + t]);
-            }
-            const __half2 h2 = __floats2half2_rn(y2[0], y2[1]);
-            hp[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int t = 0; t < 2; ++t) {
+            const int n = cb0 + j + t;
+            const float sb = (n < p.rows_b) ? __ldg(p.scale_b + n) : 0.0f;
+            y2[t] = static_cast<float>(static_cast<int32_t>(acc[j + t])) * s_row * sb;
+            if (OUT) y2[t] += __uint_as_float(oacc[j + t]);
           }
-          if (p.y_vec_ok && cb0 + 32 <= p.rows_b) {
+          const __half2 h2 = __floats2half2_rn(y2[0], y2[1]);
+          hp[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        if (p.y_vec_ok && cb0 + 32 <= p.rows_b) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<uint4*>(yrow + cb0 + 8 * q) =
-                  make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (cb0 + j < p.rows_b)
-                reinterpret_cast<uint16_t*>(yrow)[cb0 + j] =
-                    static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
-          }
-          if (p.acc_debug != nullptr) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (cb0 + j < p.rows_b)
-                p.acc_debug[static_cast<int64_t>(ra) * p.N + cb0 + j] = static_cast<int32_t>(acc[j]) >> 8;
-          }
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(yrow + cb0 + 8 * q) =
+                make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
         } else {
-          // lane owns output column n = ra; rows m = cb0 + j (tokens)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int m = cb0 + j;
-            if (m >= p.rows_b) continue;
-            float y = static_cast<float>(static_cast<int32_t>(acc[j])) * s_row * __ldg(p.scale_b + m);
-            if (OUT) y += __uint_as_float(oacc[j]);
-            p.Y[static_cast<int64_t>(m) * p.ldy + ra] = __float2half_rn(y);
-            if (p.acc_debug != nullptr)
-              p.acc_debug[static_cast<int64_t>(m) * p.N + ra] = static_cast<int32_t>(acc[j]) >> 8;
-          }
+          for (int j = 0; j < 32; ++j)
+            if (cb0 + j < p.rows_b)
+              reinterpret_cast<uint16_t*>(yrow)[cb0 + j] =
+                  static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
+        }
+        if (p.acc_debug != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (cb0 + j < p.rows_b)
+              p.acc_debug[static_cast<int64_t>(ra) * p.N + cb0 + j] = static_cast<int32_t>(acc[j]) >> 8;
         }
       }
       tc_fence_before();
@@ -424,10 +419,10 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   }
 }
 
-template <int BN, bool SWAP, bool OUT>
+template <int BN, bool OUT>
 cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& moa,
                      const CUtensorMap& mob, const PairParams& p, cudaStream_t stream) {
-  auto k = w4a4_gemm_pair_kernel<BN, SWAP, OUT>;
+  auto k = w4a4_gemm_pair_kernel<BN, OUT>;
   const int smem = PairSmem<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -438,7 +433,7 @@ cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtenso
 
 }  // namespace
 
-// Tile width for prefill without outlier columns: the fewest tile rounds over
+// Tile width without outlier columns: the fewest tile rounds over
 // the SM pairs, weighted by the width (one round of a BN-wide tile costs
 // about BN).
 int pair_tile_width(int64_t M, int64_t N, int sms) {
@@ -460,63 +455,49 @@ int pair_tile_width(int64_t M, int64_t N, int sms) {
 }
 
 qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
-  const bool swap = j.M <= 64;
   const bool out = j.n_out > 0;
-  int bn;
-  if (swap) bn = j.M <= 32 ? 32 : 64;
-  else bn = out ? 96 : pair_tile_width(j.M, j.N, sm_count());
-  const int64_t rows_a = swap ? j.N : j.M;
-  const int64_t rows_b = swap ? j.M : j.N;
+  const int bn = out ? 96 : pair_tile_width(j.M, j.N, sm_count());
   PairParams p{};
-  p.scale_a = swap ? j.w_scales : j.a_scales;
-  p.scale_b = swap ? j.a_scales : j.w_scales;
+  p.scale_a = j.a_scales;
+  p.scale_b = j.w_scales;
   p.Y = reinterpret_cast<__half*>(j.Y);
   p.ldy = j.ldy;
   p.acc_debug = j.acc_debug;
-  p.rows_a = static_cast<int32_t>(rows_a);
-  p.rows_b = static_cast<int32_t>(rows_b);
+  p.rows_a = static_cast<int32_t>(j.M);
+  p.rows_b = static_cast<int32_t>(j.N);
   p.M = static_cast<int32_t>(j.M);
   p.N = static_cast<int32_t>(j.N);
   p.kt = static_cast<int32_t>(j.Kp / 128);
   p.ot = out ? (j.n_out + kOutCols - 1) / kOutCols : 0;
-  p.tiles_a = static_cast<int32_t>((rows_a + 255) / 256);
-  p.tiles_b = static_cast<int32_t>((rows_b + bn - 1) / bn);
+  p.tiles_a = static_cast<int32_t>((j.M + 255) / 256);
+  p.tiles_b = static_cast<int32_t>((j.N + bn - 1) / bn);
   p.y_vec_ok = (reinterpret_cast<uintptr_t>(j.Y) % 16 == 0) && (j.ldy % 8 == 0);
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
-  const uint8_t* ca = swap ? j.w_codes : j.a_codes;
-  const uint8_t* cb = swap ? j.a_codes : j.w_codes;
   CUtensorMap ma{}, mb{}, moa{}, mob{};
   const uint64_t kb = static_cast<uint64_t>(j.Kp) / 2;   // packed bytes per row
   if (p.kt > 0 &&
-      (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, ca, kb, rows_a, kb, kStep, 128,
-                           CU_TENSOR_MAP_SWIZZLE_64B) ||
-       !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, cb, kb, rows_b, kb, kStep,
+      (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.a_codes, kb, j.M, kb, kSlot, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+       !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.w_codes, kb, j.N, kb, kSlot,
                            bn / 2, CU_TENSOR_MAP_SWIZZLE_NONE)))
     return QR_ERR_CUDA;
   if (out) {
-    const uint16_t* oa = swap ? j.w_out : j.x_out;
-    const uint16_t* ob = swap ? j.x_out : j.w_out;
     const uint64_t no = static_cast<uint64_t>(j.n_out);
-    if (!make_tensor_map_2d(&moa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, oa, no, rows_a, no * 2,
+    if (!make_tensor_map_2d(&moa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.x_out, no, j.M, no * 2,
                             kOutCols, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_tensor_map_2d(&mob, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ob, no, rows_b, no * 2,
+        !make_tensor_map_2d(&mob, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.w_out, no, j.N, no * 2,
                             kOutCols, bn / 2, CU_TENSOR_MAP_SWIZZLE_64B))
       return QR_ERR_CUDA;
   }
   cudaError_t e;
-  if (swap) {
-    if (bn == 32) e = out ? run_pair<32, true, true>(ma, mb, moa, mob, p, stream)
-                          : run_pair<32, true, false>(ma, mb, moa, mob, p, stream);
-    else e = out ? run_pair<64, true, true>(ma, mb, moa, mob, p, stream)
-                 : run_pair<64, true, false>(ma, mb, moa, mob, p, stream);
-  } else if (out) {
-    e = run_pair<96, false, true>(ma, mb, moa, mob, p, stream);
+  if (out) {
+    e = run_pair<96, true>(ma, mb, moa, mob, p, stream);
   } else {
     switch (bn) {
-      case 192: e = run_pair<192, false, false>(ma, mb, moa, mob, p, stream); break;
-      case 160: e = run_pair<160, false, false>(ma, mb, moa, mob, p, stream); break;
-      default: e = run_pair<128, false, false>(ma, mb, moa, mob, p, stream); break;
+      case 192: e = run_pair<192, false>(ma, mb, moa, mob, p, stream); break;
+      case 160: e = run_pair<160, false>(ma, mb, moa, mob, p, stream); break;
+      default: e = run_pair<128, false>(ma, mb, moa, mob, p, stream); break;
     }
   }
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
