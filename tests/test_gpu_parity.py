@@ -174,7 +174,7 @@ LINEAR_CASES = [
     (100, 4096, 128, 0), (65, 33, 0, 0),
     # decode: K split over 1, 2 or 4 CTAs; outlier steps only on the first
     (5, 12288, 256, 0), (33, 8192, 512, 0), (64, 384, 128, 256), (2, 1000, 2048, 32),
-    (17, 130, 8192, 0),
+    (17, 130, 8192, 0), (16, 256, 128, 256),
 ]
 
 

@@ -488,3 +488,15 @@ __device__ __forceinline__ void red_add_cluster(uint32_t cluster_addr, int32_t v
 }
 
 }  // namespace qr
+
+namespace qr {
+
+// 16-byte store into another CTA's shared memory (address from mapa_shared).
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint32_t a, uint32_t b,
+                                              uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a),
+               "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+}  // namespace qr

@@ -583,21 +583,26 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
 
 // ------------------------------------------------------------------ few rows
 
-// Few rows (decode): one CTA per row, the whole row in shared memory.  The
-// kernels above give each row one group of threads and keep it in
-// registers, which fills the GPU only with many rows; with a handful of
-// tokens a row's latency is the whole cost, so here up to 1024 threads share
-// one row.  Steps: load the row with vector loads (the outlier columns of
-// QUIK §1 removed by a block-wide prefix count over an outlier bitmap, the
-// kept columns compacted to their rotated positions), the Walsh-Hadamard
+// Few rows (decode): a cluster of CL CTAs per row, each holding a span of
+// whole rotation blocks in shared memory.  The kernels above give each row
+// one group of threads and keep it in registers, which fills the GPU only
+// with many rows; with a handful of tokens a row's latency is the whole
+// cost, so here up to CL x 1024 threads on CL SMs share one row and every
+// global load is issued up front.  Steps: load the row (vector loads) and
+// the outlier indices together; drop the outlier columns of QUIK §1 by a
+// block-wide prefix count over an outlier bitmap, each CTA keeping the kept
+// columns whose rotated positions fall in its span; run the Walsh-Hadamard
 // butterflies in passes of up to three stages through shared memory, the
-// row absmax, then quantize + pack as the other kernels do.
+// last pass also taking the span's absmax; combine the CL maxima through
+// distributed shared memory; then quantize + pack as the other kernels do.
 struct FewRowsParams {
   const __half* src;
   int64_t rows, ld;
   int32_t K, Kr, Kp, n_out;
   const int32_t* outlier_idx;
   int32_t lb, gsr, aligned;
+  int32_t cl;                 // CTAs per row (a cluster)
+  int32_t span;               // rotated elements per CTA (whole blocks, a multiple of 128)
   int32_t off_bits, off_scan;
   float clip_ratio, inv_sqrt_block;
   uint8_t* codes;
@@ -605,6 +610,13 @@ struct FewRowsParams {
   __half* out16;
   float* rot_debug;
 };
+
+constexpr int kFewMaxChunks = 4;   // 8-column chunks per thread (K <= 32768 at 1024 threads)
+
+// Shared-memory position of row element e: bits 3-4 XOR bits 6-7, so that
+// the butterfly passes with strides 8..32 hit 32 distinct banks; groups of 8
+// consecutive elements stay contiguous and aligned.
+__device__ __forceinline__ int few_swz(int e) { return e ^ (((e >> 6) & 3) << 3); }
 
 // Exclusive prefix sum over the block (blockDim a multiple of 32); `sh`
 // holds 32 ints.  Contains two __syncthreads.
@@ -644,17 +656,26 @@ __device__ __forceinline__ float block_max(float v, float* sh) {
   return m;
 }
 
-// R butterfly stages on index bits [s, s+R) of the row in shared memory.
+// R butterfly stages on index bits [s, s+R) of the row in shared memory;
+// returns the largest |value| this thread wrote.
 template <int R>
-__device__ __forceinline__ void wht_smem_pass(float* buf, int Kp, int s) {
+__device__ __forceinline__ float wht_smem_pass(float* buf, int Kp, int s) {
   constexpr int G = 1 << R;
   const int ngroups = Kp >> R;
   const int lowmask = (1 << s) - 1;
+  float am = 0.0f;
   for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
     const int base = (g & lowmask) | ((g >> s) << (s + R));
     float x[G];
+    if (R == 3 && s == 0) {                        // 8 contiguous, aligned elements
+      const float4 a = *reinterpret_cast<const float4*>(buf + few_swz(base));
+      const float4 b = *reinterpret_cast<const float4*>(buf + few_swz(base) + 4);
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+      x[4 % G] = b.x; x[5 % G] = b.y; x[6 % G] = b.z; x[7 % G] = b.w;
+    } else {
 #pragma unroll
-    for (int k = 0; k < G; ++k) x[k] = buf[base + (k << s)];
+      for (int k = 0; k < G; ++k) x[k] = buf[few_swz(base + (k << s))];
+    }
 #pragma unroll
     for (int st = 0; st < R; ++st)
 #pragma unroll
@@ -665,120 +686,143 @@ __device__ __forceinline__ void wht_smem_pass(float* buf, int Kp, int s) {
           x[k | (1 << st)] = a - b;
         }
 #pragma unroll
-    for (int k = 0; k < G; ++k) buf[base + (k << s)] = x[k];
+    for (int k = 0; k < G; ++k) am = fmaxf(am, fabsf(x[k]));
+    if (R == 3 && s == 0) {
+      *reinterpret_cast<float4*>(buf + few_swz(base)) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(buf + few_swz(base) + 4) =
+          make_float4(x[4 % G], x[5 % G], x[6 % G], x[7 % G]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < G; ++k) buf[few_swz(base + (k << s))] = x[k];
+    }
   }
+  return am;
 }
 
 template <bool CLIP>
 __global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  float* buf = reinterpret_cast<float*>(smem);                       // [Kp]
+  float* buf = reinterpret_cast<float*>(smem);                       // [span], few_swz order
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);   // outlier bitmap
   int* scan = reinterpret_cast<int*>(smem + p.off_scan);             // 32 ints
   float* red = reinterpret_cast<float*>(smem + p.off_scan + 128);    // 32 floats
+  float* maxima = reinterpret_cast<float*>(smem + p.off_scan + 256); // CL floats
   const int t = threadIdx.x, nthr = blockDim.x;
+  const int64_t row = blockIdx.x / p.cl;
+  const int cr = blockIdx.x % p.cl;                                  // rank in the cluster
+  const int e_lo = cr * p.span;                                      // this CTA's rotated span
+  const int e_hi = min(p.Kp, e_lo + p.span);
+  const int nloc = max(0, e_hi - e_lo);
   const int nchunks = (p.K + 7) >> 3;                                // 8 source columns each
   const int cpt = (nchunks + nthr - 1) / nthr;                       // chunks per thread
   const int nwords = (p.K + 31) >> 5;
-  for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
-    const __half* srow = p.src + row * p.ld;
-    if (p.n_out > 0) {
-      for (int w = t; w < nwords; w += nthr) bits[w] = 0u;
-      __syncthreads();
-      for (int j = t; j < p.n_out; j += nthr) {
-        const int c = __ldg(p.outlier_idx + j);
-        if (c >= 0 && c < p.K) atomicOr(&bits[c >> 5], 1u << (c & 31));
-        if (p.out16 != nullptr)
-          p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? srow[c] : __float2half(0.0f);
-      }
-      __syncthreads();
-    }
-    for (int e = p.Kr + t; e < p.Kp; e += nthr) buf[e] = 0.0f;
-    // this thread's chunks [c0, c0 + cpt): outliers before them, then scatter
-    const int c0 = t * cpt;
-    int before = 0;
-    if (p.n_out > 0) {
-      int cnt = 0;
-      for (int q = 0; q < cpt; ++q) {
-        const int c = c0 + q;
-        if (c < nchunks) cnt += __popc((bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu);
-      }
-      before = block_exclusive_sum(cnt, scan);
-    }
-    for (int q = 0; q < cpt; ++q) {
-      const int c = c0 + q;
-      if (c >= nchunks) break;
-      const int col0 = 8 * c;
-      float x[8];
-      if (p.aligned && col0 + 8 <= p.K) {
-        const uint4 u = ld_stream_v4(srow + col0);
-        const __half2* h = reinterpret_cast<const __half2*>(&u);
+  const int c0 = t * cpt;                                            // this thread's chunks
+  const __half* srow = p.src + row * p.ld;
+  // the row's vector loads first; their latency overlaps the outlier work
+  uint4 raw[kFewMaxChunks];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __half22float2(h[i]);
-          x[2 * i] = f.x;
-          x[2 * i + 1] = f.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = (col0 + i < p.K) ? __half2float(srow[col0 + i]) : 0.0f;
-      }
-      const uint32_t m8 = p.n_out > 0 ? (bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int e = col0 + i - before;
-        if ((m8 >> i) & 1u) {
-          ++before;
-        } else if (col0 + i < p.K && e < p.Kr) {
-          buf[e] = x[i];
-        }
-      }
+  for (int q = 0; q < kFewMaxChunks; ++q) {
+    const int col0 = 8 * (c0 + q);
+    raw[q] = make_uint4(0u, 0u, 0u, 0u);
+    if (q < cpt && p.aligned && col0 + 8 <= p.K) raw[q] = ld_stream_v4(srow + col0);
+  }
+  int before = 0;
+  if (p.n_out > 0) {
+    for (int w = t; w < nwords; w += nthr) bits[w] = 0u;
+    __syncthreads();
+    for (int j = t; j < p.n_out; j += nthr) {
+      const int c = __ldg(p.outlier_idx + j);
+      if (c >= 0 && c < p.K) atomicOr(&bits[c >> 5], 1u << (c & 31));
+      if (p.out16 != nullptr && cr == 0)
+        p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? srow[c] : __float2half(0.0f);
     }
     __syncthreads();
-    for (int s = 0; s < p.lb; s += 3) {
-      const int r = min(3, p.lb - s);
-      if (r == 3) wht_smem_pass<3>(buf, p.Kp, s);
-      else if (r == 2) wht_smem_pass<2>(buf, p.Kp, s);
-      else wht_smem_pass<1>(buf, p.Kp, s);
-      __syncthreads();
+    int cnt = 0;
+    for (int q = 0; q < cpt; ++q) {
+      const int c = c0 + q;
+      if (c < nchunks) cnt += __popc((bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu);
     }
-    const int ngroups = p.Kp >> 3;
-    float am = 0.0f;
-    for (int g = t; g < ngroups; g += nthr) {
-      const float4 a = *reinterpret_cast<const float4*>(buf + 8 * g);
-      const float4 b = *reinterpret_cast<const float4*>(buf + 8 * g + 4);
-      am = fmaxf(am, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
-      am = fmaxf(am, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
-    }
-    am = block_max(am, red);
-    const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
-    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
-    if (t == 0) p.scales[row] = s;
-    uint8_t* crow = p.codes + row * (p.Kp >> 1);
-    const int bm = (1 << p.lb) - 1;
-    for (int g = t; g < ngroups; g += nthr) {
-      float v[8];
-      if (p.gsr) {
-        // sequency position j of a block takes Hadamard output bitrev(gray(j))
+    before = block_exclusive_sum(cnt, scan);
+  }
+  // scatter the kept columns whose rotated positions are in [e_lo, e_hi);
+  // zero the padding beyond the real columns
+  for (int e = max(p.Kr, e_lo) + t; e < e_hi; e += nthr) buf[few_swz(e - e_lo)] = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int e = 8 * g + i;
-          const int j = e & bm;
-          const int nat = static_cast<int>(__brev(static_cast<unsigned>(j ^ (j >> 1))) >> (32 - p.lb));
-          v[i] = buf[(e & ~bm) + nat];
-        }
-      } else {
-        const float4 a = *reinterpret_cast<const float4*>(buf + 8 * g);
-        const float4 b = *reinterpret_cast<const float4*>(buf + 8 * g + 4);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  for (int q = 0; q < kFewMaxChunks; ++q) {
+    const int c = c0 + q;
+    if (q >= cpt || c >= nchunks) continue;
+    const int col0 = 8 * c;
+    float x[8];
+    if (p.aligned && col0 + 8 <= p.K) {
+      const __half2* h = reinterpret_cast<const __half2*>(&raw[q]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
       }
-      *reinterpret_cast<uint32_t*>(crow + 4 * g) = quant_word<CLIP>(v, r);
-      if (p.rot_debug != nullptr)
+    } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) p.rot_debug[row * p.Kp + 8 * g + i] = v[i] * p.inv_sqrt_block;
+      for (int i = 0; i < 8; ++i) x[i] = (col0 + i < p.K) ? __half2float(srow[col0 + i]) : 0.0f;
     }
-    __syncthreads();                       // buf, bits and the scratch words are reused
+    const uint32_t m8 = p.n_out > 0 ? (bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = col0 + i - before;
+      if ((m8 >> i) & 1u) {
+        ++before;
+      } else if (col0 + i < p.K && e < p.Kr && e >= e_lo && e < e_hi) {
+        buf[few_swz(e - e_lo)] = x[i];
+      }
+    }
+  }
+  __syncthreads();
+  float am = 0.0f;
+  for (int s = 0; s < p.lb; s += 3) {
+    const int r = min(3, p.lb - s);
+    if (r == 3) am = wht_smem_pass<3>(buf, nloc, s);
+    else if (r == 2) am = wht_smem_pass<2>(buf, nloc, s);
+    else am = wht_smem_pass<1>(buf, nloc, s);
+    __syncthreads();
+  }
+  if (p.lb == 0)
+    for (int e = t; e < nloc; e += nthr) am = fmaxf(am, fabsf(buf[e]));
+  am = block_max(am, red);
+  if (p.cl > 1) {
+    // every CTA of the row stores its span's maximum into every CTA
+    if (t < p.cl)
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(mapa_shared(smem_u32(maxima + cr), t)),
+                   "f"(am)
+                   : "memory");
+    cluster_sync();
+    for (int i = 0; i < p.cl; ++i) am = fmaxf(am, maxima[i]);
+  }
+  const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
+  const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
+  if (t == 0 && cr == 0) p.scales[row] = s;
+  uint8_t* crow = p.codes + row * (p.Kp >> 1);
+  const int bm = (1 << p.lb) - 1;
+  for (int g = t; g < (nloc >> 3); g += nthr) {
+    const int el = 8 * g;                          // local index of the group
+    float v[8];
+    if (p.gsr) {
+      // sequency position j of a block takes Hadamard output bitrev(gray(j))
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = (el + i) & bm;
+        const int nat = static_cast<int>(__brev(static_cast<unsigned>(j ^ (j >> 1))) >> (32 - p.lb));
+        v[i] = buf[few_swz(((el + i) & ~bm) + nat)];
+      }
+    } else {
+      const float4 a = *reinterpret_cast<const float4*>(buf + few_swz(el));
+      const float4 b = *reinterpret_cast<const float4*>(buf + few_swz(el) + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    *reinterpret_cast<uint32_t*>(crow + ((e_lo + el) >> 1)) = quant_word<CLIP>(v, r);
+    if (p.rot_debug != nullptr)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) p.rot_debug[row * p.Kp + e_lo + el + i] = v[i] * p.inv_sqrt_block;
   }
 }
 
@@ -1035,7 +1079,8 @@ int pow2_at_least(int v) {
 
 // One CTA per row while the rows do not fill the SMs.
 bool few_rows(const RowJob& job) {
-  return job.rows <= sm_count() && job.Kp <= 32768 && job.Kp > 0;
+  return job.rows <= sm_count() && job.Kp <= 32768 && job.Kp > 0 &&
+         (job.K + 7) / 8 <= 1024 * kFewMaxChunks;
 }
 
 qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
@@ -1059,22 +1104,42 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
   p.scales = job.scales;
   p.out16 = reinterpret_cast<__half*>(job.out16);
   p.rot_debug = job.rot_debug;
-  size_t off = align_up(sizeof(float) * static_cast<size_t>(job.Kp), 16);
+  // CTAs per row: up to 8 (and the SMs left per row), each a span of whole
+  // blocks that is a multiple of 128 elements
+  const int unit = std::max(1, 128 >> p.lb);                  // blocks per 128 elements
+  const int nunits = (job.Kp >> p.lb) / unit;
+  const int64_t room = std::max<int64_t>(1, sm_count() / job.rows);
+  int cl = 1;
+  while (cl * 2 <= 8 && cl * 2 <= nunits && cl * 2 <= room) cl *= 2;
+  const int units_per_cta = (nunits + cl - 1) / cl;
+  p.cl = cl;
+  p.span = units_per_cta * unit << p.lb;
+  const int64_t chunks = (job.K + 7) / 8;
+  const int64_t want = std::max<int64_t>(p.span / 8, (chunks + kFewMaxChunks - 1) / kFewMaxChunks);
+  const int threads = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(128, (want + 31) / 32 * 32)));
+  if (chunks > static_cast<int64_t>(threads) * kFewMaxChunks) return QR_ERR_UNSUPPORTED;
+  size_t off = align_up(sizeof(float) * static_cast<size_t>(p.span), 16);
   p.off_bits = static_cast<int32_t>(off);
   off = align_up(off + sizeof(uint32_t) * static_cast<size_t>((job.K + 31) / 32), 16);
   p.off_scan = static_cast<int32_t>(off);
-  off += 256;
+  off += 512;                                  // scan words, block maxima, cluster maxima
   if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
-  const int threads = std::min(1024, std::max(128, (job.Kp / 8 + 31) / 32 * 32));
-  const int grid = static_cast<int>(job.rows);
-  cudaError_t e;
-  if (rot.clip_ratio < 1.0f) {
-    e = set_smem(wht_few_rows_kernel<true>, off);
-    if (e == cudaSuccess) wht_few_rows_kernel<true><<<grid, threads, off, stream>>>(p);
-  } else {
-    e = set_smem(wht_few_rows_kernel<false>, off);
-    if (e == cudaSuccess) wht_few_rows_kernel<false><<<grid, threads, off, stream>>>(p);
-  }
+  auto k = rot.clip_ratio < 1.0f ? wht_few_rows_kernel<true> : wht_few_rows_kernel<false>;
+  cudaError_t e = set_smem(k, off);
+  if (e != cudaSuccess) return QR_ERR_CUDA;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(job.rows * cl), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = off;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }

@@ -10,10 +10,14 @@
 //    rows, zero-filled beyond M) are the shared-memory B operand.
 //  * One 128-row weight tile per cluster and K split over the cluster's KS
 //    CTAs (KS = 1, 2 or 4, chosen so that tiles x KS fills the SMs): CTA r
-//    runs a contiguous range of the K steps; CTAs r > 0 add their int32
-//    accumulators into CTA 0's shared memory (integer adds, so the sum does
-//    not depend on their order) and CTA 0 runs the epilogue.  The fp16
-//    outlier steps all run in CTA 0, so the fp32 outlier sum has one order.
+//    runs a contiguous range of the K steps.  The partial sums are then
+//    exchanged, not funnelled: CTA r owns the rows [r*128/KS, (r+1)*128/KS)
+//    of the tile, every CTA stores the other CTAs' rows of its int32
+//    partials into their shared memory (16-byte remote stores), and each CTA
+//    adds the partials of its own rows (integer adds: the order does not
+//    matter) and runs their epilogue.  The fp16 outlier steps all run in
+//    CTA 0, which sends the fp32 outlier sums with its partials, so that sum
+//    has one order.
 //  * One CTA per SM runs a deep ring of widened stages (the chain widen ->
 //    MMA -> stage free is local to the SM).
 //
@@ -64,7 +68,12 @@ struct DecodeLayout {
   static constexpr int kWideB = BN * 2 * kStep;            // SW128 K-major
   static constexpr int kOutA = OUT ? 128 * kOutCols * 2 : 0;     // SW64 K-major
   static constexpr int kOutB = OUT ? BN * kOutCols * 2 : 0;
-  static constexpr int kRed = BN * 128 * 4;                // int32 [BN][128]
+  // partials received from the other CTAs of the cluster: (KS-1) slots of
+  // 128/KS rows, each row BN int32 (+ BN fp32 outlier sums) + 4 words of
+  // padding (an odd number of 16-byte chunks per row: conflict-free rows)
+  static constexpr int kMaxKS = BN == 64 ? 2 : 4;
+  static constexpr int kRowWords = (OUT ? 2 * BN : BN) + 4;
+  static constexpr int kRed = (kMaxKS - 1) * (128 / kMaxKS) * kRowWords * 4;
   static constexpr int kFixed = kNP * (kPackA + kPackB) + kNO * (kOutA + kOutB) + kRed + 2048;
   // tensor memory: int32 accumulator, fp32 outlier accumulator, A stages
   static constexpr int kAcol = OUT ? 2 * BN : BN;
@@ -79,12 +88,13 @@ struct DecodeLayout {
   static constexpr int off_pack_b = off_pack_a + kNP * kPackA;
   static constexpr int off_red = off_pack_b + kNP * kPackB;
   static constexpr int off_bar = off_red + kRed;
-  // full_p, empty_p, full_w, empty_w, full_o, empty_o, tmem_full, red_done, drain
+  // full_p, empty_p, full_w, empty_w, full_o, empty_o, tmem_full, recv, drain
   static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 * kNO + 3;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
   static constexpr int kBytes = off_misc + 16 + 1024;
   static_assert(kNW >= 4, "stage ring");
   static_assert(kBytes <= kSmemBudget, "shared memory");
+  static_assert(BN == 32 || BN == 64, "token tile");
   static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
 };
@@ -126,11 +136,12 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   uint64_t* full_o = empty_w + kNW;          // outlier TMA landed
   uint64_t* empty_o = full_o + kNO;          // MMAs done with the outlier stage
   uint64_t* tmem_full = empty_o + kNO;       // accumulators final
-  uint64_t* red_done = tmem_full + 1;        // CTA 0: the other CTAs' sums landed
-  uint64_t* drain = red_done + 1;
+  uint64_t* recv = tmem_full + 1;            // the other CTAs' partials of my rows landed
+  uint64_t* drain = recv + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_misc);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + L::off_misc + 4);
-  int32_t* red = reinterpret_cast<int32_t*>(smem + L::off_red);
+  uint32_t* slots = reinterpret_cast<uint32_t*>(smem + L::off_red);
+  const int own_rows = 128 / p.ks;           // tile rows this CTA finishes
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -145,13 +156,11 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     for (int i = 0; i < kNW; ++i) { mbar_init(&full_w[i], 4); mbar_init(&empty_w[i], 1); }
     for (int i = 0; i < kNO; ++i) { mbar_init(&full_o[i], 1); mbar_init(&empty_o[i], 1); }
     mbar_init(tmem_full, 1);
-    mbar_init(red_done, 128 * (p.ks - 1) > 0 ? 128 * (p.ks - 1) : 1);
+    mbar_init(recv, p.ks > 1 ? (p.ks - 1) * own_rows : 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (rank == 0 && p.ks > 1)
-    for (int i = threadIdx.x; i < BN * 128; i += kThreads) red[i] = 0;
   if (warp == kProducerWarp && lane == 0) {
     if (n_int > 0) { tma_prefetch_desc(&map_w); tma_prefetch_desc(&map_x); }
     if (n_out > 0) { tma_prefetch_desc(&map_wo); tma_prefetch_desc(&map_xo); }
@@ -162,7 +171,7 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   }
   tc_fence_before();
   __syncthreads();
-  if (p.ks > 1) cluster_sync();              // CTA 0's sum buffer zeroed, barriers initialized
+  if (p.ks > 1) cluster_sync();              // every CTA's barriers initialized
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int y_w = tile * 128;                // first weight row of the tile
@@ -291,49 +300,95 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int lrow = warp * 32 + lane;
+    const int lrow = warp * 32 + lane;             // tile row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int owner = lrow / own_rows;             // the CTA that finishes this row
+    const bool has_out = OUT && p.ot > 0;
+    // scales, loaded while the MMAs run: this row's, and one token's per lane
+    // for each 32-token chunk (broadcast by shuffles in the epilogue)
     const int n = y_w + lrow;                      // output column = weight row
+    float s_row = 0.0f, sa_lane[BN / 32];
+    if (owner == rank) {
+      s_row = n < p.N ? __ldg(p.w_scales + n) * (1.0f / 256.0f) : 0.0f;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c)
+        sa_lane[c] = c * 32 + lane < p.M ? __ldg(p.a_scales + c * 32 + lane) : 0.0f;
+    }
     bool ok = mbar_wait_bounded(tmem_full, 0, abort_flag, p.status, kDevTimeoutEpilogue);
     tc_fence_after();
-    if (rank > 0) {
-      // add this CTA's partial sums into CTA 0's buffer, then signal it
-      const uint32_t red0 = mapa_shared(smem_u32(red), 0);
-      if (ok && n_int > 0) {
+    if (owner != rank) {
+      // send this row's partials (int32, and CTA 0's fp32 outlier sums)
+      const int slot = (rank - owner - 1 + p.ks) % p.ks;
+      const uint32_t dst = mapa_shared(smem_u32(slots), static_cast<uint32_t>(owner)) +
+                           4u * static_cast<uint32_t>((slot * own_rows + lrow % own_rows) * L::kRowWords);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t acc[32];
-          tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t acc[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
+        tmem_ld_wait();
+        if (n_int == 0 || !ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] = 0;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_cluster_v4(dst + 4u * (c * 32 + 4 * q), acc[4 * q], acc[4 * q + 1], acc[4 * q + 2],
+                        acc[4 * q + 3]);
+        if (has_out && rank == 0) {
+          tmem_ld_32x32b_x32(tmem_base + lane_off + BN + c * 32, acc);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j < p.M)
-              red_add_cluster(red0 + 4u * static_cast<uint32_t>((c * 32 + j) * 128 + lrow),
-                              static_cast<int32_t>(acc[j]));
+          for (int q = 0; q < 8; ++q)
+            st_cluster_v4(dst + 4u * (BN + c * 32 + 4 * q), acc[4 * q], acc[4 * q + 1],
+                          acc[4 * q + 2], acc[4 * q + 3]);
         }
       }
-      mbar_arrive_cluster(mapa_shared(smem_u32(red_done), 0));
+      mbar_arrive_cluster(mapa_shared(smem_u32(recv), static_cast<uint32_t>(owner)));
     } else {
+      // finish this row: own partial + the received ones, dequantize, store
       if (ok && p.ks > 1)
-        ok = mbar_wait_cluster_bounded(red_done, 0, abort_flag, p.status, kDevTimeoutEpilogue);
+        ok = mbar_wait_cluster_bounded(recv, 0, abort_flag, p.status, kDevTimeoutEpilogue);
       const bool n_ok = ok && n < p.N;
-      const float s_row = n_ok ? __ldg(p.w_scales + n) * (1.0f / 256.0f) : 0.0f;
+      const int r_local = lrow % own_rows;
+      const int slot0 = (0 - rank - 1 + p.ks) % p.ks;   // CTA 0's slot (outlier sums)
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t acc[32];
         uint32_t oacc[32];
+        const float sa_c = c == 0 ? sa_lane[0] : sa_lane[BN / 32 - 1];   // BN <= 64
         tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
         if (OUT) tmem_ld_32x32b_x32(tmem_base + lane_off + BN + c * 32, oacc);
         tmem_ld_wait();
-        if (!n_ok) continue;
+        if (n_int == 0) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] = 0;
+        }
+        for (int sl = 0; sl < p.ks - 1; ++sl) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              slots + (sl * own_rows + r_local) * L::kRowWords + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 v = src[q];
+            acc[4 * q] += v.x; acc[4 * q + 1] += v.y; acc[4 * q + 2] += v.z; acc[4 * q + 3] += v.w;
+          }
+        }
+        if (OUT && has_out && rank != 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              slots + (slot0 * own_rows + r_local) * L::kRowWords + BN + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 v = src[q];
+            oacc[4 * q] = v.x; oacc[4 * q + 1] = v.y; oacc[4 * q + 2] = v.z; oacc[4 * q + 3] = v.w;
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int m = c * 32 + j;
-          if (m >= p.M) continue;
-          int32_t a = n_int > 0 ? static_cast<int32_t>(acc[j]) : 0;
-          if (p.ks > 1) a += red[m * 128 + lrow];
-          float y = static_cast<float>(a) * s_row * __ldg(p.a_scales + m);
-          if (OUT && n_out > 0) y += __uint_as_float(oacc[j]);
+          const float sa = __shfl_sync(0xffffffffu, sa_c, j);
+          if (m >= p.M || !n_ok) continue;
+          const int32_t a = static_cast<int32_t>(acc[j]);
+          float y = static_cast<float>(a) * s_row * sa;
+          if (has_out) y += __uint_as_float(oacc[j]);
           p.Y[static_cast<int64_t>(m) * p.ldy + n] = __float2half_rn(y);
           if (p.acc_debug != nullptr) p.acc_debug[static_cast<int64_t>(m) * p.N + n] = a >> 8;
         }
@@ -399,7 +454,7 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
   p.M = static_cast<int32_t>(j.M);
   p.kt = static_cast<int32_t>(j.Kp / 128);
   p.ot = out ? (j.n_out + kOutCols - 1) / kOutCols : 0;
-  p.ks = decode_k_split(tiles, p.kt + p.ot, sm_count());
+  p.ks = std::min(decode_k_split(tiles, p.kt + p.ot, sm_count()), bn == 64 ? 2 : 4);
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
   CUtensorMap mw{}, mx{}, mwo{}, mxo{};
