@@ -169,9 +169,12 @@ LINEAR_CASES = [
     (65, 129, 128, 0), (128, 256, 512, 0), (200, 520, 384, 0), (300, 1000, 1024, 0),
     (4, 64, 256, 8), (16, 200, 512, 40), (64, 256, 256, 256), (100, 300, 384, 64),
     (256, 384, 256, 32), (3, 40, 0, 16), (130, 70, 0, 24),
-    # two-SM tiles: 256-row pairs, widths 128..224, ragged edges, long K
+    # two-SM tiles: 256-row pairs, widths 128 and 160, ragged edges, long K
     (257, 225, 384, 0), (512, 448, 1280, 0), (300, 1000, 11008, 0), (1000, 700, 256, 0),
     (100, 4096, 128, 0), (65, 33, 0, 0),
+    # several tiles per CTA pair with an odd number of ring slots per tile,
+    # with and without outliers (the outlier tile leaves two A stages)
+    (2048, 7104, 640, 0), (1024, 4096, 640, 64),
     # decode: K split over 1, 2 or 4 CTAs; outlier steps only on the first
     (5, 12288, 256, 0), (33, 8192, 512, 0), (64, 384, 128, 256), (2, 1000, 2048, 32),
     (17, 130, 8192, 0), (16, 256, 128, 256),

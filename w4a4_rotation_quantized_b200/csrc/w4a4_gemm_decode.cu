@@ -64,8 +64,9 @@ struct DecodeParams {
 template <int BN, bool OUT>
 struct DecodeLayout {
   static constexpr int kPackA = 128 * kSlot;               // 16 KB, 128-byte swizzle
-  static constexpr int kPackB = BN * kSlot;
-  static constexpr int kWideB = BN * 2 * kStep;            // SW128 K-major
+  static constexpr int kPackB = BN * kSlot;                // 128-byte swizzle
+  static constexpr int kWideBlk = BN * 128;                // one SW128 K-major block (128 codes)
+  static constexpr int kWideB = 2 * kWideBlk;              // a stage: two K blocks
   static constexpr int kOutA = OUT ? 128 * kOutCols * 2 : 0;     // SW64 K-major
   static constexpr int kOutB = OUT ? BN * kOutCols * 2 : 0;
   // partials received from the other CTAs of the cluster: (KS-1) slots of
@@ -77,10 +78,10 @@ struct DecodeLayout {
   static constexpr int kFixed = kNP * (kPackA + kPackB) + kNO * (kOutA + kOutB) + kRed + 2048;
   // tensor memory: int32 accumulator, fp32 outlier accumulator, A stages
   static constexpr int kAcol = OUT ? 2 * BN : BN;
-  static constexpr int kNWtmem = (512 - kAcol) / 32;
+  static constexpr int kNWtmem = (512 - kAcol) / 64;        // 64-column stages (two K steps)
   static constexpr int kNWsmem = (kSmemBudget - kFixed) / kWideB;
-  static constexpr int kNW = kNWtmem < kNWsmem ? (kNWtmem < 12 ? kNWtmem : 12)
-                                               : (kNWsmem < 12 ? kNWsmem : 12);
+  static constexpr int kNW = kNWtmem < kNWsmem ? (kNWtmem < 6 ? kNWtmem : 6)
+                                               : (kNWsmem < 6 ? kNWsmem : 6);
   static constexpr int off_wide_b = 0;                     // 1024-aligned
   static constexpr int off_out_a = off_wide_b + kNW * kWideB;
   static constexpr int off_out_b = off_out_a + kNO * kOutA;
@@ -92,10 +93,11 @@ struct DecodeLayout {
   static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 * kNO + 3;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
   static constexpr int kBytes = off_misc + 16 + 1024;
-  static_assert(kNW >= 4, "stage ring");
+  static_assert(kNW >= 3, "stage ring");
   static_assert(kBytes <= kSmemBudget, "shared memory");
   static_assert(BN == 32 || BN == 64, "token tile");
-  static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0,
+  static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0 &&
+                    kPackB % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
 };
 
@@ -130,7 +132,7 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* full_p = bars;                   // TMA landed
-  uint64_t* empty_p = full_p + kNP;          // widen done reading (both groups: 8 warps)
+  uint64_t* empty_p = full_p + kNP;          // widen group done reading (4 warps)
   uint64_t* full_w = empty_p + kNP;          // stage widened (4 warps)
   uint64_t* empty_w = full_w + kNW;          // MMAs done with the stage
   uint64_t* full_o = empty_w + kNW;          // outlier TMA landed
@@ -152,7 +154,7 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   const int n_slots = (n_int + 1) >> 1;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 8); }
+    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 4); }
     for (int i = 0; i < kNW; ++i) { mbar_init(&full_w[i], 4); mbar_init(&empty_w[i], 1); }
     for (int i = 0; i < kNO; ++i) { mbar_init(&full_o[i], 1); mbar_init(&empty_o[i], 1); }
     mbar_init(tmem_full, 1);
@@ -211,14 +213,19 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
       constexpr uint32_t idesc = idesc_i8(BN);
       constexpr uint32_t idesc_o = idesc_f16(BN);
       bool ok = true;
-      for (int it = 0; it < n_int; ++it) {
+      for (int it = 0; it < n_slots; ++it) {
         const uint32_t s = it % kNW, ph = (it / kNW) & 1;
         if (!(ok = mbar_wait_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
         tc_fence_after();
-        const uint32_t a = tmem_base + kAcol + s * 32;
-        const uint64_t db = smem_desc_kmajor(smem_u32(smem + L::off_wide_b + s * L::kWideB), 128);
+        // two K steps; past this CTA's range (odd count) both operands are
+        // zero-filled or, inside K, a step another CTA also takes: skip it
+        const int nk = (2 * it + 1 < n_int) ? 8 : 4;
+        const uint32_t a = tmem_base + kAcol + s * 64;
+        const uint64_t db0 = smem_desc_kmajor(smem_u32(smem + L::off_wide_b + s * L::kWideB), 128);
+        const uint64_t db1 = smem_desc_kmajor(smem_u32(smem + L::off_wide_b + s * L::kWideB + L::kWideBlk), 128);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) mma_i8_ts(tmem_base, a + 8 * k, db + 2 * k, idesc, (it | k) != 0);
+        for (int k = 0; k < 8; ++k)
+          if (k < nk) mma_i8_ts(tmem_base, a + 8 * k, (k < 4 ? db0 : db1) + 2 * (k & 3), idesc, (it | k) != 0);
         mma_commit(&empty_w[s]);
       }
       if (OUT && ok)
@@ -239,54 +246,55 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   } else if (warp >= 4) {
     // ------------------------------------------------------------ widen
     const int wt = threadIdx.x - 128;
-    const int group = wt >> 7;                     // takes the steps with it % 2 == group,
-    const int row = wt & 127;                      // i.e. half `group` of every ring slot;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;   // row = TMEM lane
+    const int group = wt >> 7;                     // takes the ring slots it with it % 2 == group
+    const int row = wt & 127;                      // weight row of the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int it = group; it < 2 * n_slots && ok; it += 2) {
-      const uint32_t s = (it >> 1) % kNP, ph = ((it >> 1) / kNP) & 1;
+    for (int it = group; it < n_slots && ok; it += 2) {
+      const uint32_t s = it % kNP, ph = (it / kNP) & 1;
       const uint32_t sw = it % kNW, phw = (it / kNW) & 1;
       if (!(ok = mbar_wait_bounded(&full_p[s], ph, abort_flag, p.status, kDevTimeoutWiden))) break;
-      if (it >= n_int) {                           // the unused half of the last slot
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_p[s]);
-        break;
-      }
       if (!(ok = mbar_wait_bounded(&empty_w[sw], phw ^ 1, abort_flag, p.status, kDevTimeoutWiden))) break;
       {
-        // weight row: 64 packed bytes of this half (128-byte swizzled rows)
-        // -> 128 s8 in TMEM
+        // weight row: 128 packed bytes (128-byte swizzled rows) -> 256 s8 in TMEM
         const uint8_t* pa = smem + L::off_pack_a + s * L::kPackA + row * kSlot;
-        uint32_t r[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 u = *reinterpret_cast<const uint4*>(pa + (((4 * group + c) ^ (row & 7)) << 4));
-          r[8 * c + 0] = (u.x << 4) & 0xF0F0F0F0u;
-          r[8 * c + 1] = (u.y << 4) & 0xF0F0F0F0u;
-          r[8 * c + 2] = (u.z << 4) & 0xF0F0F0F0u;
-          r[8 * c + 3] = (u.w << 4) & 0xF0F0F0F0u;
-          r[8 * c + 4] = u.x & 0xF0F0F0F0u;
-          r[8 * c + 5] = u.y & 0xF0F0F0F0u;
-          r[8 * c + 6] = u.z & 0xF0F0F0F0u;
-          r[8 * c + 7] = u.w & 0xF0F0F0F0u;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 u = *reinterpret_cast<const uint4*>(pa + (((4 * h + c) ^ (row & 7)) << 4));
+            r[8 * c + 0] = (u.x << 4) & 0xF0F0F0F0u;
+            r[8 * c + 1] = (u.y << 4) & 0xF0F0F0F0u;
+            r[8 * c + 2] = (u.z << 4) & 0xF0F0F0F0u;
+            r[8 * c + 3] = (u.w << 4) & 0xF0F0F0F0u;
+            r[8 * c + 4] = u.x & 0xF0F0F0F0u;
+            r[8 * c + 5] = u.y & 0xF0F0F0F0u;
+            r[8 * c + 6] = u.z & 0xF0F0F0F0u;
+            r[8 * c + 7] = u.w & 0xF0F0F0F0u;
+          }
+          tmem_st_32x32b_x32(tmem_base + lane_off + kAcol + sw * 64 + 32 * h, r);
         }
-        tmem_st_32x32b_x32(tmem_base + lane_off + kAcol + sw * 32, r);
       }
       {
-        // token rows: 16-byte packed chunks -> two 16-byte s8 chunks, SW128
+        // token rows (128-byte swizzled): each 16-byte packed chunk -> two
+        // 16-byte s8 chunks of the K block it belongs to, SW128
         const uint8_t* pb = smem + L::off_pack_b + s * L::kPackB;
         uint8_t* wb = smem + L::off_wide_b + sw * L::kWideB;
         for (int task = row; task < BN * 4; task += 128) {
           const int br = task >> 2, c = task & 3;
-          const uint4 u = *reinterpret_cast<const uint4*>(pb + br * kSlot + (4 * group + c) * 16);
-          uint4 ev, od;
-          ev.x = (u.x << 4) & 0xF0F0F0F0u; od.x = u.x & 0xF0F0F0F0u;
-          ev.y = (u.y << 4) & 0xF0F0F0F0u; od.y = u.y & 0xF0F0F0F0u;
-          ev.z = (u.z << 4) & 0xF0F0F0F0u; od.z = u.z & 0xF0F0F0F0u;
-          ev.w = (u.w << 4) & 0xF0F0F0F0u; od.w = u.w & 0xF0F0F0F0u;
-          uint8_t* base = wb + (br >> 3) * 1024 + (br & 7) * 128;
-          *reinterpret_cast<uint4*>(base + (((2 * c) ^ (br & 7)) << 4)) = ev;
-          *reinterpret_cast<uint4*>(base + (((2 * c + 1) ^ (br & 7)) << 4)) = od;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint4 u = *reinterpret_cast<const uint4*>(pb + br * kSlot + (((4 * h + c) ^ (br & 7)) << 4));
+            uint4 ev, od;
+            ev.x = (u.x << 4) & 0xF0F0F0F0u; od.x = u.x & 0xF0F0F0F0u;
+            ev.y = (u.y << 4) & 0xF0F0F0F0u; od.y = u.y & 0xF0F0F0F0u;
+            ev.z = (u.z << 4) & 0xF0F0F0F0u; od.z = u.z & 0xF0F0F0F0u;
+            ev.w = (u.w << 4) & 0xF0F0F0F0u; od.w = u.w & 0xF0F0F0F0u;
+            uint8_t* base = wb + h * L::kWideBlk + (br >> 3) * 1024 + (br & 7) * 128;
+            *reinterpret_cast<uint4*>(base + (((2 * c) ^ (br & 7)) << 4)) = ev;
+            *reinterpret_cast<uint4*>(base + (((2 * c + 1) ^ (br & 7)) << 4)) = od;
+          }
         }
       }
       tmem_st_wait();
@@ -463,7 +471,7 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
       (!make_tensor_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.w_codes, kb, j.N, kb, kSlot, 128,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
        !make_tensor_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.a_codes, kb, j.M, kb, kSlot, bn,
-                           CU_TENSOR_MAP_SWIZZLE_NONE)))
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
     return QR_ERR_CUDA;
   if (out) {
     const uint64_t no = static_cast<uint64_t>(j.n_out);

@@ -14,9 +14,9 @@
 //  * The B operand is widened in shared memory into the canonical
 //    128-byte-swizzled K-major layout.
 //  * A = activations (M > 64), B = weights.
-//  * The packed tiles arrive by TMA in 128-byte rows, two K steps per ring
-//    slot: the TMA unit moves a tile row by row, and at 64-byte rows its row
-//    rate, not HBM, limited the feed.
+//  * The packed tiles arrive by TMA in 128-byte rows: a ring slot, and a
+//    widened stage, holds two K steps (256 codes), so the MMA thread waits,
+//    fences and commits once per eight MMAs.
 //  * OUT: the fp16 outlier columns run as a second cta_group::2 MMA of
 //    kind::f16 into an fp32 accumulator in TMEM, added in the epilogue.
 //
@@ -26,12 +26,12 @@
 //
 // Tensor memory per CTA: two accumulator buffers (the epilogue of one tile
 // overlaps the MMAs of the next) of BN int32 columns, plus BN fp32 outlier
-// columns when OUT, and up to four 32-column A stages.
+// columns when OUT, and up to four 64-column A stages.
 //
 // Warp roles, per CTA (448 threads):
 //   warps 0-3   epilogue  (TMEM lanes = the CTA's 128 A rows of the tile)
-//   warps 4-11  widen     (two groups of four warps taking alternate K
-//                          steps: one A row per thread -> TMEM, B chunks ->
+//   warps 4-11  widen     (two groups of four warps taking alternate ring
+//                          slots: one A row per thread -> TMEM, B chunks ->
 //                          smem)
 //   warp  12    producer  (TMA of the packed and outlier tiles; no multicast)
 //   warp  13    TMEM allocation; in the even CTA one thread issues the MMAs,
@@ -61,11 +61,11 @@ constexpr int kProducerWarp = 4 + kWidenWarps;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 
-// A stages: as many 32-column stages as tensor memory holds next to the two
-// accumulator buffers, at most 4.
+// A stages: as many 64-column stages (two K steps) as tensor memory holds
+// next to the two accumulator buffers, at most 4.
 template <int BN, bool OUT>
 constexpr int widened_stages() {
-  return (512 - (OUT ? 4 : 2) * BN) / 32 < 4 ? (512 - (OUT ? 4 : 2) * BN) / 32 : 4;
+  return (512 - (OUT ? 4 : 2) * BN) / 64 < 4 ? (512 - (OUT ? 4 : 2) * BN) / 64 : 4;
 }
 
 struct PairParams {
@@ -87,8 +87,9 @@ struct PairSmem {
   static constexpr int kNW = widened_stages<BN, OUT>();
   static constexpr int kHalf = BN / 2;                     // B rows per CTA
   static constexpr int kPackA = 128 * kSlot;               // 16 KB, 128-byte swizzle
-  static constexpr int kPackB = kHalf * kSlot;
-  static constexpr int kWideB = kHalf * 2 * kStep;         // SW128 K-major
+  static constexpr int kPackB = kHalf * kSlot;             // 128-byte swizzle
+  static constexpr int kWideBlk = kHalf * 128;             // one SW128 K-major block (128 codes)
+  static constexpr int kWideB = 2 * kWideBlk;              // a stage: two K blocks
   static constexpr int kOutA = OUT ? 128 * kOutCols * 2 : 0;     // SW64 K-major
   static constexpr int kOutB = OUT ? kHalf * kOutCols * 2 : 0;
   static constexpr int off_wide_b = 0;                     // 1024-aligned
@@ -102,7 +103,8 @@ struct PairSmem {
   static constexpr int kNumBars = 2 * kNP + 2 * kNW + 3 * kNO + 5;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
   static constexpr int kBytes = off_misc + 16 + 1024;
-  static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0,
+  static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0 &&
+                    kPackB % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
 };
 
@@ -114,16 +116,16 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                       const __grid_constant__ CUtensorMap map_ob, const PairParams p) {
   using S = PairSmem<BN, OUT>;
   constexpr int kNW = S::kNW;
-  static_assert(BN % 32 == 0 && BN >= 32 && kNW >= 2, "tile width");
+  static_assert(BN % 32 == 0 && BN >= 32 && kNW >= 2 && S::kWideBlk % 1024 == 0, "tile width");
   constexpr uint32_t kColsAcc = OUT ? 2 * BN : BN;         // per accumulator buffer
   constexpr uint32_t kAcol = 2 * kColsAcc;                 // A stages in TMEM
-  static_assert(kAcol + 32 * kNW <= 512, "tensor memory");
+  static_assert(kAcol + 64 * kNW <= 512, "tensor memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::off_bar);
   uint64_t* full_p = bars;                   // local: TMA landed
-  uint64_t* empty_p = full_p + kNP;          // local: both widen groups done reading
+  uint64_t* empty_p = full_p + kNP;          // local: the widen group done reading
   uint64_t* full_w = empty_p + kNP;          // widened: 4 local warps (+ the odd CTA's relay)
   uint64_t* empty_w = full_w + kNW;          // each CTA: the pair's MMAs done with the stage
   uint64_t* full_o = empty_w + kNW;          // local: outlier TMA landed
@@ -141,7 +143,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 8); }
+    for (int i = 0; i < kNP; ++i) { mbar_init(&full_p[i], 1); mbar_init(&empty_p[i], 4); }
     for (int i = 0; i < kNW; ++i) {
       mbar_init(&full_w[i], leader ? 5 : 4);
       mbar_init(&empty_w[i], 1);
@@ -218,7 +220,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
       uint32_t wi = 0, oi = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
-        for (int ks = 0; ks < p.kt; ++ks, ++wi) {
+        for (int ps = 0; ps < slots; ++ps, ++wi) {
           const uint32_t s = wi % kNW, ph = (wi / kNW) & 1;
           if (!(ok = mbar_wait_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
           mbar_arrive_cluster_relaxed(full_w0 + s * 8);
@@ -242,14 +244,17 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
         if (!(ok = mbar_wait_cluster_bounded(&tmem_empty[buf], tph ^ 1, abort_flag, p.status, kDevTimeoutMma))) break;
         tc_fence_after();
         const uint32_t d = tmem_base + buf * kColsAcc;
-        for (int ks = 0; ks < p.kt; ++ks, ++wi) {
+        for (int ps = 0; ps < slots; ++ps, ++wi) {
           const uint32_t s = wi % kNW, ph = (wi / kNW) & 1;
           if (!(ok = mbar_wait_cluster_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
           tc_fence_after();
-          const uint32_t a = tmem_base + kAcol + s * 32;
-          const uint64_t db = smem_desc_kmajor(smem_u32(smem + S::off_wide_b + s * S::kWideB), 128);
+          // two K steps; past K (odd step count) both operands are zero-filled
+          const uint32_t a = tmem_base + kAcol + s * 64;
+          const uint64_t db0 = smem_desc_kmajor(smem_u32(smem + S::off_wide_b + s * S::kWideB), 128);
+          const uint64_t db1 = smem_desc_kmajor(smem_u32(smem + S::off_wide_b + s * S::kWideB + S::kWideBlk), 128);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mma_i8_pair_ts(d, a + 8 * k, db + 2 * k, idesc, (ks | k) != 0);
+          for (int k = 0; k < 8; ++k)
+            mma_i8_pair_ts(d, a + 8 * k, (k < 4 ? db0 : db1) + 2 * (k & 3), idesc, (ps | k) != 0);
           mma_commit_pair(&empty_w[s], 0x3);
         }
         if (OUT && ok)
@@ -272,58 +277,64 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   } else if (warp >= 4) {
     // ------------------------------------------------------------ widen
     const int wt = threadIdx.x - 128;
-    const int group = wt >> 7;                     // takes the K steps ks with ks % 2 == group,
-    const int arow = wt & 127;                     // i.e. half `group` of every ring slot
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;   // arow = TMEM lane
-    uint32_t it = 0, pi = 0;                       // steps and slots of the earlier tiles
+    const int group = wt >> 7;                     // takes the ring slots wi with wi % 2 == group
+    const int arow = wt & 127;                     // = TMEM lane (warp % 4 quadrant)
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t pi = 0;                               // slots (= stages) of the earlier tiles
     bool ok = true;
-    for (int tile = cid; tile < num_tiles && ok; tile += ncl, it += p.kt, pi += slots) {
-      for (int ks = group; ks < 2 * slots; ks += 2) {
-        const uint32_t s = (pi + (ks >> 1)) % kNP, ph = ((pi + (ks >> 1)) / kNP) & 1;
-        if (!(ok = mbar_wait_bounded(&full_p[s], ph, abort_flag, p.status, kDevTimeoutWiden))) break;
-        if (ks >= p.kt) {                          // the unused half of the last slot
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty_p[s]);
-          break;
-        }
-        const uint32_t wi = it + ks;
+    for (int tile = cid; tile < num_tiles && ok; tile += ncl, pi += slots) {
+      // Parity of the global slot index, not of the slot within the tile:
+      // a group must never run two uses of a stage ahead of the MMAs, or
+      // the parity wait on empty_w would pass a phase early (with two
+      // stages and an odd slot count, per-tile parity lets it).
+      for (int ps = (group + static_cast<int>(pi)) & 1; ps < slots; ps += 2) {
+        const uint32_t wi = pi + ps;
+        const uint32_t s = wi % kNP, ph = (wi / kNP) & 1;
         const uint32_t sw = wi % kNW, phw = (wi / kNW) & 1;
+        if (!(ok = mbar_wait_bounded(&full_p[s], ph, abort_flag, p.status, kDevTimeoutWiden))) break;
         if (!(ok = mbar_wait_cluster_bounded(&empty_w[sw], phw ^ 1, abort_flag, p.status, kDevTimeoutWiden))) break;
-        // A row: the 64 packed bytes of this half (128-byte swizzled rows) -> 128 s8 in TMEM
+        // A row: 128 packed bytes (128-byte swizzled rows) -> 256 s8 in TMEM
         {
           const uint8_t* pa = smem + S::off_pack_a + s * S::kPackA + arow * kSlot;
-          uint32_t r[32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 u = *reinterpret_cast<const uint4*>(pa + (((4 * group + c) ^ (arow & 7)) << 4));
-            r[8 * c + 0] = (u.x << 4) & 0xF0F0F0F0u;
-            r[8 * c + 1] = (u.y << 4) & 0xF0F0F0F0u;
-            r[8 * c + 2] = (u.z << 4) & 0xF0F0F0F0u;
-            r[8 * c + 3] = (u.w << 4) & 0xF0F0F0F0u;
-            r[8 * c + 4] = u.x & 0xF0F0F0F0u;
-            r[8 * c + 5] = u.y & 0xF0F0F0F0u;
-            r[8 * c + 6] = u.z & 0xF0F0F0F0u;
-            r[8 * c + 7] = u.w & 0xF0F0F0F0u;
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 u = *reinterpret_cast<const uint4*>(pa + (((4 * h + c) ^ (arow & 7)) << 4));
+              r[8 * c + 0] = (u.x << 4) & 0xF0F0F0F0u;
+              r[8 * c + 1] = (u.y << 4) & 0xF0F0F0F0u;
+              r[8 * c + 2] = (u.z << 4) & 0xF0F0F0F0u;
+              r[8 * c + 3] = (u.w << 4) & 0xF0F0F0F0u;
+              r[8 * c + 4] = u.x & 0xF0F0F0F0u;
+              r[8 * c + 5] = u.y & 0xF0F0F0F0u;
+              r[8 * c + 6] = u.z & 0xF0F0F0F0u;
+              r[8 * c + 7] = u.w & 0xF0F0F0F0u;
+            }
+            tmem_st_32x32b_x32(tmem_base + lane_off + kAcol + sw * 64 + 32 * h, r);
           }
-          tmem_st_32x32b_x32(tmem_base + lane_off + kAcol + sw * 32, r);
         }
-        // B rows: 16-byte packed chunks -> two 16-byte s8 chunks, SW128
+        // B rows (128-byte swizzled): each 16-byte packed chunk -> two 16-byte
+        // s8 chunks of the K block it belongs to, SW128
         {
           const uint8_t* pb = smem + S::off_pack_b + s * S::kPackB;
           uint8_t* wb = smem + S::off_wide_b + sw * S::kWideB;
           constexpr int kTasks = S::kHalf * 4;
-#pragma unroll 2
+#pragma unroll 1
           for (int task = arow; task < kTasks; task += kGroupThreads) {
             const int row = task >> 2, c = task & 3;
-            const uint4 u = *reinterpret_cast<const uint4*>(pb + row * kSlot + (4 * group + c) * 16);
-            uint4 ev, od;
-            ev.x = (u.x << 4) & 0xF0F0F0F0u; od.x = u.x & 0xF0F0F0F0u;
-            ev.y = (u.y << 4) & 0xF0F0F0F0u; od.y = u.y & 0xF0F0F0F0u;
-            ev.z = (u.z << 4) & 0xF0F0F0F0u; od.z = u.z & 0xF0F0F0F0u;
-            ev.w = (u.w << 4) & 0xF0F0F0F0u; od.w = u.w & 0xF0F0F0F0u;
-            uint8_t* base = wb + (row >> 3) * 1024 + (row & 7) * 128;
-            *reinterpret_cast<uint4*>(base + (((2 * c) ^ (row & 7)) << 4)) = ev;
-            *reinterpret_cast<uint4*>(base + (((2 * c + 1) ^ (row & 7)) << 4)) = od;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 u = *reinterpret_cast<const uint4*>(pb + row * kSlot + (((4 * h + c) ^ (row & 7)) << 4));
+              uint4 ev, od;
+              ev.x = (u.x << 4) & 0xF0F0F0F0u; od.x = u.x & 0xF0F0F0F0u;
+              ev.y = (u.y << 4) & 0xF0F0F0F0u; od.y = u.y & 0xF0F0F0F0u;
+              ev.z = (u.z << 4) & 0xF0F0F0F0u; od.z = u.z & 0xF0F0F0F0u;
+              ev.w = (u.w << 4) & 0xF0F0F0F0u; od.w = u.w & 0xF0F0F0F0u;
+              uint8_t* base = wb + h * S::kWideBlk + (row >> 3) * 1024 + (row & 7) * 128;
+              *reinterpret_cast<uint4*>(base + (((2 * c) ^ (row & 7)) << 4)) = ev;
+              *reinterpret_cast<uint4*>(base + (((2 * c + 1) ^ (row & 7)) << 4)) = od;
+            }
           }
         }
         tmem_st_wait();
@@ -433,25 +444,21 @@ cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtenso
 
 }  // namespace
 
-// Tile width without outlier columns: the fewest tile rounds over
-// the SM pairs, weighted by the width (one round of a BN-wide tile costs
-// about BN).
+// Tile width without outlier columns: 160 or 128 (both leave tensor memory
+// for at least three A stages next to the double-buffered accumulator; 192
+// would leave two, too shallow to hide the widen).  Cost = tile rounds over
+// the SM pairs x (width + a per-step overhead worth ~64 columns); the wider
+// tile wins within 2%.
 int pair_tile_width(int64_t M, int64_t N, int sms) {
   const int64_t ta = (M + 255) / 256;
-  const int cands[] = {192, 160, 128};
-  int64_t cost[3];
-  int64_t best_cost = -1;
-  for (int i = 0; i < 3; ++i) {
-    const int bn = cands[i];
-    const int64_t tiles = ta * ((N + bn - 1) / bn);
+  const int cands[] = {160, 128};
+  int64_t cost[2];
+  for (int i = 0; i < 2; ++i) {
+    const int64_t tiles = ta * ((N + cands[i] - 1) / cands[i]);
     const int64_t rounds = (tiles + sms / 2 - 1) / (sms / 2);
-    cost[i] = rounds * bn;
-    if (best_cost < 0 || cost[i] < best_cost) best_cost = cost[i];
+    cost[i] = rounds * (cands[i] + 64);
   }
-  // the widest tile within 2% of the cheapest (wider tiles reuse operands more)
-  for (int i = 0; i < 3; ++i)
-    if (cost[i] * 100 <= best_cost * 102) return cands[i];
-  return 128;
+  return cost[0] * 100 <= cost[1] * 102 ? 160 : 128;
 }
 
 qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
@@ -480,7 +487,7 @@ qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
       (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.a_codes, kb, j.M, kb, kSlot, 128,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
        !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.w_codes, kb, j.N, kb, kSlot,
-                           bn / 2, CU_TENSOR_MAP_SWIZZLE_NONE)))
+                           bn / 2, CU_TENSOR_MAP_SWIZZLE_128B)))
     return QR_ERR_CUDA;
   if (out) {
     const uint64_t no = static_cast<uint64_t>(j.n_out);
@@ -494,11 +501,8 @@ qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
   if (out) {
     e = run_pair<96, true>(ma, mb, moa, mob, p, stream);
   } else {
-    switch (bn) {
-      case 192: e = run_pair<192, false>(ma, mb, moa, mob, p, stream); break;
-      case 160: e = run_pair<160, false>(ma, mb, moa, mob, p, stream); break;
-      default: e = run_pair<128, false>(ma, mb, moa, mob, p, stream); break;
-    }
+    e = bn == 160 ? run_pair<160, false>(ma, mb, moa, mob, p, stream)
+                  : run_pair<128, false>(ma, mb, moa, mob, p, stream);
   }
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
