@@ -83,8 +83,8 @@ def gemm_kernel_name(M: int) -> str:
     return "w4a4_gemm_decode_kernel" if M <= DECODE_MAX_TOKENS else "w4a4_gemm_pair_kernel"
 
 
-def rotate_kernel_name(rotation: str, M: int, sms: int) -> str:
-    if rotation == "kron":
+def rotate_kernel_name(spec, M: int, sms: int) -> str:
+    if spec.rotation == "kron":
         return "kron_tc_kernel"
     return "wht_few_rows_kernel" if M <= sms else "wht_ab_kernel"
 
@@ -398,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
         "roofline": roofline,
-        "rotate_quant": {"bound": "hbm", "kernel": rotate_kernel_name(s.rotation, M, sms),
+        "rotate_quant": {"bound": "hbm", "kernel": rotate_kernel_name(s, M, sms),
                          "achieved": round(rq_gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(rq_gbs / hbm, 4), "bytes_per_launch": rq_bytes,
                          "ms_per_launch": round(rq_avg, 5)},

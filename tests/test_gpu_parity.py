@@ -71,6 +71,7 @@ ROW_CASES = [
     ("none_ragged", 200, 11, O.Rotation(O.NONE)),
     ("none_long", 8192, 3, O.Rotation(O.NONE)),
     ("had_clip", 1024, 9, O.Rotation(O.HADAMARD, block=1024, clip_ratio=0.5)),
+    ("had4096_clip", 4096, 5, O.Rotation(O.HADAMARD, block=4096, clip_ratio=0.8)),
     ("gsr_clip", 1024, 9, O.Rotation(O.GSR, block=128, clip_ratio=0.9)),
 ]
 
