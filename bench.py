@@ -171,7 +171,18 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- workload
 
-def rotation_for(wl, Q):
+def workload_signs(wl, random_signs: bool):
+    """The seeded random-sign diagonal of a randomized Hadamard (or None)."""
+    import oracle as O
+    import workloads
+    s = wl.spec
+    if not random_signs or s.rotation not in ("hadamard", "gsr"):
+        return None
+    probe = O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR}[s.rotation], block=s.block)
+    return workloads.random_signs(s.seed, O.packed_width(probe, s.K, s.n_keep_fp16))
+
+
+def rotation_for(wl, Q, signs=None):
     s = wl.spec
     import torch
     if s.rotation == "kron":
@@ -180,7 +191,18 @@ def rotation_for(wl, Q):
                           chan_scale=torch.from_numpy(wl.chan_scale).cuda(),
                           clip_ratio=s.clip_ratio)
     kind = {"hadamard": Q.HADAMARD, "gsr": Q.GSR, "none": Q.NONE}[s.rotation]
-    return Q.Rotation(kind, block=s.block, clip_ratio=s.clip_ratio)
+    return Q.Rotation(kind, block=s.block, clip_ratio=s.clip_ratio,
+                      signs=None if signs is None else torch.from_numpy(signs).cuda())
+
+
+def oracle_rotation(wl, signs=None):
+    import oracle as O
+    s = wl.spec
+    if s.rotation == "kron":
+        return O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale,
+                          clip_ratio=s.clip_ratio)
+    return O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR, "none": O.NONE}[s.rotation],
+                      block=s.block, clip_ratio=s.clip_ratio, signs=signs)
 
 
 def algorithmic_counts(wl, M, kp):
@@ -214,7 +236,8 @@ def run_ours(args, rank, world, local_rank):
     wl = workloads.make_workload(args.workload, M=args.tokens)
     s = wl.spec
     M = wl.X.shape[0]
-    rot = rotation_for(wl, Q)
+    signs = workload_signs(wl, args.random_signs)
+    rot = rotation_for(wl, Q, signs)
     idx = None
     if s.n_keep_fp16:
         idx = Q.select_outliers(torch.from_numpy(wl.X_calib).cuda(), s.n_keep_fp16)
@@ -392,7 +415,8 @@ def run_ours(args, rank, world, local_rank):
                      "fp16 in/out",
         "data": "synthetic",
         "config": {"workload": s.name, "M": M, "K": s.K, "N": s.N, "K_p": kp,
-                   "rotation": f"{s.rotation}-{s.block}" if s.rotation != "kron"
+                   "rotation": (("random-sign " if signs is not None else "") +
+                                f"{s.rotation}-{s.block}") if s.rotation != "kron"
                    else f"kron-{s.n1}x{s.n2}", "n_out": s.n_keep_fp16,
                    "clip_ratio": s.clip_ratio, "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
@@ -428,7 +452,8 @@ def aggregate_max(value_ms: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- oracle
 
-def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None):
+def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None,
+                    random_signs: bool = False):
     """Times the CPU oracle's online path on `tokens` tokens of the workload."""
     import oracle as O
     import workloads
@@ -436,12 +461,7 @@ def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None):
 
     wl = workloads.make_workload(workload, M=M_total)
     s = wl.spec
-    if s.rotation == "kron":
-        rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale,
-                         clip_ratio=s.clip_ratio)
-    else:
-        rot = O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR, "none": O.NONE}[s.rotation],
-                         block=s.block, clip_ratio=s.clip_ratio)
+    rot = oracle_rotation(wl, workload_signs(wl, random_signs))
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
     wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)     # offline, untimed
     x = wl.X[:tokens].astype(np.float64)
@@ -471,12 +491,7 @@ def run_reference(args, rank, world):
     wl = workloads.make_workload(args.workload, M=args.tokens)
     s = wl.spec
     tokens = min(wl.X.shape[0], args.reference_tokens)
-    if s.rotation == "kron":
-        rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale,
-                         clip_ratio=s.clip_ratio)
-    else:
-        rot = O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR, "none": O.NONE}[s.rotation],
-                         block=s.block, clip_ratio=s.clip_ratio)
+    rot = oracle_rotation(wl, workload_signs(wl, args.random_signs))
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
     wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)
     x = wl.X[:tokens].astype(np.float64)
@@ -525,6 +540,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-baseline-tokens", type=int, default=256)
     ap.add_argument("--reference-tokens", type=int, default=64)
+    ap.add_argument("--random-signs", action="store_true",
+                    help="randomized Hadamard: a seeded random-sign diagonal before the blocks")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -555,7 +572,8 @@ def main(argv=None):
             if world == 1 and not args.no_cpu_baseline:
                 tokens = min(args.cpu_baseline_tokens, res["config"]["M"])
                 res["cpu_baseline"] = oracle_baseline(args.workload, tokens, repeats=3,
-                                                      M_total=args.tokens)
+                                                      M_total=args.tokens,
+                                                      random_signs=args.random_signs)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

@@ -101,10 +101,18 @@ typedef struct {
   int32_t chan_mode;         /* qr_chan_mode: how chan_scale is applied */
   float clip_ratio;          /* alpha in (0, 1]: s = alpha*absmax/7, codes
                                 clamped to +-7 (1.0 = plain min-max) */
+  const int8_t* signs;       /* HADAMARD, GSR: the random-sign diagonal D of a
+                                randomized Hadamard, R = D B (rows become
+                                (x .* d) B; "random Hadamard rotations", SpinQuant
+                                review, reviewer brBn W2/A2): int8 [K_p] of +-1,
+                                8-byte aligned, applied after the outlier split
+                                and padding; NULL = no signs.  Must be NULL for
+                                the other kinds.  The weight side takes the same
+                                descriptor (D B is orthogonal). */
 } qr_rotation;
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define QR_ABI_VERSION 1
+#define QR_ABI_VERSION 2
 QR_API int32_t qr_abi_version(void);
 
 /* Human-readable name of a status code (static string). */

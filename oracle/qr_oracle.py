@@ -48,6 +48,11 @@ R9  QUIK: the outlier columns stay fp16 and unrotated; the remaining columns,
     [QK] §1 says of the original), weights by RTN instead of GPTQ.
 R10 Outlier columns are the top-k columns by infinity-norm over a calibration
     batch, ties to the lower index, returned in ascending order ([QK] §3).
+R11 A "random Hadamard rotation" ([SR] reviewer brBn W2/A2) is R = D B with
+    D a diagonal of random signs +-1 and B the block-diagonal Hadamard: a
+    row becomes (x .* d) B.  The signs act on the rotated-domain columns
+    (after the outlier split and zero padding).  D B is orthogonal, so the
+    weight side uses the same R.
 """
 from __future__ import annotations
 
@@ -103,6 +108,7 @@ class Rotation:
     P2: Optional[np.ndarray] = None
     chan_scale: Optional[np.ndarray] = None   # KRON per-channel scale c [K]
     clip_ratio: float = 1.0
+    signs: Optional[np.ndarray] = None   # HADAMARD / GSR: random +-1 diagonal d [K_p] (R11)
 
 
 def packed_width(rot: Rotation, K: int, n_out: int = 0) -> int:
@@ -137,7 +143,10 @@ def dense_rotation(rot: Rotation, k_p: int) -> np.ndarray:
     if rot.kind == KRON:
         return np.kron(rot.P1.astype(np.float64), rot.P2.astype(np.float64))
     blk = block_rotation(rot.kind, rot.block)
-    return np.kron(np.eye(k_p // rot.block), blk)
+    r = np.kron(np.eye(k_p // rot.block), blk)
+    if rot.signs is not None:
+        r = np.diag(np.asarray(rot.signs, np.float64)) @ r
+    return r
 
 
 def _apply_blocks(x: np.ndarray, blk: np.ndarray) -> np.ndarray:
@@ -164,6 +173,8 @@ def rotate_activations(x: np.ndarray, rot: Rotation) -> np.ndarray:
     if rot.kind == NONE:
         return x.copy()
     if rot.kind in (HADAMARD, GSR):
+        if rot.signs is not None:                    # R11: (x .* d) B
+            x = x * np.asarray(rot.signs, np.float64)[None, :]
         return _apply_blocks(x, block_rotation(rot.kind, rot.block))
     if rot.chan_scale is not None:
         x = x / rot.chan_scale.astype(np.float64)[None, :]
@@ -182,6 +193,8 @@ def rotate_weights(w: np.ndarray, rot: Rotation) -> np.ndarray:
     if rot.kind == NONE:
         return w.copy()
     if rot.kind in (HADAMARD, GSR):
+        if rot.signs is not None:                    # R11: D B is orthogonal
+            w = w * np.asarray(rot.signs, np.float64)[None, :]
         return _apply_blocks(w, block_rotation(rot.kind, rot.block))
     if rot.chan_scale is not None:
         w = w * rot.chan_scale.astype(np.float64)[None, :]

@@ -44,7 +44,8 @@ def gpu_rotation(r: O.Rotation) -> Q.Rotation:
                       p2=None if r.P2 is None else dev(np.asarray(r.P2, np.float32)),
                       chan_scale=None if r.chan_scale is None else dev(np.asarray(r.chan_scale,
                                                                                  np.float32)),
-                      clip_ratio=r.clip_ratio)
+                      clip_ratio=r.clip_ratio,
+                      signs=None if r.signs is None else dev(np.asarray(r.signs, np.int8)))
 
 
 def unpack(codes: torch.Tensor) -> np.ndarray:

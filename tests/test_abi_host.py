@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.qr_abi_version() == 1
+    assert L.qr_abi_version() == 2
     for s in range(6):
         assert L.status_string(s) and L.status_string(s) != "unknown status"
     assert L.status_string(99) == "unknown status"
@@ -110,6 +110,13 @@ def test_rotate_quant_argument_errors(lib):
     assert _rq(_rot(L.QR_ROT_HADAMARD, 64, clip=2.0)) == L.QR_ERR_INVALID_ARG
     assert _rq(_rot(L.QR_ROT_NONE), K=40000, ldx=40000) == L.QR_ERR_UNSUPPORTED
     assert _rq(h, M=0) == L.QR_OK                                 # empty: nothing to do
+    # random signs: HADAMARD / GSR only, 8-byte aligned
+    signed = _rot(L.QR_ROT_HADAMARD, 256)
+    signed.signs = FAKE + 4
+    assert _rq(signed) == L.QR_ERR_ALIGNMENT
+    kron = _rot(L.QR_ROT_KRON, n1=16, n2=16)
+    kron.signs = FAKE
+    assert _rq(kron) == L.QR_ERR_INVALID_ARG
 
 
 def _lin(M=16, N=16, Kp=256, a=FAKE, sa=FAKE, w=FAKE, sw=FAKE, xo=None, wo=None, n_out=0,

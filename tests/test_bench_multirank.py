@@ -1,5 +1,6 @@
 """The N>1 host logic of bench.py on CPU: two gloo ranks, max-over-ranks
 timing, and the launcher checks.  No GPU is touched."""
+import json
 import os
 import socket
 
@@ -65,3 +66,15 @@ def test_algorithmic_counts_of_the_qkv_workload():
     ops, rq, gm = bench.algorithmic_counts(wl, 2048, 4096)
     assert ops == 2.0 * 2048 * 12288 * 4096
     assert rq == 2048 * 4096 * 2 + 2048 * 4096 / 2 + 2048 * 4
+
+
+def test_reference_arm_with_random_signs(capsys):
+    # the oracle arm takes the same randomized rotation as the GPU arm
+    assert bench.main(["--impl", "reference", "--workload", "tiny_256", "--random-signs",
+                       "--steps", "2", "--warmup", "3", "--reference-tokens", "8"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["workload"] == "tiny_256"
+    import workloads
+    wl = workloads.make_workload("tiny_256")
+    d = bench.workload_signs(wl, True)
+    assert d is not None and d.shape == (256,) and bench.oracle_rotation(wl, d).signs is d

@@ -299,3 +299,42 @@ def test_graphed_layer_matches_eager(M):
         assert np.array_equal(y_graph.view(np.uint16), y_eager.view(np.uint16))
     with pytest.raises(ValueError):
         glin(dev(np.zeros((M + 1, wl.spec.K), np.float16)))
+
+
+# ---------------------------------------------------------------- randomized Hadamard
+
+SIGN_CASES = [
+    # (name, K, rows, kind, block, n_out, clip)
+    ("had4096", 4096, 9, O.HADAMARD, 4096, 0, 1.0),
+    ("had64_clip", 640, 7, O.HADAMARD, 64, 0, 0.7),
+    ("gsr128", 11008, 5, O.GSR, 128, 0, 1.0),
+    ("had4096_outliers", 8192, 6, O.HADAMARD, 4096, 256, 1.0),
+    ("had8", 256, 5, O.HADAMARD, 8, 0, 1.0),
+]
+
+
+@pytest.mark.parametrize("name,K,rows,kind,block,n_out,clip", SIGN_CASES,
+                         ids=[c[0] for c in SIGN_CASES])
+@pytest.mark.parametrize("many", [False, True], ids=["few", "many"])
+def test_rotate_quant_random_signs(name, K, rows, kind, block, n_out, clip, many):
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    idx = np.sort(rng.choice(K, size=n_out, replace=False)).astype(np.int32) if n_out else None
+    x = _rows(rng, rows, K, outl=(1,) if not n_out else idx[:2])
+    probe = O.Rotation(kind, block=block, clip_ratio=clip)
+    kp = O.packed_width(probe, K, n_out)
+    rot = O.Rotation(kind, block=block, clip_ratio=clip, signs=workloads.random_signs(7, kp))
+    for weights in (False, True):
+        gpu, ref = _run_rows(x, rot, idx, weights=weights, many=many)
+        check_side(gpu, ref, f"{name} signs", clip=clip)
+
+
+def test_layer_random_signs_end_to_end():
+    wl = workloads.make_workload("qkv_prefill_4096", M=96, N=512)
+    kp = O.packed_width(O.Rotation(O.HADAMARD, block=4096), wl.spec.K)
+    rot = O.Rotation(O.HADAMARD, block=4096, signs=workloads.random_signs(1, kp))
+    layer = Q.QuantizedLinear(dev(wl.W), gpu_rotation(rot))
+    y = layer(dev(wl.X))
+    torch.cuda.synchronize()
+    _, _, _, y_ref = O.linear_forward(wl.X.astype(np.float64), wl.W.astype(np.float64), rot)
+    assert rel_fro(host(y), y_ref) < Y_TOL
+

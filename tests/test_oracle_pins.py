@@ -370,3 +370,51 @@ def test_hadamard_bounds_weight_entries_incoherence():
     wl = workloads.make_workload("tiny_256")
     wr = O.rotate_weights(wl.W.astype(np.float64), O.Rotation(O.HADAMARD, block=256))
     assert np.abs(wr).max() <= O.incoherence_bound(wr, 0.01)
+
+
+# ---------------------------------------------------------------- randomized Hadamard (R11)
+
+def test_random_sign_hadamard_hand_example():
+    x, d, want = _golden_matrix("random_sign_hadamard4.txt")
+    rot = O.Rotation(O.HADAMARD, block=4, signs=d.astype(np.int8))
+    np.testing.assert_allclose(O.rotate_activations(x[None, :], rot)[0], want, atol=1e-12)
+    # signs applied after the rotation would give H(x) .* d instead
+    wrong = (x @ O.hadamard(4) / 2) * d
+    assert not np.allclose(wrong, want)
+
+
+@pytest.mark.parametrize("kind,block,k", [(O.HADAMARD, 64, 256), (O.GSR, 16, 128),
+                                          (O.HADAMARD, 4096, 4096)])
+def test_random_sign_rotation_is_diag_times_blocks(kind, block, k):
+    rng = np.random.default_rng(block)
+    d = workloads.random_signs(block, k)
+    x = rng.standard_normal((5, k))
+    rot = O.Rotation(kind, block=block, signs=d)
+    plain = O.Rotation(kind, block=block)
+    # an independent construction: the explicit matrix diag(d) kron(I, B)
+    r = np.diag(d.astype(np.float64)) @ np.kron(np.eye(k // block), O.block_rotation(kind, block))
+    np.testing.assert_allclose(O.rotate_activations(x, rot), x @ r, atol=1e-10)
+    np.testing.assert_allclose(O.rotate_weights(x, rot), x @ r, atol=1e-10)
+    np.testing.assert_allclose(r @ r.T, np.eye(k), atol=1e-12)          # orthogonal
+    # all-plus signs reduce to the plain rotation
+    ones = O.Rotation(kind, block=block, signs=np.ones(k, np.int8))
+    np.testing.assert_allclose(O.rotate_activations(x, ones), O.rotate_activations(x, plain),
+                               atol=0)
+
+
+def test_random_sign_rotation_keeps_invariance():
+    rng = np.random.default_rng(11)
+    K = 256
+    x = rng.standard_normal((6, K))
+    w = rng.standard_normal((5, K))
+    rot = O.Rotation(O.HADAMARD, block=128, signs=workloads.random_signs(3, K))
+    np.testing.assert_allclose(O.rotate_activations(x, rot) @ O.rotate_weights(w, rot).T,
+                               x @ w.T, atol=1e-10)
+
+
+def test_random_signs_are_seeded_and_balanced():
+    a = workloads.random_signs(5, 4096)
+    assert a.dtype == np.int8 and set(np.unique(a)) == {-1, 1}
+    assert np.array_equal(a, workloads.random_signs(5, 4096))
+    assert not np.array_equal(a, workloads.random_signs(6, 4096))
+    assert abs(int(a.sum())) < 300

@@ -31,6 +31,7 @@ class QrRotation(ctypes.Structure):
         ("chan_scale", ctypes.c_void_p),
         ("chan_mode", ctypes.c_int32),
         ("clip_ratio", ctypes.c_float),
+        ("signs", ctypes.c_void_p),
     ]
 
 
@@ -85,9 +86,9 @@ def _check(fn: str, status: int) -> None:
 
 def make_rotation(kind: int, block: int = 0, p1: int = 0, n1: int = 0, p2: int = 0, n2: int = 0,
                   chan_scale: int = 0, chan_mode: int = QR_CHAN_DIVIDE,
-                  clip_ratio: float = 1.0) -> QrRotation:
+                  clip_ratio: float = 1.0, signs: int = 0) -> QrRotation:
     return QrRotation(kind, block, p1 or None, n1, p2 or None, n2, chan_scale or None, chan_mode,
-                      clip_ratio)
+                      clip_ratio, signs or None)
 
 
 def qr_abi_version() -> int:

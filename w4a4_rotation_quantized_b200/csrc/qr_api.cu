@@ -115,6 +115,10 @@ static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t 
   if (kp > 32768 || K > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
   if (n_out > 0 && (K > 32768 || n_out > 8192)) return QR_ERR_UNSUPPORTED;
   if (kp > 0 && !aligned16(codes)) return QR_ERR_ALIGNMENT;
+  if (rot->signs != nullptr) {
+    if (rot->kind != QR_ROT_HADAMARD && rot->kind != QR_ROT_GSR) return QR_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(rot->signs) % 8 != 0) return QR_ERR_ALIGNMENT;
+  }
   RowJob job{};
   job.src = src;
   job.rows = rows;

@@ -129,6 +129,7 @@ struct WhtParams {
   int64_t rows, ld;
   int32_t K, Kr, Kp, n_out;
   const int32_t* outlier_idx;
+  const int8_t* signs;        // random-sign diagonal [Kp] or null
   int32_t lb;                 // butterflies on in-block index bits [0, lb)
   int32_t nb;                 // blocks per row, Kp >> lb
   int32_t gsr;                // sequency order within blocks
@@ -142,6 +143,7 @@ struct WhtParams {
   __half* out16;
   float* rot_debug;
   int32_t off_buf, buf_bytes, off_red, off_kept, off_idx;   // shared-memory carve-up
+  int32_t off_signs;          // the sign diagonal as bits [Kp/8] (signs != null)
   // ring mode: rows stream into shared memory by bulk copies
   int32_t ring_slots, ring_row_bytes, off_ring, off_bars, rows_per_block;
   int32_t* status;
@@ -183,6 +185,30 @@ __device__ __forceinline__ void copy_outliers(const WhtParams& p, const __half* 
       const int c = __ldg(p.outlier_idx + j);
       p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? srow[c] : __float2half(0.0f);
     }
+}
+
+// Randomized Hadamard.  The CTA first packs the int8 sign diagonal into a
+// bitmask in shared memory (bit j of byte i: element 8i + j is negated; only
+// the sign bit of each int8 entry is read); then 8 consecutive rotated-domain
+// values [e, e+8) flip their sign bits where the diagonal is negative.  The
+// flip is exact.
+__device__ __forceinline__ void build_sign_bits(const int8_t* signs, int kp, uint8_t* bits) {
+  for (int i = threadIdx.x; i < kp / 8; i += blockDim.x) {
+    const uint2 d = __ldg(reinterpret_cast<const uint2*>(signs) + i);
+    uint32_t b = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      b |= ((d.x >> (8 * j + 7)) & 1u) << j;
+      b |= ((d.y >> (8 * j + 7)) & 1u) << (4 + j);
+    }
+    bits[i] = static_cast<uint8_t>(b);
+  }
+}
+
+__device__ __forceinline__ void apply_signs8(const uint8_t* bits, int e, float (&x)[8]) {
+  const uint32_t b = bits[e >> 3];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((b >> i) & 1u) << 31));
 }
 
 // Shared-memory position of rotated element e: 8 floats of padding after
@@ -253,6 +279,11 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
   const int rg = threadIdx.x / nt;
   const int t = threadIdx.x - rg * nt;
   const int lane = threadIdx.x & 31;
+  uint8_t* sbits = smem + p.off_signs;
+  if (p.signs != nullptr) {
+    build_sign_bits(p.signs, p.Kp, sbits);
+    __syncthreads();
+  }
   uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
   if (p.n_out > 0) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
                                     reinterpret_cast<int32_t*>(smem + p.off_idx));
@@ -349,6 +380,7 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
         } else {
           load8(p, srow, kept, e, x);
         }
+        if (p.signs != nullptr) apply_signs8(sbits, e, x);
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[8 * h + i] = x[i];
       }
@@ -514,6 +546,11 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
   const int nt = p.nt;
   const int rg = threadIdx.x / nt;
   const int t = threadIdx.x - rg * nt;
+  uint8_t* sbits = smem + p.off_signs;
+  if (p.signs != nullptr) {
+    build_sign_bits(p.signs, p.Kp, sbits);
+    __syncthreads();
+  }
   uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
   if (p.n_out > 0) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
                                     reinterpret_cast<int32_t*>(smem + p.off_idx));
@@ -533,6 +570,7 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
       float x[8];
       if (g < ngroups) {
         load8(p, srow, kept, 8 * g, x);
+        if (p.signs != nullptr) apply_signs8(sbits, 8 * g, x);
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) x[i] = 0.0f;
@@ -600,6 +638,7 @@ struct FewRowsParams {
   int64_t rows, ld;
   int32_t K, Kr, Kp, n_out;
   const int32_t* outlier_idx;
+  const int8_t* signs;        // random-sign diagonal [Kp] or null
   int32_t lb, gsr, aligned;
   int32_t cl;                 // CTAs per row (a cluster)
   int32_t span;               // rotated elements per CTA (whole blocks, a multiple of 128)
@@ -772,7 +811,9 @@ __global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams 
       if ((m8 >> i) & 1u) {
         ++before;
       } else if (col0 + i < p.K && e < p.Kr && e >= e_lo && e < e_hi) {
-        buf[few_swz(e - e_lo)] = x[i];
+        float xv = x[i];
+        if (p.signs != nullptr && __ldg(p.signs + e) < 0) xv = -xv;
+        buf[few_swz(e - e_lo)] = xv;
       }
     }
   }
@@ -1094,6 +1135,7 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
   p.Kp = job.Kp;
   p.n_out = job.n_out;
   p.outlier_idx = job.outlier_idx;
+  p.signs = (rot.kind == QR_ROT_HADAMARD || rot.kind == QR_ROT_GSR) ? rot.signs : nullptr;
   const int block = (rot.kind == QR_ROT_NONE) ? 1 : rot.block;
   p.lb = ilog2(block);
   p.gsr = rot.kind == QR_ROT_GSR;
@@ -1155,6 +1197,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.Kp = job.Kp;
   p.n_out = job.n_out;
   p.outlier_idx = job.outlier_idx;
+  p.signs = (rot.kind == QR_ROT_HADAMARD || rot.kind == QR_ROT_GSR) ? rot.signs : nullptr;
   const int block = (rot.kind == QR_ROT_NONE) ? 1 : rot.block;
   const int lb = ilog2(block);
   p.lb = lb;
@@ -1207,6 +1250,9 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   if (job.n_out > 0) off = align_up(off + sizeof(uint16_t) * job.Kr, 16);
   p.off_idx = static_cast<int32_t>(off);
   if (job.n_out > 0) off = align_up(off + sizeof(int32_t) * job.n_out, 16);
+  const size_t sign_bytes = p.signs != nullptr ? static_cast<size_t>(job.Kp / 8) : 0;
+  p.off_signs = static_cast<int32_t>(off);
+  off = align_up(off + sign_bytes, 16);
   if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
 
   p.status = device_status_word();
@@ -1228,7 +1274,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
     const size_t buf_off = roff;
     roff = align_up(roff + static_cast<size_t>(p.buf_bytes) * groups, 128);
     const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - static_cast<int64_t>(roff) -
-                         16 * per_block - 16 - 1024) / row_bytes;
+                         16 * per_block - 16 - 1024 - static_cast<int64_t>(sign_bytes)) / row_bytes;
     const int slots = static_cast<int>(std::min<int64_t>(per_block, fit));
     if (slots >= 1 && groups * nt + 32 <= bound) {
       p.off_red = 0;
@@ -1241,6 +1287,8 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
       p.rows_per_block = static_cast<int32_t>(per_block);
       p.rows_per_cta = groups;                                   // row groups
       off = p.off_bars + 16 * static_cast<size_t>(slots) + 16;
+      p.off_signs = static_cast<int32_t>(align_up(off, 16));
+      off = p.off_signs + sign_bytes;
       grid = static_cast<int>((job.rows + per_block - 1) / per_block);
     } else {
       ring = false;

@@ -38,6 +38,7 @@ class Rotation:
     chan_scale: Optional[torch.Tensor] = None   # fp32 [n1*n2]
     chan_mode: int = L.QR_CHAN_DIVIDE
     clip_ratio: float = 1.0
+    signs: Optional[torch.Tensor] = None    # int8 [K_p] of +-1 (HADAMARD, GSR): R = D B
     _c: Optional[L.QrRotation] = field(default=None, repr=False)
 
     def c(self) -> L.QrRotation:
@@ -46,11 +47,15 @@ class Rotation:
                 _need_cuda(t, torch.float32, "rotation tensor")
                 if not t.is_contiguous():
                     raise ValueError("rotation tensors must be contiguous")
+        if self.signs is not None:
+            _need_cuda(self.signs, torch.int8, "signs")
+            if not self.signs.is_contiguous():
+                raise ValueError("signs must be contiguous")
         n1 = 0 if self.p1 is None else self.p1.shape[0]
         n2 = 0 if self.p2 is None else self.p2.shape[0]
         self._c = L.make_rotation(self.kind, self.block, _ptr(self.p1) or 0, n1,
                                   _ptr(self.p2) or 0, n2, _ptr(self.chan_scale) or 0,
-                                  self.chan_mode, self.clip_ratio)
+                                  self.chan_mode, self.clip_ratio, _ptr(self.signs) or 0)
         return self._c
 
 

@@ -184,3 +184,11 @@ def random_codes_rows(rng: np.random.Generator, rows: int, cols: int) -> np.ndar
     pos = rng.integers(cols, size=rows)
     q[np.arange(rows), pos] = np.where(rng.random(rows) < 0.5, 7, -7)
     return q
+
+
+def random_signs(seed: int, k_p: int) -> np.ndarray:
+    """A seeded random +-1 diagonal of length k_p (int8), the input of a
+    randomized Hadamard rotation.  Drawn here so that both the oracle and the
+    CUDA path receive the same signs."""
+    rng = np.random.default_rng([seed, 99])
+    return np.where(rng.random(k_p) < 0.5, -1, 1).astype(np.int8)
