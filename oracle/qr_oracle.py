@@ -53,6 +53,13 @@ R11 A "random Hadamard rotation" ([SR] reviewer brBn W2/A2) is R = D B with
     row becomes (x .* d) B.  The signs act on the rotated-domain columns
     (after the outlier split and zero padding).  D B is orthogonal, so the
     weight side uses the same R.
+R12 QUIK's activations are asymmetric per token, dynamic ([QK] §1).  Read
+    as min-max over the unsigned range [0, 15]: lo = alpha*min, hi =
+    alpha*max, s = (hi - lo)/15, zero point z = round(-lo/s), q =
+    clamp(round(x/s) + z, 0, 15), dequantized s*(q - z); both decisions in
+    float32, half to even.  The codes are stored as the signed nibble
+    q - 8 (two's complement, [-8, 7]) with the zero point z - 8, so that
+    s*(q - z) = s*((q - 8) - (z - 8)) and the same integer GEMM applies.
 """
 from __future__ import annotations
 
@@ -233,6 +240,46 @@ def quantize_rows(xr: np.ndarray, clip_ratio: float = 1.0) -> Quantized:
     return Quantized(codes=q, scales=s, quotient=v)
 
 
+@dataclass
+class AsymQuantized:
+    codes: np.ndarray        # int8 [rows x K_p]: q - 8, in [-8, 7]
+    scales: np.ndarray       # float32 [rows]
+    zeros: np.ndarray        # int32 [rows]: z - 8
+    quotient: np.ndarray     # float32 x/s before rounding (tie window)
+    zero_quotient: np.ndarray  # float32 -lo/s before rounding (tie window of z)
+
+
+def quantize_rows_asym(xr: np.ndarray, clip_ratio: float = 1.0) -> AsymQuantized:
+    """Asymmetric per-row min-max quantization to 4-bit codes (R12).
+
+    [QK] QUIK量化 §1: activations are quantized asymmetrically per token,
+    dynamically; weights stay symmetric (quantize_rows).
+    """
+    x32 = np.asarray(xr, dtype=np.float64).astype(np.float32)
+    rows = x32.shape[0]
+    if x32.shape[1]:
+        lo = (np.float32(clip_ratio) * np.min(x32, axis=1)).astype(np.float32)
+        hi = (np.float32(clip_ratio) * np.max(x32, axis=1)).astype(np.float32)
+    else:
+        lo = hi = np.zeros(rows, np.float32)
+    s = ((hi - lo) / np.float32(15)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    zq = (-lo / safe).astype(np.float32)
+    zq[s == 0] = 0.0
+    z = np.rint(zq).astype(np.int64)
+    v = (x32 / safe[:, None]).astype(np.float32)
+    v[s == 0] = 0.0
+    q = np.clip(np.rint(v).astype(np.int64) + z[:, None], 0, 15)
+    return AsymQuantized(codes=(q - 8).astype(np.int8), scales=s, zeros=(z - 8).astype(np.int32),
+                         quotient=v, zero_quotient=zq)
+
+
+def dequant_asym_rows(q: AsymQuantized) -> np.ndarray:
+    """X_hat = s * (codes - zeros) in float64 (R12)."""
+    return np.asarray(q.scales, np.float64)[:, None] * (
+        q.codes.astype(np.float64) - q.zeros.astype(np.float64)[:, None])
+
+
 def pack_int4(q: np.ndarray) -> np.ndarray:
     """Two's-complement nibbles, two per byte, element 2j in the low nibble."""
     q = np.asarray(q, dtype=np.int64)
@@ -362,6 +409,39 @@ def linear(a: Side, w: Side):
     acc = int_gemm(a.q.codes, w.q.codes)
     y = dequant_epilogue(acc, a.q.scales, w.q.scales, a.fp16_part, w.fp16_part)
     return acc, y
+
+
+def quantize_activations_asym(x: np.ndarray, rot: Rotation,
+                              outlier_idx: Optional[np.ndarray] = None) -> Side:
+    """The online activation path with QUIK's asymmetric quantizer (R12)."""
+    x_in, x_out = split_outliers(x, outlier_idx)
+    n_out = 0 if outlier_idx is None else len(outlier_idx)
+    k_p = packed_width(rot, np.asarray(x).shape[1], n_out)
+    xr = rotate_activations(pad_columns(np.asarray(x_in, np.float64), k_p), rot)
+    q = quantize_rows_asym(xr, rot.clip_ratio)
+    return Side(xr, q, pack_int4(q.codes), np.asarray(x_out, np.float16))
+
+
+def linear_asym(a: Side, w: Side):
+    """(acc, Y) for asymmetric activation codes: acc = sum (q_a - 8) q_w
+    (what the integer GEMM accumulates), Y = fp16(X_hat W_hat^T + X_out
+    W_out^T) with X_hat = s_a (codes - zeros), W_hat = s_w q_w, formed in
+    float64 from the dequantized operands ([QK] §1, §4; R12)."""
+    acc = int_gemm(a.q.codes, w.q.codes)
+    x_hat = dequant_asym_rows(a.q)
+    w_hat = np.asarray(w.q.scales, np.float64)[:, None] * w.q.codes.astype(np.float64)
+    y = x_hat @ w_hat.T
+    if a.fp16_part.shape[1]:
+        y = y + np.asarray(a.fp16_part, np.float64) @ np.asarray(w.fp16_part, np.float64).T
+    return acc, y.astype(np.float16)
+
+
+def linear_forward_asym(x, w, rot: Rotation, outlier_idx=None):
+    """The whole layer with asymmetric activations and symmetric weights."""
+    a = quantize_activations_asym(x, rot, outlier_idx)
+    ws = quantize_weights(w, rot, outlier_idx)
+    acc, y = linear_asym(a, ws)
+    return a, ws, acc, y
 
 
 def linear_forward(x, w, rot: Rotation, outlier_idx=None):

@@ -418,3 +418,60 @@ def test_random_signs_are_seeded_and_balanced():
     assert np.array_equal(a, workloads.random_signs(5, 4096))
     assert not np.array_equal(a, workloads.random_signs(6, 4096))
     assert abs(int(a.sum())) < 300
+
+
+# ---------------------------------------------------------------- asymmetric activations (R12)
+
+def test_asym_quantizer_hand_example():
+    for r in read_golden_rows("quantizer_asym_1x4.txt"):
+        v = [float(t) for t in r]
+        x, codes, scale, zero = np.array(v[:4]), np.array(v[4:8]), v[8], v[9]
+        q = O.quantize_rows_asym(x[None, :])
+        assert np.array_equal(q.codes[0], codes.astype(np.int8))
+        assert q.scales[0] == np.float32(scale) and q.zeros[0] == zero
+
+
+def test_asym_quantizer_properties():
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal((6, 300)),
+                        np.abs(rng.standard_normal((3, 300))) + 2.0,     # all positive
+                        np.zeros((1, 300))])
+    q = O.quantize_rows_asym(x)
+    assert q.codes.min() >= -8 and q.codes.max() <= 7
+    xhat = O.dequant_asym_rows(q)
+    s = q.scales.astype(np.float64)[:, None]
+    assert np.all(np.abs(xhat - x) <= s / 2 * (1 + 1e-5) + 1e-12)    # half a step, unclipped
+    assert not xhat[-1].any() and q.scales[-1] == 0
+    # each row's minimum lands on the bottom code (q = 0)
+    assert np.array_equal(q.codes[np.arange(10), np.argmin(x, axis=1)][:-1], np.full(9, -8))
+    # clipping shrinks the range and clamps into [0, 15]
+    qc = O.quantize_rows_asym(x, clip_ratio=0.5)
+    assert qc.codes.min() >= -8 and qc.codes.max() <= 7
+    assert np.all(qc.scales[:-1] < q.scales[:-1])
+
+
+def test_asym_beats_symmetric_on_one_sided_rows():
+    # QUIK's reason for asymmetric activations: rows far from symmetric
+    rng = np.random.default_rng(9)
+    a = rng.standard_normal((64, 512))
+    x = a / (1 + np.exp(-a))                       # SiLU: bounded below, long upper tail
+    e_asym = np.abs(O.dequant_asym_rows(O.quantize_rows_asym(x)) - x).mean()
+    qs = O.quantize_rows(x)
+    e_sym = np.abs(qs.scales.astype(np.float64)[:, None] * qs.codes - x).mean()
+    assert e_asym < 0.75 * e_sym
+
+
+def test_asym_linear_matches_the_dequantized_product():
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((5, 256)).astype(np.float16)
+    w = (rng.standard_normal((7, 256)) * 0.05).astype(np.float16)
+    rot = O.Rotation(O.HADAMARD, block=128)
+    a, ws, acc, y = O.linear_forward_asym(x.astype(np.float64), w.astype(np.float64), rot)
+    # acc is the integer product of the stored codes; the zero point enters
+    # only through X_hat: Y = s_a s_w (acc - z' sum_k q_w)
+    zsum = a.q.zeros.astype(np.int64)[:, None] * ws.q.codes.astype(np.int64).sum(axis=1)[None, :]
+    alt = (acc - zsum) * a.q.scales.astype(np.float64)[:, None] * ws.q.scales.astype(np.float64)[None, :]
+    np.testing.assert_allclose(y.astype(np.float64), alt, rtol=2e-3, atol=1e-3)
+    # and the layer tracks X W^T
+    ref = x.astype(np.float64) @ w.astype(np.float64).T
+    assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.2
