@@ -205,8 +205,10 @@ def oracle_rotation(wl, signs=None):
                       block=s.block, clip_ratio=s.clip_ratio, signs=signs)
 
 
-def algorithmic_counts(wl, M, kp):
-    """Algorithmic work of one step (padding excluded)."""
+def algorithmic_counts(wl, M, kp, asym=False):
+    """Algorithmic work of one step (padding excluded).  Asymmetric activations
+    add a zero point per token (written, then read) and a code sum per weight
+    row (read)."""
     s = wl.spec
     K, N = s.K, s.N
     n_out = s.n_keep_fp16
@@ -216,6 +218,9 @@ def algorithmic_counts(wl, M, kp):
     rq_bytes = M * K * 2 + M * k_int / 2 + M * 4 + M * n_out * 2
     # GEMM: read codes, scales and outlier columns, write Y
     gemm_bytes = (M + N) * k_int / 2 + (M + N) * 4 + (M + N) * n_out * 2 + M * N * 2
+    if asym:
+        rq_bytes += M * 4
+        gemm_bytes += (M + N) * 4
     return gemm_ops, rq_bytes, gemm_bytes
 
 
@@ -242,37 +247,51 @@ def run_ours(args, rank, world, local_rank):
     if s.n_keep_fp16:
         idx = Q.select_outliers(torch.from_numpy(wl.X_calib).cuda(), s.n_keep_fp16)
     kp = Q.packed_k(rot, s.K, s.n_keep_fp16)
-    gemm_ops, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp)
+    asym = args.asym_activations
+    gemm_ops, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp, asym)
 
     # input sets: enough copies that one pass over them exceeds L2 twice
     x0 = torch.from_numpy(wl.X).cuda()
     w0 = torch.from_numpy(wl.W).cuda()
     t_pack0 = torch.cuda.Event(enable_timing=True)
     t_pack1 = torch.cuda.Event(enable_timing=True)
-    Q.QuantizedLinear(w0, rot, idx)                   # warm-up (module load, attributes)
+    Q.QuantizedLinear(w0, rot, idx, asym)            # warm-up (module load, attributes)
     torch.cuda.synchronize()
     t_pack0.record()
-    layer0 = Q.QuantizedLinear(w0, rot, idx)
+    layer0 = Q.QuantizedLinear(w0, rot, idx, asym)
     t_pack1.record()
     torch.cuda.synchronize()
     pack_ms = t_pack0.elapsed_time(t_pack1)
-    set_bytes = x0.numel() * 2 + layer0.w_codes.numel() + 4 * s.N + \
+    set_bytes = x0.numel() * 2 + layer0.w_codes.numel() + (8 if asym else 4) * s.N + \
         (0 if layer0.w_out is None else layer0.w_out.numel() * 2)
     nsets = max(2, math.ceil(2 * L2_BYTES / set_bytes))
     xs = [x0] + [x0.clone() for _ in range(nsets - 1)]
-    wsets = [(layer0.w_codes, layer0.w_scales, layer0.w_out)]
+    wsets = [(layer0.w_codes, layer0.w_scales, layer0.w_out, layer0.w_sums)]
     for _ in range(nsets - 1):
         wsets.append((layer0.w_codes.clone(), layer0.w_scales.clone(),
-                      None if layer0.w_out is None else layer0.w_out.clone()))
+                      None if layer0.w_out is None else layer0.w_out.clone(),
+                      None if layer0.w_sums is None else layer0.w_sums.clone()))
     del w0
     y = torch.empty((M, s.N), dtype=torch.float16, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        x = xs[i % nsets]
-        wc, wsc, wo = wsets[i % nsets]
+    def rq(x):
+        if asym:
+            codes, scales, zeros, x_out, _ = Q.rotate_quant_asym(x, rot, idx)
+            return codes, scales, x_out, zeros
         codes, scales, x_out, _ = Q.rotate_quant(x, rot, idx)
-        Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
+        return codes, scales, x_out, None
+
+    def linear(a, wset):
+        codes, scales, x_out, zeros = a
+        wc, wsc, wo, wsum = wset
+        if asym:
+            Q.w4a4_linear_asym(codes, scales, zeros, wc, wsc, wsum, x_out, wo, out=y)
+        else:
+            Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
+
+    def step(i):
+        linear(rq(xs[i % nsets]), wsets[i % nsets])
 
     for i in range(args.warmup):
         step(i)
@@ -284,13 +303,11 @@ def run_ours(args, rank, world, local_rank):
     # region replays them in turn; events between replays give each kernel's
     # device time.  A last pair of graphs takes the K mod G remaining steps.
     def rot_pass(n):
-        return [Q.rotate_quant(xs[i], rot, idx)[:3] for i in range(n)]
+        return [rq(xs[i]) for i in range(n)]
 
     def gemm_pass(outs, n):
         for i in range(n):
-            codes, scales, x_out = outs[i]
-            wc, wsc, wo = wsets[i]
-            Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
+            linear(outs[i], wsets[i])
 
     def capture(fn):
         g = torch.cuda.CUDAGraph()
@@ -418,7 +435,9 @@ def run_ours(args, rank, world, local_rank):
                    "rotation": (("random-sign " if signs is not None else "") +
                                 f"{s.rotation}-{s.block}") if s.rotation != "kron"
                    else f"kron-{s.n1}x{s.n2}", "n_out": s.n_keep_fp16,
-                   "clip_ratio": s.clip_ratio, "parallelism": f"replicas x{world}",
+                   "clip_ratio": s.clip_ratio,
+                   "activations": "asymmetric per-token" if asym else "symmetric per-token",
+                   "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
         "roofline": roofline,
@@ -452,8 +471,16 @@ def aggregate_max(value_ms: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- oracle
 
+def oracle_step(O, asym: bool):
+    """The oracle's online path: activation quantizer, then the linear."""
+    if asym:
+        return lambda x, rot, idx, wside: O.linear_asym(
+            O.quantize_activations_asym(x, rot, idx), wside)
+    return lambda x, rot, idx, wside: O.linear(O.quantize_activations(x, rot, idx), wside)
+
+
 def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None,
-                    random_signs: bool = False):
+                    random_signs: bool = False, asym: bool = False):
     """Times the CPU oracle's online path on `tokens` tokens of the workload."""
     import oracle as O
     import workloads
@@ -465,11 +492,11 @@ def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None,
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
     wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)     # offline, untimed
     x = wl.X[:tokens].astype(np.float64)
+    run = oracle_step(O, asym)
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
-        a = O.quantize_activations(x, rot, idx)
-        O.linear(a, wside)
+        run(x, rot, idx, wside)
         times.append(time.perf_counter() - t0)
     gemm_ops, _, _ = algorithmic_counts(wl, tokens, 0)
     sec = statistics.median(times)
@@ -495,10 +522,10 @@ def run_reference(args, rank, world):
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
     wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)
     x = wl.X[:tokens].astype(np.float64)
+    run = oracle_step(O, args.asym_activations)
 
     def step():
-        a = O.quantize_activations(x, rot, idx)
-        O.linear(a, wside)
+        run(x, rot, idx, wside)
 
     for _ in range(args.warmup):
         step()
@@ -518,7 +545,8 @@ def run_reference(args, rank, world):
         "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": s.name, "M": tokens, "K": s.K, "N": s.N,
-                   "parallelism": "host cores"},
+                   "activations": "asymmetric per-token" if args.asym_activations
+                   else "symmetric per-token", "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
@@ -542,6 +570,8 @@ def main(argv=None):
     ap.add_argument("--reference-tokens", type=int, default=64)
     ap.add_argument("--random-signs", action="store_true",
                     help="randomized Hadamard: a seeded random-sign diagonal before the blocks")
+    ap.add_argument("--asym-activations", action="store_true",
+                    help="QUIK's asymmetric per-token activation quantizer (zero point per token)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -573,7 +603,8 @@ def main(argv=None):
                 tokens = min(args.cpu_baseline_tokens, res["config"]["M"])
                 res["cpu_baseline"] = oracle_baseline(args.workload, tokens, repeats=3,
                                                       M_total=args.tokens,
-                                                      random_signs=args.random_signs)
+                                                      random_signs=args.random_signs,
+                                                      asym=args.asym_activations)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

@@ -190,6 +190,47 @@ QR_API qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales,
                          uint16_t* Y, int64_t ldy, int32_t* acc_debug,
                          qr_stream stream);
 
+/* ----------------------------------------------------------------------
+ * Asymmetric per-token activations ("QUIK：LLM上的一种4-bit推理方法",
+ * QUIK量化 §1: activations are quantized asymmetrically per token and
+ * dynamically, weights symmetrically).
+ *
+ * qr_rotate_quant_asym: as qr_rotate_quant, but each rotated row x is
+ * quantized over [0, 15]: lo = alpha*min(x), hi = alpha*max(x),
+ * s = (hi - lo)/15, z = round(-lo/s), q = clamp(round(x/s) + z, 0, 15)
+ * (float32, half to even).  Codes are stored as the signed nibble q - 8
+ * (same packing as qr_rotate_quant), scales[m] = s, zeros[m] = z - 8
+ * (int32 [M], device), so x ~= s * (code - zero).  A zero row gets s = 0.
+ * Not for QR_ROT_KRON (UNSUPPORTED).  Errors as qr_rotate_quant, plus
+ * INVALID_ARG for a null zeros with M > 0. */
+QR_API qr_status qr_rotate_quant_asym(const qr_rotation* rot, const uint16_t* X, int64_t M,
+                                      int64_t K, int64_t ldx, const int32_t* outlier_idx,
+                                      int32_t n_out, uint8_t* a_codes, float* a_scales,
+                                      int32_t* a_zeros, uint16_t* x_out, float* x_rot_debug,
+                                      qr_stream stream);
+
+/* Per weight row, the sum of its packed signed codes: w_sums[n] =
+ * sum_k q_w[n, k] (int32 [N], device), for the zero-point term of
+ * qr_w4a4_linear_asym.  Offline, once per layer.  w_codes [N x K_p/2],
+ * 16-byte aligned; K_p % 128 == 0.  Errors: INVALID_ARG, ALIGNMENT. */
+QR_API qr_status qr_weight_code_sums(const uint8_t* w_codes, int64_t N, int64_t K_p,
+                                     int32_t* w_sums, qr_stream stream);
+
+/* qr_w4a4_linear for asymmetric activation codes:
+ *   acc[m, n] = sum_k code_a[m, k] q_w[n, k]          (int32, exact)
+ *   Y[m, n]   = fp16( (acc - zero_a[m] * w_sums[n]) * s_a[m] * s_w[n]
+ *                     + X_out[m] . W_out[n] )
+ * i.e. the product of the dequantized operands s_a (code - zero) and
+ * s_w q_w.  a_zeros int32 [M], w_sums int32 [N] from qr_weight_code_sums;
+ * acc_debug receives acc.  Other arguments and errors as qr_w4a4_linear,
+ * plus INVALID_ARG for a null a_zeros or w_sums. */
+QR_API qr_status qr_w4a4_linear_asym(const uint8_t* a_codes, const float* a_scales,
+                                     const int32_t* a_zeros, const uint8_t* w_codes,
+                                     const float* w_scales, const int32_t* w_sums, int64_t M,
+                                     int64_t N, int64_t K_p, const uint16_t* x_out,
+                                     const uint16_t* w_out, int32_t n_out, uint16_t* Y,
+                                     int64_t ldy, int32_t* acc_debug, qr_stream stream);
+
 /* QUIK calibration (QUIK §3: outliers are the columns with the largest
  * infinity-norm over a calibration batch).  Writes the k selected column
  * indices of X_calib [T x ldx] (fp16, ldx >= K) to idx_out[k] in ascending

@@ -105,6 +105,39 @@ def tile_side(ref: O.Side, reps: int) -> O.Side:
     return O.Side(rotated=t(ref.rotated), q=q, packed=t(ref.packed), fp16_part=t(ref.fp16_part))
 
 
+def check_side_asym(gpu, ref: O.Side, what: str, clip: float = 1.0):
+    """Compares (codes, scales, zeros, fp16 part, rotated) from the GPU with an
+    oracle Side of asymmetric activation codes (zero points exact except
+    where -lo/s lies within the tie window of a half; such rows' codes are
+    not compared)."""
+    codes, scales, zeros, out16, rot = gpu
+    q = ref.q
+    if rot is not None and ref.rotated.shape[1]:
+        r = host(rot).astype(np.float64)
+        norm = np.linalg.norm(ref.rotated, axis=1)
+        err = np.abs(r - ref.rotated).max(axis=1)
+        assert not (err > ROT_TOL * np.maximum(norm, 1e-30)).any(), f"{what}: rotated rows off"
+    norm = np.linalg.norm(ref.rotated, axis=1)
+    ref_s = q.scales.astype(np.float64)
+    allowed = clip * 2 * ROT_TOL * norm / 15.0 + SCALE_TOL * ref_s
+    off = np.abs(host(scales).astype(np.float64) - ref_s)
+    assert np.all(off <= allowed), f"{what}: scales off by up to {(off / np.maximum(ref_s, 1e-30)).max():.3g}"
+    zq = q.zero_quotient.astype(np.float64)
+    ztie = np.abs(np.abs(zq - np.rint(zq)) - 0.5) < TIE_WINDOW
+    gz = host(zeros).astype(np.int64)
+    assert np.array_equal(gz[~ztie], q.zeros.astype(np.int64)[~ztie]), f"{what}: zero points differ"
+    got = unpack(codes)
+    want = q.codes
+    v = q.quotient.astype(np.float64)
+    tie = (np.abs(np.abs(v - np.rint(v)) - 0.5) < TIE_WINDOW) | ztie[:, None]
+    diff = got != want
+    assert not (diff & ~tie).any(), f"{what}: {int((diff & ~tie).sum())} codes differ outside ties"
+    if out16 is not None:
+        np.testing.assert_array_equal(host(out16).view(np.uint16),
+                                      np.asarray(ref.fp16_part, np.float16).view(np.uint16))
+    return int(diff.sum())
+
+
 def rel_fro(a, b) -> float:
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)

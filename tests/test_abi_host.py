@@ -148,3 +148,24 @@ def test_calibration_argument_errors(lib):
     assert L.qr_invert_transpose(FAKE, 0, FAKE, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG
     assert L.qr_invert_transpose(FAKE, 200, FAKE, FAKE, None, check=False) == L.QR_ERR_UNSUPPORTED
     assert L.qr_invert_transpose(None, 4, FAKE, FAKE, None, check=False) == L.QR_ERR_INVALID_ARG
+
+
+def test_asymmetric_entry_points_argument_errors(lib):
+    h = _rot(L.QR_ROT_HADAMARD, 256)
+    rq = lambda rot, zeros=FAKE, M=4: L.qr_rotate_quant_asym(
+        rot, FAKE, M, 256, 256, None, 0, FAKE, FAKE, zeros, None, None, None, check=False)
+    assert rq(h, zeros=None) == L.QR_ERR_INVALID_ARG
+    assert rq(_rot(L.QR_ROT_KRON, n1=16, n2=16)) == L.QR_ERR_UNSUPPORTED
+    assert rq(h, zeros=None, M=0) == L.QR_OK
+    sums = lambda N=8, Kp=256, codes=FAKE, out=FAKE: L.qr_weight_code_sums(codes, N, Kp, out, None,
+                                                                          check=False)
+    assert sums(Kp=100) == L.QR_ERR_INVALID_ARG
+    assert sums(out=None) == L.QR_ERR_INVALID_ARG
+    assert sums(codes=FAKE + 4) == L.QR_ERR_ALIGNMENT
+    assert sums(N=0) == L.QR_OK
+    lin = lambda za=FAKE, ws=FAKE: L.qr_w4a4_linear_asym(FAKE, FAKE, za, FAKE, FAKE, ws, 16, 16, 256,
+                                                         None, None, 0, FAKE, 16, None, None,
+                                                         check=False)
+    assert lin(za=None) == L.QR_ERR_INVALID_ARG
+    assert lin(ws=None) == L.QR_ERR_INVALID_ARG
+

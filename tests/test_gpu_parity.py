@@ -10,7 +10,7 @@ import torch
 import oracle as O
 import w4a4_rotation_quantized_b200 as Q
 import workloads
-from tests.gpu_helpers import (Y_TOL, check_side, dev, gpu_rotation, host,
+from tests.gpu_helpers import (Y_TOL, check_side, check_side_asym, dev, gpu_rotation, host,
                                oracle_rows_from_gpu_codes, rel_fro, require_gpu, tile_rows,
                                tile_side, unpack)
 
@@ -337,4 +337,104 @@ def test_layer_random_signs_end_to_end():
     torch.cuda.synchronize()
     _, _, _, y_ref = O.linear_forward(wl.X.astype(np.float64), wl.W.astype(np.float64), rot)
     assert rel_fro(host(y), y_ref) < Y_TOL
+
+
+# ---------------------------------------------------------------- asymmetric activations
+
+ASYM_CASES = [
+    # (name, K, rows, kind, block, n_out, clip)
+    ("had4096", 4096, 9, O.HADAMARD, 4096, 0, 1.0),
+    ("gsr128", 11008, 5, O.GSR, 128, 0, 1.0),
+    ("had64_clip", 640, 7, O.HADAMARD, 64, 0, 0.8),
+    ("none_ragged", 200, 6, O.NONE, 1, 0, 1.0),
+    ("had4096_outliers", 8192, 6, O.HADAMARD, 4096, 256, 1.0),
+    ("had8", 256, 5, O.HADAMARD, 8, 0, 1.0),
+]
+
+
+@pytest.mark.parametrize("name,K,rows,kind,block,n_out,clip", ASYM_CASES,
+                         ids=[c[0] for c in ASYM_CASES])
+@pytest.mark.parametrize("many", [False, True], ids=["few", "many"])
+def test_rotate_quant_asym(name, K, rows, kind, block, n_out, clip, many):
+    rng = np.random.default_rng(zlib.crc32(name.encode()) + 5)
+    idx = np.sort(rng.choice(K, size=n_out, replace=False)).astype(np.int32) if n_out else None
+    x = _rows(rng, rows, K, outl=(1,) if not n_out else idx[:2])
+    x[0] = 0                                         # a zero row
+    x[1] = np.abs(x[1]) + np.float16(1.0)            # a row far from zero
+    rot = O.Rotation(kind, block=block, clip_ratio=clip)
+    reps = 1
+    x_run = x
+    if many:
+        x_run, reps = tile_rows(x)
+    ig = None if idx is None else dev(idx)
+    gpu = Q.rotate_quant_asym(dev(x_run), gpu_rotation(rot), ig, debug=True)
+    torch.cuda.synchronize()
+    ref = O.quantize_activations_asym(x.astype(np.float64), rot, idx)
+    if reps > 1:
+        codes, scales, zeros, out16, dbg = gpu
+        rows0 = x.shape[0]
+        for r in range(reps):
+            sl = slice(r * rows0, (r + 1) * rows0)
+            check_side_asym((codes[sl], scales[sl], zeros[sl], None if out16 is None else out16[sl],
+                             dbg[sl]), ref, f"{name} asym copy {r}", clip=clip)
+    else:
+        check_side_asym(gpu, ref, f"{name} asym", clip=clip)
+    assert host(gpu[1])[0] == 0
+
+
+def test_weight_code_sums():
+    rng = np.random.default_rng(4)
+    q = rng.integers(-7, 8, size=(300, 1280)).astype(np.int8)
+    got = host(Q.weight_code_sums(dev(O.pack_int4(q))))
+    assert np.array_equal(got, q.astype(np.int64).sum(axis=1))
+
+
+ASYM_LINEAR_CASES = [(1, 512, 1024, 0), (16, 8192, 512, 0), (64, 384, 256, 64), (40, 1000, 2048, 32),
+                     (300, 1000, 1024, 0), (257, 225, 384, 32)]
+
+
+@pytest.mark.parametrize("M,N,K,n_out", ASYM_LINEAR_CASES)
+def test_linear_asym_matches_oracle(M, N, K, n_out):
+    rng = np.random.default_rng(M * 7 + N + K)
+    qa = rng.integers(-8, 8, size=(M, K)).astype(np.int8)
+    qw = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+    za = rng.integers(-20, 20, size=M).astype(np.int32)
+    sa = rng.uniform(0.01, 0.2, M).astype(np.float32)
+    sw = rng.uniform(0.001, 0.01, N).astype(np.float32)
+    xo = (rng.standard_normal((M, n_out)) * 3).astype(np.float16) if n_out else None
+    wo = (rng.standard_normal((N, n_out)) * 0.02).astype(np.float16) if n_out else None
+    w_codes = dev(O.pack_int4(qw))
+    sums = Q.weight_code_sums(w_codes)
+    y, acc = Q.w4a4_linear_asym(dev(O.pack_int4(qa)), dev(sa), dev(za), w_codes, dev(sw), sums,
+                                None if xo is None else dev(xo), None if wo is None else dev(wo),
+                                acc_debug=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(acc).astype(np.int64), O.int_gemm(qa, qw))
+    aq = O.AsymQuantized(codes=qa, scales=sa, zeros=za, quotient=None, zero_quotient=None)
+    a_side = O.Side(rotated=None, q=aq, packed=None,
+                    fp16_part=xo if xo is not None else np.zeros((M, 0), np.float16))
+    w_side = O.Side(rotated=None, q=O.Quantized(codes=qw, scales=sw, quotient=None), packed=None,
+                    fp16_part=wo if wo is not None else np.zeros((N, 0), np.float16))
+    _, want = O.linear_asym(a_side, w_side)
+    assert rel_fro(host(y), want) < 1e-3
+
+
+@pytest.mark.parametrize("name,M,N", [("quik_decode_8192", 1, 1024), ("quik_decode_8192", 64, 1024),
+                                      ("qkv_prefill_4096", 96, 512)])
+def test_layer_asym_end_to_end(name, M, N):
+    wl = workloads.make_workload(name, M=M, N=N)
+    rot = _oracle_rotation(wl)
+    idx = idx_g = None
+    if wl.spec.n_keep_fp16:
+        idx = O.select_outliers(wl.X_calib, wl.spec.n_keep_fp16)
+        idx_g = Q.select_outliers(dev(wl.X_calib), wl.spec.n_keep_fp16)
+    layer = Q.QuantizedLinear(dev(wl.W), gpu_rotation(rot), idx_g, asym_activations=True)
+    y = layer(dev(wl.X))
+    torch.cuda.synchronize()
+    _, _, _, y_ref = O.linear_forward_asym(wl.X.astype(np.float64), wl.W.astype(np.float64), rot,
+                                           idx)
+    assert rel_fro(host(y), y_ref) < Y_TOL
+    g = Q.GraphedLinear(layer, M)
+    y2 = host(g(torch.from_numpy(wl.X).pin_memory())).copy()
+    assert np.array_equal(y2.view(np.uint16), host(y).view(np.uint16))
 

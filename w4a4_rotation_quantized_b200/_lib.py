@@ -16,7 +16,8 @@ QR_CHAN_DIVIDE, QR_CHAN_MULTIPLY = 0, 1
 
 EXPORTED = ("qr_abi_version", "qr_status_string", "qr_packed_k", "qr_rotate_quant",
             "qr_pack_weights", "qr_w4a4_linear", "qr_select_outliers",
-            "qr_invert_transpose", "qr_device_status")
+            "qr_invert_transpose", "qr_device_status", "qr_rotate_quant_asym",
+            "qr_weight_code_sums", "qr_w4a4_linear_asym")
 
 
 class QrRotation(ctypes.Structure):
@@ -66,6 +67,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qr_select_outliers": (ctypes.c_int, [vp, i64, i64, i64, i32, vp, vp]),
         "qr_invert_transpose": (ctypes.c_int, [vp, i32, vp, vp, vp]),
         "qr_device_status": (ctypes.c_int, [ctypes.POINTER(i32)]),
+        "qr_rotate_quant_asym": (ctypes.c_int, [rot_p, vp, i64, i64, i64, vp, i32, vp, vp, vp, vp,
+                                                vp, vp]),
+        "qr_weight_code_sums": (ctypes.c_int, [vp, i64, i64, vp, vp]),
+        "qr_w4a4_linear_asym": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, i32,
+                                               vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -123,6 +129,31 @@ def qr_w4a4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K_p, x_out, w_out
                                n_out, Y, ldy, acc_debug, stream)
     if check:
         _check("qr_w4a4_linear", st)
+    return st
+
+
+def qr_rotate_quant_asym(rot, X, M, K, ldx, outlier_idx, n_out, codes, scales, zeros, x_out,
+                         x_rot_debug, stream, *, check=True):
+    st = load().qr_rotate_quant_asym(ctypes.byref(rot), X, M, K, ldx, outlier_idx, n_out, codes,
+                                     scales, zeros, x_out, x_rot_debug, stream)
+    if check:
+        _check("qr_rotate_quant_asym", st)
+    return st
+
+
+def qr_weight_code_sums(w_codes, N, K_p, w_sums, stream, *, check=True):
+    st = load().qr_weight_code_sums(w_codes, N, K_p, w_sums, stream)
+    if check:
+        _check("qr_weight_code_sums", st)
+    return st
+
+
+def qr_w4a4_linear_asym(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, M, N, K_p, x_out,
+                        w_out, n_out, Y, ldy, acc_debug, stream, *, check=True):
+    st = load().qr_w4a4_linear_asym(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, M, N,
+                                    K_p, x_out, w_out, n_out, Y, ldy, acc_debug, stream)
+    if check:
+        _check("qr_w4a4_linear_asym", st)
     return st
 
 

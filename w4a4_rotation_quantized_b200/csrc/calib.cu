@@ -1,5 +1,7 @@
-// calib.cu -- offline helpers: QUIK outlier-column selection and the inverse
-// transpose of a Kronecker factor.  Both run once per layer, in one CTA.
+// calib.cu -- offline helpers: QUIK outlier-column selection, the inverse
+// transpose of a Kronecker factor (both once per layer, in one CTA), and the
+// per-row sums of packed weight codes that the asymmetric-activation
+// epilogue needs.
 #include <cuda_fp16.h>
 
 #include "qr_internal.h"
@@ -144,7 +146,41 @@ __global__ void __launch_bounds__(kInvThreads) invert_transpose_kernel(
   if (tid == 0) *info = 0;
 }
 
+// Row sums of packed signed 4-bit codes: sums[row] = sum_k q[row, k].  With
+// asymmetric activations s_a (q_a - z_a) the GEMM's integer product of the
+// stored codes needs - z_a * sums[n] (QUIK §1: activations asymmetric per
+// token).  One warp per row, 16 bytes (32 codes) per lane per step.
+__global__ void __launch_bounds__(256) code_row_sums_kernel(const uint8_t* __restrict__ codes,
+                                                            int64_t rows, int64_t row_bytes,
+                                                            int32_t* __restrict__ sums) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const uint8_t* r = codes + row * row_bytes;
+  int32_t acc = 0;
+  for (int64_t b = 16 * lane; b < row_bytes; b += 16 * 32) {
+    const uint4 u = *reinterpret_cast<const uint4*>(r + b);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)                       // sign-extend each nibble
+        acc += static_cast<int32_t>(w[i] << (28 - 4 * j)) >> 28;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) sums[row] = acc;
+}
+
 }  // namespace
+
+qr_status launch_code_row_sums(const uint8_t* codes, int64_t rows, int64_t kp, int32_t* sums,
+                               cudaStream_t stream) {
+  if (rows == 0) return QR_OK;
+  const int64_t blocks = (rows + 7) / 8;
+  code_row_sums_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(codes, rows, kp / 2, sums);
+  return cudaGetLastError() == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+}
 
 qr_status launch_select_outliers(const uint16_t* x, int64_t T, int64_t K, int64_t ld, int32_t k,
                                  int32_t* idx_out, cudaStream_t stream) {

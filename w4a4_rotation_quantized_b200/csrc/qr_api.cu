@@ -99,7 +99,8 @@ static int64_t packed_k(const qr_rotation* rot, int64_t K, int32_t n_out) {
 
 static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t rows, int64_t K,
                            int64_t ld, const int32_t* outlier_idx, int32_t n_out, uint8_t* codes,
-                           float* scales, uint16_t* out16, float* rot_debug, qr_stream stream) {
+                           float* scales, int32_t* zeros, uint16_t* out16, float* rot_debug,
+                           qr_stream stream) {
   if (rot == nullptr || rows < 0 || K < 0 || n_out < 0 || n_out > K) return QR_ERR_INVALID_ARG;
   const int64_t kp = packed_k(rot, K, n_out);
   if (kp < 0) {
@@ -119,6 +120,7 @@ static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t 
     if (rot->kind != QR_ROT_HADAMARD && rot->kind != QR_ROT_GSR) return QR_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(rot->signs) % 8 != 0) return QR_ERR_ALIGNMENT;
   }
+  if (zeros != nullptr && rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
   RowJob job{};
   job.src = src;
   job.rows = rows;
@@ -131,6 +133,7 @@ static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t 
   job.rot = rot;
   job.codes = codes;
   job.scales = scales;
+  job.zeros = zeros;
   job.out16 = n_out > 0 ? out16 : nullptr;
   job.rot_debug = rot_debug;
   return launch_rotate_quant(job, reinterpret_cast<cudaStream_t>(stream));
@@ -163,21 +166,44 @@ int64_t qr_packed_k(const qr_rotation* rot, int64_t K, int32_t n_out) {
 qr_status qr_rotate_quant(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
                           int64_t ldx, const int32_t* outlier_idx, int32_t n_out, uint8_t* codes,
                           float* scales, uint16_t* x_out, float* x_rot_debug, qr_stream stream) {
-  return rows_call(rot, X, M, K, ldx, outlier_idx, n_out, codes, scales, x_out, x_rot_debug,
-                   stream);
+  return rows_call(rot, X, M, K, ldx, outlier_idx, n_out, codes, scales, nullptr, x_out,
+                   x_rot_debug, stream);
+}
+
+qr_status qr_rotate_quant_asym(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                               int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
+                               uint8_t* codes, float* scales, int32_t* zeros, uint16_t* x_out,
+                               float* x_rot_debug, qr_stream stream) {
+  if (zeros == nullptr && M > 0) return QR_ERR_INVALID_ARG;
+  return rows_call(rot, X, M, K, ldx, outlier_idx, n_out, codes, scales, zeros, x_out,
+                   x_rot_debug, stream);
 }
 
 qr_status qr_pack_weights(const qr_rotation* rot_w, const uint16_t* W, int64_t N, int64_t K,
                           int64_t ldw, const int32_t* outlier_idx, int32_t n_out, uint8_t* w_codes,
                           float* w_scales, uint16_t* w_out, float* w_rot_debug, qr_stream stream) {
-  return rows_call(rot_w, W, N, K, ldw, outlier_idx, n_out, w_codes, w_scales, w_out, w_rot_debug,
-                   stream);
+  return rows_call(rot_w, W, N, K, ldw, outlier_idx, n_out, w_codes, w_scales, nullptr, w_out,
+                   w_rot_debug, stream);
 }
 
-qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales, const uint8_t* w_codes,
-                         const float* w_scales, int64_t M, int64_t N, int64_t K_p,
-                         const uint16_t* x_out, const uint16_t* w_out, int32_t n_out, uint16_t* Y,
-                         int64_t ldy, int32_t* acc_debug, qr_stream stream) {
+qr_status qr_weight_code_sums(const uint8_t* w_codes, int64_t N, int64_t K_p, int32_t* w_sums,
+                              qr_stream stream) {
+  if (N < 0 || K_p < 0 || K_p % 128 != 0) return QR_ERR_INVALID_ARG;
+  if (N == 0) return QR_OK;
+  if (w_sums == nullptr || (K_p > 0 && w_codes == nullptr)) return QR_ERR_INVALID_ARG;
+  if (K_p > 0 && !aligned16(w_codes)) return QR_ERR_ALIGNMENT;
+  return launch_code_row_sums(w_codes, N, K_p, w_sums, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace qr {
+
+static qr_status linear_call(const uint8_t* a_codes, const float* a_scales, const int32_t* a_zeros,
+                             const uint8_t* w_codes, const float* w_scales, const int32_t* w_sums,
+                             int64_t M, int64_t N, int64_t K_p, const uint16_t* x_out,
+                             const uint16_t* w_out, int32_t n_out, uint16_t* Y, int64_t ldy,
+                             int32_t* acc_debug, qr_stream stream) {
   if (M < 0 || N < 0 || K_p < 0 || n_out < 0) return QR_ERR_INVALID_ARG;
   if (K_p % 128 != 0) return QR_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return QR_OK;
@@ -192,8 +218,10 @@ qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales, const ui
   GemmJob j{};
   j.a_codes = a_codes;
   j.a_scales = a_scales;
+  j.a_zeros = a_zeros;
   j.w_codes = w_codes;
   j.w_scales = w_scales;
+  j.w_sums = w_sums;
   j.M = M;
   j.N = N;
   j.Kp = K_p;
@@ -204,6 +232,29 @@ qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales, const ui
   j.ldy = ldy;
   j.acc_debug = acc_debug;
   return launch_w4a4_gemm(j, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace qr
+
+extern "C" {
+
+qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales, const uint8_t* w_codes,
+                         const float* w_scales, int64_t M, int64_t N, int64_t K_p,
+                         const uint16_t* x_out, const uint16_t* w_out, int32_t n_out, uint16_t* Y,
+                         int64_t ldy, int32_t* acc_debug, qr_stream stream) {
+  return linear_call(a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, M, N, K_p, x_out,
+                     w_out, n_out, Y, ldy, acc_debug, stream);
+}
+
+qr_status qr_w4a4_linear_asym(const uint8_t* a_codes, const float* a_scales,
+                              const int32_t* a_zeros, const uint8_t* w_codes,
+                              const float* w_scales, const int32_t* w_sums, int64_t M, int64_t N,
+                              int64_t K_p, const uint16_t* x_out, const uint16_t* w_out,
+                              int32_t n_out, uint16_t* Y, int64_t ldy, int32_t* acc_debug,
+                              qr_stream stream) {
+  if (M > 0 && N > 0 && (a_zeros == nullptr || w_sums == nullptr)) return QR_ERR_INVALID_ARG;
+  return linear_call(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, M, N, K_p, x_out,
+                     w_out, n_out, Y, ldy, acc_debug, stream);
 }
 
 qr_status qr_select_outliers(const uint16_t* X_calib, int64_t T, int64_t K, int64_t ldx,

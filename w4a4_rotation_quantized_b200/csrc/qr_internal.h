@@ -30,6 +30,7 @@ struct RowJob {
   const qr_rotation* rot;
   uint8_t* codes;             // [rows x Kp/2]
   float* scales;              // [rows]
+  int32_t* zeros;             // [rows] zero points (asymmetric activations) or null
   uint16_t* out16;            // [rows x n_out] or null
   float* rot_debug;           // [rows x Kp] or null
 };
@@ -43,7 +44,9 @@ qr_status launch_kron_tc(const RowJob& job, cudaStream_t stream);
 
 struct GemmJob {
   const uint8_t* a_codes; const float* a_scales;
+  const int32_t* a_zeros;     // asymmetric activations: zero points [M], else null
   const uint8_t* w_codes; const float* w_scales;
+  const int32_t* w_sums;      // with a_zeros: per weight row, the sum of its codes [N]
   int64_t M, N, Kp;
   const uint16_t* x_out; const uint16_t* w_out; int32_t n_out;
   uint16_t* Y; int64_t ldy;
@@ -68,6 +71,9 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
 
 qr_status launch_select_outliers(const uint16_t* x, int64_t T, int64_t K, int64_t ld,
                                  int32_t k, int32_t* idx_out, cudaStream_t stream);
+
+qr_status launch_code_row_sums(const uint8_t* codes, int64_t rows, int64_t kp, int32_t* sums,
+                               cudaStream_t stream);
 
 qr_status launch_invert_transpose(const float* P, int32_t n, float* out, int32_t* info,
                                   cudaStream_t stream);

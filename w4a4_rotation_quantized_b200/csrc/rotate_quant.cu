@@ -43,9 +43,11 @@ constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
 // product; the integer then sits in the low mantissa bits, and its low four
 // bits are its two's-complement nibble.
 template <bool CLIP>
-__device__ __forceinline__ uint32_t quant_nibble(float v, float r) {
-  float t = fmaf(v, r, kRoundMagic);
-  if (CLIP) t = fminf(fmaxf(t, kRoundMagic - 7.0f), kRoundMagic + 7.0f);
+__device__ __forceinline__ uint32_t quant_nibble(float v, float r, float c = kRoundMagic,
+                                                 float lo = kRoundMagic - 7.0f,
+                                                 float hi = kRoundMagic + 7.0f) {
+  float t = fmaf(v, r, c);
+  if (CLIP) t = fminf(fmaxf(t, lo), hi);
   return __float_as_uint(t) & 0xFu;
 }
 
@@ -62,16 +64,18 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // byte permutes gather the even and the odd codes, and one shift and one
 // 3-input logic op interleave their nibbles.
 template <bool CLIP>
-__device__ __forceinline__ uint32_t quant_word(const float (&v)[8], float r) {
+__device__ __forceinline__ uint32_t quant_word(const float (&v)[8], float r, float c = kRoundMagic,
+                                               float lo = kRoundMagic - 7.0f,
+                                               float hi = kRoundMagic + 7.0f) {
   uint32_t b[8];
-  const uint64_t r2 = f2_pack(r, r), c2 = f2_pack(kRoundMagic, kRoundMagic);
+  const uint64_t r2 = f2_pack(r, r), c2 = f2_pack(c, c);
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     float t0, t1;
     f2_unpack(f2_fma(f2_pack(v[i], v[i + 1]), r2, c2), t0, t1);
     if (CLIP) {
-      t0 = fminf(fmaxf(t0, kRoundMagic - 7.0f), kRoundMagic + 7.0f);
-      t1 = fminf(fmaxf(t1, kRoundMagic - 7.0f), kRoundMagic + 7.0f);
+      t0 = fminf(fmaxf(t0, lo), hi);
+      t1 = fminf(fmaxf(t1, lo), hi);
     }
     b[i] = __float_as_uint(t0);
     b[i + 1] = __float_as_uint(t1);
@@ -140,6 +144,7 @@ struct WhtParams {
   float clip_ratio, inv_sqrt_block;
   uint8_t* codes;
   float* scales;
+  int32_t* zeros;             // asymmetric activations: zero points [rows] (null: symmetric)
   __half* out16;
   float* rot_debug;
   int32_t off_buf, buf_bytes, off_red, off_kept, off_idx;   // shared-memory carve-up
@@ -220,6 +225,47 @@ __device__ __forceinline__ int swz(int e) {
   return e + ((e >> SH) << 3);
 }
 
+// Per-row quantizer: codes are the low nibble of fma(v, r, c) clamped to
+// [lo, hi] (CLIP).  Symmetric (min-max over [-7, 7]): c = 1.5*2^23, bounds
+// +-7.  Asymmetric (QUIK's per-token activations, min-max over [0, 15]
+// stored as q - 8): c = 1.5*2^23 + z - 8, bounds [-8, 7], and the kernels
+// always clamp.  v are the unnormalized transform outputs; inv_sqrt folds
+// the 1/sqrt(b) of the rotation into the scale.
+struct RowQ { float r, c, lo, hi; };
+
+__device__ __forceinline__ RowQ sym_row_q(float am, float clip, float inv_sqrt, float* scale_out) {
+  if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 7.0f;
+  return RowQ{(am > 0.0f) ? 7.0f / (clip * am) : 0.0f, kRoundMagic, kRoundMagic - 7.0f,
+              kRoundMagic + 7.0f};
+}
+
+__device__ __forceinline__ RowQ asym_row_q(float mn, float mx, float clip, float inv_sqrt,
+                                           float* scale_out, int32_t* zero_out) {
+  const float lo = clip * mn, hi = clip * mx;
+  const float range = hi - lo;
+  const float r = range > 0.0f ? 15.0f / range : 0.0f;
+  const float z = range > 0.0f ? rintf(-lo * r) : 0.0f;
+  if (scale_out != nullptr) {
+    *scale_out = range * inv_sqrt / 15.0f;
+    *zero_out = static_cast<int32_t>(z) - 8;
+  }
+  return RowQ{r, kRoundMagic + (z - 8.0f), kRoundMagic - 8.0f, kRoundMagic + 7.0f};
+}
+
+// Maximum over a row group (any sign).
+__device__ __forceinline__ float row_max(float v, float* red, int rg, int t, int nt) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int nw = nt >> 5;
+  if (nw > 1) {
+    if ((t & 31) == 0) red[t >> 5] = v;
+    row_barrier(rg, nt);
+    v = -INFINITY;
+    for (int w = 0; w < nw; ++w) v = fmaxf(v, red[w]);
+  }
+  return v;
+}
+
 // Reduce a row's absmax over its row group; returns the maximum.
 __device__ __forceinline__ float row_absmax(float am, float* red, int rg, int t, int nt) {
 #pragma unroll
@@ -288,7 +334,7 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
   if (p.n_out > 0) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
                                     reinterpret_cast<int32_t*>(smem + p.off_idx));
   float* buf = reinterpret_cast<float*>(smem + p.off_buf + static_cast<size_t>(rg) * p.buf_bytes);
-  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 16;
+  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 32;
   const int items_a = p.nb * TA, items_b = p.nb * TB;
 
   // Ring mode: the CTA owns rows [row0, row1); a producer warp (after the
@@ -415,10 +461,26 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
 #pragma unroll
       for (int j = 0; j < EB; ++j) am = fmaxf(am, fabsf(v[k][j]));
     }
-    am = row_absmax(am, red, rg, t, nt);
-    const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
-    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
-    if (t == 0) p.scales[row] = s;
+    RowQ q;
+    if (p.zeros == nullptr) {
+      am = row_absmax(am, red, rg, t, nt);
+      q = sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
+    } else {
+      float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+      for (int k = 0; k < ITEMS; ++k)
+        if (t + k * nt < items_b)
+#pragma unroll
+          for (int j = 0; j < EB; ++j) {
+            mx = fmaxf(mx, v[k][j]);
+            mn = fminf(mn, v[k][j]);
+          }
+      mx = row_max(mx, red, rg, t, nt);
+      mn = -row_max(-mn, red + 16, rg, t, nt);
+      q = asym_row_q(mn, mx, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr,
+                     p.zeros + row);
+    }
+    const float r = q.r;
     uint8_t* crow = p.codes + row * (p.Kp >> 1);
 
     if (p.rot_debug != nullptr) {
@@ -457,7 +519,7 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
           float q8[8];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) q8[jj] = v[k][8 * wb + jj];
-          uint32_t W = quant_word<CLIP>(q8, r);
+          uint32_t W = quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
           // Transpose the 8x8 nibble block held by the lanes with tb_low =
           // 0..7: swap 16-bit halves with lane^4, bytes with lane^2 (byte
           // permutes), nibbles with lane^1 (rotate + 3-input logic op).
@@ -487,7 +549,7 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
           const int p1 = a0, p2 = a1 ^ a0, p3 = a2 ^ p2;   // p_{LB-1}, p_{LB-2}, p_{LB-3}
           uint32_t nib[EB];
 #pragma unroll
-          for (int j = 0; j < EB; ++j) nib[j] = quant_nibble<CLIP>(v[k][j], r);
+          for (int j = 0; j < EB; ++j) nib[j] = quant_nibble<CLIP>(v[k][j], r, q.c, q.lo, q.hi);
 #pragma unroll
           for (int f = 0; f < (1 << (MB - 3)); ++f) {
             const int kw = f | (p3 << (MB - 3)) | (p2 << (MB - 2)) | (p1 << (MB - 1));
@@ -519,7 +581,7 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
               const int rev = static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - LB));
               n = gray_inverse(rev);
             }
-            cb[(blk << LB) + n] = static_cast<uint8_t>(quant_nibble<CLIP>(v[k][j], r));
+            cb[(blk << LB) + n] = static_cast<uint8_t>(quant_nibble<CLIP>(v[k][j], r, q.c, q.lo, q.hi));
           }
         }
       }
@@ -554,7 +616,7 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
   uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
   if (p.n_out > 0) build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept,
                                     reinterpret_cast<int32_t*>(smem + p.off_idx));
-  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 16;
+  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 32;
   const int lb = p.lb;
   const int ngroups = p.Kp >> 3;
   const int64_t row_step = static_cast<int64_t>(gridDim.x) * p.rows_per_cta;
@@ -591,10 +653,26 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
         am = fmaxf(am, fabsf(x[i]));
       }
     }
-    am = row_absmax(am, red, rg, t, nt);
-    const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
-    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
-    if (t == 0) p.scales[row] = s;
+    RowQ q;
+    if (p.zeros == nullptr) {
+      am = row_absmax(am, red, rg, t, nt);
+      q = sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
+    } else {
+      float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+      for (int k = 0; k < ITEMS; ++k)
+        if (t + k * nt < ngroups)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            mx = fmaxf(mx, v[k][i]);
+            mn = fminf(mn, v[k][i]);
+          }
+      mx = row_max(mx, red, rg, t, nt);
+      mn = -row_max(-mn, red + 16, rg, t, nt);
+      q = asym_row_q(mn, mx, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr,
+                     p.zeros + row);
+    }
+    const float r = q.r;
     uint8_t* crow = p.codes + row * (p.Kp >> 1);
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
@@ -609,7 +687,7 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
             const int rev = static_cast<int>(__brev(static_cast<unsigned>(i & bm)) >> (32 - lb));
             pos = (i & ~bm) + gray_inverse(rev);
           }
-          W |= quant_nibble<CLIP>(v[k][i], r) << (4 * pos);
+          W |= quant_nibble<CLIP>(v[k][i], r, q.c, q.lo, q.hi) << (4 * pos);
           if (p.rot_debug != nullptr) p.rot_debug[row * p.Kp + 8 * g + pos] = v[k][i] * p.inv_sqrt_block;
         }
         *reinterpret_cast<uint32_t*>(crow + 4 * g) = W;
@@ -646,6 +724,7 @@ struct FewRowsParams {
   float clip_ratio, inv_sqrt_block;
   uint8_t* codes;
   float* scales;
+  int32_t* zeros;             // asymmetric activations: zero points [rows] (null: symmetric)
   __half* out16;
   float* rot_debug;
 };
@@ -682,14 +761,15 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* sh) {
   return (w > 0 ? sh[w - 1] : 0) + x - v;
 }
 
-// Maximum over the block; `sh` holds 32 floats.  Contains two __syncthreads.
+// Maximum over the block (any sign); `sh` holds 32 floats.  Contains two
+// __syncthreads.
 __device__ __forceinline__ float block_max(float v, float* sh) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   if (lane == 0) sh[w] = v;
   __syncthreads();
-  float m = 0.0f;
+  float m = -INFINITY;
   for (int i = 0; i < nw; ++i) m = fmaxf(m, sh[i]);
   __syncthreads();
   return m;
@@ -738,14 +818,14 @@ __device__ __forceinline__ float wht_smem_pass(float* buf, int Kp, int s) {
   return am;
 }
 
-template <bool CLIP>
-__global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams p) {
+template <bool CLIP, bool ASYM, bool SIGNS>
+__global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   float* buf = reinterpret_cast<float*>(smem);                       // [span], few_swz order
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);   // outlier bitmap
   int* scan = reinterpret_cast<int*>(smem + p.off_scan);             // 32 ints
   float* red = reinterpret_cast<float*>(smem + p.off_scan + 128);    // 32 floats
-  float* maxima = reinterpret_cast<float*>(smem + p.off_scan + 256); // CL floats
+  float* maxima = reinterpret_cast<float*>(smem + p.off_scan + 256); // 2 x CL floats
   const int t = threadIdx.x, nthr = blockDim.x;
   const int64_t row = blockIdx.x / p.cl;
   const int cr = blockIdx.x % p.cl;                                  // rank in the cluster
@@ -812,7 +892,7 @@ __global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams 
         ++before;
       } else if (col0 + i < p.K && e < p.Kr && e >= e_lo && e < e_hi) {
         float xv = x[i];
-        if (p.signs != nullptr && __ldg(p.signs + e) < 0) xv = -xv;
+        if (SIGNS && __ldg(p.signs + e) < 0) xv = -xv;
         buf[few_swz(e - e_lo)] = xv;
       }
     }
@@ -828,19 +908,37 @@ __global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams 
   }
   if (p.lb == 0)
     for (int e = t; e < nloc; e += nthr) am = fmaxf(am, fabsf(buf[e]));
-  am = block_max(am, red);
-  if (p.cl > 1) {
-    // every CTA of the row stores its span's maximum into every CTA
-    if (t < p.cl)
-      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(mapa_shared(smem_u32(maxima + cr), t)),
-                   "f"(am)
-                   : "memory");
-    cluster_sync();
-    for (int i = 0; i < p.cl; ++i) am = fmaxf(am, maxima[i]);
+  // symmetric: the span's absmax; asymmetric: its max and -min
+  float m0 = am, m1 = 0.0f;
+  if (ASYM) {
+    m0 = -INFINITY;
+    m1 = -INFINITY;
+    for (int e = t; e < nloc; e += nthr) {
+      m0 = fmaxf(m0, buf[e]);
+      m1 = fmaxf(m1, -buf[e]);
+    }
+    m1 = block_max(m1, red);
   }
-  const float s = (p.clip_ratio * (am * p.inv_sqrt_block)) / 7.0f;
-  const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
-  if (t == 0 && cr == 0) p.scales[row] = s;
+  m0 = block_max(m0, red);
+  if (p.cl > 1) {
+    // every CTA of the row stores its span's maxima into every CTA
+    if (t < p.cl) {
+      const uint32_t dst = mapa_shared(smem_u32(maxima + cr), t);
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst), "f"(m0) : "memory");
+      if (ASYM) asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst + 32u), "f"(m1) : "memory");
+    }
+    cluster_sync();
+    for (int i = 0; i < p.cl; ++i) {
+      m0 = fmaxf(m0, maxima[i]);
+      if (ASYM) m1 = fmaxf(m1, maxima[8 + i]);
+    }
+  }
+  const bool lead = t == 0 && cr == 0;
+  const RowQ q = !ASYM
+                     ? sym_row_q(m0, p.clip_ratio, p.inv_sqrt_block, lead ? p.scales + row : nullptr)
+                     : asym_row_q(-m1, m0, p.clip_ratio, p.inv_sqrt_block,
+                                  lead ? p.scales + row : nullptr, p.zeros + row);
+  const float r = q.r;
   uint8_t* crow = p.codes + row * (p.Kp >> 1);
   const int bm = (1 << p.lb) - 1;
   for (int g = t; g < (nloc >> 3); g += nthr) {
@@ -860,7 +958,7 @@ __global__ void __launch_bounds__(1024) wht_few_rows_kernel(const FewRowsParams 
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
       v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
-    *reinterpret_cast<uint32_t*>(crow + ((e_lo + el) >> 1)) = quant_word<CLIP>(v, r);
+    *reinterpret_cast<uint32_t*>(crow + ((e_lo + el) >> 1)) = quant_word<CLIP>(v, r, q.c, q.lo, q.hi);
     if (p.rot_debug != nullptr)
 #pragma unroll
       for (int i = 0; i < 8; ++i) p.rot_debug[row * p.Kp + e_lo + el + i] = v[i] * p.inv_sqrt_block;
@@ -1144,6 +1242,7 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
   p.inv_sqrt_block = static_cast<float>(1.0 / std::sqrt(static_cast<double>(block)));
   p.codes = job.codes;
   p.scales = job.scales;
+  p.zeros = job.zeros;
   p.out16 = reinterpret_cast<__half*>(job.out16);
   p.rot_debug = job.rot_debug;
   // CTAs per row: up to 8 (and the SMs left per row), each a span of whole
@@ -1166,7 +1265,17 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
   p.off_scan = static_cast<int32_t>(off);
   off += 512;                                  // scan words, block maxima, cluster maxima
   if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
-  auto k = rot.clip_ratio < 1.0f ? wht_few_rows_kernel<true> : wht_few_rows_kernel<false>;
+  // asymmetric codes always clamp (their bounds are [-8, 7])
+  using Kfn = void (*)(FewRowsParams);
+  Kfn k;
+  if (p.signs != nullptr)
+    k = job.zeros != nullptr    ? wht_few_rows_kernel<true, true, true>
+        : rot.clip_ratio < 1.0f ? wht_few_rows_kernel<true, false, true>
+                                : wht_few_rows_kernel<false, false, true>;
+  else
+    k = job.zeros != nullptr    ? wht_few_rows_kernel<true, true, false>
+        : rot.clip_ratio < 1.0f ? wht_few_rows_kernel<true, false, false>
+                                : wht_few_rows_kernel<false, false, false>;
   cudaError_t e = set_smem(k, off);
   if (e != cudaSuccess) return QR_ERR_CUDA;
   cudaLaunchConfig_t cfg{};
@@ -1208,6 +1317,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.inv_sqrt_block = static_cast<float>(1.0 / std::sqrt(static_cast<double>(block)));
   p.codes = job.codes;
   p.scales = job.scales;
+  p.zeros = job.zeros;
   p.out16 = reinterpret_cast<__half*>(job.out16);
   p.rot_debug = job.rot_debug;
   if (job.Kp > 32768) return QR_ERR_UNSUPPORTED;
@@ -1240,7 +1350,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
 
   size_t off = 0;
   p.off_red = static_cast<int32_t>(off);
-  off = align_up(off + sizeof(float) * 16 * R, 16);
+  off = align_up(off + sizeof(float) * 32 * R, 16);
   p.off_buf = static_cast<int32_t>(off);
   // fp32 row buffer with the layout-B padding: 8 floats after every 8*eb
   // elements (swz<3 + MB>), plus 8 spare
@@ -1270,7 +1380,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
     int groups = static_cast<int>(std::min<int64_t>(max_groups, per_block));
     while (groups > 1 && groups * nt + 32 > bound) --groups;
     // layout: red | row-group buffers | ring slots | barriers
-    size_t roff = align_up(sizeof(float) * 16 * groups, 16);
+    size_t roff = align_up(sizeof(float) * 32 * groups, 16);
     const size_t buf_off = roff;
     roff = align_up(roff + static_cast<size_t>(p.buf_bytes) * groups, 128);
     const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - static_cast<int64_t>(roff) -
@@ -1295,7 +1405,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
     }
   }
   const int threads = ring ? p.rows_per_cta * nt + 32 : R * nt;
-  const bool clip = rot.clip_ratio < 1.0f;
+  const bool clip = rot.clip_ratio < 1.0f || job.zeros != nullptr;   // asymmetric codes clamp
   cudaError_t e;
   if (small)
     e = clip ? dispatch_small<true>(items, p, threads, off, stream)

@@ -52,6 +52,8 @@ constexpr int kSmemBudget = 227 * 1024;
 struct DecodeParams {
   const float* w_scales;           // [N]
   const float* a_scales;           // [M]
+  const int32_t* a_zeros;          // asymmetric activations: zero point per token [M], else null
+  const int32_t* w_sums;           // with a_zeros: code sum per weight row [N]
   __half* Y;
   int64_t ldy;
   int32_t* acc_debug;              // [M x N] or null
@@ -118,7 +120,7 @@ __device__ __forceinline__ StepRange step_range(int r, int ks, int kt, int ot) {
   return StepRange{i0, min(kt, i0 + q), 0, 0};
 }
 
-template <int BN, bool OUT>
+template <int BN, bool OUT, bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
                         const __grid_constant__ CUtensorMap map_x,
@@ -315,6 +317,8 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     // scales, loaded while the MMAs run: this row's, and one token's per lane
     // for each 32-token chunk (broadcast by shuffles in the epilogue)
     const int n = y_w + lrow;                      // output column = weight row
+    // asymmetric activations: acc - 256 * zero[m] * w_sum[n] (the accumulator is 256 x)
+    constexpr bool asym = ASYM;
     float s_row = 0.0f, sa_lane[BN / 32];
     if (owner == rank) {
       s_row = n < p.N ? __ldg(p.w_scales + n) * (1.0f / 256.0f) : 0.0f;
@@ -364,6 +368,10 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
         uint32_t acc[32];
         uint32_t oacc[32];
         const float sa_c = c == 0 ? sa_lane[0] : sa_lane[BN / 32 - 1];   // BN <= 64
+        const float wsum = (asym && n < p.N) ? static_cast<float>(__ldg(p.w_sums + n)) : 0.0f;
+        const float za_c = (asym && c * 32 + lane < p.M)
+                               ? 256.0f * static_cast<float>(__ldg(p.a_zeros + c * 32 + lane))
+                               : 0.0f;
         tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
         if (OUT) tmem_ld_32x32b_x32(tmem_base + lane_off + BN + c * 32, oacc);
         tmem_ld_wait();
@@ -393,9 +401,12 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
         for (int j = 0; j < 32; ++j) {
           const int m = c * 32 + j;
           const float sa = __shfl_sync(0xffffffffu, sa_c, j);
+          const float za = __shfl_sync(0xffffffffu, za_c, j);
           if (m >= p.M || !n_ok) continue;
           const int32_t a = static_cast<int32_t>(acc[j]);
-          float y = static_cast<float>(a) * s_row * sa;
+          float af = static_cast<float>(a);
+          if (asym) af = fmaf(-za, wsum, af);
+          float y = af * s_row * sa;
           if (has_out) y += __uint_as_float(oacc[j]);
           p.Y[static_cast<int64_t>(m) * p.ldy + n] = __float2half_rn(y);
           if (p.acc_debug != nullptr) p.acc_debug[static_cast<int64_t>(m) * p.N + n] = a >> 8;
@@ -413,11 +424,11 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   }
 }
 
-template <int BN, bool OUT>
+template <int BN, bool OUT, bool ASYM>
 cudaError_t run_decode(const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& mwo,
                        const CUtensorMap& mxo, const DecodeParams& p, int tiles,
                        cudaStream_t stream) {
-  auto k = w4a4_gemm_decode_kernel<BN, OUT>;
+  auto k = w4a4_gemm_decode_kernel<BN, OUT, ASYM>;
   const int smem = DecodeLayout<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -455,6 +466,8 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
   DecodeParams p{};
   p.w_scales = j.w_scales;
   p.a_scales = j.a_scales;
+  p.a_zeros = j.a_zeros;
+  p.w_sums = j.w_sums;
   p.Y = reinterpret_cast<__half*>(j.Y);
   p.ldy = j.ldy;
   p.acc_debug = j.acc_debug;
@@ -483,10 +496,13 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
   }
   const int t = static_cast<int>(tiles);
   cudaError_t e;
-  if (bn == 32) e = out ? run_decode<32, true>(mw, mx, mwo, mxo, p, t, stream)
-                        : run_decode<32, false>(mw, mx, mwo, mxo, p, t, stream);
-  else e = out ? run_decode<64, true>(mw, mx, mwo, mxo, p, t, stream)
-               : run_decode<64, false>(mw, mx, mwo, mxo, p, t, stream);
+  const bool asym = p.a_zeros != nullptr;
+#define QR_RUN_DECODE(B, O)                                                        \
+  (asym ? run_decode<B, O, true>(mw, mx, mwo, mxo, p, t, stream)                   \
+        : run_decode<B, O, false>(mw, mx, mwo, mxo, p, t, stream))
+  if (bn == 32) e = out ? QR_RUN_DECODE(32, true) : QR_RUN_DECODE(32, false);
+  else e = out ? QR_RUN_DECODE(64, true) : QR_RUN_DECODE(64, false);
+#undef QR_RUN_DECODE
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
 

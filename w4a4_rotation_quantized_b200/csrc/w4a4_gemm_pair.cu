@@ -71,6 +71,8 @@ constexpr int widened_stages() {
 struct PairParams {
   const float* scale_a;            // per A-side row
   const float* scale_b;            // per B-side row
+  const int32_t* a_zeros;          // asymmetric activations: zero point per row, else null
+  const int32_t* w_sums;           // with a_zeros: code sum per weight row
   __half* Y;
   int64_t ldy;
   int32_t* acc_debug;              // [M x N] or null
@@ -108,7 +110,7 @@ struct PairSmem {
                 "swizzled tiles need 1024-byte alignment");
 };
 
-template <int BN, bool OUT>
+template <int BN, bool OUT, bool ASYM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                       const __grid_constant__ CUtensorMap map_b,
@@ -362,6 +364,9 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
       const int ra = ta * 256 + static_cast<int>(rank) * 128 + lrow;   // A-side row
       const bool ra_ok = ra < p.rows_a;
       const float s_row = ra_ok ? __ldg(p.scale_a + ra) * (1.0f / 256.0f) : 0.0f;
+      // asymmetric activations: acc - 256 * zero * w_sum (the accumulator is 256 x)
+      constexpr bool asym = ASYM;
+      const float zrow = (asym && ra_ok) ? 256.0f * static_cast<float>(__ldg(p.a_zeros + ra)) : 0.0f;
       const uint32_t t_acc = tmem_base + lane_off + buf * kColsAcc;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -390,7 +395,9 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
           for (int t = 0; t < 2; ++t) {
             const int n = cb0 + j + t;
             const float sb = (n < p.rows_b) ? __ldg(p.scale_b + n) : 0.0f;
-            y2[t] = static_cast<float>(static_cast<int32_t>(acc[j + t])) * s_row * sb;
+            float a = static_cast<float>(static_cast<int32_t>(acc[j + t]));
+            if (asym && n < p.rows_b) a = fmaf(-zrow, static_cast<float>(__ldg(p.w_sums + n)), a);
+            y2[t] = a * s_row * sb;
             if (OUT) y2[t] += __uint_as_float(oacc[j + t]);
           }
           const __half2 h2 = __floats2half2_rn(y2[0], y2[1]);
@@ -433,7 +440,8 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
 template <int BN, bool OUT>
 cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& moa,
                      const CUtensorMap& mob, const PairParams& p, cudaStream_t stream) {
-  auto k = w4a4_gemm_pair_kernel<BN, OUT>;
+  auto k = p.a_zeros != nullptr ? w4a4_gemm_pair_kernel<BN, OUT, true>
+                                : w4a4_gemm_pair_kernel<BN, OUT, false>;
   const int smem = PairSmem<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -467,6 +475,8 @@ qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
   PairParams p{};
   p.scale_a = j.a_scales;
   p.scale_b = j.w_scales;
+  p.a_zeros = j.a_zeros;
+  p.w_sums = j.w_sums;
   p.Y = reinterpret_cast<__half*>(j.Y);
   p.ldy = j.ldy;
   p.acc_debug = j.acc_debug;

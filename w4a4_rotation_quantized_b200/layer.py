@@ -88,7 +88,7 @@ def packed_k(rot: Rotation, K: int, n_out: int = 0) -> int:
     return kp
 
 
-def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool):
+def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool, asym: bool = False):
     _need_cuda(x, torch.float16, "input")
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("input must be a 2-D row-major tensor")
@@ -105,6 +105,12 @@ def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool):
     scales = torch.empty(rows, dtype=torch.float32, device=dev)
     out16 = torch.empty((rows, n_out), dtype=torch.float16, device=dev) if n_out else None
     dbg = torch.empty((rows, kp), dtype=torch.float32, device=dev) if debug else None
+    if asym:
+        zeros = torch.empty(rows, dtype=torch.int32, device=dev)
+        fn(crot, x.data_ptr(), rows, K, x.stride(0), _ptr(outlier_idx) if n_out else None, n_out,
+           codes.data_ptr(), scales.data_ptr(), zeros.data_ptr(), _ptr(out16), _ptr(dbg),
+           _stream())
+        return codes, scales, zeros, out16, dbg
     fn(crot, x.data_ptr(), rows, K, x.stride(0), _ptr(outlier_idx) if n_out else None, n_out,
        codes.data_ptr(), scales.data_ptr(), _ptr(out16), _ptr(dbg), _stream())
     return codes, scales, out16, dbg
@@ -113,6 +119,20 @@ def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool):
 def rotate_quant(x, rot: Rotation, outlier_idx=None, debug: bool = False):
     """Online activation path: (codes, scales, x_out, x_rot or None)."""
     return _rows(L.qr_rotate_quant, rot, x, outlier_idx, debug)
+
+
+def rotate_quant_asym(x, rot: Rotation, outlier_idx=None, debug: bool = False):
+    """Online activation path with QUIK's asymmetric per-token quantizer:
+    (codes, scales, zeros, x_out, x_rot or None); x ~= scale * (code - zero)."""
+    return _rows(L.qr_rotate_quant_asym, rot, x, outlier_idx, debug, asym=True)
+
+
+def weight_code_sums(w_codes: torch.Tensor) -> torch.Tensor:
+    """Per weight row, the sum of its packed codes (int32 [N])."""
+    N, kp2 = w_codes.shape
+    sums = torch.empty(N, dtype=torch.int32, device=w_codes.device)
+    L.qr_weight_code_sums(w_codes.data_ptr(), N, 2 * kp2, sums.data_ptr(), _stream())
+    return sums
 
 
 def pack_weights(w, rot_w: Rotation, outlier_idx=None, debug: bool = False):
@@ -135,6 +155,23 @@ def w4a4_linear(a_codes, a_scales, w_codes, w_scales, x_out=None, w_out=None,
     return y, acc
 
 
+def w4a4_linear_asym(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, x_out=None,
+                     w_out=None, out: Optional[torch.Tensor] = None, acc_debug: bool = False):
+    """Y = fp16((acc - zero_a w_sums) * sa * sw + x_out w_out^T) for asymmetric
+    activation codes; returns (Y, acc or None)."""
+    M, kp2 = a_codes.shape
+    N = w_codes.shape[0]
+    n_out = 0 if x_out is None else x_out.shape[1]
+    dev = a_codes.device
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev) if acc_debug else None
+    L.qr_w4a4_linear_asym(a_codes.data_ptr(), a_scales.data_ptr(), a_zeros.data_ptr(),
+                          w_codes.data_ptr(), w_scales.data_ptr(), w_sums.data_ptr(), M, N,
+                          2 * kp2, _ptr(x_out), _ptr(w_out), n_out, y.data_ptr(), y.stride(0),
+                          _ptr(acc), _stream())
+    return y, acc
+
+
 def select_outliers(x_calib: torch.Tensor, k: int) -> torch.Tensor:
     """QUIK calibration: the k columns of largest infinity-norm, ascending."""
     _need_cuda(x_calib, torch.float16, "x_calib")
@@ -148,14 +185,22 @@ def select_outliers(x_calib: torch.Tensor, k: int) -> torch.Tensor:
 class QuantizedLinear:
     """A linear layer held as rotated 4-bit weights; forward() is the online path."""
 
-    def __init__(self, weight: torch.Tensor, rot: Rotation, outlier_idx=None):
+    def __init__(self, weight: torch.Tensor, rot: Rotation, outlier_idx=None,
+                 asym_activations: bool = False):
         self.rot = rot
         self.rot_w = weight_rotation(rot)
         self.outlier_idx = outlier_idx
+        self.asym = asym_activations
         self.w_codes, self.w_scales, self.w_out, _ = pack_weights(weight, self.rot_w, outlier_idx)
+        self.w_sums = weight_code_sums(self.w_codes) if asym_activations else None
         self.out_features, self.in_features = weight.shape
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
+        if self.asym:
+            codes, scales, zeros, x_out, _ = rotate_quant_asym(x, self.rot, self.outlier_idx)
+            y, _ = w4a4_linear_asym(codes, scales, zeros, self.w_codes, self.w_scales, self.w_sums,
+                                    x_out, self.w_out)
+            return y
         codes, scales, x_out, _ = rotate_quant(x, self.rot, self.outlier_idx)
         y, _ = w4a4_linear(codes, scales, self.w_codes, self.w_scales, x_out, self.w_out)
         return y
