@@ -81,6 +81,7 @@ struct PairParams {
   int32_t kt, ot;                  // int4 K steps, outlier steps
   int32_t tiles_a, tiles_b;        // 256-row A tiles, BN-row B tiles
   int32_t y_vec_ok;
+  int32_t y_tma;                   // Y leaves through tensor stores (map_y is valid)
   int32_t* status;
 };
 
@@ -99,15 +100,23 @@ struct PairSmem {
   static constexpr int off_out_b = off_out_a + kNO * kOutA;
   static constexpr int off_pack_a = off_out_b + kNO * kOutB;
   static constexpr int off_pack_b = off_pack_a + kNP * kPackA;
-  static constexpr int off_bar = off_pack_b + kNP * kPackB;
+  // epilogue: per warp, two staging boxes of 32 rows x 32 fp16 columns
+  // (64-byte swizzle, for the tensor store) and the tile's B-side scales
+  // (and, asymmetric, code sums) as floats
+  static constexpr int kYBox = 32 * 64;
+  static constexpr int kSbFloats = 2 * BN;
+  static constexpr int off_ystage = off_pack_b + kNP * kPackB;
+  static constexpr int off_sb = off_ystage + 4 * 2 * kYBox;
+  static constexpr int off_bar = off_sb + 4 * kSbFloats * 4;
   // full_p, empty_p, full_w, empty_w, full_o, full_o2, empty_o,
   // tmem_full[2], tmem_empty[2], drain
   static constexpr int kNumBars = 2 * kNP + 2 * kNW + 3 * kNO + 5;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
   static constexpr int kBytes = off_misc + 16 + 1024;
   static_assert(off_out_a % 1024 == 0 && off_out_b % 1024 == 0 && off_pack_a % 1024 == 0 &&
-                    kPackB % 1024 == 0,
+                    kPackB % 1024 == 0 && off_ystage % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
+  static_assert(kBytes <= 227 * 1024, "shared memory");
 };
 
 template <int BN, bool OUT, bool ASYM>
@@ -115,7 +124,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                       const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_oa,
-                      const __grid_constant__ CUtensorMap map_ob, const PairParams p) {
+                      const __grid_constant__ CUtensorMap map_ob,
+                      const __grid_constant__ CUtensorMap map_y, const PairParams p) {
   using S = PairSmem<BN, OUT>;
   constexpr int kNW = S::kNW;
   static_assert(BN % 32 == 0 && BN >= 32 && kNW >= 2 && S::kWideBlk % 1024 == 0, "tile width");
@@ -351,22 +361,36 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Lane = A-side row (output row m), 32 output columns per chunk.  The
+    // tile's B-side scales sit in a per-warp shared-memory copy (read as
+    // broadcast float4); the fp16 results go to a per-warp 32 x 32 staging
+    // box that one lane hands to a tensor store, double-buffered, so the
+    // warp never issues scattered global stores.
     const int lrow = warp * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tmem_empty0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
-    uint32_t tcount = 0;
+    float* sb_w = reinterpret_cast<float*>(smem + S::off_sb) + warp * S::kSbFloats;
+    uint8_t* ystage = smem + S::off_ystage + warp * 2 * S::kYBox;
+    uint32_t tcount = 0, nbox = 0;
     bool ok = true;
     for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++tcount) {
       const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
       const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
+      __syncwarp();                                // the previous tile's readers are done
+      for (int i = lane; i < BN; i += 32) {
+        const int n = tb * BN + i;
+        const bool n_ok = n < p.rows_b;
+        sb_w[i] = n_ok ? __ldg(p.scale_b + n) : 0.0f;
+        if (ASYM) sb_w[BN + i] = n_ok ? static_cast<float>(__ldg(p.w_sums + n)) : 0.0f;
+      }
+      __syncwarp();
       if (!(ok = mbar_wait_cluster_bounded(&tmem_full[buf], tph, abort_flag, p.status, kDevTimeoutEpilogue))) break;
       tc_fence_after();
       const int ra = ta * 256 + static_cast<int>(rank) * 128 + lrow;   // A-side row
       const bool ra_ok = ra < p.rows_a;
       const float s_row = ra_ok ? __ldg(p.scale_a + ra) * (1.0f / 256.0f) : 0.0f;
       // asymmetric activations: acc - 256 * zero * w_sum (the accumulator is 256 x)
-      constexpr bool asym = ASYM;
-      const float zrow = (asym && ra_ok) ? 256.0f * static_cast<float>(__ldg(p.a_zeros + ra)) : 0.0f;
+      const float zrow = (ASYM && ra_ok) ? 256.0f * static_cast<float>(__ldg(p.a_zeros + ra)) : 0.0f;
       const uint32_t t_acc = tmem_base + lane_off + buf * kColsAcc;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -375,57 +399,79 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
         tmem_ld_32x32b_x32(t_acc + c * 32, acc);
         if (OUT) tmem_ld_32x32b_x32(t_acc + BN + c * 32, oacc);
         tmem_ld_wait();
-        if (p.kt == 0) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[j] = 0;
-        }
-        if (OUT && p.ot == 0) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) oacc[j] = 0;
-        }
-        const int cb0 = tb * BN + c * 32;          // first B-side row of this chunk
-        if (!ra_ok) continue;
-        // lane owns output row m = ra; columns n = cb0 + j
-        __half* yrow = p.Y + static_cast<int64_t>(ra) * p.ldy;
+        const bool kz = p.kt == 0, oz = OUT && p.ot == 0;
+        const int cb0 = tb * BN + c * 32;          // first B-side row (output column) of the chunk
+        const float4* sb4 = reinterpret_cast<const float4*>(sb_w + c * 32);
+        const float4* ws4 = reinterpret_cast<const float4*>(sb_w + BN + c * 32);
         uint32_t hp[16];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float y2[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int n = cb0 + j + t;
-            const float sb = (n < p.rows_b) ? __ldg(p.scale_b + n) : 0.0f;
-            float a = static_cast<float>(static_cast<int32_t>(acc[j + t]));
-            if (asym && n < p.rows_b) a = fmaf(-zrow, static_cast<float>(__ldg(p.w_sums + n)), a);
-            y2[t] = a * s_row * sb;
-            if (OUT) y2[t] += __uint_as_float(oacc[j + t]);
+        for (int q = 0; q < 8; ++q) {
+          const float4 sb = sb4[q];
+          const float sbv[4] = {sb.x, sb.y, sb.z, sb.w};
+          float wsv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if (ASYM) {
+            const float4 w = ws4[q];
+            wsv[0] = w.x; wsv[1] = w.y; wsv[2] = w.z; wsv[3] = w.w;
           }
-          const __half2 h2 = __floats2half2_rn(y2[0], y2[1]);
-          hp[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          float y[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int j = 4 * q + t;
+            float a = kz ? 0.0f : static_cast<float>(static_cast<int32_t>(acc[j]));
+            if (ASYM) a = fmaf(-zrow, wsv[t], a);
+            y[t] = a * s_row * sbv[t];
+            if (OUT && !oz) y[t] += __uint_as_float(oacc[j]);
+          }
+          const __half2 h0 = __floats2half2_rn(y[0], y[1]);
+          const __half2 h1 = __floats2half2_rn(y[2], y[3]);
+          hp[2 * q] = *reinterpret_cast<const uint32_t*>(&h0);
+          hp[2 * q + 1] = *reinterpret_cast<const uint32_t*>(&h1);
         }
-        if (p.y_vec_ok && cb0 + 32 <= p.rows_b) {
+        if (p.y_tma) {
+          // box row = lane: 64 bytes as four 16-byte chunks, chunk index
+          // XOR (row / 2) % 4 (the 64-byte swizzle of the tensor map)
+          uint8_t* box = ystage + (nbox & 1) * S::kYBox;
+          if (lane == 0 && nbox >= 2) bulk_wait_group_read<1>();
+          __syncwarp();
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(yrow + cb0 + 8 * q) =
+            *reinterpret_cast<uint4*>(box + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
                 make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
-        } else {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_y, box, cb0, ta * 256 + static_cast<int>(rank) * 128 + warp * 32);
+            bulk_commit_group();
+          }
+          ++nbox;
+        } else if (ra_ok) {
+          __half* yrow = p.Y + static_cast<int64_t>(ra) * p.ldy;
+          if (p.y_vec_ok && cb0 + 32 <= p.rows_b) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (cb0 + j < p.rows_b)
-              reinterpret_cast<uint16_t*>(yrow)[cb0 + j] =
-                  static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(yrow + cb0 + 8 * q) =
+                  make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (cb0 + j < p.rows_b)
+                reinterpret_cast<uint16_t*>(yrow)[cb0 + j] =
+                    static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
+          }
         }
-        if (p.acc_debug != nullptr) {
+        if (p.acc_debug != nullptr && ra_ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (cb0 + j < p.rows_b)
-              p.acc_debug[static_cast<int64_t>(ra) * p.N + cb0 + j] = static_cast<int32_t>(acc[j]) >> 8;
+              p.acc_debug[static_cast<int64_t>(ra) * p.N + cb0 + j] =
+                  kz ? 0 : static_cast<int32_t>(acc[j]) >> 8;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty0 + buf * 8);
     }
+    if (lane == 0) bulk_wait_group<0>();           // tensor stores done before the CTA ends
   }
 
   tc_fence_before();
@@ -439,14 +485,15 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
 
 template <int BN, bool OUT>
 cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& moa,
-                     const CUtensorMap& mob, const PairParams& p, cudaStream_t stream) {
+                     const CUtensorMap& mob, const CUtensorMap& my, const PairParams& p,
+                     cudaStream_t stream) {
   auto k = p.a_zeros != nullptr ? w4a4_gemm_pair_kernel<BN, OUT, true>
                                 : w4a4_gemm_pair_kernel<BN, OUT, false>;
   const int smem = PairSmem<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int clusters = std::min(p.tiles_a * p.tiles_b, sm_count() / 2);
-  k<<<2 * clusters, kThreads, smem, stream>>>(ma, mb, moa, mob, p);
+  k<<<2 * clusters, kThreads, smem, stream>>>(ma, mb, moa, mob, my, p);
   return cudaGetLastError();
 }
 
@@ -489,6 +536,12 @@ qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
   p.tiles_a = static_cast<int32_t>((j.M + 255) / 256);
   p.tiles_b = static_cast<int32_t>((j.N + bn - 1) / bn);
   p.y_vec_ok = (reinterpret_cast<uintptr_t>(j.Y) % 16 == 0) && (j.ldy % 8 == 0);
+  // Y through tensor stores: boxes of 32 columns x 32 rows, 64-byte swizzle
+  CUtensorMap my{};
+  p.y_tma = p.y_vec_ok &&
+            make_tensor_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.Y, static_cast<uint64_t>(j.N),
+                               static_cast<uint64_t>(j.M), static_cast<uint64_t>(j.ldy) * 2, 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_64B);
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
   CUtensorMap ma{}, mb{}, moa{}, mob{};
@@ -509,10 +562,10 @@ qr_status launch_w4a4_gemm_pair(const GemmJob& j, cudaStream_t stream) {
   }
   cudaError_t e;
   if (out) {
-    e = run_pair<96, true>(ma, mb, moa, mob, p, stream);
+    e = run_pair<96, true>(ma, mb, moa, mob, my, p, stream);
   } else {
-    e = bn == 160 ? run_pair<160, false>(ma, mb, moa, mob, p, stream)
-                  : run_pair<128, false>(ma, mb, moa, mob, p, stream);
+    e = bn == 160 ? run_pair<160, false>(ma, mb, moa, mob, my, p, stream)
+                  : run_pair<128, false>(ma, mb, moa, mob, my, p, stream);
   }
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
