@@ -414,6 +414,25 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
+// 1-D bulk copy from this CTA's shared memory to shared memory of a CTA of
+// the cluster (addresses 16-byte aligned, size a multiple of 16); the bytes
+// are counted on the destination CTA's mbarrier `dst_bar` (a cluster
+// address).  The source must stay untouched until the destination has seen
+// its barrier complete.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* src,
+                                                     uint32_t bytes, uint32_t dst_bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "r"(smem_u32(src)), "r"(bytes), "r"(dst_bar)
+      : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;

@@ -60,6 +60,7 @@ struct DecodeParams {
   int32_t N, M;
   int32_t kt, ot;                  // int4 K steps, outlier steps
   int32_t ks;                      // CTAs splitting K in a cluster
+  int32_t y_tma;                   // Y leaves through tensor stores (map_y is valid)
   int32_t* status;
 };
 
@@ -77,7 +78,8 @@ struct DecodeLayout {
   static constexpr int kMaxKS = BN == 64 ? 2 : 4;
   static constexpr int kRowWords = (OUT ? 2 * BN : BN) + 4;
   static constexpr int kRed = (kMaxKS - 1) * (128 / kMaxKS) * kRowWords * 4;
-  static constexpr int kFixed = kNP * (kPackA + kPackB) + kNO * (kOutA + kOutB) + kRed + 2048;
+  static constexpr int kTok = 2 * BN * 4;                  // token scales (+ 256 x zero points)
+  static constexpr int kFixed = kNP * (kPackA + kPackB) + kNO * (kOutA + kOutB) + kRed + kTok + 2048;
   // tensor memory: int32 accumulator, fp32 outlier accumulator, A stages
   static constexpr int kAcol = OUT ? 2 * BN : BN;
   static constexpr int kNWtmem = (512 - kAcol) / 64;        // 64-column stages (two K steps)
@@ -90,7 +92,14 @@ struct DecodeLayout {
   static constexpr int off_pack_a = off_out_b + kNO * kOutB;
   static constexpr int off_pack_b = off_pack_a + kNP * kPackA;
   static constexpr int off_red = off_pack_b + kNP * kPackB;
-  static constexpr int off_bar = off_red + kRed;
+  static constexpr int off_tok = off_red + kRed;
+  static constexpr int off_bar = off_tok + kTok;
+  // after the main loop the widened-stage area holds the epilogue staging:
+  // the rows this CTA sends (int32 partials and outlier sums, kRowWords per
+  // row), then the fp16 output box [tokens][owned rows] of the tensor store
+  static constexpr int kSendBytes = (128 - 128 / kMaxKS) * kRowWords * 4;
+  static constexpr int off_ybox = (kSendBytes + 1023) / 1024 * 1024;
+  static_assert(off_ybox + BN * 128 * 2 <= kNW * kWideB, "epilogue staging");
   // full_p, empty_p, full_w, empty_w, full_o, empty_o, tmem_full, recv, drain
   static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 * kNO + 3;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
@@ -125,7 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
                         const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_wo,
-                        const __grid_constant__ CUtensorMap map_xo, const DecodeParams p) {
+                        const __grid_constant__ CUtensorMap map_xo,
+                        const __grid_constant__ CUtensorMap map_y, const DecodeParams p) {
   using L = DecodeLayout<BN, OUT>;
   constexpr int kNW = L::kNW;
   constexpr uint32_t kAcol = L::kAcol;
@@ -160,10 +170,13 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     for (int i = 0; i < kNW; ++i) { mbar_init(&full_w[i], 4); mbar_init(&empty_w[i], 1); }
     for (int i = 0; i < kNO; ++i) { mbar_init(&full_o[i], 1); mbar_init(&empty_o[i], 1); }
     mbar_init(tmem_full, 1);
-    mbar_init(recv, p.ks > 1 ? (p.ks - 1) * own_rows : 1);
+    mbar_init(recv, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // the other CTAs' partials of my rows arrive by bulk copies
+    if (p.ks > 1)
+      mbar_arrive_expect_tx(recv, static_cast<uint32_t>((p.ks - 1) * own_rows * L::kRowWords * 4));
   }
   if (warp == kProducerWarp && lane == 0) {
     if (n_int > 0) { tma_prefetch_desc(&map_w); tma_prefetch_desc(&map_x); }
@@ -310,68 +323,82 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Lane = tile row (output column n).  Rows another CTA owns: the int32
+    // partials (and CTA 0's fp32 outlier sums) are staged in this CTA's
+    // shared memory and sent with one bulk copy per warp into the owner's
+    // receive slot.  Owned rows: partials added, dequantized with the token
+    // scales staged in shared memory, written as fp16 into a [token][row]
+    // box that one thread hands to a tensor store.
     const int lrow = warp * 32 + lane;             // tile row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int owner = lrow / own_rows;             // the CTA that finishes this row
     const bool has_out = OUT && p.ot > 0;
-    // scales, loaded while the MMAs run: this row's, and one token's per lane
-    // for each 32-token chunk (broadcast by shuffles in the epilogue)
     const int n = y_w + lrow;                      // output column = weight row
+    float* tok = reinterpret_cast<float*>(smem + L::off_tok);   // [BN] scales, [BN] 256 x zeros
+    if (warp == 0)
+      for (int i = lane; i < BN; i += 32) {
+        tok[i] = i < p.M ? __ldg(p.a_scales + i) : 0.0f;
+        if (ASYM) tok[BN + i] = i < p.M ? 256.0f * static_cast<float>(__ldg(p.a_zeros + i)) : 0.0f;
+      }
+    named_barrier(1, 128);                         // the four epilogue warps
     // asymmetric activations: acc - 256 * zero[m] * w_sum[n] (the accumulator is 256 x)
-    constexpr bool asym = ASYM;
-    float s_row = 0.0f, sa_lane[BN / 32];
-    if (owner == rank) {
-      s_row = n < p.N ? __ldg(p.w_scales + n) * (1.0f / 256.0f) : 0.0f;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
-        sa_lane[c] = c * 32 + lane < p.M ? __ldg(p.a_scales + c * 32 + lane) : 0.0f;
+    float s_row = 0.0f, wsum = 0.0f;
+    if (owner == rank && n < p.N) {
+      s_row = __ldg(p.w_scales + n) * (1.0f / 256.0f);
+      if (ASYM) wsum = static_cast<float>(__ldg(p.w_sums + n));
     }
     bool ok = mbar_wait_bounded(tmem_full, 0, abort_flag, p.status, kDevTimeoutEpilogue);
     tc_fence_after();
     if (owner != rank) {
-      // send this row's partials (int32, and CTA 0's fp32 outlier sums)
-      const int slot = (rank - owner - 1 + p.ks) % p.ks;
-      const uint32_t dst = mapa_shared(smem_u32(slots), static_cast<uint32_t>(owner)) +
-                           4u * static_cast<uint32_t>((slot * own_rows + lrow % own_rows) * L::kRowWords);
+      // rows sent, in order: all rows but the owned block
+      const int srow = lrow < rank * own_rows ? lrow : lrow - own_rows;
+      uint32_t* stg = reinterpret_cast<uint32_t*>(smem + L::off_wide_b) + srow * L::kRowWords;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t acc[32];
         tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
         tmem_ld_wait();
-        if (n_int == 0 || !ok) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[j] = 0;
-        }
+        const bool zero = n_int == 0 || !ok;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          st_cluster_v4(dst + 4u * (c * 32 + 4 * q), acc[4 * q], acc[4 * q + 1], acc[4 * q + 2],
-                        acc[4 * q + 3]);
+          *reinterpret_cast<uint4*>(stg + c * 32 + 4 * q) =
+              zero ? make_uint4(0u, 0u, 0u, 0u)
+                   : make_uint4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
         if (has_out && rank == 0) {
           tmem_ld_32x32b_x32(tmem_base + lane_off + BN + c * 32, acc);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            st_cluster_v4(dst + 4u * (BN + c * 32 + 4 * q), acc[4 * q], acc[4 * q + 1],
-                          acc[4 * q + 2], acc[4 * q + 3]);
+            *reinterpret_cast<uint4*>(stg + BN + c * 32 + 4 * q) =
+                make_uint4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
         }
       }
-      mbar_arrive_cluster(mapa_shared(smem_u32(recv), static_cast<uint32_t>(owner)));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        // this warp's 32 rows are contiguous both here and in the owner's slot
+        const int slot = (rank - owner - 1 + p.ks) % p.ks;
+        const uint32_t dst = mapa_shared(smem_u32(slots), static_cast<uint32_t>(owner)) +
+                             4u * static_cast<uint32_t>((slot * own_rows + lrow % own_rows) * L::kRowWords);
+        bulk_copy_to_cluster(dst, stg, 32u * L::kRowWords * 4u,
+                             mapa_shared(smem_u32(recv), static_cast<uint32_t>(owner)));
+      }
     } else {
       // finish this row: own partial + the received ones, dequantize, store
-      if (ok && p.ks > 1)
-        ok = mbar_wait_cluster_bounded(recv, 0, abort_flag, p.status, kDevTimeoutEpilogue);
+      if (p.ks > 1) {
+        const bool got = mbar_wait_cluster_bounded(recv, 0, abort_flag, p.status, kDevTimeoutEpilogue);
+        ok = ok && got;
+      }
       const bool n_ok = ok && n < p.N;
       const int r_local = lrow % own_rows;
       const int slot0 = (0 - rank - 1 + p.ks) % p.ks;   // CTA 0's slot (outlier sums)
+      __half* ybox = reinterpret_cast<__half*>(smem + L::off_wide_b + L::off_ybox);
+      const float4* tok4 = reinterpret_cast<const float4*>(tok);
+      const float4* zer4 = reinterpret_cast<const float4*>(tok + BN);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t acc[32];
         uint32_t oacc[32];
-        const float sa_c = c == 0 ? sa_lane[0] : sa_lane[BN / 32 - 1];   // BN <= 64
-        const float wsum = (asym && n < p.N) ? static_cast<float>(__ldg(p.w_sums + n)) : 0.0f;
-        const float za_c = (asym && c * 32 + lane < p.M)
-                               ? 256.0f * static_cast<float>(__ldg(p.a_zeros + c * 32 + lane))
-                               : 0.0f;
         tmem_ld_32x32b_x32(tmem_base + lane_off + c * 32, acc);
         if (OUT) tmem_ld_32x32b_x32(tmem_base + lane_off + BN + c * 32, oacc);
         tmem_ld_wait();
@@ -397,19 +424,61 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
             oacc[4 * q] = v.x; oacc[4 * q + 1] = v.y; oacc[4 * q + 2] = v.z; oacc[4 * q + 3] = v.w;
           }
         }
+        // dequantize all 32 tokens first (no branches: independent chains),
+        // then store them
+        uint32_t hp[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = c * 32 + j;
-          const float sa = __shfl_sync(0xffffffffu, sa_c, j);
-          const float za = __shfl_sync(0xffffffffu, za_c, j);
-          if (m >= p.M || !n_ok) continue;
-          const int32_t a = static_cast<int32_t>(acc[j]);
-          float af = static_cast<float>(a);
-          if (asym) af = fmaf(-za, wsum, af);
-          float y = af * s_row * sa;
-          if (has_out) y += __uint_as_float(oacc[j]);
-          p.Y[static_cast<int64_t>(m) * p.ldy + n] = __float2half_rn(y);
-          if (p.acc_debug != nullptr) p.acc_debug[static_cast<int64_t>(m) * p.N + n] = a >> 8;
+        for (int q = 0; q < 8; ++q) {
+          const float4 sa4 = tok4[c * 8 + q];
+          const float sav[4] = {sa4.x, sa4.y, sa4.z, sa4.w};
+          float zav[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if (ASYM) {
+            const float4 z4 = zer4[c * 8 + q];
+            zav[0] = z4.x; zav[1] = z4.y; zav[2] = z4.z; zav[3] = z4.w;
+          }
+          float y[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int j = 4 * q + t;
+            float af = static_cast<float>(static_cast<int32_t>(acc[j]));
+            if (ASYM) af = fmaf(-zav[t], wsum, af);
+            y[t] = af * s_row * sav[t];
+            if (has_out) y[t] += __uint_as_float(oacc[j]);
+          }
+          const __half2 h0 = __floats2half2_rn(y[0], y[1]);
+          const __half2 h1 = __floats2half2_rn(y[2], y[3]);
+          hp[2 * q] = *reinterpret_cast<const uint32_t*>(&h0);
+          hp[2 * q + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+        }
+        if (p.y_tma) {
+          uint16_t* yb = reinterpret_cast<uint16_t*>(ybox) + c * 32 * own_rows + r_local;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            yb[j * own_rows] = static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
+        } else if (n_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < p.M)
+              reinterpret_cast<uint16_t*>(p.Y)[static_cast<int64_t>(c * 32 + j) * p.ldy + n] =
+                  static_cast<uint16_t>(hp[j / 2] >> (16 * (j & 1)));
+        }
+        if (p.acc_debug != nullptr && n_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < p.M)
+              p.acc_debug[static_cast<int64_t>(c * 32 + j) * p.N + n] = static_cast<int32_t>(acc[j]) >> 8;
+        }
+      }
+      if (p.y_tma) {
+        // rows past N and tokens past M fall outside the tensor: not written
+        fence_proxy_async_smem();
+        named_barrier(2, static_cast<uint32_t>(own_rows));   // the owner warps
+        if (r_local == 0) {
+          if (ok) {
+            tma_store_2d(&map_y, ybox, y_w + rank * own_rows, 0);
+            bulk_commit_group();
+          }
+          bulk_wait_group<0>();
         }
       }
     }
@@ -426,8 +495,8 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
 
 template <int BN, bool OUT, bool ASYM>
 cudaError_t run_decode(const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& mwo,
-                       const CUtensorMap& mxo, const DecodeParams& p, int tiles,
-                       cudaStream_t stream) {
+                       const CUtensorMap& mxo, const CUtensorMap& my, const DecodeParams& p,
+                       int tiles, cudaStream_t stream) {
   auto k = w4a4_gemm_decode_kernel<BN, OUT, ASYM>;
   const int smem = DecodeLayout<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -444,7 +513,7 @@ cudaError_t run_decode(const CUtensorMap& mw, const CUtensorMap& mx, const CUten
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k, mw, mx, mwo, mxo, p);
+  e = cudaLaunchKernelEx(&cfg, k, mw, mx, mwo, mxo, my, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -476,6 +545,13 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
   p.kt = static_cast<int32_t>(j.Kp / 128);
   p.ot = out ? (j.n_out + kOutCols - 1) / kOutCols : 0;
   p.ks = std::min(decode_k_split(tiles, p.kt + p.ot, sm_count()), bn == 64 ? 2 : 4);
+  // Y through tensor stores: per owner block, a box of (128 / KS) rows x BN tokens
+  CUtensorMap my{};
+  p.y_tma = (reinterpret_cast<uintptr_t>(j.Y) % 16 == 0) && (j.ldy % 8 == 0) &&
+            make_tensor_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.Y, static_cast<uint64_t>(j.N),
+                               static_cast<uint64_t>(j.M), static_cast<uint64_t>(j.ldy) * 2,
+                               static_cast<uint32_t>(128 / p.ks), static_cast<uint32_t>(bn),
+                               CU_TENSOR_MAP_SWIZZLE_NONE);
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
   CUtensorMap mw{}, mx{}, mwo{}, mxo{};
@@ -498,8 +574,8 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
   cudaError_t e;
   const bool asym = p.a_zeros != nullptr;
 #define QR_RUN_DECODE(B, O)                                                        \
-  (asym ? run_decode<B, O, true>(mw, mx, mwo, mxo, p, t, stream)                   \
-        : run_decode<B, O, false>(mw, mx, mwo, mxo, p, t, stream))
+  (asym ? run_decode<B, O, true>(mw, mx, mwo, mxo, my, p, t, stream)               \
+        : run_decode<B, O, false>(mw, mx, mwo, mxo, my, p, t, stream))
   if (bn == 32) e = out ? QR_RUN_DECODE(32, true) : QR_RUN_DECODE(32, false);
   else e = out ? QR_RUN_DECODE(64, true) : QR_RUN_DECODE(64, false);
 #undef QR_RUN_DECODE
