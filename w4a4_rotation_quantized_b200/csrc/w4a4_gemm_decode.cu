@@ -24,7 +24,9 @@
 // Warp roles (448 threads):
 //   warps 0-3   epilogue (TMEM lane = weight row of the tile)
 //   warps 4-11  widen (two groups of four warps taking alternate K steps)
-//   warp  12    producer (TMA; no multicast)
+//   warp  12    producers (TMA; no multicast): lane 0 the packed ring, lane 1
+//               the fp16 outlier ring, whose steps the MMA thread interleaves
+//               with the int steps
 //   warp  13    TMEM allocation and the MMA-issuing thread
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -114,15 +116,17 @@ struct DecodeLayout {
 
 // K steps of CTA `r` of a cluster of `ks`: int steps [i0, i1), outlier steps
 // [o0, o1).  CTA 0 takes every outlier step and a share of the int steps
-// that evens out the totals; the other CTAs split the rest of the int steps.
-// Int ranges start at even steps (a ring slot holds two).
+// that evens out the totals, an outlier step counting as 2/5 of an int step
+// (its MMAs are short and its loads overlap the int ring); the other CTAs
+// split the rest of the int steps.  Int ranges start at even steps (a ring
+// slot holds two).
 struct StepRange { int i0, i1, o0, o1; };
 
 __device__ __forceinline__ StepRange step_range(int r, int ks, int kt, int ot) {
   StepRange s{0, kt, 0, ot};
   if (ks == 1) return s;
-  const int per = (kt + ot + ks - 1) / ks;
-  const int first = min(kt, (max(0, per - ot) + 1) & ~1);
+  const int per = (5 * kt + 2 * ot + 5 * ks - 1) / (5 * ks);
+  const int first = min(kt, (max(0, per - (2 * ot + 4) / 5) + 1) & ~1);
   if (r == 0) return StepRange{0, first, 0, ot};
   const int q = (((kt - first + ks - 2) / (ks - 1)) + 1) & ~1;
   const int i0 = min(kt, first + (r - 1) * q);
@@ -206,21 +210,23 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
         tma_load_2d(smem + L::off_pack_a + s * L::kPackA, &map_w, &full_p[s], x, y_w);
         tma_load_2d(smem + L::off_pack_b + s * L::kPackB, &map_x, &full_p[s], x, 0);
       }
-      uint32_t ot = 0;
-      if (OUT && ok)
-        for (int os = sr.o0; os < sr.o1; ++os, ++ot) {
-          const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
-          if (!(ok = mbar_wait_bounded(&empty_o[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
-          mbar_arrive_expect_tx(&full_o[s], L::kOutA + L::kOutB);
-          tma_load_2d(smem + L::off_out_a + s * L::kOutA, &map_wo, &full_o[s], os * kOutCols, y_w);
-          tma_load_2d(smem + L::off_out_b + s * L::kOutB, &map_xo, &full_o[s], os * kOutCols, 0);
-        }
-      if (!ok) {
+      if (!ok)
         for (uint32_t i = (it > kNP ? it - kNP : 0); i < it; ++i)
           mbar_wait_bounded(&full_p[i % kNP], (i / kNP) & 1, abort_flag, nullptr, 0, kDrainLimitNs);
+    } else if (OUT && lane == 1 && n_out > 0) {
+      // the outlier ring, beside the int ring, so that its loads overlap it
+      bool ok = true;
+      uint32_t ot = 0;
+      for (int os = sr.o0; os < sr.o1; ++os, ++ot) {
+        const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
+        if (!(ok = mbar_wait_bounded(&empty_o[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
+        mbar_arrive_expect_tx(&full_o[s], L::kOutA + L::kOutB);
+        tma_load_2d(smem + L::off_out_a + s * L::kOutA, &map_wo, &full_o[s], os * kOutCols, y_w);
+        tma_load_2d(smem + L::off_out_b + s * L::kOutB, &map_xo, &full_o[s], os * kOutCols, 0);
+      }
+      if (!ok)
         for (uint32_t i = (ot > kNO ? ot - kNO : 0); i < ot; ++i)
           mbar_wait_bounded(&full_o[i % kNO], (i / kNO) & 1, abort_flag, nullptr, 0, kDrainLimitNs);
-      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA
@@ -228,6 +234,19 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
       constexpr uint32_t idesc = idesc_i8(BN);
       constexpr uint32_t idesc_o = idesc_f16(BN);
       bool ok = true;
+      int ot = 0;                                // outlier steps done
+      // one fp16 outlier step (two K16 MMAs into the fp32 accumulator)
+      auto outlier_step = [&]() {
+        const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
+        if (!(ok = mbar_wait_bounded(&full_o[s], ph, abort_flag, p.status, kDevTimeoutMma))) return;
+        tc_fence_after();
+        const uint64_t da = smem_desc_kmajor(smem_u32(smem + L::off_out_a + s * L::kOutA), 64);
+        const uint64_t db = smem_desc_kmajor(smem_u32(smem + L::off_out_b + s * L::kOutB), 64);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) mma_f16(tmem_base + BN, da + 2 * k, db + 2 * k, idesc_o, (ot | k) != 0);
+        mma_commit(&empty_o[s]);
+        ++ot;
+      };
       for (int it = 0; it < n_slots; ++it) {
         const uint32_t s = it % kNW, ph = (it / kNW) & 1;
         if (!(ok = mbar_wait_bounded(&full_w[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
@@ -242,18 +261,13 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
         for (int k = 0; k < 8; ++k)
           if (k < nk) mma_i8_ts(tmem_base, a + 8 * k, (k < 4 ? db0 : db1) + 2 * (k & 3), idesc, (it | k) != 0);
         mma_commit(&empty_w[s]);
-      }
-      if (OUT && ok)
-        for (int ot = 0; ot < n_out; ++ot) {
-          const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
-          if (!(ok = mbar_wait_bounded(&full_o[s], ph, abort_flag, p.status, kDevTimeoutMma))) break;
-          tc_fence_after();
-          const uint64_t da = smem_desc_kmajor(smem_u32(smem + L::off_out_a + s * L::kOutA), 64);
-          const uint64_t db = smem_desc_kmajor(smem_u32(smem + L::off_out_b + s * L::kOutB), 64);
-#pragma unroll
-          for (int k = 0; k < 2; ++k) mma_f16(tmem_base + BN, da + 2 * k, db + 2 * k, idesc_o, (ot | k) != 0);
-          mma_commit(&empty_o[s]);
+        if (OUT && it >= 1 && ot < n_out) {
+          outlier_step();
+          if (!ok) break;
         }
+      }
+      if (OUT)
+        while (ok && ot < n_out) outlier_step();
       if (ok) mma_commit(tmem_full);
       mma_commit(drain);
       mbar_wait_bounded(drain, 0, abort_flag, p.status, kDevTimeoutDrain, kDrainLimitNs);
