@@ -137,6 +137,20 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with it may start while
+// the previous kernel on the stream is still running; grid_dep_wait blocks
+// the thread until that kernel has completed and its writes are visible (a
+// no-op for a kernel launched without it), so every thread calls it before
+// its first global-memory access.  grid_dep_launch lets the next kernel's
+// CTAs be scheduled (they then run up to their own grid_dep_wait).
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy (tensor core) reads of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {

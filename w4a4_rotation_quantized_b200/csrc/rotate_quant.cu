@@ -317,6 +317,8 @@ struct AbBounds {
 
 template <int MB, int HA, int ITEMS, bool CLIP, int OUT, bool RING>
 __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(const WhtParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   constexpr int LB = 3 + MB + HA;
   constexpr int EA = 8 << HA, TA = 1 << MB;
   constexpr int EB = 1 << MB, TB = 8 << HA;
@@ -604,6 +606,8 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
 // consecutive elements, all block bits are inside a thread.
 template <int ITEMS, bool CLIP>
 __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   extern __shared__ __align__(16) uint8_t smem[];
   const int nt = p.nt;
   const int rg = threadIdx.x / nt;
@@ -820,6 +824,8 @@ __device__ __forceinline__ float wht_smem_pass(float* buf, int Kp, int s) {
 
 template <bool CLIP, bool ASYM, bool SIGNS>
 __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   extern __shared__ __align__(16) uint8_t smem[];
   float* buf = reinterpret_cast<float*>(smem);                       // [span], few_swz order
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);   // outlier bitmap
@@ -1136,8 +1142,8 @@ cudaError_t launch_rows_kernel(Kernel k, const WhtParams& p, int threads, size_t
   const int64_t want = (p.rows + p.rows_per_cta - 1) / p.rows_per_cta;
   const int64_t cap = static_cast<int64_t>(std::max(per_sm, 1)) * sm_count();
   const int grid = static_cast<int>(std::min(want, cap));
-  k<<<grid, threads, smem, s>>>(p);
-  return cudaGetLastError();
+  e = launch_pdl(k, dim3(grid), dim3(threads), smem, s, 1, p);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 // Ring-mode launch: one CTA per SM (at most one per row), contiguous rows.
@@ -1146,8 +1152,8 @@ cudaError_t launch_ring_kernel(Kernel k, const WhtParams& p, int threads, size_t
                                int grid, cudaStream_t s) {
   cudaError_t e = set_smem(k, smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, threads, smem, s>>>(p);
-  return cudaGetLastError();
+  e = launch_pdl(k, dim3(grid), dim3(threads), smem, s, 1, p);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <int MB, int HA, int OUT, bool CLIP, bool RING>
@@ -1278,19 +1284,8 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
                                 : wht_few_rows_kernel<false, false, false>;
   cudaError_t e = set_smem(k, off);
   if (e != cudaSuccess) return QR_ERR_CUDA;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(job.rows * cl), 1, 1);
-  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
-  cfg.dynamicSmemBytes = off;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k, p);
+  e = launch_pdl(k, dim3(static_cast<unsigned>(job.rows * cl)), dim3(static_cast<unsigned>(threads)),
+                 off, stream, static_cast<unsigned>(cl), p);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }

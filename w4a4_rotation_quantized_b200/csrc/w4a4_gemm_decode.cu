@@ -195,6 +195,8 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   if (p.ks > 1) cluster_sync();              // every CTA's barriers initialized
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();                           // the previous kernel's outputs are visible
+  grid_dep_launch();
   const int y_w = tile * 128;                // first weight row of the tile
 
   if (warp == kProducerWarp) {
@@ -515,19 +517,8 @@ cudaError_t run_decode(const CUtensorMap& mw, const CUtensorMap& mx, const CUten
   const int smem = DecodeLayout<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles * p.ks), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.ks);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k, mw, mx, mwo, mxo, my, p);
+  e = launch_pdl(k, dim3(static_cast<unsigned>(tiles * p.ks)), dim3(kThreads), smem, stream,
+                 static_cast<unsigned>(p.ks), mw, mx, mwo, mxo, my, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

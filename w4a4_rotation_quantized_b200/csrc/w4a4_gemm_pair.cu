@@ -183,6 +183,8 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   cluster_sync();                            // barriers of both CTAs initialized
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();                           // the previous kernel's outputs are visible
+  grid_dep_launch();
 
   const int num_tiles = p.tiles_a * p.tiles_b;
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
@@ -493,8 +495,8 @@ cudaError_t run_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int clusters = std::min(p.tiles_a * p.tiles_b, sm_count() / 2);
-  k<<<2 * clusters, kThreads, smem, stream>>>(ma, mb, moa, mob, my, p);
-  return cudaGetLastError();
+  e = launch_pdl(k, dim3(2 * clusters), dim3(kThreads), smem, stream, 1, ma, mb, moa, mob, my, p);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 }  // namespace
