@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
 // cost, so here up to CL x 1024 threads on CL SMs share one row and every
 // global load is issued up front.  Steps: load the row (vector loads) and
 // the outlier indices together; drop the outlier columns of QUIK §1 by a
-// block-wide prefix count over an outlier bitmap, each CTA keeping the kept
+// binary search of the ascending outlier list, each CTA keeping the kept
 // columns whose rotated positions fall in its span; run the Walsh-Hadamard
 // butterflies in passes of up to three stages through shared memory, the
 // last pass also taking the span's absmax; combine the CL maxima through
@@ -739,31 +739,6 @@ constexpr int kFewMaxChunks = 4;   // 8-column chunks per thread (K <= 32768 at 
 // the butterfly passes with strides 8..32 hit 32 distinct banks; groups of 8
 // consecutive elements stay contiguous and aligned.
 __device__ __forceinline__ int few_swz(int e) { return e ^ (((e >> 6) & 3) << 3); }
-
-// Exclusive prefix sum over the block (blockDim a multiple of 32); `sh`
-// holds 32 ints.  Contains two __syncthreads.
-__device__ __forceinline__ int block_exclusive_sum(int v, int* sh) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    int s = lane < nw ? sh[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    sh[lane] = s;
-  }
-  __syncthreads();
-  return (w > 0 ? sh[w - 1] : 0) + x - v;
-}
 
 // Maximum over the block (any sign); `sh` holds 32 floats.  Contains two
 // __syncthreads.
@@ -828,8 +803,7 @@ __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsPara
   grid_dep_launch();
   extern __shared__ __align__(16) uint8_t smem[];
   float* buf = reinterpret_cast<float*>(smem);                       // [span], few_swz order
-  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);   // outlier bitmap
-  int* scan = reinterpret_cast<int*>(smem + p.off_scan);             // 32 ints
+  int* sidx = reinterpret_cast<int*>(smem + p.off_bits);             // the outlier columns
   float* red = reinterpret_cast<float*>(smem + p.off_scan + 128);    // 32 floats
   float* maxima = reinterpret_cast<float*>(smem + p.off_scan + 256); // 2 x CL floats
   const int t = threadIdx.x, nthr = blockDim.x;
@@ -840,7 +814,6 @@ __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsPara
   const int nloc = max(0, e_hi - e_lo);
   const int nchunks = (p.K + 7) >> 3;                                // 8 source columns each
   const int cpt = (nchunks + nthr - 1) / nthr;                       // chunks per thread
-  const int nwords = (p.K + 31) >> 5;
   const int c0 = t * cpt;                                            // this thread's chunks
   const __half* srow = p.src + row * p.ld;
   // the row's vector loads first; their latency overlaps the outlier work
@@ -851,23 +824,25 @@ __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsPara
     raw[q] = make_uint4(0u, 0u, 0u, 0u);
     if (q < cpt && p.aligned && col0 + 8 <= p.K) raw[q] = ld_stream_v4(srow + col0);
   }
+  // `before` = outlier columns left of this thread's first column: a binary
+  // search of the (strictly ascending) outlier list staged in shared memory
   int before = 0;
   if (p.n_out > 0) {
-    for (int w = t; w < nwords; w += nthr) bits[w] = 0u;
-    __syncthreads();
     for (int j = t; j < p.n_out; j += nthr) {
       const int c = __ldg(p.outlier_idx + j);
-      if (c >= 0 && c < p.K) atomicOr(&bits[c >> 5], 1u << (c & 31));
+      sidx[j] = c;
       if (p.out16 != nullptr && cr == 0)
         p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? srow[c] : __float2half(0.0f);
     }
     __syncthreads();
-    int cnt = 0;
-    for (int q = 0; q < cpt; ++q) {
-      const int c = c0 + q;
-      if (c < nchunks) cnt += __popc((bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu);
+    int lo = 0, hi = p.n_out;
+    const int col_first = 8 * c0;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sidx[mid] < col_first) lo = mid + 1;
+      else hi = mid;
     }
-    before = block_exclusive_sum(cnt, scan);
+    before = lo;
   }
   // scatter the kept columns whose rotated positions are in [e_lo, e_hi);
   // zero the padding beyond the real columns
@@ -890,7 +865,13 @@ __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsPara
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = (col0 + i < p.K) ? __half2float(srow[col0 + i]) : 0.0f;
     }
-    const uint32_t m8 = p.n_out > 0 ? (bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
+    // outlier columns of this chunk: the next entries of the list below col0 + 8
+    uint32_t m8 = 0u;
+    for (int k = before; k < p.n_out && k < before + 8; ++k) {
+      const int d = sidx[k] - col0;
+      if (d >= 8) break;
+      if (d >= 0) m8 |= 1u << d;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = col0 + i - before;
@@ -1267,9 +1248,9 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
   if (chunks > static_cast<int64_t>(threads) * kFewMaxChunks) return QR_ERR_UNSUPPORTED;
   size_t off = align_up(sizeof(float) * static_cast<size_t>(p.span), 16);
   p.off_bits = static_cast<int32_t>(off);
-  off = align_up(off + sizeof(uint32_t) * static_cast<size_t>((job.K + 31) / 32), 16);
+  off = align_up(off + sizeof(int32_t) * static_cast<size_t>(std::max(job.n_out, 1)), 16);
   p.off_scan = static_cast<int32_t>(off);
-  off += 512;                                  // scan words, block maxima, cluster maxima
+  off += 512;                                  // block maxima, cluster maxima
   if (off > static_cast<size_t>(max_smem_optin())) return QR_ERR_UNSUPPORTED;
   // asymmetric codes always clamp (their bounds are [-8, 7])
   using Kfn = void (*)(FewRowsParams);
