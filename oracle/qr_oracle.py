@@ -60,6 +60,17 @@ R12 QUIK's activations are asymmetric per token, dynamic ([QK] §1).  Read
     float32, half to even.  The codes are stored as the signed nibble
     q - 8 (two's complement, [-8, 7]) with the zero point z - 8, so that
     s*(q - z) = s*((q - 8) - (z - 8)) and the same integer GEMM applies.
+R13 The KV-cache path.  R3 ([SR] reviewer brBn Q2/A2; [QS] §3, Fig 5) is
+    the same orthogonal matrix applied to the query and key rows of every
+    head after RoPE, so that (q R3)(k R3)^T = q k^T; the pages do not say
+    which matrix it is, and it is read as the normalized Hadamard of the
+    head dimension, H_d / sqrt(d) (QuaRot's online rotation, [QS] §2).
+    [QS] §3 remarks that the query branch should carry R3^{-1}; for the
+    symmetric Hadamard R3^{-1} = R3^T = R3, so both readings agree.  The
+    KV cache is quantized group-wise asymmetrically with groups of 128
+    ([FQ] §3 量化设置), read as 4 bits with the R12 quantizer applied to
+    each group of consecutive values of a token's (heads x head_dim) row:
+    keys after R3, values as they are; queries stay fp16.
 """
 from __future__ import annotations
 
@@ -450,6 +461,58 @@ def linear_forward(x, w, rot: Rotation, outlier_idx=None):
     ws = quantize_weights(w, rot, outlier_idx)
     acc, y = linear(a, ws)
     return a, ws, acc, y
+
+
+# --------------------------------------------------------------------------
+# KV cache: R3 on queries and keys, group-wise asymmetric KV quantization
+# --------------------------------------------------------------------------
+
+def rotate_heads(x: np.ndarray, head_dim: int) -> np.ndarray:
+    """Each head's slice of a token row times H_d / sqrt(d) (R13)."""
+    x = np.asarray(x, np.float64)
+    t, w = x.shape
+    if w % head_dim:
+        raise ValueError("row width must be a multiple of head_dim")
+    h = hadamard(head_dim) / np.sqrt(head_dim)
+    return (x.reshape(t, w // head_dim, head_dim) @ h).reshape(t, w)
+
+
+@dataclass
+class GroupQuantized:
+    codes: np.ndarray        # int8 [tokens x width]: q - 8, in [-8, 7]
+    scales: np.ndarray       # float32 [tokens x width/group]
+    zeros: np.ndarray        # int32 [tokens x width/group]: z - 8
+    quotient: np.ndarray     # float32 [tokens x width] x/s before rounding
+    zero_quotient: np.ndarray  # float32 [tokens x width/group]
+
+
+def quantize_groups_asym(x: np.ndarray, group: int) -> GroupQuantized:
+    """Group-wise asymmetric 4-bit quantization (R13): every `group`
+    consecutive values of a row are one row of the R12 quantizer."""
+    x = np.asarray(x, np.float64)
+    t, w = x.shape
+    if w % group:
+        raise ValueError("row width must be a multiple of the group size")
+    q = quantize_rows_asym(x.reshape(t * (w // group), group))
+    return GroupQuantized(codes=q.codes.reshape(t, w), scales=q.scales.reshape(t, w // group),
+                          zeros=q.zeros.reshape(t, w // group),
+                          quotient=q.quotient.reshape(t, w),
+                          zero_quotient=q.zero_quotient.reshape(t, w // group))
+
+
+def dequant_groups_asym(q: GroupQuantized, group: int) -> np.ndarray:
+    """s * (codes - zeros) per group, float64."""
+    t, w = q.codes.shape
+    s = np.repeat(np.asarray(q.scales, np.float64), group, axis=1)
+    z = np.repeat(q.zeros.astype(np.float64), group, axis=1)
+    return s * (q.codes.astype(np.float64) - z)
+
+
+def kv_quantize(q: np.ndarray, k: np.ndarray, v: np.ndarray, head_dim: int, group: int = 128):
+    """The online KV-cache step (R13): (q R3, Q_g(k R3), Q_g(v)); q, k, v
+    are [tokens x heads*head_dim] after RoPE."""
+    return (rotate_heads(q, head_dim), quantize_groups_asym(rotate_heads(k, head_dim), group),
+            quantize_groups_asym(v, group))
 
 
 # --------------------------------------------------------------------------

@@ -475,3 +475,86 @@ def test_asym_linear_matches_the_dequantized_product():
     # and the layer tracks X W^T
     ref = x.astype(np.float64) @ w.astype(np.float64).T
     assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.2
+
+
+# ---------------------------------------------------------------- KV cache (R13)
+
+def _sylvester(n):
+    """H[i, j] = (-1)^popcount(i & j), written out independently."""
+    return np.array([[(-1) ** bin(i & j).count("1") for j in range(n)] for i in range(n)], float)
+
+
+def test_rotate_heads_hand_example():
+    row = _golden_matrix("rotate_heads_2x4.txt")[0]
+    np.testing.assert_allclose(O.rotate_heads(row[None, :8], 4)[0], row[8:], atol=1e-12)
+
+
+@pytest.mark.parametrize("head_dim,heads", [(4, 3), (64, 2), (128, 3)])
+def test_rotate_heads_is_block_diagonal_hadamard(head_dim, heads):
+    rng = np.random.default_rng(head_dim + heads)
+    x = rng.standard_normal((5, heads * head_dim))
+    r = np.kron(np.eye(heads), _sylvester(head_dim) / np.sqrt(head_dim))
+    np.testing.assert_allclose(O.rotate_heads(x, head_dim), x @ r, atol=1e-10)
+
+
+def test_r3_keeps_every_heads_attention_scores():
+    # (q R3)(k R3)^T = q k^T head by head, the identity the review answer gives
+    rng = np.random.default_rng(31)
+    d, heads = 128, 4
+    q = rng.standard_normal((6, heads * d))
+    k = rng.standard_normal((9, heads * d))
+    qr, kr = O.rotate_heads(q, d), O.rotate_heads(k, d)
+    for h in range(heads):
+        sl = slice(h * d, (h + 1) * d)
+        np.testing.assert_allclose(qr[:, sl] @ kr[:, sl].T, q[:, sl] @ k[:, sl].T, atol=1e-9)
+
+
+def test_r3_inverse_reading_coincides_for_hadamard():
+    # the notes' R3^{-1} on the query branch equals R3 for the symmetric Hadamard
+    h = _sylvester(128) / np.sqrt(128)
+    np.testing.assert_allclose(np.linalg.inv(h), h, atol=1e-12)
+
+
+def test_group_quantizer_is_rows_of_the_asym_quantizer():
+    # the two hand-worked 1x4 rows side by side form one 8-wide row of two groups
+    rows = [[float(t) for t in r] for r in read_golden_rows("quantizer_asym_1x4.txt")]
+    x = np.array([rows[0][:4] + rows[1][:4]])
+    g = O.quantize_groups_asym(x, 4)
+    assert np.array_equal(g.codes[0], np.array(rows[0][4:8] + rows[1][4:8], np.int8))
+    assert list(g.scales[0]) == [rows[0][8], rows[1][8]]
+    assert list(g.zeros[0]) == [rows[0][9], rows[1][9]]
+
+
+def test_group_quantizer_properties():
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((7, 512)) * np.linspace(0.1, 5.0, 512)
+    x[3, 128:256] = 2.5                                   # a constant group
+    g = O.quantize_groups_asym(x, 128)
+    assert g.codes.shape == x.shape and g.scales.shape == (7, 4) and g.zeros.shape == (7, 4)
+    assert g.codes.min() >= -8 and g.codes.max() <= 7
+    xh = O.dequant_groups_asym(g, 128)
+    s = np.repeat(g.scales.astype(np.float64), 128, axis=1)
+    assert np.all(np.abs(xh - x)[s > 0] <= (s / 2 * (1 + 1e-5) + 1e-12)[s > 0])
+    assert g.scales[3, 1] == 0 and not xh[3, 128:256].any()
+
+
+def test_kv_quantize_keeps_scores_close_and_rotation_helps_keys():
+    # keys with a few large channels: R3 spreads them over the head, so the
+    # g128 4-bit keys give attention scores closer to the exact ones
+    rng = np.random.default_rng(33)
+    d, heads = 128, 4
+    q = rng.standard_normal((16, heads * d))
+    k = rng.standard_normal((64, heads * d))
+    k[:, [5, 140, 300, 420]] *= 25.0
+    v = rng.standard_normal((64, heads * d))
+    qr, kq, vq = O.kv_quantize(q, k, v, d, 128)
+    kr_hat = O.dequant_groups_asym(kq, 128)
+    plain = O.dequant_groups_asym(O.quantize_groups_asym(k, 128), 128)
+    exact = [q[:, h * d:(h + 1) * d] @ k[:, h * d:(h + 1) * d].T for h in range(heads)]
+    rot = [qr[:, h * d:(h + 1) * d] @ kr_hat[:, h * d:(h + 1) * d].T for h in range(heads)]
+    unrot = [q[:, h * d:(h + 1) * d] @ plain[:, h * d:(h + 1) * d].T for h in range(heads)]
+    err_rot = sum(np.linalg.norm(a - b) for a, b in zip(rot, exact)) / sum(map(np.linalg.norm, exact))
+    err_unrot = sum(np.linalg.norm(a - b) for a, b in zip(unrot, exact)) / sum(map(np.linalg.norm, exact))
+    assert err_rot < 0.1 and err_rot < err_unrot
+    v_hat = O.dequant_groups_asym(vq, 128)
+    assert np.linalg.norm(v_hat - v) / np.linalg.norm(v) < 0.1
