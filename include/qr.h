@@ -249,6 +249,34 @@ QR_API qr_status qr_select_outliers(const uint16_t* X_calib, int64_t T, int64_t 
 QR_API qr_status qr_invert_transpose(const float* P, int32_t n, float* out,
                               int32_t* info, qr_stream stream);
 
+/* ----------------------------------------------------------------------
+ * KV cache ("SpinQuant: LLM Quantization with Learned Rotations" review,
+ * reviewer brBn Q2/A2: the same R3 on the query and key rows after RoPE,
+ * (q R3)(k R3)^T = q k^T; FlatQuant §3, quantization setting: the KV cache
+ * quantized group-wise asymmetrically, groups of 128).  R3 is the
+ * normalized Hadamard of the head dimension, H_d / sqrt(d), on every head.
+ *
+ * Q, K, V   fp16 [tokens x heads*head_dim], contiguous rows (the layout
+ *           after the projections and RoPE), device
+ * q_rot     fp16 [tokens x heads*head_dim]: Q with R3 on every head
+ * k_codes   uint8 [tokens x heads*head_dim/2]: K with R3 on every head,
+ *           then each run of `group` consecutive values of a row quantized
+ *           as by qr_rotate_quant_asym (4-bit, asymmetric, codes q - 8 packed
+ *           two per byte, element 2j in the low nibble); k_scales float32
+ *           and k_zeros int32 [tokens x heads*head_dim/group]
+ * v_codes, v_scales, v_zeros: the same for V without a rotation
+ * Q/q_rot, the four K arrays and the four V arrays are each all given or
+ * all NULL (a part that is NULL is skipped).  Caller-owned device memory;
+ * Q and q_rot 16-byte aligned, k_codes and v_codes 16-byte aligned.
+ * head_dim in {32, 64, 128, 256}; group a multiple of 128 and of head_dim
+ * that divides heads*head_dim (UNSUPPORTED otherwise).  Errors: INVALID_ARG
+ * for negative sizes or a partly given side, ALIGNMENT, CUDA. */
+QR_API qr_status qr_kv_quantize(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                int64_t tokens, int32_t heads, int32_t head_dim, int32_t group,
+                                uint16_t* q_rot, uint8_t* k_codes, float* k_scales,
+                                int32_t* k_zeros, uint8_t* v_codes, float* v_scales,
+                                int32_t* v_zeros, qr_stream stream);
+
 /* Reads, and clears, the current device's status word that kernels set when
  * a bounded wait ran out.  Synchronizes the device.  *code_out = 0 when no
  * kernel reported anything. */

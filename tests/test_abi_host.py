@@ -169,3 +169,24 @@ def test_asymmetric_entry_points_argument_errors(lib):
     assert lin(za=None) == L.QR_ERR_INVALID_ARG
     assert lin(ws=None) == L.QR_ERR_INVALID_ARG
 
+
+
+def test_kv_quantize_argument_errors(lib):
+    # every call here fails validation (or has no tokens): nothing launches
+    def kv(q=FAKE, k=FAKE, v=FAKE, tokens=4, heads=4, d=128, g=128, qr=FAKE, kc=FAKE, ks=FAKE,
+           kz=FAKE, vc=FAKE, vs=FAKE, vz=FAKE):
+        return L.qr_kv_quantize(q, k, v, tokens, heads, d, g, qr, kc, ks, kz, vc, vs, vz, None,
+                                check=False)
+    assert kv(tokens=-1) == L.QR_ERR_INVALID_ARG
+    assert kv(heads=0) == L.QR_ERR_INVALID_ARG
+    assert kv(d=96) == L.QR_ERR_UNSUPPORTED
+    assert kv(g=192) == L.QR_ERR_UNSUPPORTED            # not a multiple of 128
+    assert kv(d=256, g=128) == L.QR_ERR_UNSUPPORTED      # a group must hold whole heads
+    assert kv(heads=3, d=128, g=256) == L.QR_ERR_UNSUPPORTED   # width not a multiple of g
+    assert kv(qr=None) == L.QR_ERR_INVALID_ARG           # Q without its output
+    assert kv(kz=None) == L.QR_ERR_INVALID_ARG           # a partly given K side
+    assert kv(v=None) == L.QR_ERR_INVALID_ARG            # V outputs without V
+    assert kv(q=FAKE + 2) == L.QR_ERR_ALIGNMENT
+    assert kv(tokens=0) == L.QR_OK
+    assert kv(q=None, k=None, v=None, qr=None, kc=None, ks=None, kz=None, vc=None, vs=None,
+              vz=None) == L.QR_OK

@@ -10,6 +10,7 @@ is its ctypes binding plus torch-facing helpers.
 from . import _lib  # noqa: F401
 from .layer import (GSR, HADAMARD, KRON, NONE, GraphedLinear, QuantizedLinear,  # noqa: F401
                     Rotation,
-                    invert_transpose, pack_weights, packed_k, rotate_quant, rotate_quant_asym,
+                    invert_transpose, kv_quantize, pack_weights, packed_k, rotate_quant,
+                    rotate_quant_asym,
                     select_outliers, w4a4_linear, w4a4_linear_asym, weight_code_sums,
                     weight_rotation)

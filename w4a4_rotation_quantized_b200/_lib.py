@@ -17,7 +17,7 @@ QR_CHAN_DIVIDE, QR_CHAN_MULTIPLY = 0, 1
 EXPORTED = ("qr_abi_version", "qr_status_string", "qr_packed_k", "qr_rotate_quant",
             "qr_pack_weights", "qr_w4a4_linear", "qr_select_outliers",
             "qr_invert_transpose", "qr_device_status", "qr_rotate_quant_asym",
-            "qr_weight_code_sums", "qr_w4a4_linear_asym")
+            "qr_weight_code_sums", "qr_w4a4_linear_asym", "qr_kv_quantize")
 
 
 class QrRotation(ctypes.Structure):
@@ -72,6 +72,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qr_weight_code_sums": (ctypes.c_int, [vp, i64, i64, vp, vp]),
         "qr_w4a4_linear_asym": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, i32,
                                                vp, i64, vp, vp]),
+        "qr_kv_quantize": (ctypes.c_int, [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                          vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -154,6 +156,15 @@ def qr_w4a4_linear_asym(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, M
                                     K_p, x_out, w_out, n_out, Y, ldy, acc_debug, stream)
     if check:
         _check("qr_w4a4_linear_asym", st)
+    return st
+
+
+def qr_kv_quantize(Q, K, V, tokens, heads, head_dim, group, q_rot, k_codes, k_scales, k_zeros,
+                   v_codes, v_scales, v_zeros, stream, *, check=True):
+    st = load().qr_kv_quantize(Q, K, V, tokens, heads, head_dim, group, q_rot, k_codes, k_scales,
+                               k_zeros, v_codes, v_scales, v_zeros, stream)
+    if check:
+        _check("qr_kv_quantize", st)
     return st
 
 

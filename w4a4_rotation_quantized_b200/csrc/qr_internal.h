@@ -103,6 +103,19 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
 qr_status launch_select_outliers(const uint16_t* x, int64_t T, int64_t K, int64_t ld,
                                  int32_t k, int32_t* idx_out, cudaStream_t stream);
 
+// R3 on query rows: `vectors` contiguous head vectors of head_dim (32, 64,
+// 128 or 256) fp16 values, each times H_d / sqrt(d), written as fp16.
+qr_status launch_head_rotate(const uint16_t* src, uint16_t* dst, int64_t vectors, int head_dim,
+                             cudaStream_t stream);
+
+// KV-cache codes: `groups` rows of `group` (128 or 256) contiguous fp16
+// values, each quantized asymmetrically to 4 bits (codes q - 8 packed two per
+// byte, scale and zero point per row), R3 (Hadamard of head_dim, a power of
+// two dividing the group) applied first when `rotate`.
+qr_status launch_kv_group_quant(const uint16_t* src, int64_t groups, int group, int head_dim,
+                                bool rotate, uint8_t* codes, float* scales, int32_t* zeros,
+                                cudaStream_t stream);
+
 qr_status launch_code_row_sums(const uint8_t* codes, int64_t rows, int64_t kp, int32_t* sums,
                                cudaStream_t stream);
 

@@ -27,6 +27,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "qr_device.cuh"
 #include "qr_internal.h"
@@ -1442,7 +1443,108 @@ qr_status launch_kron_rows(const RowJob& job, cudaStream_t stream) {
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
 
+// KV-cache groups: one warp per group of G = 32 E consecutive values (a
+// token's heads are contiguous, so a group holds G / D whole heads).  Lane L
+// holds elements [E L, E L + E): R3's butterflies over the bits below
+// log2(D) run in registers (element bits) and by xor shuffles (lane bits);
+// the group's min and max come from two warp reductions; the asymmetric
+// 4-bit codes use the same fma-and-clamp as the row kernels, with 1/sqrt(D)
+// folded into the scale; each lane stores its E nibbles (E / 2 bytes, a
+// coalesced 32 E / 2-byte row per warp) and lane 0 the scale and zero point.
+template <int E, bool ROT>
+__global__ void __launch_bounds__(256) kv_group_quant_kernel(const __half* __restrict__ src,
+                                                             int64_t groups, int head_bits,
+                                                             float inv_sqrt, uint8_t* codes,
+                                                             float* scales, int32_t* zeros) {
+  grid_dep_wait();
+  grid_dep_launch();
+  constexpr int G = 32 * E;
+  constexpr int LE = E == 4 ? 2 : 3;
+  static_assert(E == 4 || E == 8, "groups of 128 or 256");
+  using V = typename std::conditional<E == 4, uint2, uint4>::type;
+  using C = typename std::conditional<E == 4, uint16_t, uint32_t>::type;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; g < groups;
+       g += nwarps) {
+    const V raw = *reinterpret_cast<const V*>(src + g * G + lane * E);
+    const __half* h = reinterpret_cast<const __half*>(&raw);
+    float x[E];
+#pragma unroll
+    for (int j = 0; j < E; ++j) x[j] = __half2float(h[j]);
+    if (ROT) {
+#pragma unroll
+      for (int b = 0; b < LE; ++b)
+        if (b < head_bits)
+#pragma unroll
+          for (int j = 0; j < E; ++j)
+            if (!(j & (1 << b))) {
+              const float a = x[j], c = x[j | (1 << b)];
+              x[j] = a + c;
+              x[j | (1 << b)] = a - c;
+            }
+#pragma unroll
+      for (int lb = 0; lb < 5; ++lb)
+        if (LE + lb < head_bits) {
+          const bool upper = (lane >> lb) & 1;
+#pragma unroll
+          for (int j = 0; j < E; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[j], 1 << lb);
+            x[j] = upper ? o - x[j] : x[j] + o;
+          }
+        }
+    }
+    float mx = x[0], mn = x[0];
+#pragma unroll
+    for (int j = 1; j < E; ++j) {
+      mx = fmaxf(mx, x[j]);
+      mn = fminf(mn, x[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    const RowQ q = asym_row_q(mn, mx, 1.0f, inv_sqrt, lane == 0 ? scales + g : nullptr, zeros + g);
+    C packed = 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j)
+      packed |= static_cast<C>(quant_nibble<true>(x[j], q.r, q.c, q.lo, q.hi) << (4 * j));
+    *reinterpret_cast<C*>(codes + g * (G / 2) + lane * (E / 2)) = packed;
+  }
+}
+
 }  // namespace
+
+// Group-wise asymmetric KV-cache codes over rows of `group` (128 or 256)
+// contiguous values, R3 (the Hadamard of head_dim, a power of two dividing
+// the group) applied first when `rotate`.
+qr_status launch_kv_group_quant(const uint16_t* src, int64_t groups, int group, int head_dim,
+                                bool rotate, uint8_t* codes, float* scales, int32_t* zeros,
+                                cudaStream_t stream) {
+  if (groups == 0) return QR_OK;
+  int hb = 0;
+  while ((1 << hb) < head_dim) ++hb;
+  const float inv_sqrt = rotate ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)))
+                                : 1.0f;
+  const int64_t blocks = std::min<int64_t>((groups + 7) / 8, static_cast<int64_t>(sm_count()) * 8);
+  const auto* x = reinterpret_cast<const __half*>(src);
+  cudaError_t e;
+  if (group == 128)
+    e = rotate ? launch_pdl(kv_group_quant_kernel<4, true>, dim3(static_cast<unsigned>(blocks)),
+                            dim3(256), 0, stream, 1, x, groups, hb, inv_sqrt, codes, scales, zeros)
+               : launch_pdl(kv_group_quant_kernel<4, false>, dim3(static_cast<unsigned>(blocks)),
+                            dim3(256), 0, stream, 1, x, groups, hb, inv_sqrt, codes, scales, zeros);
+  else if (group == 256)
+    e = rotate ? launch_pdl(kv_group_quant_kernel<8, true>, dim3(static_cast<unsigned>(blocks)),
+                            dim3(256), 0, stream, 1, x, groups, hb, inv_sqrt, codes, scales, zeros)
+               : launch_pdl(kv_group_quant_kernel<8, false>, dim3(static_cast<unsigned>(blocks)),
+                            dim3(256), 0, stream, 1, x, groups, hb, inv_sqrt, codes, scales, zeros);
+  else
+    return QR_ERR_UNSUPPORTED;
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+}
 
 qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream) {
   if (job.rows == 0) return QR_OK;

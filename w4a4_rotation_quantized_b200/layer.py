@@ -172,6 +172,40 @@ def w4a4_linear_asym(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, x_ou
     return y, acc
 
 
+def kv_quantize(q: Optional[torch.Tensor], k: Optional[torch.Tensor], v: Optional[torch.Tensor],
+                head_dim: int, group: int = 128):
+    """The KV-cache step after RoPE: R3 (H_d / sqrt(d) per head) on q and k,
+    group-wise asymmetric 4-bit codes for k (after R3) and v.  Inputs are
+    fp16 [tokens, heads*head_dim] row-major (any may be None).  Returns
+    (q_rot, (k_codes, k_scales, k_zeros), (v_codes, v_scales, v_zeros)),
+    None for a part not given."""
+    given = [t for t in (q, k, v) if t is not None]
+    if not given:
+        raise ValueError("nothing to do")
+    tokens, width = given[0].shape
+    for t in given:
+        _need_cuda(t, torch.float16, "input")
+        if t.shape != (tokens, width) or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous [tokens, heads*head_dim] tensors")
+    if width % head_dim:
+        raise ValueError("width must be a multiple of head_dim")
+    heads = width // head_dim
+    dev = given[0].device
+    q_rot = torch.empty_like(q) if q is not None else None
+
+    def side(t):
+        if t is None:
+            return None
+        return (torch.empty((tokens, width // 2), dtype=torch.uint8, device=dev),
+                torch.empty((tokens, width // group), dtype=torch.float32, device=dev),
+                torch.empty((tokens, width // group), dtype=torch.int32, device=dev))
+    ks, vs = side(k), side(v)
+    p = lambda tup, i: None if tup is None else tup[i].data_ptr()
+    L.qr_kv_quantize(_ptr(q), _ptr(k), _ptr(v), tokens, heads, head_dim, group, _ptr(q_rot),
+                     p(ks, 0), p(ks, 1), p(ks, 2), p(vs, 0), p(vs, 1), p(vs, 2), _stream())
+    return q_rot, ks, vs
+
+
 def select_outliers(x_calib: torch.Tensor, k: int) -> torch.Tensor:
     """QUIK calibration: the k columns of largest infinity-norm, ascending."""
     _need_cuda(x_calib, torch.float16, "x_calib")
