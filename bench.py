@@ -555,6 +555,156 @@ def run_reference(args, rank, world):
     }
 
 
+# --------------------------------------------------------------------------- KV cache
+
+KV_METRIC = "KV-cache R3 + g128 4-bit quantization GB/s at 1 B200, % of HBM"
+
+
+def kv_bytes(s, tokens):
+    """Algorithmic bytes of one KV step: read q, k, v; write q R3, the k and v
+    codes (half a byte per value) and a float scale + int32 zero per group."""
+    w = s.heads * s.head_dim
+    return tokens * w * 2 * 4 + 2 * (tokens * w // 2 + tokens * (w // s.group) * 8)
+
+
+def run_kv(args, rank, world, local_rank):
+    import torch
+    import w4a4_rotation_quantized_b200 as Q
+    import workloads
+    from w4a4_rotation_quantized_b200 import build as B
+
+    torch.cuda.set_device(local_rank)
+    if rank == 0:
+        B.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    Q._lib.load()
+    s, q, k, v = workloads.make_kv(args.workload, args.tokens)
+    T = q.shape[0]
+    byts = kv_bytes(s, T)
+    nsets = max(2, math.ceil(2 * L2_BYTES / (3 * q.nbytes)))
+    sets = [tuple(torch.from_numpy(a).cuda() for a in (q, k, v)) for _ in range(nsets)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        a, b, c = sets[i % nsets]
+        return Q.kv_quantize(a, b, c, s.head_dim, s.group)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        keep = [step(i) for i in range(nsets)]
+    g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, args.steps // nsets)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    sampler.stop()
+    del keep
+    if Q._lib.qr_device_status() != 0:
+        raise RuntimeError("a kernel reported a device status")
+    steps = reps * nsets
+    ms = aggregate_max(e0.elapsed_time(e1), world) / steps
+    peaks, peak_src = load_peaks()
+    gbs = byts / (ms * 1e-3) / 1e9
+    # end to end with host buffers: q, k, v in, every output out
+    hq, hk, hv = (torch.from_numpy(a).pin_memory() for a in (q, k, v))
+    e2e_steps = min(args.steps, 20)
+    d_in = [torch.empty_like(t, device="cuda") for t in (hq, hk, hv)]
+    r = step(0)
+    outs_h = [torch.empty_like(r[0], device="cpu").pin_memory()] + \
+        [torch.empty_like(t, device="cpu").pin_memory() for part in r[1:] for t in part]
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        for d, h in zip(d_in, (hq, hk, hv)):
+            d.copy_(h, non_blocking=True)
+        r = Q.kv_quantize(d_in[0], d_in[1], d_in[2], s.head_dim, s.group)
+        flat = [r[0]] + [t for part in r[1:] for t in part]
+        for h, d in zip(outs_h, flat):
+            h.copy_(d, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = aggregate_max(a0.elapsed_time(a1), world) / e2e_steps
+    return {
+        "metric": KV_METRIC, "value": round(world * byts / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "precision": "fp16 in, fp32 rotation, 4-bit asymmetric codes + fp32 scale/int32 zero "
+                     "per group, fp16 queries out",
+        "data": "synthetic",
+        "config": {"workload": s.name, "tokens": T, "heads": s.heads, "head_dim": s.head_dim,
+                   "group": s.group, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotate over {nsets} copies"},
+        "roofline": {"bound": "hbm", "kernel": "kv_group_quant_kernel + head_rotate_kernel",
+                     "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "peak_source": f"{peak_src} HBM copy bandwidth",
+                     "algorithmic_bytes_per_launch": byts, "traffic": None},
+        "e2e": {"value": round(world * byts / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": int(hq.nbytes + hk.nbytes + hv.nbytes),
+                "d2h_bytes_per_step": int(sum(h.nbytes for h in outs_h)), "steps": e2e_steps,
+                "api": "kv_quantize"},
+        "gpu_launches": 3 * steps,
+        "clocks": sampler.summary(t0, t1),
+    }
+
+
+def run_kv_reference(args, rank, world):
+    """The oracle's KV step on the host cores (rank 0)."""
+    if rank != 0:
+        return None
+    import oracle as O
+    import workloads
+    s, q, k, v = workloads.make_kv(args.workload, min(args.reference_tokens,
+                                                      args.tokens or workloads.KV_SPECS[
+                                                          args.workload].tokens))
+    q64, k64, v64 = (a.astype(np.float64) for a in (q, k, v))
+    for _ in range(args.warmup):
+        O.kv_quantize(q64, k64, v64, s.head_dim, s.group)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.kv_quantize(q64, k64, v64, s.head_dim, s.group)
+    sec = (time.perf_counter() - t0) / args.steps
+    from threadpoolctl import threadpool_info
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    value = kv_bytes(s, q.shape[0]) / sec / 1e9
+    sample = f"{q.shape[0]} of {s.tokens} tokens of {s.name} per step through the oracle"
+    return {
+        "impl": "reference", "metric": KV_METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": s.name, "tokens": q.shape[0], "heads": s.heads,
+                   "head_dim": s.head_dim, "group": s.group, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 # --------------------------------------------------------------------------- main
 
 def main(argv=None):
@@ -582,8 +732,10 @@ def main(argv=None):
     if world != args.gpus:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
 
+    import workloads
+    kv = args.workload in workloads.KV_SPECS
     if args.impl == "reference":
-        res = run_reference(args, rank, world)
+        res = run_kv_reference(args, rank, world) if kv else run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
         return 0
@@ -597,8 +749,15 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res = run_ours(args, rank, world, local_rank)
-        if rank == 0:
+        res = run_kv(args, rank, world, local_rank) if kv else run_ours(args, rank, world,
+                                                                         local_rank)
+        if rank == 0 and kv and world == 1 and not args.no_cpu_baseline:
+            ref = run_kv_reference(argparse.Namespace(
+                workload=args.workload, tokens=args.tokens, reference_tokens=64, warmup=1,
+                steps=3), 0, 1)
+            res["cpu_baseline"] = ref["cpu_baseline"]
+            print(json.dumps(res), flush=True)
+        elif rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 tokens = min(args.cpu_baseline_tokens, res["config"]["M"])
                 res["cpu_baseline"] = oracle_baseline(args.workload, tokens, repeats=3,

@@ -78,3 +78,17 @@ def test_reference_arm_with_random_signs(capsys):
     wl = workloads.make_workload("tiny_256")
     d = bench.workload_signs(wl, True)
     assert d is not None and d.shape == (256,) and bench.oracle_rotation(wl, d).signs is d
+
+
+def test_kv_cache_reference_arm(capsys):
+    # the KV-cache workload's reference arm: the oracle's R3 + g128 step
+    assert bench.main(["--impl", "reference", "--workload", "kv_cache_llama2_7b", "--steps", "1",
+                       "--warmup", "3", "--reference-tokens", "4"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.KV_METRIC
+    assert line["config"]["tokens"] == 4 and line["config"]["group"] == 128
+    import workloads
+    s = workloads.KV_SPECS["kv_cache_llama2_7b"]
+    # q, k, v read, q written (fp16); k and v codes (half a byte) + scale and zero per group
+    w = s.heads * s.head_dim
+    assert bench.kv_bytes(s, 4) == 4 * w * 8 + 2 * (4 * w // 2 + 4 * (w // 128) * 8)

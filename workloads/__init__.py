@@ -192,3 +192,43 @@ def random_signs(seed: int, k_p: int) -> np.ndarray:
     CUDA path receive the same signs."""
     rng = np.random.default_rng([seed, 99])
     return np.where(rng.random(k_p) < 0.5, -1, 1).astype(np.int8)
+
+
+# --------------------------------------------------------------------------
+# KV cache (the R3 rotation of queries and keys, group-wise KV quantization)
+# --------------------------------------------------------------------------
+
+@dataclass
+class KVSpec:
+    name: str
+    tokens: int
+    heads: int
+    head_dim: int
+    group: int
+    seed: int
+    n_outlier_channels: int      # key channels scaled by outlier_scale
+    outlier_scale: float
+
+
+KV_SPECS = {
+    # LLaMA-2-7B attention: 32 heads of 128, a 2048-token prefill
+    "kv_cache_llama2_7b": KVSpec("kv_cache_llama2_7b", tokens=2048, heads=32, head_dim=128,
+                                 group=128, seed=20261208, n_outlier_channels=32,
+                                 outlier_scale=20.0),
+}
+
+
+def make_kv(name: str, tokens: Optional[int] = None):
+    """Seeded post-RoPE q, k, v (fp16 [tokens x heads*head_dim]): N(0,1), with
+    a few key channels scaled up (the outlier channels rotation spreads)."""
+    s = KV_SPECS[name]
+    t = s.tokens if tokens is None else tokens
+    w = s.heads * s.head_dim
+    rng = np.random.default_rng(s.seed)
+    ch = np.sort(rng.choice(w, size=s.n_outlier_channels, replace=False))
+    g = np.random.default_rng([s.seed, 1])
+    q = g.standard_normal((t, w), dtype=np.float32)
+    k = g.standard_normal((t, w), dtype=np.float32)
+    v = g.standard_normal((t, w), dtype=np.float32)
+    k[:, ch] *= np.float32(s.outlier_scale)
+    return s, q.astype(np.float16), k.astype(np.float16), v.astype(np.float16)
