@@ -71,6 +71,21 @@ R13 The KV-cache path.  R3 ([SR] reviewer brBn Q2/A2; [QS] §3, Fig 5) is
     ([FQ] §3 量化设置), read as 4 bits with the R12 quantizer applied to
     each group of consecutive values of a token's (heads x head_dim) row:
     keys after R3, values as they are; queries stay fp16.
+R14 QUIK's 8-bit layers ([QK] QUIK量化, results: the LLaMA-2 down_proj in
+    INT8 with the outlier count raised in proportion to its input width;
+    QUIK-8B: every layer INT8).  Read as the R1/R2 quantizer with b = 8:
+    codes in [-127, 127], s = alpha * absmax / 127, round half to even in
+    float32, stored one int8 per value; the outlier count of a layer of K
+    inputs is round(256 * K / 4096) (688 for K = 11008).
+R15 FP4 on Blackwell ([SR] reviewer brBn W3/A3 names a W-fp4/A-fp4 benchmark
+    on Blackwell's fp4 tensor cores as planned work, with no format).  Read as the e2m1 element type with a per-row
+    fp32 scale, the direct analogue of R2: s = alpha * absmax / 6, each
+    x/s (float32) rounded to the nearest e2m1 value {0, 0.5, 1, 1.5, 2, 3,
+    4, 6} (with sign), ties to the even mantissa, saturating at 6.  The
+    e2m1 nibble is sign (bit 3), exponent (bits 2-1, bias 1), mantissa
+    (bit 0); +-0 both decode to 0.  The integers 5 and 7 of the INT4 grid
+    are not representable, so FP4 is a different quantizer, not a
+    re-encoding of the INT4 codes.
 """
 from __future__ import annotations
 
@@ -232,8 +247,9 @@ class Quantized:
     quotient: np.ndarray     # float32 x/s before rounding (for the tie window)
 
 
-def quantize_rows(xr: np.ndarray, clip_ratio: float = 1.0) -> Quantized:
-    """Symmetric per-row min-max quantization to 4-bit codes.
+def quantize_rows(xr: np.ndarray, clip_ratio: float = 1.0, bits: int = 4) -> Quantized:
+    """Symmetric per-row min-max quantization to `bits`-bit codes (4, or 8
+    for QUIK's INT8 layers, R14).
 
     [SR] Q1/A1: min-max quantization scales each row into the symmetric
     range (R1, R2); [FQ] §3 量化设置: activations per token, weights per
@@ -242,13 +258,64 @@ def quantize_rows(xr: np.ndarray, clip_ratio: float = 1.0) -> Quantized:
     """
     x32 = np.asarray(xr, dtype=np.float64).astype(np.float32)
     absmax = np.max(np.abs(x32), axis=1) if x32.shape[1] else np.zeros(x32.shape[0], np.float32)
-    s = (np.float32(clip_ratio) * absmax) / np.float32(QMAX)
+    qmax = QMAX if bits == 4 else 2 ** (bits - 1) - 1
+    s = (np.float32(clip_ratio) * absmax) / np.float32(qmax)
     s = s.astype(np.float32)
     safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
     v = (x32 / safe[:, None]).astype(np.float32)
     v[s == 0] = 0.0
-    q = np.clip(np.rint(v), -QMAX, QMAX).astype(np.int8)
+    q = np.clip(np.rint(v), -qmax, qmax).astype(np.int8)
     return Quantized(codes=q, scales=s, quotient=v)
+
+
+def quik_outlier_count(K: int) -> int:
+    """Outlier columns of a QUIK layer of K inputs (R14): 256 per 4096."""
+    return int(np.rint(256 * K / 4096))
+
+
+# e2m1 magnitudes by 3-bit code (exponent, mantissa); R15
+E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+@dataclass
+class Fp4Quantized:
+    codes: np.ndarray        # uint8 [rows x K_p]: e2m1 nibbles (sign bit 3)
+    scales: np.ndarray       # float32 [rows]
+    quotient: np.ndarray     # float32 x/s before rounding (tie window)
+
+
+def e2m1_round(v: np.ndarray) -> np.ndarray:
+    """Nearest e2m1 value of each v (float), ties to the even mantissa,
+    saturating at +-6 (R15); returns the 4-bit codes."""
+    v = np.asarray(v, np.float64)
+    mag = np.minimum(np.abs(v), 6.0)
+    d = np.abs(mag[..., None] - E2M1)                   # distance to every grid value
+    best = np.min(d, axis=-1, keepdims=True)
+    cand = d == best                                    # one, or two at a tie
+    even = (np.arange(8) % 2 == 0)                      # mantissa bit 0 clear
+    pick = np.where(cand.sum(-1, keepdims=True) > 1, cand & even, cand)
+    code = np.argmax(pick, axis=-1).astype(np.uint8)
+    return code | np.where((v < 0) & (code > 0), 8, 0).astype(np.uint8)
+
+
+def e2m1_value(code: np.ndarray) -> np.ndarray:
+    code = np.asarray(code, np.int64)
+    return np.where(code & 8, -1.0, 1.0) * E2M1[code & 7]
+
+
+def quantize_rows_fp4(xr: np.ndarray, clip_ratio: float = 1.0) -> Fp4Quantized:
+    """Per-row e2m1 quantization with an fp32 scale (R15)."""
+    x32 = np.asarray(xr, dtype=np.float64).astype(np.float32)
+    absmax = np.max(np.abs(x32), axis=1) if x32.shape[1] else np.zeros(x32.shape[0], np.float32)
+    s = ((np.float32(clip_ratio) * absmax) / np.float32(6)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    v = (x32 / safe[:, None]).astype(np.float32)
+    v[s == 0] = 0.0
+    return Fp4Quantized(codes=e2m1_round(v), scales=s, quotient=v)
+
+
+def dequant_fp4_rows(q: Fp4Quantized) -> np.ndarray:
+    return np.asarray(q.scales, np.float64)[:, None] * e2m1_value(q.codes)
 
 
 @dataclass
@@ -323,7 +390,8 @@ def int_gemm(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
     """
     a = np.asarray(qa, dtype=np.float64)
     w = np.asarray(qw, dtype=np.float64)
-    if a.shape[1] * QMAX * QMAX >= 2 ** 53:
+    big = max(1.0, float(np.abs(a).max(initial=0.0)), float(np.abs(w).max(initial=0.0)))
+    if a.shape[1] * big * big >= 2 ** 53:
         raise ValueError("K too large for an exact float64 dot product")
     return np.rint(a @ w.T).astype(np.int64)
 

@@ -558,3 +558,75 @@ def test_kv_quantize_keeps_scores_close_and_rotation_helps_keys():
     assert err_rot < 0.1 and err_rot < err_unrot
     v_hat = O.dequant_groups_asym(vq, 128)
     assert np.linalg.norm(v_hat - v) / np.linalg.norm(v) < 0.1
+
+
+# ---------------------------------------------------------------- 8-bit layers (R14)
+
+def test_int8_quantizer_hand_example():
+    v = [float(t) for t in read_golden_rows("quantizer_int8_1x8.txt")[0]]
+    q = O.quantize_rows(np.array([v[:8]]), bits=8)
+    assert np.array_equal(q.codes[0], np.array(v[8:16], np.int8))
+    assert q.scales[0] == np.float32(v[16])
+
+
+def test_int8_quantizer_properties_and_exact_products():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((9, 700)) * np.exp(rng.standard_normal((9, 1)))
+    q = O.quantize_rows(x, bits=8)
+    assert q.codes.min() >= -127 and q.codes.max() <= 127
+    assert np.all(np.abs(q.codes).max(axis=1) == 127)
+    s = q.scales.astype(np.float64)[:, None]
+    assert np.all(np.abs(s * q.codes - x) <= s / 2 * (1 + 1e-5) + 1e-12)
+    # the exact integer GEMM at the 8-bit extremes (brute force)
+    a = np.full((2, 11008), 127, np.int8)
+    a[1, ::2] = -127
+    w = np.full((3, 11008), -127, np.int8)
+    acc = O.int_gemm(a, w)
+    brute = [[sum(int(p) * int(r) for p, r in zip(a[i], w[j])) for j in range(3)] for i in range(2)]
+    assert acc.tolist() == brute and abs(acc).max() < 2 ** 31
+
+
+def test_quik_outlier_count_scales_with_width():
+    assert O.quik_outlier_count(4096) == 256
+    assert O.quik_outlier_count(11008) == 688          # the INT8 down_proj
+    assert O.quik_outlier_count(8192) == 512
+
+
+# ---------------------------------------------------------------- FP4 (R15)
+
+def test_fp4_quantizer_hand_example():
+    v = [float(t) for t in read_golden_rows("fp4_e2m1_1x12.txt")[0]]
+    q = O.quantize_rows_fp4(np.array([v[:12]]))
+    assert np.array_equal(q.codes[0], np.array(v[12:24], np.uint8))
+    assert q.scales[0] == np.float32(v[24])
+
+
+def test_e2m1_grid_and_rounding():
+    # every code decodes to the grid, and rounding a grid value returns it
+    vals = O.e2m1_value(np.arange(16))
+    assert sorted(set(np.abs(vals))) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(16):
+        if c != 8:                                   # -0 rounds to +0
+            assert O.e2m1_round(np.array([vals[c]]))[0] == c
+    # nearest value: brute force over a fine sweep (ties excluded)
+    xs = np.linspace(-7, 7, 2801)
+    got = O.e2m1_value(O.e2m1_round(xs))
+    grid = np.concatenate([-O.E2M1[::-1], O.E2M1])
+    near = grid[np.argmin(np.abs(np.clip(xs, -6, 6)[:, None] - grid[None, :]), axis=1)]
+    mids = (O.E2M1[1:] + O.E2M1[:-1]) / 2
+    tie = np.isin(np.round(np.abs(xs), 9), np.round(mids, 9))
+    assert np.array_equal(got[~tie], near[~tie])
+
+
+def test_fp4_quantizer_error_bound():
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((6, 256))
+    q = O.quantize_rows_fp4(x)
+    xh = O.dequant_fp4_rows(q)
+    s = q.scales.astype(np.float64)[:, None]
+    v = np.abs(x) / s
+    # half the grid gap at each magnitude: 0.25 below 2, 0.5 below 4, 1 up to 6
+    gap = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0))
+    assert np.all(np.abs(xh - x) <= gap * s * (1 + 1e-5) + 1e-12)
+    # each row's largest value lands on the top of the grid (6 s = absmax)
+    np.testing.assert_allclose(np.abs(xh).max(axis=1), np.abs(x).max(axis=1), rtol=1e-6)
