@@ -12,12 +12,13 @@
 //    CTAs (KS = 1, 2 or 4, chosen so that tiles x KS fills the SMs): CTA r
 //    runs a contiguous range of the K steps.  The partial sums are then
 //    exchanged, not funnelled: CTA r owns the rows [r*128/KS, (r+1)*128/KS)
-//    of the tile, every CTA stores the other CTAs' rows of its int32
-//    partials into their shared memory (16-byte remote stores), and each CTA
-//    adds the partials of its own rows (integer adds: the order does not
-//    matter) and runs their epilogue.  The fp16 outlier steps all run in
-//    CTA 0, which sends the fp32 outlier sums with its partials, so that sum
-//    has one order.
+//    of the tile; every CTA stages the other CTAs' rows of its int32
+//    partials in its own shared memory and sends each warp's 32 rows with
+//    one shared-to-shared bulk copy into the owner's receive slot, and each
+//    CTA adds the partials of its own rows (integer adds: the order does not
+//    matter) and runs their epilogue, ending in one tensor store of the fp16
+//    [token][row] box.  The fp16 outlier steps all run in CTA 0, which sends
+//    the fp32 outlier sums with its partials, so that sum has one order.
 //  * One CTA per SM runs a deep ring of widened stages (the chain widen ->
 //    MMA -> stage free is local to the SM).
 //
