@@ -180,7 +180,8 @@ def test_kv_quantize_argument_errors(lib):
     assert kv(tokens=-1) == L.QR_ERR_INVALID_ARG
     assert kv(heads=0) == L.QR_ERR_INVALID_ARG
     assert kv(d=96) == L.QR_ERR_UNSUPPORTED
-    assert kv(g=192) == L.QR_ERR_UNSUPPORTED            # not a multiple of 128
+    assert kv(g=192) == L.QR_ERR_UNSUPPORTED            # groups of 128 or 256
+    assert kv(g=512, heads=8) == L.QR_ERR_UNSUPPORTED
     assert kv(d=256, g=128) == L.QR_ERR_UNSUPPORTED      # a group must hold whole heads
     assert kv(heads=3, d=128, g=256) == L.QR_ERR_UNSUPPORTED   # width not a multiple of g
     assert kv(qr=None) == L.QR_ERR_INVALID_ARG           # Q without its output

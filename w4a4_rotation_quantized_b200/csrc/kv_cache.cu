@@ -4,9 +4,9 @@
 // the query and key rows of every head after RoPE, so that
 // (q R3)(k R3)^T = q k^T; here R3 is the normalized Hadamard of the head
 // dimension.  The keys are rotated and quantized group-wise (groups of 128,
-// asymmetric 4-bit, the KV-cache setting of FlatQuant §3) by the row
-// kernels of rotate_quant.cu on a [tokens * width / group, group] view; the
-// queries stay fp16 and only need the rotation, which this kernel does.
+// asymmetric 4-bit, the KV-cache setting of FlatQuant §3) by
+// kv_group_quant_kernel in rotate_quant.cu, one warp per group; the queries
+// stay fp16 and only need the rotation, which this kernel does.
 //
 // One warp per head vector of D = 32 E elements: lane L holds elements
 // [E L, E L + E) (one vector load), the low log2(E) butterfly stages run in

@@ -203,7 +203,8 @@ qr_status qr_kv_quantize(const uint16_t* Q, const uint16_t* K, const uint16_t* V
   if (head_dim != 32 && head_dim != 64 && head_dim != 128 && head_dim != 256)
     return QR_ERR_UNSUPPORTED;
   const int64_t width = static_cast<int64_t>(heads) * head_dim;
-  if (group % 128 != 0 || group % head_dim != 0 || width % group != 0) return QR_ERR_UNSUPPORTED;
+  if ((group != 128 && group != 256) || group % head_dim != 0 || width % group != 0)
+    return QR_ERR_UNSUPPORTED;
   // each side is all there or all absent
   if ((Q == nullptr) != (q_rot == nullptr)) return QR_ERR_INVALID_ARG;
   const bool k_any = K || k_codes || k_scales || k_zeros, k_all = K && k_codes && k_scales && k_zeros;
@@ -213,39 +214,17 @@ qr_status qr_kv_quantize(const uint16_t* Q, const uint16_t* K, const uint16_t* V
   if (Q != nullptr && (!aligned16(Q) || !aligned16(q_rot))) return QR_ERR_ALIGNMENT;
   if (tokens * width > (int64_t(1) << 40)) return QR_ERR_UNSUPPORTED;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // keys and values: rows of `group` values, one quantization group each;
-  // groups of 128 and 256 run one warp per group, larger ones the row kernels
+  // keys and values: rows of `group` values, one quantization group each,
+  // one warp per group
   const int64_t rows = tokens * (width / group);
-  qr_status st = QR_OK;
   if ((k_all && (!aligned16(K) || !aligned16(k_codes))) ||
       (v_all && (!aligned16(V) || !aligned16(v_codes))))
     return QR_ERR_ALIGNMENT;
-  if (group <= 256) {
-    if (k_all) st = launch_kv_group_quant(K, rows, group, head_dim, true, k_codes, k_scales, k_zeros, s);
-    if (st == QR_OK && v_all)
-      st = launch_kv_group_quant(V, rows, group, head_dim, false, v_codes, v_scales, v_zeros, s);
-    if (st == QR_OK && Q != nullptr) st = launch_head_rotate(Q, q_rot, tokens * heads, head_dim, s);
-    return st;
-  }
-  if (k_all) {
-    qr_rotation r3{};
-    r3.kind = QR_ROT_HADAMARD;
-    r3.block = head_dim;
-    r3.clip_ratio = 1.0f;
-    st = rows_call(&r3, K, rows, group, group, nullptr, 0, k_codes, k_scales, k_zeros, nullptr,
-                   nullptr, stream);
-    if (st != QR_OK) return st;
-  }
-  if (v_all) {
-    qr_rotation none{};
-    none.kind = QR_ROT_NONE;
-    none.block = 1;
-    none.clip_ratio = 1.0f;
-    st = rows_call(&none, V, rows, group, group, nullptr, 0, v_codes, v_scales, v_zeros, nullptr,
-                   nullptr, stream);
-    if (st != QR_OK) return st;
-  }
-  if (Q != nullptr) st = launch_head_rotate(Q, q_rot, tokens * heads, head_dim, s);
+  qr_status st = QR_OK;
+  if (k_all) st = launch_kv_group_quant(K, rows, group, head_dim, true, k_codes, k_scales, k_zeros, s);
+  if (st == QR_OK && v_all)
+    st = launch_kv_group_quant(V, rows, group, head_dim, false, v_codes, v_scales, v_zeros, s);
+  if (st == QR_OK && Q != nullptr) st = launch_head_rotate(Q, q_rot, tokens * heads, head_dim, s);
   return st;
 }
 
