@@ -31,6 +31,8 @@ template <> struct HalfVec<2> { using T = uint32_t; };
 template <> struct HalfVec<4> { using T = uint2; };
 template <> struct HalfVec<8> { using T = uint4; };
 
+constexpr int kBatch = 4;
+
 template <int E>
 __global__ void __launch_bounds__(256) head_rotate_kernel(const __half* __restrict__ src,
                                                           __half* __restrict__ dst,
@@ -42,38 +44,48 @@ __global__ void __launch_bounds__(256) head_rotate_kernel(const __half* __restri
   using V = typename HalfVec<E>::T;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       v < vectors; v += nwarps) {
-    const V raw = *reinterpret_cast<const V*>(src + v * D + lane * E);
-    const __half* h = reinterpret_cast<const __half*>(&raw);
-    float x[E];
+  // kBatch head vectors per warp and iteration, their loads issued together
+  for (int64_t v0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kBatch;
+       v0 < vectors; v0 += nwarps * kBatch) {
+    V raws[kBatch];
 #pragma unroll
-    for (int j = 0; j < E; ++j) x[j] = __half2float(h[j]);
-    // stages on the element bits held by the thread
+    for (int u = 0; u < kBatch; ++u)
+      if (v0 + u < vectors) raws[u] = *reinterpret_cast<const V*>(src + (v0 + u) * D + lane * E);
 #pragma unroll
-    for (int b = 0; b < LE; ++b)
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t v = v0 + u;
+      if (v >= vectors) break;                       // uniform over the warp
+      const V raw = raws[u];
+      const __half* h = reinterpret_cast<const __half*>(&raw);
+      float x[E];
 #pragma unroll
-      for (int j = 0; j < E; ++j)
-        if (!(j & (1 << b))) {
-          const float a = x[j], c = x[j | (1 << b)];
-          x[j] = a + c;
-          x[j | (1 << b)] = a - c;
+      for (int j = 0; j < E; ++j) x[j] = __half2float(h[j]);
+      // stages on the element bits held by the thread
+#pragma unroll
+      for (int b = 0; b < LE; ++b)
+#pragma unroll
+        for (int j = 0; j < E; ++j)
+          if (!(j & (1 << b))) {
+            const float a = x[j], c = x[j | (1 << b)];
+            x[j] = a + c;
+            x[j | (1 << b)] = a - c;
+          }
+      // stages on the lane bits: the partner lane holds the other element
+#pragma unroll
+      for (int lb = 0; lb < 5; ++lb) {
+        const bool upper = (lane >> lb) & 1;
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+          const float o = __shfl_xor_sync(0xffffffffu, x[j], 1 << lb);
+          x[j] = upper ? o - x[j] : x[j] + o;
         }
-    // stages on the lane bits: the partner lane holds the other element
-#pragma unroll
-    for (int lb = 0; lb < 5; ++lb) {
-      const bool upper = (lane >> lb) & 1;
-#pragma unroll
-      for (int j = 0; j < E; ++j) {
-        const float o = __shfl_xor_sync(0xffffffffu, x[j], 1 << lb);
-        x[j] = upper ? o - x[j] : x[j] + o;
       }
-    }
-    V out;
-    __half* oh = reinterpret_cast<__half*>(&out);
+      V out;
+      __half* oh = reinterpret_cast<__half*>(&out);
 #pragma unroll
-    for (int j = 0; j < E; ++j) oh[j] = __float2half_rn(x[j] * scale);
-    *reinterpret_cast<V*>(dst + v * D + lane * E) = out;
+      for (int j = 0; j < E; ++j) oh[j] = __float2half_rn(x[j] * scale);
+      *reinterpret_cast<V*>(dst + v * D + lane * E) = out;
+    }
   }
 }
 
@@ -81,7 +93,7 @@ template <int E>
 cudaError_t run_head_rotate(const uint16_t* src, uint16_t* dst, int64_t vectors,
                             cudaStream_t stream) {
   constexpr int kWarps = 8;
-  const int64_t blocks = std::min<int64_t>((vectors + kWarps - 1) / kWarps,
+  const int64_t blocks = std::min<int64_t>((vectors + kWarps * kBatch - 1) / (kWarps * kBatch),
                                            static_cast<int64_t>(sm_count()) * 8);
   const float scale = static_cast<float>(1.0 / std::sqrt(32.0 * E));
   return launch_pdl(head_rotate_kernel<E>, dim3(static_cast<unsigned>(blocks)), dim3(32 * kWarps),

@@ -1451,6 +1451,8 @@ qr_status launch_kron_rows(const RowJob& job, cudaStream_t stream) {
 // 4-bit codes use the same fma-and-clamp as the row kernels, with 1/sqrt(D)
 // folded into the scale; each lane stores its E nibbles (E / 2 bytes, a
 // coalesced 32 E / 2-byte row per warp) and lane 0 the scale and zero point.
+constexpr int kKvBatch = 4;
+
 template <int E, bool ROT>
 __global__ void __launch_bounds__(256) kv_group_quant_kernel(const __half* __restrict__ src,
                                                              int64_t groups, int head_bits,
@@ -1465,52 +1467,63 @@ __global__ void __launch_bounds__(256) kv_group_quant_kernel(const __half* __res
   using C = typename std::conditional<E == 4, uint16_t, uint32_t>::type;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; g < groups;
-       g += nwarps) {
-    const V raw = *reinterpret_cast<const V*>(src + g * G + lane * E);
-    const __half* h = reinterpret_cast<const __half*>(&raw);
-    float x[E];
+  // kKvBatch groups per warp and iteration: their loads are issued together,
+  // so that enough bytes are in flight to cover the memory latency
+  for (int64_t g0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kKvBatch;
+       g0 < groups; g0 += nwarps * kKvBatch) {
+    V raws[kKvBatch];
 #pragma unroll
-    for (int j = 0; j < E; ++j) x[j] = __half2float(h[j]);
-    if (ROT) {
+    for (int u = 0; u < kKvBatch; ++u)
+      if (g0 + u < groups) raws[u] = *reinterpret_cast<const V*>(src + (g0 + u) * G + lane * E);
 #pragma unroll
-      for (int b = 0; b < LE; ++b)
-        if (b < head_bits)
+    for (int u = 0; u < kKvBatch; ++u) {
+      const int64_t g = g0 + u;
+      if (g >= groups) break;                        // uniform over the warp
+      const V raw = raws[u];
+      const __half* h = reinterpret_cast<const __half*>(&raw);
+      float x[E];
 #pragma unroll
-          for (int j = 0; j < E; ++j)
-            if (!(j & (1 << b))) {
-              const float a = x[j], c = x[j | (1 << b)];
-              x[j] = a + c;
-              x[j | (1 << b)] = a - c;
+      for (int j = 0; j < E; ++j) x[j] = __half2float(h[j]);
+      if (ROT) {
+#pragma unroll
+        for (int b = 0; b < LE; ++b)
+          if (b < head_bits)
+#pragma unroll
+            for (int j = 0; j < E; ++j)
+              if (!(j & (1 << b))) {
+                const float a = x[j], c = x[j | (1 << b)];
+                x[j] = a + c;
+                x[j | (1 << b)] = a - c;
+              }
+#pragma unroll
+        for (int lb = 0; lb < 5; ++lb)
+          if (LE + lb < head_bits) {
+            const bool upper = (lane >> lb) & 1;
+#pragma unroll
+            for (int j = 0; j < E; ++j) {
+              const float o = __shfl_xor_sync(0xffffffffu, x[j], 1 << lb);
+              x[j] = upper ? o - x[j] : x[j] + o;
             }
-#pragma unroll
-      for (int lb = 0; lb < 5; ++lb)
-        if (LE + lb < head_bits) {
-          const bool upper = (lane >> lb) & 1;
-#pragma unroll
-          for (int j = 0; j < E; ++j) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[j], 1 << lb);
-            x[j] = upper ? o - x[j] : x[j] + o;
           }
-        }
-    }
-    float mx = x[0], mn = x[0];
+      }
+      float mx = x[0], mn = x[0];
 #pragma unroll
-    for (int j = 1; j < E; ++j) {
-      mx = fmaxf(mx, x[j]);
-      mn = fminf(mn, x[j]);
-    }
+      for (int j = 1; j < E; ++j) {
+        mx = fmaxf(mx, x[j]);
+        mn = fminf(mn, x[j]);
+      }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    }
-    const RowQ q = asym_row_q(mn, mx, 1.0f, inv_sqrt, lane == 0 ? scales + g : nullptr, zeros + g);
-    C packed = 0;
+      for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      const RowQ q = asym_row_q(mn, mx, 1.0f, inv_sqrt, lane == 0 ? scales + g : nullptr, zeros + g);
+      C packed = 0;
 #pragma unroll
-    for (int j = 0; j < E; ++j)
-      packed |= static_cast<C>(quant_nibble<true>(x[j], q.r, q.c, q.lo, q.hi) << (4 * j));
-    *reinterpret_cast<C*>(codes + g * (G / 2) + lane * (E / 2)) = packed;
+      for (int j = 0; j < E; ++j)
+        packed |= static_cast<C>(quant_nibble<true>(x[j], q.r, q.c, q.lo, q.hi) << (4 * j));
+      *reinterpret_cast<C*>(codes + g * (G / 2) + lane * (E / 2)) = packed;
+    }
   }
 }
 
@@ -1527,7 +1540,8 @@ qr_status launch_kv_group_quant(const uint16_t* src, int64_t groups, int group, 
   while ((1 << hb) < head_dim) ++hb;
   const float inv_sqrt = rotate ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)))
                                 : 1.0f;
-  const int64_t blocks = std::min<int64_t>((groups + 7) / 8, static_cast<int64_t>(sm_count()) * 8);
+  const int64_t blocks = std::min<int64_t>((groups + 8 * kKvBatch - 1) / (8 * kKvBatch),
+                                           static_cast<int64_t>(sm_count()) * 8);
   const auto* x = reinterpret_cast<const __half*>(src);
   cudaError_t e;
   if (group == 128)
