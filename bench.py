@@ -7,8 +7,9 @@ One step is one pass of the layer's online hot path over one batch: rotate +
 quantize the activations (one kernel) and the W4A4 GEMM with its fused
 dequant/outlier epilogue (one kernel).  The weights are rotated and packed
 once, offline, before timing (their time is reported separately).  Default
-workload: the LLaMA-2-7B-shaped fused QKV prefill, X[2048 x 4096] through a
-full 4096-point Hadamard into W[12288 x 4096].
+workload: the largest one-GPU layer, the LLaMA-3-70B-shaped FlatQuant gate+up
+prefill, X[4096 x 8192] through the Kronecker transform P1 (128x128) kron P2
+(64x64) with per-channel scales and clip ratio 0.9, into W[57344 x 8192].
 
 Timing: W warm-up steps, then exactly K steps bracketed by a barrier and a
 device synchronize on both sides, CUDA events on the launching stream, max
@@ -171,15 +172,22 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- workload
 
-def workload_signs(wl, random_signs: bool):
-    """The seeded random-sign diagonal of a randomized Hadamard (or None)."""
-    import oracle as O
+def workload_signs(wl, random_signs: bool, packed_width: int):
+    """The seeded random-sign diagonal of a randomized Hadamard over the
+    `packed_width` rotated columns (or None).  Each arm sizes it with its own
+    implementation's packed width."""
     import workloads
     s = wl.spec
     if not random_signs or s.rotation not in ("hadamard", "gsr"):
         return None
-    probe = O.Rotation({"hadamard": O.HADAMARD, "gsr": O.GSR}[s.rotation], block=s.block)
-    return workloads.random_signs(s.seed, O.packed_width(probe, s.K, s.n_keep_fp16))
+    return workloads.random_signs(s.seed, packed_width)
+
+
+def oracle_signs(wl, random_signs: bool):
+    """workload_signs for the oracle legs (CPU baseline, reference arm)."""
+    import oracle as O
+    return workload_signs(wl, random_signs,
+                          O.packed_width(oracle_rotation(wl), wl.spec.K, wl.spec.n_keep_fp16))
 
 
 def rotation_for(wl, Q, signs=None):
@@ -205,12 +213,12 @@ def oracle_rotation(wl, signs=None):
                       block=s.block, clip_ratio=s.clip_ratio, signs=signs)
 
 
-def algorithmic_counts(wl, M, kp, asym=False):
+def algorithmic_counts(wl, M, kp, asym=False, N=None):
     """Algorithmic work of one step (padding excluded).  Asymmetric activations
     add a zero point per token (written, then read) and a code sum per weight
-    row (read)."""
+    row (read).  N overrides the output width (a sample of the weight rows)."""
     s = wl.spec
-    K, N = s.K, s.N
+    K, N = s.K, (s.N if N is None else N)
     n_out = s.n_keep_fp16
     k_int = K - n_out
     gemm_ops = 2.0 * M * N * k_int + 2.0 * M * N * n_out
@@ -222,6 +230,14 @@ def algorithmic_counts(wl, M, kp, asym=False):
         rq_bytes += M * 4
         gemm_bytes += (M + N) * 4
     return gemm_ops, rq_bytes, gemm_bytes
+
+
+def kron_split_flops(wl, M):
+    """Tensor-core FLOPs of the Kronecker transform of M rows: the two small
+    products vec(P1^T mat(x) P2), 2 M K (n1 + n2) FLOPs, three times over for
+    the fp16 hi/lo split (hi*hi + hi*lo + lo*hi) that keeps fp32 accuracy."""
+    s = wl.spec
+    return 3.0 * 2.0 * M * s.K * (s.n1 + s.n2)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -241,7 +257,8 @@ def run_ours(args, rank, world, local_rank):
     wl = workloads.make_workload(args.workload, M=args.tokens)
     s = wl.spec
     M = wl.X.shape[0]
-    signs = workload_signs(wl, args.random_signs)
+    signs = workload_signs(wl, args.random_signs,
+                           Q.packed_k(rotation_for(wl, Q), s.K, s.n_keep_fp16))
     rot = rotation_for(wl, Q, signs)
     idx = None
     if s.n_keep_fp16:
@@ -395,19 +412,22 @@ def run_ours(args, rank, world, local_rank):
     rq_gbs = rq_bytes / (rq_avg * 1e-3) / 1e9
     int8_sust = peaks["bf16_tflops_sustained"] * INT8_PER_BF16
     int8_burst = peaks["bf16_tflops"] * INT8_PER_BF16
+    timed_s = elapsed_ms * 1e-3
     hbm = peaks["hbm_gbs"]
     clocks = sampler.summary(t0, t1)
     sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
     gemm_name = gemm_kernel_name(M)
-    # the GEMM's bound: tensor cores above the ridge point, HBM below it
-    tensor_bound = gemm_ops / gemm_bytes >= int8_sust * 1e12 / (hbm * 1e9)
+    # the GEMM's bound: tensor cores above the ridge point, HBM below it.
+    # The denominator is the burst figure (the timed region is well under a
+    # second of GPU time); the sustained and datasheet fractions ride along.
+    tensor_bound = gemm_ops / gemm_bytes >= int8_burst * 1e12 / (hbm * 1e9)
     if tensor_bound:
         roofline = {"bound": "tensor", "kernel": gemm_name, "achieved": round(gemm_tops, 1),
-                    "peak": round(int8_sust, 1), "unit": "TOP/s",
-                    "frac": round(gemm_tops / int8_sust, 4),
-                    "peak_source": f"{peak_src} bf16 sustained x {INT8_PER_BF16:g} (nominal "
-                                   f"INT8:BF16)",
-                    "frac_of_burst": round(gemm_tops / int8_burst, 4),
+                    "peak": round(int8_burst, 1), "unit": "TOP/s",
+                    "frac": round(gemm_tops / int8_burst, 4),
+                    "peak_source": f"{peak_src} bf16 burst x {INT8_PER_BF16:g} (nominal "
+                                   f"INT8:BF16); timed region {timed_s:.3f} s",
+                    "frac_of_sustained": round(gemm_tops / int8_sust, 4),
                     "frac_of_datasheet_4500": round(gemm_tops / DATASHEET_INT8_TOPS, 4)}
     else:
         roofline = {"bound": "hbm", "kernel": gemm_name, "achieved": round(gemm_gbs, 1),
@@ -441,10 +461,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
         "roofline": roofline,
-        "rotate_quant": {"bound": "hbm", "kernel": rotate_kernel_name(s, M, sms),
-                         "achieved": round(rq_gbs, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(rq_gbs / hbm, 4), "bytes_per_launch": rq_bytes,
-                         "ms_per_launch": round(rq_avg, 5)},
+        "rotate_quant": rotate_quant_roofline(wl, M, rq_bytes, rq_avg, peaks, peak_src,
+                                              rotate_kernel_name(s, M, sms)),
         "gemm_hbm_bytes_per_launch": gemm_bytes,
         "offline_weight_pack_ms": round(pack_ms, 3),
         "e2e": {"value": round(world * gemm_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
@@ -455,6 +473,40 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     return result
+
+
+def rotate_quant_roofline(wl, M, rq_bytes, rq_ms, peaks, peak_src, kernel):
+    """Roofline of the rotate+quantize launch.  Hadamard and GSR rows are
+    HBM-bound.  The Kronecker transform is bounded by the slower of HBM and
+    its split-precision tensor-core FLOPs (fp16 operands, so the bf16 rate);
+    frac is the bound's time over the measured time."""
+    hbm = peaks["hbm_gbs"]
+    sec = rq_ms * 1e-3
+    gbs = rq_bytes / sec / 1e9
+    out = {"kernel": kernel, "bytes_per_launch": rq_bytes, "ms_per_launch": round(rq_ms, 5),
+           "hbm_achieved_gbs": round(gbs, 1), "hbm_peak_gbs": hbm,
+           "hbm_frac": round(gbs / hbm, 4)}
+    if wl.spec.rotation != "kron":
+        out.update({"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(gbs / hbm, 4),
+                    "peak_source": f"{peak_src} HBM copy bandwidth"})
+        return out
+    flops = kron_split_flops(wl, M)
+    tfs = flops / sec / 1e12
+    t_hbm = rq_bytes / (hbm * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    out.update({"tensor_flops_per_launch": flops, "tensor_achieved_tflops": round(tfs, 1),
+                "tensor_peak_tflops": peaks["bf16_tflops"],
+                "tensor_frac": round(tfs / peaks["bf16_tflops"], 4)})
+    if t_tc >= t_hbm:
+        out.update({"bound": "tensor", "achieved": round(tfs, 1), "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(t_tc / sec, 4),
+                    "peak_source": f"{peak_src} bf16 burst (fp16 operands run at the bf16 rate)"})
+    else:
+        out.update({"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(t_hbm / sec, 4),
+                    "peak_source": f"{peak_src} HBM copy bandwidth"})
+    return out
 
 
 def aggregate_max(value_ms: float, world: int) -> float:
@@ -479,49 +531,76 @@ def oracle_step(O, asym: bool):
     return lambda x, rot, idx, wside: O.linear(O.quantize_activations(x, rot, idx), wside)
 
 
-def oracle_baseline(workload: str, tokens: int, repeats: int = 1, M_total=None,
-                    random_signs: bool = False, asym: bool = False):
-    """Times the CPU oracle's online path on `tokens` tokens of the workload."""
+def _oracle_threads():
+    from threadpoolctl import threadpool_info
+    return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+
+
+def oracle_sample(workload: str, tokens: int, rows, M_total=None, random_signs: bool = False):
+    """The oracle's inputs for a bounded sample of the workload: the first
+    `tokens` tokens and the first `rows` weight rows (all of them when rows
+    is None), with the weights prepared (offline, untimed)."""
     import oracle as O
     import workloads
-    from threadpoolctl import threadpool_info
-
-    wl = workloads.make_workload(workload, M=M_total)
+    wl = workloads.make_workload(workload, M=M_total, N=rows)
     s = wl.spec
-    rot = oracle_rotation(wl, workload_signs(wl, random_signs))
+    rot = oracle_rotation(wl, oracle_signs(wl, random_signs))
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
-    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)     # offline, untimed
+    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)
     x = wl.X[:tokens].astype(np.float64)
+    return wl, rot, idx, wside, x
+
+
+def oracle_baseline(workload: str, tokens: int, rows, repeats: int = 1, M_total=None,
+                    random_signs: bool = False, asym: bool = False, st_tokens: int = 32):
+    """Times the CPU oracle's online path on a bounded sample of the workload
+    (`tokens` tokens against `rows` weight rows) on the host cores, and once
+    more single-threaded on `st_tokens` of those tokens."""
+    import oracle as O
+    from threadpoolctl import threadpool_limits
+
+    wl, rot, idx, wside, x = oracle_sample(workload, tokens, rows, M_total, random_signs)
+    n_rows = wl.W.shape[0]
     run = oracle_step(O, asym)
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
         run(x, rot, idx, wside)
         times.append(time.perf_counter() - t0)
-    gemm_ops, _, _ = algorithmic_counts(wl, tokens, 0)
+    gemm_ops, _, _ = algorithmic_counts(wl, x.shape[0], 0, N=n_rows)
     sec = statistics.median(times)
-    threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    threads = _oracle_threads()
+    st = min(st_tokens, x.shape[0])
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        run(x[:st], rot, idx, wside)
+        st_sec = time.perf_counter() - t0
+    st_ops, _, _ = algorithmic_counts(wl, st, 0, N=n_rows)
     return {"value": round(gemm_ops / sec / 1e12, 6), "unit": "TOPS", "cores": threads,
             "kind": "oracle", "seconds_per_sample": round(sec, 3),
-            "sample": f"{tokens} of {wl.X.shape[0]} tokens of {workload} through the oracle's "
-                      f"online path (rotate+quantize+integer GEMM+epilogue), median of {repeats}; "
-                      f"weights prepared untimed"}
+            "sample": f"{x.shape[0]} of {wl.spec.M} tokens x {n_rows} of {wl.spec.N} weight rows "
+                      f"of {workload} through the oracle's online path (rotate+quantize+integer "
+                      f"GEMM+epilogue), median of {repeats}; weights prepared untimed",
+            "single_thread": {"value": round(st_ops / st_sec / 1e12, 6), "unit": "TOPS",
+                              "cores": 1, "seconds_per_sample": round(st_sec, 3),
+                              "sample": f"{st} tokens x {n_rows} weight rows, one run"}}
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm, on the host cores."""
+    """The oracle as the reference arm, on the host cores: each step runs the
+    oracle's online path on a bounded sample of the workload."""
     if rank != 0:
         return None
     import oracle as O
     import workloads
 
-    wl = workloads.make_workload(args.workload, M=args.tokens)
+    spec = workloads.SPECS[args.workload]
+    M_all = args.tokens or spec.M
+    tokens = min(M_all, args.reference_tokens)
+    rows = min(spec.N, args.reference_rows)
+    wl, rot, idx, wside, x = oracle_sample(args.workload, tokens, rows, args.tokens,
+                                           args.random_signs)
     s = wl.spec
-    tokens = min(wl.X.shape[0], args.reference_tokens)
-    rot = oracle_rotation(wl, workload_signs(wl, args.random_signs))
-    idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
-    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)
-    x = wl.X[:tokens].astype(np.float64)
     run = oracle_step(O, args.asym_activations)
 
     def step():
@@ -533,18 +612,17 @@ def run_reference(args, rank, world):
     for _ in range(args.steps):
         step()
     sec = (time.perf_counter() - t0) / args.steps
-    gemm_ops, _, _ = algorithmic_counts(wl, tokens, 0)
-    from threadpoolctl import threadpool_info
-    threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    gemm_ops, _, _ = algorithmic_counts(wl, tokens, 0, N=rows)
+    threads = _oracle_threads()
     value = gemm_ops / sec / 1e12
-    sample = (f"{tokens} of {wl.X.shape[0]} tokens of {s.name} per step through the oracle's "
-              f"online path; weights prepared untimed")
+    sample = (f"{tokens} of {M_all} tokens x {rows} of {s.N} weight rows of {s.name} per step "
+              f"through the oracle's online path; weights prepared untimed")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": s.name, "M": tokens, "K": s.K, "N": s.N,
+        "config": {"workload": s.name, "M": tokens, "K": s.K, "N": rows,
                    "activations": "asymmetric per-token" if args.asym_activations
                    else "symmetric per-token", "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": threads,
@@ -713,11 +791,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qkv_prefill_4096")
+    ap.add_argument("--workload", default="flatquant_gate_up_8192")
     ap.add_argument("--tokens", type=int, default=None, help="override the token count M")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-baseline-tokens", type=int, default=256)
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=512)
+    ap.add_argument("--cpu-baseline-rows", type=int, default=8192,
+                    help="weight rows in the CPU baseline's sample (capped at N)")
     ap.add_argument("--reference-tokens", type=int, default=64)
+    ap.add_argument("--reference-rows", type=int, default=4096,
+                    help="weight rows in the reference arm's per-step sample (capped at N)")
     ap.add_argument("--random-signs", action="store_true",
                     help="randomized Hadamard: a seeded random-sign diagonal before the blocks")
     ap.add_argument("--asym-activations", action="store_true",
@@ -760,7 +842,8 @@ def main(argv=None):
         elif rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 tokens = min(args.cpu_baseline_tokens, res["config"]["M"])
-                res["cpu_baseline"] = oracle_baseline(args.workload, tokens, repeats=3,
+                rows = min(args.cpu_baseline_rows, res["config"]["N"])
+                res["cpu_baseline"] = oracle_baseline(args.workload, tokens, rows, repeats=3,
                                                       M_total=args.tokens,
                                                       random_signs=args.random_signs,
                                                       asym=args.asym_activations)

@@ -267,7 +267,7 @@ QR_API qr_status qr_invert_transpose(const float* P, int32_t n, float* out,
  * v_codes, v_scales, v_zeros: the same for V without a rotation
  * Q/q_rot, the four K arrays and the four V arrays are each all given or
  * all NULL (a part that is NULL is skipped).  Caller-owned device memory;
- * Q and q_rot 16-byte aligned, k_codes and v_codes 16-byte aligned.
+ * Q, K, V, q_rot, k_codes and v_codes 16-byte aligned (ALIGNMENT otherwise).
  * head_dim in {32, 64, 128, 256}; group 128 or 256, a multiple of head_dim
  * that divides heads*head_dim (UNSUPPORTED otherwise).  Errors: INVALID_ARG
  * for negative sizes or a partly given side, ALIGNMENT, CUDA. */

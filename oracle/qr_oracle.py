@@ -30,8 +30,13 @@ R1  Codes are symmetric in [-(2^(b-1)-1), 2^(b-1)-1] = [-7, 7] for 4 bits;
     the range printed in [SR] Q1/A1 is garbled, -8 is never produced.
 R2  Scale s = alpha * absmax / 7 (min-max, [SR] Q1/A1), alpha the clip ratio
     ([FQ] §2.3 clipping, applied to both sides); codes are clamped to +-7.
-R3  Rounding is round-half-to-even; the code decision is taken in float32,
-    the precision the CUDA kernels take it in.
+R3  Rounding is round-half-to-even.  The pages fix neither the rounding rule
+    nor the precision of x/s; the scale is a float32 number (one per row,
+    the type the layer hands from one step to the next), so the quotient is
+    formed in float32 from the float32 rotated value and scale.  Forming it
+    in another precision moves a code only where x/s lies within a few
+    float32 ulps of a half-integer, inside the 1e-4 tie window that the
+    parity rule leaves open.
 R4  An all-zero row gets s = 0 and all-zero codes.
 R5  Hadamard matrices are Sylvester-ordered, scaled by 1/sqrt(n).
 R6  X' = X R and W' = W R^{-T} with W stored [N out x K in], so that

@@ -1,6 +1,8 @@
 """The N>1 host logic of bench.py on CPU: two gloo ranks, max-over-ranks
 timing, and the launcher checks.  No GPU is touched."""
 import json
+
+import numpy as np
 import os
 import socket
 
@@ -76,8 +78,21 @@ def test_reference_arm_with_random_signs(capsys):
     assert line["impl"] == "reference" and line["config"]["workload"] == "tiny_256"
     import workloads
     wl = workloads.make_workload("tiny_256")
-    d = bench.workload_signs(wl, True)
+    d = bench.oracle_signs(wl, True)
     assert d is not None and d.shape == (256,) and bench.oracle_rotation(wl, d).signs is d
+    # the GPU arm sizes the same signs from its own packed width
+    assert np.array_equal(bench.workload_signs(wl, True, 256), d)
+
+
+def test_gpu_arm_never_reaches_the_oracle():
+    # the GPU arm, and every helper it calls to shape its inputs, imports and
+    # calls nothing from the oracle; only the CPU-baseline and reference legs do
+    import inspect
+    for fn in (bench.run_ours, bench.workload_signs, bench.rotation_for, bench.run_kv,
+               bench.rotate_quant_roofline, bench.algorithmic_counts, bench.kron_split_flops):
+        src = inspect.getsource(fn)
+        assert "import oracle" not in src and "O." not in src, fn.__name__
+        assert "oracle_signs" not in src and "oracle_rotation" not in src, fn.__name__
 
 
 def test_kv_cache_reference_arm(capsys):

@@ -58,7 +58,11 @@ KV_CASES = [
     (1, 32, 128, 128),
     (129, 4, 256, 256),
     (64, 8, 32, 128),
-    (1000, 2, 128, 128),          # many rows: the row-group kernels
+    (1000, 2, 128, 128),          # 2000 groups: one pass of the warps
+    # 40000 groups, more than the grid's warps x groups per warp (at most
+    # sm_count * 8 blocks * 8 warps * 4 groups, 37888 on 148 SMs): the
+    # grid-stride loop runs a second iteration with a ragged batch tail
+    (20000, 2, 128, 128),
 ]
 
 

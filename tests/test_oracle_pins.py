@@ -160,6 +160,17 @@ def test_computational_invariance(kind, block, k):
     np.testing.assert_allclose(np.linalg.norm(xr, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
 
 
+def test_rmsnorm_hand_worked_rows():
+    # x_i <- x_i / ||x_i|| per row (the QuaRot/SpinQuant notes, §1): fixes the
+    # value, which the commutation identity below cannot (any row-wise
+    # normalisation, the identity map included, commutes with Q).
+    from fractions import Fraction
+    for r in read_golden_rows("rmsnorm_3x3.txt"):
+        x = np.array([[float(v) for v in r[:3]]])
+        want = np.array([[float(Fraction(v)) for v in r[3:]]])
+        np.testing.assert_allclose(O.rmsnorm(x), want, rtol=0, atol=1e-15)
+
+
 def test_rmsnorm_commutes_with_rotation():
     # RMSNorm(X) = RMSNorm(X Q^T) Q for orthogonal Q (the QuaRot/SpinQuant notes, §1).
     rng = np.random.default_rng(7)
@@ -364,6 +375,17 @@ def test_rotation_reduces_error_on_outlier_inputs():
         act[name] = np.linalg.norm(deq - a.rotated) / np.linalg.norm(a.rotated)
     assert errs["had"] < errs["none"], errs
     assert act["had"] < 0.6 * act["none"], act
+
+
+def test_incoherence_bound_hand_worked():
+    # mu ||W||_F / sqrt(mn), mu = 2 ln(4mn/delta) (SpinQuant review, reviewer
+    # Jf43 W1/A1): values worked by hand; a log2, a dropped factor 2 or a
+    # missing sqrt(mn) each changes them.
+    for r in read_golden_rows("incoherence_bound.txt"):
+        m, n, delta = int(r[0]), int(r[1]), float(r[2])
+        w = np.array([float(v) for v in r[3:3 + m * n]]).reshape(m, n)
+        want = float(r[3 + m * n]) * np.log(2.0)
+        assert abs(O.incoherence_bound(w, delta) - want) <= 1e-12 * want
 
 
 def test_hadamard_bounds_weight_entries_incoherence():

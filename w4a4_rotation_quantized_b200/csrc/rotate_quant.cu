@@ -1485,9 +1485,10 @@ __global__ void __launch_bounds__(256) kv_group_quant_kernel(const __half* __res
 #pragma unroll
       for (int j = 0; j < E; ++j) x[j] = __half2float(h[j]);
       if (ROT) {
+        // head_dim >= 32 (qr_kv_quantize rejects smaller heads), so
+        // head_bits >= 5 > LE: every element bit is a butterfly stage.
 #pragma unroll
         for (int b = 0; b < LE; ++b)
-          if (b < head_bits)
 #pragma unroll
             for (int j = 0; j < E; ++j)
               if (!(j & (1 << b))) {
