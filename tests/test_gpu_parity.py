@@ -142,6 +142,45 @@ def test_kron_flatquant_factors_with_outliers():
     check_side(gpu, ref, "flatquant+outliers", clip=0.9)
 
 
+def _kron_rows_any_magnitude(wl, m, rng):
+    """Rows of every magnitude for the tensor-core Kronecker kernel: norms
+    from ~1e-2 to ~1e5, a zero row, a constant row, and a row whose x/c
+    exceeds the fp16 range (60000 on a channel with c < 0.9)."""
+    x = rng.standard_normal((m, 8192)).astype(np.float32)
+    x *= (10.0 ** rng.uniform(-4.0, 3.3, size=m)).astype(np.float32)[:, None]
+    x[1] = 0.0
+    x[2] = 0.75
+    ch = int(np.argmin(wl.chan_scale))
+    x[3, ch] = 60000.0
+    return x.astype(np.float16)
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 16, 2 * 148 * 3 + 1])
+def test_kron_tc_rows_of_any_magnitude(m):
+    # one token, one pair, a short pair, and three pairs on most CTAs with a
+    # short last pair; per-token power-of-two normalization keeps every fp16
+    # operand in range
+    wl = workloads.make_workload("flatquant_gate_up_8192", M=8, N=8)
+    rng = np.random.default_rng(1000 + m)
+    x = _kron_rows_any_magnitude(wl, max(m, 4), rng)[:m]
+    rot = O.Rotation(O.KRON, P1=wl.P1, P2=wl.P2, chan_scale=wl.chan_scale, clip_ratio=0.9)
+    gpu, ref = _run_rows(x, rot)
+    check_side(gpu, ref, f"kron tc m={m}", clip=0.9)
+    gpu, ref = _run_rows(x, rot, weights=True)
+    check_side(gpu, ref, f"kron tc weights m={m}", clip=0.9)
+
+
+def test_kron_tc_factor_scales_and_no_channel_scale():
+    # P1 and P2 far from unit scale (normalized by powers of two inside the
+    # kernel), no per-channel scale, no clipping
+    wl = workloads.make_workload("flatquant_gate_up_8192", M=40, N=8)
+    p1 = (wl.P1 * np.float32(3e-3)).astype(np.float32)
+    p2 = (wl.P2 * np.float32(250.0)).astype(np.float32)
+    rot = O.Rotation(O.KRON, P1=p1, P2=p2, chan_scale=None, clip_ratio=1.0)
+    gpu, ref = _run_rows(wl.X, rot)
+    check_side(gpu, ref, "kron tc scaled factors")
+
+
 def test_invert_transpose_matches_numpy():
     wl = workloads.make_workload("flatquant_gate_up_8192", M=1, N=1)
     for p in (wl.P1, wl.P2):

@@ -6,20 +6,37 @@
 // small matrices, Y = P1^T mat(x / c) P2, then quantized per token; the page
 // fuses the two small matmuls with the quantization into one kernel.
 //
-// Here, per token, with mat(x) = X [128 x 64] (row a = x[64a .. 64a+63]):
-//   stage 1  T  = X P2        MMA M = a (128), N = d (64), K = b (64)
-//   stage 2  Y  = P1^T T      MMA M = c (128), N = d (64), K = a (128)
-// Stage 2's B operand is T read "MN-major" (row a of T holds the 64 d's
-// contiguously), so each thread writes its own TMEM row of T straight back to
-// shared memory without a transpose.  fp16 operands carry ~11 bits; every
-// fp32 operand is split into hi = fp16(v) and lo = fp16(v - hi), and each
-// product is hi*hi + hi*lo + lo*hi accumulated in fp32 (relative error about
-// 2^-22), which keeps the rotated rows well inside 1e-5 of the row norm.
+// Shapes: n1 = 128, n2 = 64; mat(x) = X [128 x 64], row a = x[64a .. 64a+63].
+// Per token, two stages on tcgen05 MMAs (M = 128, fp32 accumulators in TMEM):
+//   stage 1  T = X P2        A = X (TMEM, lane a), B = [P2 | P2 lo] (smem)
+//   stage 2  Y = P1^T T      A = P1^T (TMEM, lane c), B = [T_0 | T_1] (smem)
+// fp16 operands carry 11 bits, so every operand v is split into hi = fp16(v)
+// and lo = fp16(v - hi).  Stage 1 puts P2's hi and lo side by side along N
+// (N = 128): the MMAs with X_hi and X_lo give all four cross terms in two
+// column halves that the converter adds.  Stage 2 takes two tokens side by
+// side along N (N = 128) and sums P1hi.Thi + P1hi.Tlo + P1lo.Thi.  Measured
+// tcgen05 rates with A in TMEM (max(64, N/2) clocks per M128 K16 MMA) make
+// both stages run at the full tensor rate: 8 + 12 MMAs of 64 clocks per
+// token.  The dropped lo.lo term is ~2^-22 of each product.
 //
-// One CTA of 128 threads per SM, persistent over tokens; thread i owns TMEM
-// lane i (row a in stage 1, row c in stage 2).  Supports n1 = 128, n2 = 64,
-// no outlier split, 16-byte aligned rows; other shapes use the CUDA-core
-// kernel.
+// Range: each token is scaled by a power of two sigma that puts max|x/c|
+// in [2^7, 2^8), and P1, P2 by powers of two that put their largest entries
+// in [1, 2).  Then no fp16 operand overflows (|T| < 2^15) and the lo parts of
+// everything that matters at the 1e-5 row-norm level stay normal fp16
+// numbers, for any fp16 input.  The scale factors are exact, so the codes
+// equal those of the unscaled arithmetic and the scale is divided back out.
+//
+// Warp roles (one CTA of 17 warps per SM, persistent over pairs of tokens):
+//   warp 0      TMEM allocation, and one thread issuing every MMA
+//   warps 1-8   loaders: x -> x/c -> per-token max -> sigma -> hi/lo -> TMEM
+//               (16 lanes x 4 threads per row, so each warp load touches 8
+//               rows of 64 contiguous bytes; the K order inside a row is
+//               permuted to the store layout and P2's rows follow it)
+//   warps 9-16  converters (stage-1 accumulators -> hi/lo T tiles in smem)
+//               and the epilogue (absmax over the token, codes, scale)
+// MMA issue order, per pair p: S1(2p), S2(p-1) first half, S1(2p+1),
+// S2(p-1) second half, so that the converter's work on one token overlaps
+// the tensor core's work on another.  Every wait is bounded.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -32,8 +49,34 @@ namespace qr {
 namespace {
 
 constexpr int kN1 = 128, kN2 = 64;
-constexpr int kThreadsTc = 128;
+constexpr int kLoadWarps = 8, kPostWarps = 8;
+constexpr int kThreadsTc = 32 * (1 + kLoadWarps + kPostWarps);     // 544
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+constexpr int kXSlots = 8;              // per-token max exchange slots
+
+// TMEM columns (512 allocated)
+constexpr uint32_t kColA1 = 0;          // 2 slots x (X hi 32 | X lo 32)
+constexpr uint32_t kColD1 = 128;        // stage 1: [x P2hi | x P2lo], 128 fp32
+constexpr uint32_t kColP1 = 256;        // P1^T hi 64 | lo 64
+constexpr uint32_t kColD2 = 384;        // stage 2: two tokens x 64 fp32
+
+// shared memory (byte offsets from a 1 KB-aligned base)
+constexpr int kBp2Bytes = 128 * 128;    // 128 rows (n) x 64 fp16 (K), SW128 K-major
+constexpr int kTokT = 128 * 128;        // one token's T, hi or lo: 128 K-rows x 64 fp16
+constexpr int kB2Slot = 4 * kTokT;      // T hi (2 tokens) | T lo (2 tokens)
+constexpr int off_bp2 = 0;
+constexpr int off_b2 = off_bp2 + kBp2Bytes;
+constexpr int off_bar = off_b2 + 2 * kB2Slot;
+// barriers (8 bytes each)
+constexpr int kBarXFull = 0, kBarXEmpty = 2, kBarD1Full = 4, kBarD1Empty = 5,
+              kBarB2Full = 6, kBarB2Empty = 8, kBarD2Full = 10, kBarD2Empty = 11,
+              kBarXMax = 12, kBarYMax = 12 + kXSlots, kBarDrain = kBarYMax + 4,
+              kNumBars = kBarDrain + 1;
+constexpr int off_redx = off_bar + 8 * kNumBars;            // float [kXSlots][8]
+constexpr int off_redy = off_redx + 4 * kXSlots * 8;        // float [2][2][4]
+constexpr int off_pmax = off_redy + 4 * 16;                 // float [17][2]
+constexpr int off_misc = off_pmax + 8 * 17;                 // tmem slot, abort flag
+constexpr int kSmemTc = off_misc + 16 + 1024;
 
 struct KronTcParams {
   const __half* src;
@@ -49,19 +92,6 @@ struct KronTcParams {
   int32_t* status;
 };
 
-// shared-memory carve-up (bytes, 1024-aligned regions)
-constexpr int kA1 = kN1 * kN2 * 2;           // X hi or lo: 128 rows x 128 B
-constexpr int kB1 = kN2 * kN2 * 2;           // P2^T hi or lo: 64 rows x 128 B
-constexpr int kA2 = kN1 * kN1 * 2;           // P1^T hi or lo: two K-halves of 128 x 128 B
-constexpr int kB2 = kN1 * kN2 * 2;           // T hi or lo: 128 K-rows x 128 B (MN-major)
-constexpr int off_a1h = 0, off_a1l = off_a1h + kA1;
-constexpr int off_b1h = off_a1l + kA1, off_b1l = off_b1h + kB1;
-constexpr int off_a2h = off_b1l + kB1, off_a2l = off_a2h + kA2;
-constexpr int off_b2h = off_a2l + kA2, off_b2l = off_b2h + kB2;
-constexpr int off_bar = off_b2l + kB2;
-constexpr int off_red = off_bar + 32;
-constexpr int kSmemTc = off_red + 64 + 1024;
-
 // byte offset of 16-byte chunk j of row r in a 128-byte-swizzled tile whose
 // rows are 128 bytes (8-row atoms of 1 KB)
 __device__ __forceinline__ int sw128(int r, int j) {
@@ -73,29 +103,51 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Splits 8 fp32 values into fp16 hi and lo parts (hi = fp16(v), lo = fp16(v - hi)).
-__device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo) {
-  float h[8];
+// hi = fp16(a), lo = fp16(a - hi), for a pair of values, packed.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 f = __half22float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  float la, lb;
+  f2_unpack(f2_sub(f2_pack(a, b), f2_pack(f.x, f.y)), la, lb);
+  lo = pack_h2(la, lb);
+}
+
+__device__ __forceinline__ void tmem_st_16x256b_x2(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+
+// A power of two f with f * m in [2^e, 2^(e+1)) for finite m > 0; 1 otherwise.
+__device__ __forceinline__ float pow2_normalizer(float m, int e) {
+  const uint32_t bits = __float_as_uint(m);
+  const int ex = static_cast<int>((bits >> 23) & 0xFFu);
+  if (!(m > 0.0f) || ex == 0xFF) return 1.0f;
+  const int f = min(254, max(1, e + 254 - ex));
+  return __uint_as_float(static_cast<uint32_t>(f) << 23);
+}
+
+// K order of stage 1: the MMA's K index kk (TMEM column kk/2 of a row)
+// holds x[a][perm_b(kk)], so that thread c of a row group loads the
+// contiguous b ranges [8c, 8c+8) and [32+8c, 32+8c+8) and stores them with
+// the 16x256b layout (block k, register pair e, half hf).
+__host__ __device__ __forceinline__ int perm_b(int kk) {
+  const int k = kk >> 4, c = (kk >> 2) & 3, e = (kk >> 1) & 1, hf = kk & 1;
+  return 32 * (k >> 1) + 8 * c + 4 * (k & 1) + 2 * e + hf;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) h[i] = __half2float(__float2half_rn(v[i]));
-  hi = make_uint4(pack_h2(h[0], h[1]), pack_h2(h[2], h[3]), pack_h2(h[4], h[5]),
-                  pack_h2(h[6], h[7]));
-  lo = make_uint4(pack_h2(v[0] - h[0], v[1] - h[1]), pack_h2(v[2] - h[2], v[3] - h[3]),
-                  pack_h2(v[4] - h[4], v[5] - h[5]), pack_h2(v[6] - h[6], v[7] - h[7]));
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
-// Descriptors: K-major SW128 (rows of 128 bytes, SBO 1 KB) and MN-major
-// SW128 (128-byte rows along N, 8 K-rows per 1 KB atom, SBO 1 KB).
-__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t addr) {
-  const uint64_t start = (addr >> 4) & 0x3FFFu;
-  const uint64_t lbo = (8192u >> 4);          // stride between 64-wide N atoms (one atom here)
-  const uint64_t sbo = (1024u >> 4);
-  return start | (lbo << 16) | (sbo << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// kind::f16 instruction descriptors: D f32, A/B f16, M=128, N=64;
-// stage 2 reads B MN-major (bit 16).
-constexpr uint32_t kIdescS1 = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+// Kind::f16 instruction descriptor: D f32, A/B f16, M = 128, N = 128; A from
+// TMEM, B K-major (stage 1) or MN-major (stage 2, bit 16).
+constexpr uint32_t kIdescS1 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescS2 = kIdescS1 | (1u << 16);
 
 template <bool CLIP>
@@ -103,207 +155,403 @@ __global__ void __launch_bounds__(kThreadsTc, 1) kron_tc_kernel(const KronTcPara
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + off_bar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 16);
-  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + off_bar + 20);
-  float* red = reinterpret_cast<float*>(smem + off_red);
-  const int i = threadIdx.x;                 // = TMEM lane = row a / row c
-  const int warp = i >> 5, lane = i & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + off_bar);
+  volatile float* red_x = reinterpret_cast<volatile float*>(smem + off_redx);
+  volatile float* red_y = reinterpret_cast<volatile float*>(smem + off_redy);
+  float* pmax = reinterpret_cast<float*>(smem + off_pmax);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_misc);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + off_misc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- constants: P2^T (rows d, K = b) and P1^T (rows c, K = a), hi/lo
-  if (i < kN2) {
-    for (int j = 0; j < 8; ++j) {
-      float v[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = p.p2[(8 * j + e) * kN2 + i];     // P2[b][d = i]
-      uint4 hi, lo;
-      split8(v, hi, lo);
-      *reinterpret_cast<uint4*>(smem + off_b1h + sw128(i, j)) = hi;
-      *reinterpret_cast<uint4*>(smem + off_b1l + sw128(i, j)) = lo;
+  // this CTA's pairs of tokens: pair P = blockIdx.x + i * gridDim.x holds rows
+  // 2P and 2P + 1; an odd row count leaves the last pair one token short
+  const int64_t npairs = (p.rows + 1) >> 1;
+  const int np = static_cast<int>((npairs - 1 - blockIdx.x) / gridDim.x + 1);
+  const bool short_tail =
+      (p.rows & 1) && (blockIdx.x + static_cast<int64_t>(np - 1) * gridDim.x == npairs - 1);
+  const int ntok = 2 * np - (short_tail ? 1 : 0);
+  auto row_of = [&](int t) -> int64_t {
+    return 2 * (blockIdx.x + static_cast<int64_t>(t >> 1) * gridDim.x) + (t & 1);
+  };
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kBarXFull + i], kLoadWarps);
+      mbar_init(&bars[kBarXEmpty + i], 1);
+      mbar_init(&bars[kBarB2Full + i], 2 * kPostWarps);
+      mbar_init(&bars[kBarB2Empty + i], 1);
     }
-  }
-  for (int j = 0; j < 16; ++j) {                                         // a = 8j .. 8j+7
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = p.p1[(8 * j + e) * kN1 + i];      // P1[a][c = i]
-    uint4 hi, lo;
-    split8(v, hi, lo);
-    const int half = j >> 3, jj = j & 7;
-    *reinterpret_cast<uint4*>(smem + off_a2h + half * (kA2 / 2) + sw128(i, jj)) = hi;
-    *reinterpret_cast<uint4*>(smem + off_a2l + half * (kA2 / 2) + sw128(i, jj)) = lo;
-  }
-  // per-thread channel factors of the 64 channels this thread owns (a = i)
-  float cf[64];
-#pragma unroll
-  for (int b = 0; b < 64; ++b) {
-    float c = 1.0f;
-    if (p.chan != nullptr) {
-      const float cv = p.chan[i * 64 + b];
-      c = p.chan_multiply ? cv : 1.0f / cv;
-    }
-    cf[b] = c;
-  }
-  if (i == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bars[kBarD1Full], 1);
+    mbar_init(&bars[kBarD1Empty], kPostWarps);
+    mbar_init(&bars[kBarD2Full], 1);
+    mbar_init(&bars[kBarD2Empty], kPostWarps);
+    for (int i = 0; i < kXSlots; ++i) mbar_init(&bars[kBarXMax + i], kLoadWarps);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[kBarYMax + i], 4);
+    mbar_init(&bars[kBarDrain], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 128);
-    tmem_relinquish();
+  grid_dep_wait();
+  grid_dep_launch();
+
+  // ---- prologue: power-of-two normalizers of P1 and P2
+  {
+    float m1 = 0.0f, m2 = 0.0f;
+    for (int i = threadIdx.x; i < kN1 * kN1; i += kThreadsTc) m1 = fmaxf(m1, fabsf(p.p1[i]));
+    for (int i = threadIdx.x; i < kN2 * kN2; i += kThreadsTc) m2 = fmaxf(m2, fabsf(p.p2[i]));
+    m1 = warp_max(m1);
+    m2 = warp_max(m2);
+    if (lane == 0) {
+      pmax[2 * warp] = m1;
+      pmax[2 * warp + 1] = m2;
+    }
   }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t d1 = tmem, d2 = tmem + 64;
-
-  uint32_t phase = 0;
-  bool ok = true;
-  // prefetch of this thread's 64 halves of the first token
-  uint4 nx[8];
-  int64_t row = blockIdx.x;
-  if (row < p.rows) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.src + row * p.ld + i * 64);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) nx[q] = __ldg(src + q);
-  }
-  for (; row < p.rows && ok; row += gridDim.x) {
-    // ---- X row a = i, scaled, split, into the stage-1 A tiles
-    uint4 cx[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) cx[q] = nx[q];
-    const int64_t next = row + gridDim.x;
-    if (next < p.rows) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.src + next * p.ld + i * 64);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) nx[q] = __ldg(src + q);
+  float rho1, rho2;
+  {
+    float m1 = 0.0f, m2 = 0.0f;
+    for (int w = 0; w < kThreadsTc / 32; ++w) {
+      m1 = fmaxf(m1, pmax[2 * w]);
+      m2 = fmaxf(m2, pmax[2 * w + 1]);
     }
+    rho1 = pow2_normalizer(m1, 0);
+    rho2 = pow2_normalizer(m2, 0);
+  }
+  const int q = warp & 3;                              // TMEM lane quadrant
+  const uint32_t quad_off = static_cast<uint32_t>(32 * q) << 16;
+  float cf[32];                                        // loaders: channel factors
+  float cfmax = 0.0f;
+  if (warp >= 1 && warp <= kLoadWarps) {
+    const int h = (warp - 1) >> 2;
+    // P1^T (rows c = lane row, K = a in [64h, 64h+64)) -> TMEM, hi | lo
+    const int c = 32 * q + lane;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const __half2* h = reinterpret_cast<const __half2*>(&cx[q]);
+    for (int hf = 0; hf < 2; ++hf) {
+      uint32_t hw[16], lw[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int a = 64 * h + 32 * hf + 2 * j;
+        split2(p.p1[a * kN1 + c] * rho1, p.p1[(a + 1) * kN1 + c] * rho1, hw[j], lw[j]);
+      }
+      tmem_st_32x32b_x16(tmem + quad_off + kColP1 + 32 * h + 16 * hf, hw);
+      tmem_st_32x32b_x16(tmem + quad_off + kColP1 + 64 + 32 * h + 16 * hf, lw);
+    }
+    // channel factors of the 32 values this thread loads per token: rows
+    // g and g+8 of its 16-lane half, b in [8c', 8c'+8) and [32+8c', 32+8c'+8)
+    const int g = lane >> 2, cq = lane & 3;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int a = 32 * q + 16 * h + g + 8 * rr;
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float f = 1.0f;
+          if (p.chan != nullptr) {
+            const float cv = p.chan[a * kN2 + 32 * u + 8 * cq + e];
+            f = p.chan_multiply ? cv : 1.0f / cv;
+          }
+          cf[16 * rr + 8 * u + e] = f;
+          cfmax = fmaxf(cfmax, fabsf(f));
+        }
+    }
+    tmem_st_wait();
+  } else if (warp > kLoadWarps) {
+    // [P2 hi | P2 lo] as stage 1's B: row n, K index kk holds P2[perm_b(kk)][n % 64]
+    const int idx = threadIdx.x - 32 * (1 + kLoadWarps);
+    for (int cid = idx; cid < 128 * 8; cid += 32 * kPostWarps) {
+      const int n = cid & 127, ch = cid >> 7, d = n & 63;
       float v[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h[e]);
-        v[2 * e] = f.x * cf[8 * q + 2 * e];
-        v[2 * e + 1] = f.y * cf[8 * q + 2 * e + 1];
-      }
-      uint4 hi, lo;
-      split8(v, hi, lo);
-      *reinterpret_cast<uint4*>(smem + off_a1h + sw128(i, q)) = hi;
-      *reinterpret_cast<uint4*>(smem + off_a1l + sw128(i, q)) = lo;
+      for (int e = 0; e < 8; ++e) v[e] = p.p2[perm_b(8 * ch + e) * kN2 + d] * rho2;
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) split2(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+      const uint32_t* w = (n < 64) ? hi : lo;
+      *reinterpret_cast<uint4*>(smem + off_bp2 + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- stage 1: T = X P2  (hi*hi + hi*lo + lo*hi)
-    if (i == 0) {
-      tc_fence_after();
-      const uint32_t a_h = smem_u32(smem + off_a1h), a_l = smem_u32(smem + off_a1l);
-      const uint32_t b_h = smem_u32(smem + off_b1h), b_l = smem_u32(smem + off_b1l);
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const uint32_t o = 32 * s;
-        mma_f16(d1, smem_desc_kmajor(a_h + o, 128), smem_desc_kmajor(b_h + o, 128), kIdescS1, s > 0);
-        mma_f16(d1, smem_desc_kmajor(a_h + o, 128), smem_desc_kmajor(b_l + o, 128), kIdescS1, 1);
-        mma_f16(d1, smem_desc_kmajor(a_l + o, 128), smem_desc_kmajor(b_h + o, 128), kIdescS1, 1);
-      }
-      mma_commit(bar);
-    }
-    if (!(ok = mbar_wait_bounded(bar, phase, abort_flag, p.status, kDevTimeoutMma))) break;
-    phase ^= 1;
-    tc_fence_after();
-    // ---- T row a = i (64 fp32) -> hi/lo, MN-major stage-2 B tiles
-    {
-      uint32_t t[64];
-      uint32_t (&t0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&t[0]);
-      uint32_t (&t1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&t[32]);
-      tmem_ld_32x32b_x32(d1 + lane_off, t0);
-      tmem_ld_32x32b_x32(d1 + lane_off + 32, t1);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(t[8 * j + e]);
-        uint4 hi, lo;
-        split8(v, hi, lo);
-        *reinterpret_cast<uint4*>(smem + off_b2h + sw128(i, j)) = hi;
-        *reinterpret_cast<uint4*>(smem + off_b2l + sw128(i, j)) = lo;
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- stage 2: Y = P1^T T  (K = a in 8 steps of 16)
-    if (i == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint32_t ao = (s >> 2) * (kA2 / 2) + 32 * (s & 3);
-        const uint32_t bo = 2048 * s;
-        const uint64_t ah = smem_desc_kmajor(smem_u32(smem + off_a2h) + ao, 128);
-        const uint64_t al = smem_desc_kmajor(smem_u32(smem + off_a2l) + ao, 128);
-        const uint64_t bh = desc_mn_sw128(smem_u32(smem + off_b2h) + bo);
-        const uint64_t bl = desc_mn_sw128(smem_u32(smem + off_b2l) + bo);
-        mma_f16(d2, ah, bh, kIdescS2, s > 0);
-        mma_f16(d2, ah, bl, kIdescS2, 1);
-        mma_f16(d2, al, bh, kIdescS2, 1);
-      }
-      mma_commit(bar);
-    }
-    if (!(ok = mbar_wait_bounded(bar, phase, abort_flag, p.status, kDevTimeoutMma))) break;
-    phase ^= 1;
-    tc_fence_after();
-    // ---- Y row c = i: absmax over the token, quantize, pack, store
-    uint32_t y[64];
-    uint32_t (&y0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&y[0]);
-    uint32_t (&y1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&y[32]);
-    tmem_ld_32x32b_x32(d2 + lane_off, y0);
-    tmem_ld_32x32b_x32(d2 + lane_off + 32, y1);
-    tmem_ld_wait();
-    float am = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 64; ++j) am = fmaxf(am, fabsf(__uint_as_float(y[j])));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-    if (lane == 0) red[warp] = am;
-    tc_fence_before();
-    __syncthreads();
-    am = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    const float s = (p.clip_ratio * am) / 7.0f;
-    const float r = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
-    if (i == 0) p.scales[row] = s;
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float t = fmaf(__uint_as_float(y[8 * j + e]), r, kMagic);
-        if (CLIP) t = fminf(fmaxf(t, kMagic - 7.0f), kMagic + 7.0f);
-        word |= (__float_as_uint(t) & 0xFu) << (4 * e);
-      }
-      w[j] = word;
-    }
-    uint4* cdst = reinterpret_cast<uint4*>(p.codes + row * (kN1 * kN2 / 2) + i * 32);
-    cdst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    cdst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    if (p.rot_debug != nullptr) {
-      float* dd = p.rot_debug + row * (kN1 * kN2) + i * 64;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) dd[j] = __uint_as_float(y[j]);
-    }
-    __syncthreads();     // red, A1, B2 are reused by the next token
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  auto wait = [&](int b, uint32_t parity, int32_t code) -> bool {
+    return mbar_wait_bounded(&bars[b], parity, abort_flag, p.status, code);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t bp2 = smem_u32(smem + off_bp2);
+      auto s1 = [&](int t) -> bool {
+        const int j = t & 1;
+        if (!wait(kBarXFull + j, (t >> 1) & 1, kDevTimeoutMma)) return false;
+        if (t >= 1 && !wait(kBarD1Empty, (t - 1) & 1, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t a = tmem + kColA1 + 64 * j;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_f16_ts(tmem + kColD1, a + 8 * k, smem_desc_kmajor(bp2 + 32 * k, 128), kIdescS1, k > 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_f16_ts(tmem + kColD1, a + 32 + 8 * k, smem_desc_kmajor(bp2 + 32 * k, 128), kIdescS1, 1);
+        mma_commit(&bars[kBarXEmpty + j]);
+        mma_commit(&bars[kBarD1Full]);
+        return true;
+      };
+      auto s2 = [&](int pr, int half) -> bool {
+        const int sl = pr & 1;
+        if (half == 0) {
+          if (!wait(kBarB2Full + sl, (pr >> 1) & 1, kDevTimeoutMma)) return false;
+          if (pr >= 1 && !wait(kBarD2Empty, (pr - 1) & 1, kDevTimeoutMma)) return false;
+          tc_fence_after();
+        }
+        const uint32_t bh = smem_u32(smem + off_b2 + sl * kB2Slot), bl = bh + 2 * kTokT;
+#pragma unroll
+        for (int s = 4 * half; s < 4 * half + 4; ++s) {
+          const uint64_t dh = smem_desc_mn_sw128(bh + 2048 * s, kTokT);
+          const uint64_t dl = smem_desc_mn_sw128(bl + 2048 * s, kTokT);
+          mma_f16_ts(tmem + kColD2, tmem + kColP1 + 8 * s, dh, kIdescS2, s > 0);
+          mma_f16_ts(tmem + kColD2, tmem + kColP1 + 8 * s, dl, kIdescS2, 1);
+          mma_f16_ts(tmem + kColD2, tmem + kColP1 + 64 + 8 * s, dh, kIdescS2, 1);
+        }
+        if (half == 1) {
+          mma_commit(&bars[kBarB2Empty + sl]);
+          mma_commit(&bars[kBarD2Full]);
+        }
+        return true;
+      };
+      bool ok = true;
+      for (int pr = 0; pr < np && ok; ++pr) {
+        ok = s1(2 * pr);
+        if (ok && pr > 0) ok = s2(pr - 1, 0);
+        if (ok && 2 * pr + 1 < ntok) ok = s1(2 * pr + 1);
+        if (ok && pr > 0) ok = s2(pr - 1, 1);
+      }
+      if (ok) ok = s2(np - 1, 0);
+      if (ok) s2(np - 1, 1);
+      mma_commit(&bars[kBarDrain]);
+      mbar_wait_bounded(&bars[kBarDrain], 0, abort_flag, p.status, kDevTimeoutDrain,
+                        kDrainLimitNs);
+    }
+  } else if (warp <= kLoadWarps) {
+    // ------------------------------------------------------------ loaders
+    const int h = (warp - 1) >> 2, wi = warp - 1;
+    const int g = lane >> 2, cq = lane & 3;
+    const int a0 = 32 * q + 16 * h + g;                // rows a0 and a0 + 8
+    const uint32_t lanes16 = static_cast<uint32_t>(32 * q + 16 * h) << 16;
+    auto load = [&](uint4 (&b)[4], int t) {
+      const __half* base = p.src + row_of(t) * p.ld;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          b[2 * rr + u] = __ldg(reinterpret_cast<const uint4*>(
+              base + (a0 + 8 * rr) * kN2 + 32 * u + 8 * cq));
+    };
+    // One token: per-token normalizer sigma, hi/lo split, TMEM store.  sigma
+    // comes from an upper bound of max|x/c| (each thread's max|x| times its
+    // largest channel factor), exchanged among the loader warps: it keeps
+    // sigma |x/c| below 2^8 and is within a factor max(c)/min(c) of tight.
+    auto step = [&](uint4 (&b)[4], int t) -> bool {
+      __half2 hm = __float2half2_rn(0.0f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2* hx = reinterpret_cast<const __half2*>(&b[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hm = __hmax2(hm, __habs2(hx[e]));
+      }
+      const float2 hmf = __half22float2(hm);
+      const float m = warp_max(fmaxf(hmf.x, hmf.y) * cfmax);
+      const int xs = t & (kXSlots - 1);
+      if (lane == 0) {
+        red_x[xs * 8 + wi] = m;
+        mbar_arrive(&bars[kBarXMax + xs]);
+      }
+      if (!wait(kBarXMax + xs, (t >> 3) & 1, kDevTimeoutProducer)) return false;
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, red_x[xs * 8 + i]);
+      const float sg = pow2_normalizer(mx, 7);
+      const uint64_t sg2 = f2_pack(sg, sg), zero2 = f2_pack(0.0f, 0.0f);
+      if (t >= 2 && !wait(kBarXEmpty + (t & 1), ((t >> 1) - 1) & 1, kDevTimeoutProducer))
+        return false;
+      tc_fence_after();
+      const uint32_t col = tmem + lanes16 + kColA1 + 64 * (t & 1);
+      // registers of the 16x256b stores: block k, lane half rr, column pair
+      // e: K indices 16k + 4cq + 2e + {0, 1} of row a0 + 8rr, i.e. b =
+      // 32(k>>1) + 8cq + 4(k&1) + 2e + {0, 1}: elements 4(k&1) + 2e, +1 of
+      // load b[2rr + (k>>1)].  Two stores of two blocks each.
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        uint32_t hw[8], lw[8];
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int k = 2 * k2 + kk;
+              const int li = 2 * rr + (k >> 1), el = 4 * (k & 1) + 2 * e;
+              const float2 f = __half22float2(reinterpret_cast<const __half2*>(&b[li])[el >> 1]);
+              const int ci = 8 * li + el;
+              const uint64_t v = f2_fma(f2_fma(f2_pack(f.x, f.y), f2_pack(cf[ci], cf[ci + 1]), zero2),
+                                        sg2, zero2);
+              float v0, v1;
+              f2_unpack(v, v0, v1);
+              split2(v0, v1, hw[4 * kk + 2 * rr + e], lw[4 * kk + 2 * rr + e]);
+            }
+        tmem_st_16x256b_x2(col + 16 * k2, hw);
+        tmem_st_16x256b_x2(col + 32 + 16 * k2, lw);
+      }
+      if (t + 2 < ntok) load(b, t + 2);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarXFull + (t & 1)]);
+      return true;
+    };
+    uint4 b0[4], b1[4];
+    if (ntok > 0) load(b0, 0);
+    if (ntok > 1) load(b1, 1);
+    bool ok = true;
+    for (int t = 0; t < ntok && ok; t += 2) {
+      ok = step(b0, t);
+      if (ok && t + 1 < ntok) ok = step(b1, t + 1);
+    }
+  } else {
+    // ------------------------------------------------------------ converters + epilogue
+    const int h = (warp - 1 - kLoadWarps) >> 2;
+    const int r = 32 * q + lane;                       // TMEM lane: row a, then row c
+    auto conv = [&](int t) -> bool {
+      const int pr = t >> 1, j = t & 1, sl = pr & 1;
+      if (!wait(kBarD1Full, t & 1, kDevTimeoutWiden)) return false;
+      tc_fence_after();
+      uint32_t u[32], w[32];
+      tmem_ld_32x32b_x32(tmem + quad_off + kColD1 + 32 * h, u);
+      tmem_ld_32x32b_x32(tmem + quad_off + kColD1 + 64 + 32 * h, w);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarD1Empty]);
+      uint32_t hw[16], lw[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float t0, t1;
+        f2_unpack(f2_add(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])),
+                         f2_pack(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]))),
+                  t0, t1);
+        split2(t0, t1, hw[i], lw[i]);
+      }
+      if (j == 0 && pr >= 2 && !wait(kBarB2Empty + sl, ((pr >> 1) - 1) & 1, kDevTimeoutWiden))
+        return false;
+      uint8_t* th = smem + off_b2 + sl * kB2Slot + j * kTokT;
+      uint8_t* tl = th + 2 * kTokT;
+#pragma unroll
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const int ch = 4 * h + m4;
+        *reinterpret_cast<uint4*>(th + sw128(r, ch)) =
+            make_uint4(hw[4 * m4], hw[4 * m4 + 1], hw[4 * m4 + 2], hw[4 * m4 + 3]);
+        *reinterpret_cast<uint4*>(tl + sw128(r, ch)) =
+            make_uint4(lw[4 * m4], lw[4 * m4 + 1], lw[4 * m4 + 2], lw[4 * m4 + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarB2Full + sl]);
+      return true;
+    };
+    auto epi = [&](int pr) -> bool {
+      const int t = 2 * pr + h;
+      if (!wait(kBarD2Full, pr & 1, kDevTimeoutEpilogue)) return false;
+      tc_fence_after();
+      uint32_t y[64];
+      tmem_ld_32x32b_x32(tmem + quad_off + kColD2 + 64 * h,
+                         *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
+      tmem_ld_32x32b_x32(tmem + quad_off + kColD2 + 64 * h + 32,
+                         *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarD2Empty]);
+      if (t >= ntok) return true;                      // the missing token of a short pair
+      float am = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) am = fmaxf(am, fabsf(__uint_as_float(y[i])));
+      am = warp_max(am);
+      const int ys = pr & 1;
+      if (lane == 0) {
+        red_y[(ys * 2 + h) * 4 + q] = am;
+        mbar_arrive(&bars[kBarYMax + 2 * ys + h]);
+      }
+      if (!wait(kBarYMax + 2 * ys + h, (pr >> 1) & 1, kDevTimeoutEpilogue)) return false;
+      am = fmaxf(fmaxf(red_y[(ys * 2 + h) * 4 + 0], red_y[(ys * 2 + h) * 4 + 1]),
+                 fmaxf(red_y[(ys * 2 + h) * 4 + 2], red_y[(ys * 2 + h) * 4 + 3]));
+      // the token's normalizer, from the loaders' exchange slot (still intact:
+      // the loaders reuse it only eight tokens later)
+      const int xs = t & (kXSlots - 1);
+      if (!wait(kBarXMax + xs, (t >> 3) & 1, kDevTimeoutEpilogue)) return false;
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, red_x[xs * 8 + i]);
+      const float unscale = (1.0f / pow2_normalizer(mx, 7)) * (1.0f / rho1) * (1.0f / rho2);
+      const float rcp = (am > 0.0f) ? 7.0f / (p.clip_ratio * am) : 0.0f;
+      const int64_t row = row_of(t);
+      if (r == 0) p.scales[row] = ((p.clip_ratio * am) / 7.0f) * unscale;
+      uint32_t wd[8];
+#pragma unroll
+      for (int jw = 0; jw < 8; ++jw) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float v = fmaf(__uint_as_float(y[8 * jw + e]), rcp, kMagic);
+          if (CLIP) v = fminf(fmaxf(v, kMagic - 7.0f), kMagic + 7.0f);
+          word |= (__float_as_uint(v) & 0xFu) << (4 * e);
+        }
+        wd[jw] = word;
+      }
+      uint4* cdst = reinterpret_cast<uint4*>(p.codes + row * (kN1 * kN2 / 2) + r * 32);
+      cdst[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      cdst[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+      if (p.rot_debug != nullptr) {
+        float4* dd = reinterpret_cast<float4*>(p.rot_debug + row * (kN1 * kN2) + r * 64);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          dd[i] = make_float4(__uint_as_float(y[4 * i]) * unscale,
+                              __uint_as_float(y[4 * i + 1]) * unscale,
+                              __uint_as_float(y[4 * i + 2]) * unscale,
+                              __uint_as_float(y[4 * i + 3]) * unscale);
+      }
+      return true;
+    };
+    bool ok = true;
+    for (int pr = 0; pr < np && ok; ++pr) {
+      ok = conv(2 * pr);
+      if (ok) {
+        if (2 * pr + 1 < ntok) {
+          ok = conv(2 * pr + 1);
+        } else {                                       // short pair: nothing to convert
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kBarB2Full + (pr & 1)]);
+        }
+      }
+      if (ok && pr > 0) ok = epi(pr - 1);
+    }
+    if (ok) epi(np - 1);
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -312,12 +560,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) kron_tc_kernel(const KronTcPara
 bool kron_tc_supported(const RowJob& job) {
   const qr_rotation& rot = *job.rot;
   return rot.n1 == kN1 && rot.n2 == kN2 && job.n_out == 0 && job.Kp == kN1 * kN2 &&
-         (reinterpret_cast<uintptr_t>(job.src) % 16 == 0) && (job.ld % 8 == 0) &&
-         (reinterpret_cast<uintptr_t>(job.codes) % 16 == 0);
+         job.zeros == nullptr && (reinterpret_cast<uintptr_t>(job.src) % 16 == 0) &&
+         (job.ld % 8 == 0) && (reinterpret_cast<uintptr_t>(job.codes) % 16 == 0) &&
+         (job.rot_debug == nullptr || reinterpret_cast<uintptr_t>(job.rot_debug) % 16 == 0);
 }
 
 qr_status launch_kron_tc(const RowJob& job, cudaStream_t stream) {
   const qr_rotation& rot = *job.rot;
+  if (job.rows == 0) return QR_OK;
   KronTcParams p{};
   p.src = reinterpret_cast<const __half*>(job.src);
   p.rows = job.rows;
@@ -332,14 +582,17 @@ qr_status launch_kron_tc(const RowJob& job, cudaStream_t stream) {
   p.rot_debug = job.rot_debug;
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
-  const int grid = static_cast<int>(std::min<int64_t>(job.rows, sm_count()));
+  const int64_t npairs = (job.rows + 1) / 2;
+  const int grid = static_cast<int>(std::min<int64_t>(npairs, sm_count()));
   cudaError_t e;
   if (rot.clip_ratio < 1.0f) {
     e = cudaFuncSetAttribute(kron_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
-    if (e == cudaSuccess) kron_tc_kernel<true><<<grid, kThreadsTc, kSmemTc, stream>>>(p);
+    if (e == cudaSuccess)
+      e = launch_pdl(kron_tc_kernel<true>, dim3(grid), dim3(kThreadsTc), kSmemTc, stream, 1, p);
   } else {
     e = cudaFuncSetAttribute(kron_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
-    if (e == cudaSuccess) kron_tc_kernel<false><<<grid, kThreadsTc, kSmemTc, stream>>>(p);
+    if (e == cudaSuccess)
+      e = launch_pdl(kron_tc_kernel<false>, dim3(grid), dim3(kThreadsTc), kSmemTc, stream, 1, p);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;

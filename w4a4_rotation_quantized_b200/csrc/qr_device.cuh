@@ -17,6 +17,7 @@ enum DeviceCode : int32_t {
   kDevTimeoutMma = 0x103,
   kDevTimeoutEpilogue = 0x104,
   kDevTimeoutDrain = 0x105,
+  kDevTimeoutSelfCheck = 0x1FF,
 };
 
 // A wait gives up after this long (globaltimer nanoseconds).  A healthy
@@ -558,6 +559,47 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint32_t a,
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a),
                "r"(b), "r"(c), "r"(d)
                : "memory");
+}
+
+}  // namespace qr
+
+namespace qr {
+
+// D(tmem, fp32) (+)= A(tmem) x B(smem)^T, fp16 operands, M = 128 (one CTA).
+// A holds two fp16 K-elements per 32-bit column (element 2j in the low half).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Stores four blocks of 8 consecutive 32-bit columns of 16 TMEM lanes
+// (lanes taddr.lane .. +15) in the MMA accumulator-fragment order: thread
+// 4g + c holds, for block k, registers 4k..4k+3 = (lane g, col 8k+2c),
+// (lane g, col 8k+2c+1), (lane g+8, col 8k+2c), (lane g+8, col 8k+2c+1).
+__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte-swizzled
+// canonical layout: atoms of 64 fp16 along MN (128-byte rows) by 8 rows
+// along K (1 KB); `atom_stride` bytes between atoms along MN (LBO), 1 KB
+// between 8-row groups along K (SBO).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t smem_addr, uint32_t atom_stride) {
+  const uint64_t start = (smem_addr >> 4) & 0x3FFFu;
+  const uint64_t lbo = (atom_stride >> 4) & 0x3FFFu;
+  const uint64_t sbo = 1024u >> 4;
+  return start | (lbo << 16) | (sbo << 32) | (1ull << 46) | (2ull << 61);
 }
 
 }  // namespace qr
