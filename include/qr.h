@@ -277,10 +277,31 @@ QR_API qr_status qr_kv_quantize(const uint16_t* Q, const uint16_t* K, const uint
                                 int32_t* k_zeros, uint8_t* v_codes, float* v_scales,
                                 int32_t* v_zeros, qr_stream stream);
 
+/* Codes a kernel records in the device status word when one of its bounded
+ * waits runs out (the role that gave up); 0 = nothing recorded. */
+#define QR_DEV_TIMEOUT_PRODUCER  0x101   /* a loader / producer role */
+#define QR_DEV_TIMEOUT_WIDEN     0x102   /* an operand-conversion role */
+#define QR_DEV_TIMEOUT_MMA       0x103   /* the MMA-issuing thread */
+#define QR_DEV_TIMEOUT_EPILOGUE  0x104   /* an epilogue role */
+#define QR_DEV_TIMEOUT_DRAIN     0x105   /* draining in-flight work on abort */
+#define QR_DEV_TIMEOUT_SELFCHECK 0x1FF   /* qr_check_wait_timeout */
+
 /* Reads, and clears, the current device's status word that kernels set when
  * a bounded wait ran out.  Synchronizes the device.  *code_out = 0 when no
  * kernel reported anything. */
 QR_API qr_status qr_device_status(int32_t* code_out);
+
+/* Failure-detection self-check.  The pages have no counterpart: this checks
+ * the library's own guard against a wait that never ends.  Launches one
+ * thread on `stream` that waits, for at most limit_ns nanoseconds, on an
+ * mbarrier that nothing ever arrives on, through the same bounded-wait
+ * routine every kernel of the library uses.  The wait runs out, records
+ * QR_DEV_TIMEOUT_SELFCHECK in the device status word (unless a code is
+ * already there) and the kernel returns normally: no fault, no trap, and the
+ * CUDA context stays usable.  Read and clear the code with
+ * qr_device_status().  limit_ns in [1000, 100000000] (1 us to 0.1 s).
+ * Errors: INVALID_ARG for a limit outside that range, CUDA. */
+QR_API qr_status qr_check_wait_timeout(int64_t limit_ns, qr_stream stream);
 
 #ifdef __cplusplus
 }

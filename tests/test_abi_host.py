@@ -191,3 +191,9 @@ def test_kv_quantize_argument_errors(lib):
     assert kv(tokens=0) == L.QR_OK
     assert kv(q=None, k=None, v=None, qr=None, kc=None, ks=None, kz=None, vc=None, vs=None,
               vz=None) == L.QR_OK
+
+
+def test_wait_selfcheck_argument_errors(lib):
+    # the limit is validated on the host, before any launch
+    for bad in (0, 999, 100000001, -5):
+        assert L.qr_check_wait_timeout(bad, None, check=False) == L.QR_ERR_INVALID_ARG

@@ -17,7 +17,11 @@ QR_CHAN_DIVIDE, QR_CHAN_MULTIPLY = 0, 1
 EXPORTED = ("qr_abi_version", "qr_status_string", "qr_packed_k", "qr_rotate_quant",
             "qr_pack_weights", "qr_w4a4_linear", "qr_select_outliers",
             "qr_invert_transpose", "qr_device_status", "qr_rotate_quant_asym",
-            "qr_weight_code_sums", "qr_w4a4_linear_asym", "qr_kv_quantize")
+            "qr_weight_code_sums", "qr_w4a4_linear_asym", "qr_kv_quantize",
+            "qr_check_wait_timeout")
+
+# codes of the device status word (qr_device_status)
+QR_DEV_TIMEOUT_SELFCHECK = 0x1FF
 
 
 class QrRotation(ctypes.Structure):
@@ -74,6 +78,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                vp, i64, vp, vp]),
         "qr_kv_quantize": (ctypes.c_int, [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                           vp, vp]),
+        "qr_check_wait_timeout": (ctypes.c_int, [i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -186,3 +191,10 @@ def qr_device_status() -> int:
     code = ctypes.c_int32(0)
     _check("qr_device_status", load().qr_device_status(ctypes.byref(code)))
     return code.value
+
+
+def qr_check_wait_timeout(limit_ns: int, stream, *, check=True) -> int:
+    st = load().qr_check_wait_timeout(limit_ns, stream)
+    if check:
+        _check("qr_check_wait_timeout", st)
+    return st

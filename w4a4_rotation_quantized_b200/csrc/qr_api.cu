@@ -5,9 +5,17 @@
 #include <cmath>
 #include <mutex>
 
+#include "qr_device.cuh"
 #include "qr_internal.h"
 
 namespace qr {
+
+static_assert(QR_DEV_TIMEOUT_PRODUCER == kDevTimeoutProducer &&
+                  QR_DEV_TIMEOUT_WIDEN == kDevTimeoutWiden && QR_DEV_TIMEOUT_MMA == kDevTimeoutMma &&
+                  QR_DEV_TIMEOUT_EPILOGUE == kDevTimeoutEpilogue &&
+                  QR_DEV_TIMEOUT_DRAIN == kDevTimeoutDrain &&
+                  QR_DEV_TIMEOUT_SELFCHECK == kDevTimeoutSelfCheck,
+              "status codes of the header and of the kernels");
 
 namespace {
 
@@ -304,6 +312,12 @@ qr_status qr_invert_transpose(const float* P, int32_t n, float* out, int32_t* in
   if (P == nullptr || out == nullptr || info == nullptr || n < 1) return QR_ERR_INVALID_ARG;
   if (n > 128) return QR_ERR_UNSUPPORTED;
   return launch_invert_transpose(P, n, out, info, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qr_status qr_check_wait_timeout(int64_t limit_ns, qr_stream stream) {
+  if (limit_ns < 1000 || limit_ns > 100000000) return QR_ERR_INVALID_ARG;
+  return launch_wait_selfcheck(static_cast<uint64_t>(limit_ns),
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 qr_status qr_device_status(int32_t* code_out) {

@@ -119,6 +119,9 @@ qr_status launch_kv_group_quant(const uint16_t* src, int64_t groups, int group, 
 qr_status launch_code_row_sums(const uint8_t* codes, int64_t rows, int64_t kp, int32_t* sums,
                                cudaStream_t stream);
 
+// One thread waits, with the given limit, on an mbarrier nothing arrives on.
+qr_status launch_wait_selfcheck(uint64_t limit_ns, cudaStream_t stream);
+
 qr_status launch_invert_transpose(const float* P, int32_t n, float* out, int32_t* info,
                                   cudaStream_t stream);
 
