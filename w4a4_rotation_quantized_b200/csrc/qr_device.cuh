@@ -577,20 +577,6 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
-// Stores four blocks of 8 consecutive 32-bit columns of 16 TMEM lanes
-// (lanes taddr.lane .. +15) in the MMA accumulator-fragment order: thread
-// 4g + c holds, for block k, registers 4k..4k+3 = (lane g, col 8k+2c),
-// (lane g, col 8k+2c+1), (lane g+8, col 8k+2c), (lane g+8, col 8k+2c+1).
-__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
 // Shared-memory descriptor of an MN-major operand in the 128-byte-swizzled
 // canonical layout: atoms of 64 fp16 along MN (128-byte rows) by 8 rows
 // along K (1 KB); `atom_stride` bytes between atoms along MN (LBO), 1 KB

@@ -336,7 +336,11 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
           constexpr int kTasks = S::kHalf * 4;
 #pragma unroll 1
           for (int task = arow; task < kTasks; task += kGroupThreads) {
-            const int row = task >> 2, c = task & 3;
+            // eight consecutive threads take eight consecutive rows (one
+            // 128-byte swizzle atom) at the same chunk c: their 16-byte reads
+            // (chunk (4h + c) ^ row) and writes ((2c, 2c+1) ^ row) then fall in
+            // eight distinct bank groups
+            const int row = (task & 7) | ((task >> 5) << 3), c = (task >> 3) & 3;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint4 u = *reinterpret_cast<const uint4*>(pb + row * kSlot + (((4 * h + c) ^ (row & 7)) << 4));
