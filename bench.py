@@ -461,8 +461,10 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
         "roofline": roofline,
-        "rotate_quant": rotate_quant_roofline(wl, M, rq_bytes, rq_avg, peaks, peak_src,
-                                              rotate_kernel_name(s, M, sms)),
+        "rotate_quant": dict(rotate_quant_roofline(wl, M, rq_bytes, rq_avg, peaks, peak_src,
+                                                   rotate_kernel_name(s, M, sms)),
+                             traffic=dram_traffic(rotate_kernel_name(s, M, sms), s.name)
+                             if M == s.M else None),
         "gemm_hbm_bytes_per_launch": gemm_bytes,
         "offline_weight_pack_ms": round(pack_ms, 3),
         "e2e": {"value": round(world * gemm_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
