@@ -54,6 +54,7 @@ KERNEL_SOURCES = {
     "wht_ab_kernel": ["rotate_quant.cu", "qr_device.cuh"],
     "wht_few_rows_kernel": ["rotate_quant.cu", "qr_device.cuh"],
     "kron_tc_kernel": ["kron_tc.cu", "qr_device.cuh"],
+    "w8a8_gemm_kernel": ["w8a8_gemm.cu", "qr_device.cuh"],
 }
 DECODE_MAX_TOKENS = 64          # the GEMM runs its decode kernel up to here
 
@@ -80,7 +81,9 @@ def dram_traffic(kernel: str, workload: str):
     return rec.get("bytes")
 
 
-def gemm_kernel_name(M: int) -> str:
+def gemm_kernel_name(M: int, bits: int = 4) -> str:
+    if bits == 8:
+        return "w8a8_gemm_kernel"
     return "w4a4_gemm_decode_kernel" if M <= DECODE_MAX_TOKENS else "w4a4_gemm_pair_kernel"
 
 
@@ -216,16 +219,18 @@ def oracle_rotation(wl, signs=None):
 def algorithmic_counts(wl, M, kp, asym=False, N=None):
     """Algorithmic work of one step (padding excluded).  Asymmetric activations
     add a zero point per token (written, then read) and a code sum per weight
-    row (read).  N overrides the output width (a sample of the weight rows)."""
+    row (read).  N overrides the output width (a sample of the weight rows).
+    Codes take half a byte each, or one byte in an 8-bit layer."""
     s = wl.spec
     K, N = s.K, (s.N if N is None else N)
+    cb = s.bits / 8.0                       # bytes per code
     n_out = s.n_keep_fp16
     k_int = K - n_out
     gemm_ops = 2.0 * M * N * k_int + 2.0 * M * N * n_out
     # rotate+quant: read X, write packed codes, scales (and the fp16 outlier copy)
-    rq_bytes = M * K * 2 + M * k_int / 2 + M * 4 + M * n_out * 2
+    rq_bytes = M * K * 2 + M * k_int * cb + M * 4 + M * n_out * 2
     # GEMM: read codes, scales and outlier columns, write Y
-    gemm_bytes = (M + N) * k_int / 2 + (M + N) * 4 + (M + N) * n_out * 2 + M * N * 2
+    gemm_bytes = (M + N) * k_int * cb + (M + N) * 4 + (M + N) * n_out * 2 + M * N * 2
     if asym:
         rq_bytes += M * 4
         gemm_bytes += (M + N) * 4
@@ -265,6 +270,9 @@ def run_ours(args, rank, world, local_rank):
         idx = Q.select_outliers(torch.from_numpy(wl.X_calib).cuda(), s.n_keep_fp16)
     kp = Q.packed_k(rot, s.K, s.n_keep_fp16)
     asym = args.asym_activations
+    bits = s.bits
+    if bits == 8 and asym:
+        raise SystemExit("the 8-bit layers take symmetric activations")
     gemm_ops, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp, asym)
 
     # input sets: enough copies that one pass over them exceeds L2 twice
@@ -272,10 +280,10 @@ def run_ours(args, rank, world, local_rank):
     w0 = torch.from_numpy(wl.W).cuda()
     t_pack0 = torch.cuda.Event(enable_timing=True)
     t_pack1 = torch.cuda.Event(enable_timing=True)
-    Q.QuantizedLinear(w0, rot, idx, asym)            # warm-up (module load, attributes)
+    Q.QuantizedLinear(w0, rot, idx, asym, bits)      # warm-up (module load, attributes)
     torch.cuda.synchronize()
     t_pack0.record()
-    layer0 = Q.QuantizedLinear(w0, rot, idx, asym)
+    layer0 = Q.QuantizedLinear(w0, rot, idx, asym, bits)
     t_pack1.record()
     torch.cuda.synchronize()
     pack_ms = t_pack0.elapsed_time(t_pack1)
@@ -296,6 +304,9 @@ def run_ours(args, rank, world, local_rank):
         if asym:
             codes, scales, zeros, x_out, _ = Q.rotate_quant_asym(x, rot, idx)
             return codes, scales, x_out, zeros
+        if bits == 8:
+            codes, scales, x_out, _ = Q.rotate_quant8(x, rot, idx)
+            return codes, scales, x_out, None
         codes, scales, x_out, _ = Q.rotate_quant(x, rot, idx)
         return codes, scales, x_out, None
 
@@ -304,6 +315,8 @@ def run_ours(args, rank, world, local_rank):
         wc, wsc, wo, wsum = wset
         if asym:
             Q.w4a4_linear_asym(codes, scales, zeros, wc, wsc, wsum, x_out, wo, out=y)
+        elif bits == 8:
+            Q.w8a8_linear(codes, scales, wc, wsc, x_out, wo, out=y)
         else:
             Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
 
@@ -416,7 +429,7 @@ def run_ours(args, rank, world, local_rank):
     hbm = peaks["hbm_gbs"]
     clocks = sampler.summary(t0, t1)
     sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
-    gemm_name = gemm_kernel_name(M)
+    gemm_name = gemm_kernel_name(M, bits)
     # the GEMM's bound: tensor cores above the ridge point, HBM below it.
     # The denominator is the burst figure (the timed region is well under a
     # second of GPU time); the sustained and datasheet fractions ride along.
@@ -448,8 +461,8 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "s8",
-        "precision": "int4 codes on s8 tensor-core MMA, s32 accumulate; fp32 rotation; "
-                     "fp16 in/out",
+        "precision": (f"int{bits} codes on s8 tensor-core MMA, s32 accumulate; fp32 rotation; "
+                      "fp16 in/out"),
         "data": "synthetic",
         "config": {"workload": s.name, "M": M, "K": s.K, "N": s.N, "K_p": kp,
                    "rotation": (("random-sign " if signs is not None else "") +
@@ -457,6 +470,7 @@ def run_ours(args, rank, world, local_rank):
                    else f"kron-{s.n1}x{s.n2}", "n_out": s.n_keep_fp16,
                    "clip_ratio": s.clip_ratio,
                    "activations": "asymmetric per-token" if asym else "symmetric per-token",
+                   "bits": bits,
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
@@ -525,12 +539,12 @@ def aggregate_max(value_ms: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- oracle
 
-def oracle_step(O, asym: bool):
+def oracle_step(O, asym: bool, bits: int = 4):
     """The oracle's online path: activation quantizer, then the linear."""
     if asym:
         return lambda x, rot, idx, wside: O.linear_asym(
             O.quantize_activations_asym(x, rot, idx), wside)
-    return lambda x, rot, idx, wside: O.linear(O.quantize_activations(x, rot, idx), wside)
+    return lambda x, rot, idx, wside: O.linear(O.quantize_activations(x, rot, idx, bits), wside)
 
 
 def _oracle_threads():
@@ -548,7 +562,7 @@ def oracle_sample(workload: str, tokens: int, rows, M_total=None, random_signs: 
     s = wl.spec
     rot = oracle_rotation(wl, oracle_signs(wl, random_signs))
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
-    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx)
+    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx, s.bits)
     x = wl.X[:tokens].astype(np.float64)
     return wl, rot, idx, wside, x
 
@@ -563,7 +577,7 @@ def oracle_baseline(workload: str, tokens: int, rows, repeats: int = 1, M_total=
 
     wl, rot, idx, wside, x = oracle_sample(workload, tokens, rows, M_total, random_signs)
     n_rows = wl.W.shape[0]
-    run = oracle_step(O, asym)
+    run = oracle_step(O, asym, wl.spec.bits)
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
@@ -603,7 +617,7 @@ def run_reference(args, rank, world):
     wl, rot, idx, wside, x = oracle_sample(args.workload, tokens, rows, args.tokens,
                                            args.random_signs)
     s = wl.spec
-    run = oracle_step(O, args.asym_activations)
+    run = oracle_step(O, args.asym_activations, s.bits)
 
     def step():
         run(x, rot, idx, wside)

@@ -111,8 +111,9 @@ typedef struct {
                                 descriptor (D B is orthogonal). */
 } qr_rotation;
 
-/* ABI version of this header (bumped on any incompatible change). */
-#define QR_ABI_VERSION 2
+/* ABI version of this header (bumped on any change to the entry points;
+ * 3 added the 8-bit calls and qr_check_wait_timeout). */
+#define QR_ABI_VERSION 3
 QR_API int32_t qr_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -189,6 +190,36 @@ QR_API qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales,
                          const uint16_t* x_out, const uint16_t* w_out, int32_t n_out,
                          uint16_t* Y, int64_t ldy, int32_t* acc_debug,
                          qr_stream stream);
+
+/* ----------------------------------------------------------------------
+ * 8-bit layers ("QUIK：LLM上的一种4-bit推理方法", QUIK量化, results: the
+ * LLaMA-2 down_proj stays in INT8 with its outlier count raised in
+ * proportion to its input width, round(256 K / 4096) = 688 for K = 11008;
+ * QUIK-8B runs every layer in INT8).  The same steps as the 4-bit calls with
+ * the symmetric quantizer on 8 bits: scales = alpha * max|x'| / 127, codes =
+ * clamp(round_half_even(x' / s), -127, 127), one int8 per code, rows of K_p
+ * bytes (K_p from qr_packed_k, as for 4 bits).
+ *
+ * qr_rotate_quant8 / qr_pack_weights8: arguments and errors as
+ * qr_rotate_quant / qr_pack_weights, with codes int8 [rows x K_p] (16-byte
+ * aligned); Kronecker descriptors are UNSUPPORTED.
+ * qr_w8a8_linear: as qr_w4a4_linear for int8 codes [M x K_p] and
+ * [N x K_p] (16-byte aligned, K_p % 128 == 0, K_p <= 65536):
+ *   acc[m, n] = sum_k qa[m, k] qw[n, k]   (exact int32: |acc| <= 127^2 K_p)
+ *   Y[m, n]   = fp16(acc * a_scales[m] * w_scales[n] + X_out[m] . W_out[n]) */
+QR_API qr_status qr_rotate_quant8(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                                  int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
+                                  int8_t* codes, float* scales, uint16_t* x_out,
+                                  float* x_rot_debug, qr_stream stream);
+QR_API qr_status qr_pack_weights8(const qr_rotation* rot_w, const uint16_t* W, int64_t N,
+                                  int64_t K, int64_t ldw, const int32_t* outlier_idx,
+                                  int32_t n_out, int8_t* w_codes, float* w_scales,
+                                  uint16_t* w_out, float* w_rot_debug, qr_stream stream);
+QR_API qr_status qr_w8a8_linear(const int8_t* a_codes, const float* a_scales,
+                                const int8_t* w_codes, const float* w_scales, int64_t M,
+                                int64_t N, int64_t K_p, const uint16_t* x_out,
+                                const uint16_t* w_out, int32_t n_out, uint16_t* Y, int64_t ldy,
+                                int32_t* acc_debug, qr_stream stream);
 
 /* ----------------------------------------------------------------------
  * Asymmetric per-token activations ("QUIK：LLM上的一种4-bit推理方法",

@@ -466,26 +466,32 @@ class Side:
     fp16_part: np.ndarray    # the outlier columns, fp16 [rows x n_out]
 
 
+def _stored(q: Quantized, bits: int) -> np.ndarray:
+    """Codes as stored: two nibbles per byte (4 bits), one int8 each (8 bits, R14)."""
+    return pack_int4(q.codes) if bits == 4 else q.codes.astype(np.int8)
+
+
 def quantize_activations(x: np.ndarray, rot: Rotation,
-                         outlier_idx: Optional[np.ndarray] = None) -> Side:
-    """Online activation path: outlier split, rotation, per-token quantization."""
+                         outlier_idx: Optional[np.ndarray] = None, bits: int = 4) -> Side:
+    """Online activation path: outlier split, rotation, per-token quantization
+    (4-bit codes, or 8-bit for QUIK's INT8 layers, R14)."""
     x_in, x_out = split_outliers(x, outlier_idx)
     n_out = 0 if outlier_idx is None else len(outlier_idx)
     k_p = packed_width(rot, np.asarray(x).shape[1], n_out)
     xr = rotate_activations(pad_columns(np.asarray(x_in, np.float64), k_p), rot)
-    q = quantize_rows(xr, rot.clip_ratio)
-    return Side(xr, q, pack_int4(q.codes), np.asarray(x_out, np.float16))
+    q = quantize_rows(xr, rot.clip_ratio, bits)
+    return Side(xr, q, _stored(q, bits), np.asarray(x_out, np.float16))
 
 
 def quantize_weights(w: np.ndarray, rot: Rotation,
-                     outlier_idx: Optional[np.ndarray] = None) -> Side:
+                     outlier_idx: Optional[np.ndarray] = None, bits: int = 4) -> Side:
     """Offline weight path: the same split, W R^{-T}, per-channel RTN ([QS] §2)."""
     w_in, w_out = split_outliers(w, outlier_idx)
     n_out = 0 if outlier_idx is None else len(outlier_idx)
     k_p = packed_width(rot, np.asarray(w).shape[1], n_out)
     wr = rotate_weights(pad_columns(np.asarray(w_in, np.float64), k_p), rot)
-    q = quantize_rows(wr, rot.clip_ratio)
-    return Side(wr, q, pack_int4(q.codes), np.asarray(w_out, np.float16))
+    q = quantize_rows(wr, rot.clip_ratio, bits)
+    return Side(wr, q, _stored(q, bits), np.asarray(w_out, np.float16))
 
 
 def linear(a: Side, w: Side):
@@ -528,10 +534,10 @@ def linear_forward_asym(x, w, rot: Rotation, outlier_idx=None):
     return a, ws, acc, y
 
 
-def linear_forward(x, w, rot: Rotation, outlier_idx=None):
-    """The whole layer: Y ~= X W^T through rotated 4-bit codes."""
-    a = quantize_activations(x, rot, outlier_idx)
-    ws = quantize_weights(w, rot, outlier_idx)
+def linear_forward(x, w, rot: Rotation, outlier_idx=None, bits: int = 4):
+    """The whole layer: Y ~= X W^T through rotated 4-bit (or 8-bit, R14) codes."""
+    a = quantize_activations(x, rot, outlier_idx, bits)
+    ws = quantize_weights(w, rot, outlier_idx, bits)
     acc, y = linear(a, ws)
     return a, ws, acc, y
 

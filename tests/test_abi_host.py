@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.qr_abi_version() == 2
+    assert L.qr_abi_version() == 3
     for s in range(6):
         assert L.status_string(s) and L.status_string(s) != "unknown status"
     assert L.status_string(99) == "unknown status"
@@ -197,3 +197,24 @@ def test_wait_selfcheck_argument_errors(lib):
     # the limit is validated on the host, before any launch
     for bad in (0, 999, 100000001, -5):
         assert L.qr_check_wait_timeout(bad, None, check=False) == L.QR_ERR_INVALID_ARG
+
+
+def test_int8_entry_points_argument_errors(lib):
+    # the 8-bit calls validate like the 4-bit ones; nothing launches here
+    h = _rot(L.QR_ROT_HADAMARD, 256)
+    def rq8(rot, codes=FAKE, M=4, K=512):
+        return L.qr_rotate_quant8(rot, FAKE, M, K, K, None, 0, codes, FAKE, None, None, None,
+                                  check=False)
+    assert rq8(h, codes=FAKE + 8) == L.QR_ERR_ALIGNMENT
+    assert rq8(h, M=-1) == L.QR_ERR_INVALID_ARG
+    assert rq8(h, M=0) == L.QR_OK
+    assert rq8(_rot(L.QR_ROT_KRON, n1=16, n2=32), K=512) == L.QR_ERR_UNSUPPORTED
+    assert L.qr_pack_weights8(h, FAKE, 4, 512, 512, None, 0, None, FAKE, None, None, None,
+                              check=False) == L.QR_ERR_INVALID_ARG
+    def lin8(Kp=256, a=FAKE, n_out=0, xo=None, wo=None, M=16):
+        return L.qr_w8a8_linear(a, FAKE, FAKE, FAKE, M, 16, Kp, xo, wo, n_out, FAKE, 16, None,
+                                None, check=False)
+    assert lin8(Kp=200) == L.QR_ERR_INVALID_ARG
+    assert lin8(a=FAKE + 4) == L.QR_ERR_ALIGNMENT
+    assert lin8(n_out=12, xo=FAKE, wo=FAKE) == L.QR_ERR_UNSUPPORTED
+    assert lin8(M=0) == L.QR_OK

@@ -608,6 +608,28 @@ def test_int8_quantizer_properties_and_exact_products():
     assert acc.tolist() == brute and abs(acc).max() < 2 ** 31
 
 
+@pytest.mark.parametrize("kind", [O.NONE, O.HADAMARD, O.GSR])
+def test_int8_layer_on_exactly_representable_rows(kind):
+    # 8-bit codes through the whole activation / weight / linear path (R14):
+    # rows built so that x R = qa and w R = qw, integer codes with absmax 127,
+    # give those codes, unit scales and the exact integer product
+    rng = np.random.default_rng(43)
+    k, m, n = 256, 5, 7
+    def codes(rows):
+        q = rng.integers(-127, 128, size=(rows, k)).astype(np.int64)
+        q[np.arange(rows), rng.integers(k, size=rows)] = np.where(rng.random(rows) < 0.5, 127, -127)
+        return q
+    qa, qw = codes(m), codes(n)
+    rot = O.Rotation(kind, block=32 if kind == O.GSR else 64)
+    r = O.dense_rotation(rot, k)
+    a, ws, acc, y = O.linear_forward(qa @ r.T, qw @ r.T, rot, bits=8)
+    assert np.array_equal(a.q.codes, qa) and np.array_equal(ws.q.codes, qw)
+    assert a.packed.dtype == np.int8 and a.packed.shape == (m, k)
+    np.testing.assert_allclose(a.q.scales, 1.0, rtol=1e-6)
+    np.testing.assert_allclose(ws.q.scales, 1.0, rtol=1e-6)
+    assert np.array_equal(acc, qa @ qw.T)
+
+
 def test_quik_outlier_count_scales_with_width():
     assert O.quik_outlier_count(4096) == 256
     assert O.quik_outlier_count(11008) == 688          # the INT8 down_proj

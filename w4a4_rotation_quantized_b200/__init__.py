@@ -11,6 +11,6 @@ from . import _lib  # noqa: F401
 from .layer import (GSR, HADAMARD, KRON, NONE, GraphedLinear, QuantizedLinear,  # noqa: F401
                     Rotation,
                     invert_transpose, kv_quantize, pack_weights, packed_k, rotate_quant,
-                    rotate_quant_asym,
+                    pack_weights8, rotate_quant8, rotate_quant_asym, w8a8_linear,
                     select_outliers, w4a4_linear, w4a4_linear_asym, weight_code_sums,
                     weight_rotation)

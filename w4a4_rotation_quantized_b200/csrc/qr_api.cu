@@ -108,7 +108,7 @@ static int64_t packed_k(const qr_rotation* rot, int64_t K, int32_t n_out) {
 static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t rows, int64_t K,
                            int64_t ld, const int32_t* outlier_idx, int32_t n_out, uint8_t* codes,
                            float* scales, int32_t* zeros, uint16_t* out16, float* rot_debug,
-                           qr_stream stream) {
+                           qr_stream stream, int bits = 4) {
   if (rot == nullptr || rows < 0 || K < 0 || n_out < 0 || n_out > K) return QR_ERR_INVALID_ARG;
   const int64_t kp = packed_k(rot, K, n_out);
   if (kp < 0) {
@@ -129,7 +129,9 @@ static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t 
     if (reinterpret_cast<uintptr_t>(rot->signs) % 8 != 0) return QR_ERR_ALIGNMENT;
   }
   if (zeros != nullptr && rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
+  if (bits == 8 && rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
   RowJob job{};
+  job.bits = bits;
   job.src = src;
   job.rows = rows;
   job.K = K;
@@ -244,7 +246,7 @@ static qr_status linear_call(const uint8_t* a_codes, const float* a_scales, cons
                              const uint8_t* w_codes, const float* w_scales, const int32_t* w_sums,
                              int64_t M, int64_t N, int64_t K_p, const uint16_t* x_out,
                              const uint16_t* w_out, int32_t n_out, uint16_t* Y, int64_t ldy,
-                             int32_t* acc_debug, qr_stream stream) {
+                             int32_t* acc_debug, qr_stream stream, int bits = 4) {
   if (M < 0 || N < 0 || K_p < 0 || n_out < 0) return QR_ERR_INVALID_ARG;
   if (K_p % 128 != 0) return QR_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return QR_OK;
@@ -272,7 +274,8 @@ static qr_status linear_call(const uint8_t* a_codes, const float* a_scales, cons
   j.Y = Y;
   j.ldy = ldy;
   j.acc_debug = acc_debug;
-  return launch_w4a4_gemm(j, reinterpret_cast<cudaStream_t>(stream));
+  return bits == 8 ? launch_w8a8_gemm(j, reinterpret_cast<cudaStream_t>(stream))
+                   : launch_w4a4_gemm(j, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace qr
@@ -312,6 +315,29 @@ qr_status qr_invert_transpose(const float* P, int32_t n, float* out, int32_t* in
   if (P == nullptr || out == nullptr || info == nullptr || n < 1) return QR_ERR_INVALID_ARG;
   if (n > 128) return QR_ERR_UNSUPPORTED;
   return launch_invert_transpose(P, n, out, info, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qr_status qr_rotate_quant8(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                           int64_t ldx, const int32_t* outlier_idx, int32_t n_out, int8_t* codes,
+                           float* scales, uint16_t* x_out, float* x_rot_debug, qr_stream stream) {
+  return rows_call(rot, X, M, K, ldx, outlier_idx, n_out, reinterpret_cast<uint8_t*>(codes), scales,
+                   nullptr, x_out, x_rot_debug, stream, 8);
+}
+
+qr_status qr_pack_weights8(const qr_rotation* rot_w, const uint16_t* W, int64_t N, int64_t K,
+                           int64_t ldw, const int32_t* outlier_idx, int32_t n_out, int8_t* w_codes,
+                           float* w_scales, uint16_t* w_out, float* w_rot_debug, qr_stream stream) {
+  return rows_call(rot_w, W, N, K, ldw, outlier_idx, n_out, reinterpret_cast<uint8_t*>(w_codes),
+                   w_scales, nullptr, w_out, w_rot_debug, stream, 8);
+}
+
+qr_status qr_w8a8_linear(const int8_t* a_codes, const float* a_scales, const int8_t* w_codes,
+                         const float* w_scales, int64_t M, int64_t N, int64_t K_p,
+                         const uint16_t* x_out, const uint16_t* w_out, int32_t n_out, uint16_t* Y,
+                         int64_t ldy, int32_t* acc_debug, qr_stream stream) {
+  return linear_call(reinterpret_cast<const uint8_t*>(a_codes), a_scales, nullptr,
+                     reinterpret_cast<const uint8_t*>(w_codes), w_scales, nullptr, M, N, K_p,
+                     x_out, w_out, n_out, Y, ldy, acc_debug, stream, 8);
 }
 
 qr_status qr_check_wait_timeout(int64_t limit_ns, qr_stream stream) {

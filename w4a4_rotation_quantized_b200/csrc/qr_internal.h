@@ -64,6 +64,7 @@ struct RowJob {
   int32_t* zeros;             // [rows] zero points (asymmetric activations) or null
   uint16_t* out16;            // [rows x n_out] or null
   float* rot_debug;           // [rows x Kp] or null
+  int32_t bits;               // code width: 4 (packed nibbles) or 8 (one int8 per code)
 };
 
 qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream);
@@ -85,6 +86,10 @@ struct GemmJob {
 };
 
 qr_status launch_w4a4_gemm(const GemmJob& job, cudaStream_t stream);
+
+// 8-bit codes (one int8 per code, rows of K_p bytes): TMA-fed tcgen05
+// kind::i8 MMAs with both operands in shared memory.
+qr_status launch_w8a8_gemm(const GemmJob& job, cudaStream_t stream);
 
 // M > 64: 2-SM tcgen05 MMA with the activation operand in TMEM, fp16
 // outlier columns as a second MMA.

@@ -100,6 +100,38 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return u;
 }
 
+// Eight 8-bit codes round_half_even(v[i] * r) (clamped to [lo, hi] when
+// CLIP), one byte each, v[0] first: the low byte of each fma with 1.5*2^23
+// is the code's two's-complement byte; byte permutes gather them.
+template <bool CLIP>
+__device__ __forceinline__ uint2 quant_bytes8(const float (&v)[8], float r, float c, float lo,
+                                              float hi) {
+  uint32_t b[8];
+  const uint64_t r2 = f2_pack(r, r), c2 = f2_pack(c, c);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float t0, t1;
+    f2_unpack(f2_fma(f2_pack(v[i], v[i + 1]), r2, c2), t0, t1);
+    if (CLIP) {
+      t0 = fminf(fmaxf(t0, lo), hi);
+      t1 = fminf(fmaxf(t1, lo), hi);
+    }
+    b[i] = __float_as_uint(t0);
+    b[i + 1] = __float_as_uint(t1);
+  }
+  return make_uint2(prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x4000u), 0x7610u),
+                    prmt(prmt(b[4], b[5], 0x0040u), prmt(b[6], b[7], 0x4000u), 0x7610u));
+}
+
+// One 8-bit code round_half_even(v * r) (clamped to [lo, hi] when CLIP) as
+// its two's-complement byte.
+template <bool CLIP>
+__device__ __forceinline__ uint32_t quant_byte(float v, float r, float c, float lo, float hi) {
+  float t = fmaf(v, r, c);
+  if (CLIP) t = fminf(fmaxf(t, lo), hi);
+  return __float_as_uint(t) & 0xFFu;
+}
+
 // Inverse of the binary-reflected Gray code on 8 bits.
 __device__ __forceinline__ int gray_inverse(int g) {
   g ^= g >> 1;
@@ -153,6 +185,7 @@ struct WhtParams {
   // ring mode: rows stream into shared memory by bulk copies
   int32_t ring_slots, ring_row_bytes, off_ring, off_bars, rows_per_block;
   int32_t* status;
+  int32_t bits8;              // 8-bit codes (one int8 per code) instead of nibbles
 };
 
 // Loads 8 consecutive rotated-domain elements [e, e+8) of a row as fp32:
@@ -238,6 +271,14 @@ __device__ __forceinline__ RowQ sym_row_q(float am, float clip, float inv_sqrt, 
   if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 7.0f;
   return RowQ{(am > 0.0f) ? 7.0f / (clip * am) : 0.0f, kRoundMagic, kRoundMagic - 7.0f,
               kRoundMagic + 7.0f};
+}
+
+// 8-bit symmetric codes (QUIK's INT8 layers): s = alpha * absmax / 127,
+// codes clamped to +-127.
+__device__ __forceinline__ RowQ sym_row_q8(float am, float clip, float inv_sqrt, float* scale_out) {
+  if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 127.0f;
+  return RowQ{(am > 0.0f) ? 127.0f / (clip * am) : 0.0f, kRoundMagic, kRoundMagic - 127.0f,
+              kRoundMagic + 127.0f};
 }
 
 __device__ __forceinline__ RowQ asym_row_q(float mn, float mx, float clip, float inv_sqrt,
@@ -467,7 +508,8 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
     RowQ q;
     if (p.zeros == nullptr) {
       am = row_absmax(am, red, rg, t, nt);
-      q = sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
+      q = p.bits8 ? sym_row_q8(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr)
+                  : sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
     } else {
       float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
@@ -484,7 +526,7 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
                      p.zeros + row);
     }
     const float r = q.r;
-    uint8_t* crow = p.codes + row * (p.Kp >> 1);
+    uint8_t* crow = p.codes + row * (p.bits8 ? p.Kp : (p.Kp >> 1));
 
     if (p.rot_debug != nullptr) {
 #pragma unroll
@@ -506,7 +548,32 @@ __global__ void __launch_bounds__(AbBounds<MB, HA, ITEMS>::value) wht_ab_kernel(
       }
     }
 
-    if constexpr (OUT == 0) {
+    if (p.bits8) {
+      // 8-bit codes: one byte each through shared memory at its output
+      // position, then copied out in 16-byte pieces
+      row_barrier(rg, nt);                 // every thread is done reading buf
+      uint8_t* cb = reinterpret_cast<uint8_t*>(buf);
+#pragma unroll
+      for (int k = 0; k < ITEMS; ++k) {
+        const int w = t + k * nt;
+        if (w < items_b) {
+          const int blk = w >> (3 + HA), tb = w & (TB - 1);
+          const int e0 = (blk << LB) + (tb & 7) + ((tb >> 3) << (3 + MB));
+#pragma unroll
+          for (int j = 0; j < EB; ++j) {
+            int n = (e0 & ((1 << LB) - 1)) + 8 * j;
+            if (p.gsr) {
+              const int rev = static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - LB));
+              n = gray_inverse(rev);
+            }
+            cb[(blk << LB) + n] = static_cast<uint8_t>(quant_byte<CLIP>(v[k][j], r, q.c, q.lo, q.hi));
+          }
+        }
+      }
+      row_barrier(rg, nt);
+      for (int e = 16 * t; e < p.Kp; e += 16 * nt)
+        *reinterpret_cast<uint4*>(crow + e) = *reinterpret_cast<const uint4*>(cb + e);
+    } else if constexpr (OUT == 0) {
       static_assert(MB >= 3, "nibble transposes need 8 values per lane");
       const int l = lane & 7;
       const uint32_t sel4 = (l & 4) ? 0x3276u : 0x5410u;
@@ -661,7 +728,8 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
     RowQ q;
     if (p.zeros == nullptr) {
       am = row_absmax(am, red, rg, t, nt);
-      q = sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
+      q = p.bits8 ? sym_row_q8(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr)
+                  : sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
     } else {
       float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
@@ -678,12 +746,12 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
                      p.zeros + row);
     }
     const float r = q.r;
-    uint8_t* crow = p.codes + row * (p.Kp >> 1);
+    uint8_t* crow = p.codes + row * (p.bits8 ? p.Kp : (p.Kp >> 1));
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
       const int g = t + k * nt;
       if (g < ngroups) {
-        uint32_t W = 0;
+        uint32_t W = 0, B0 = 0, B1 = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           int pos = i;
@@ -692,10 +760,18 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
             const int rev = static_cast<int>(__brev(static_cast<unsigned>(i & bm)) >> (32 - lb));
             pos = (i & ~bm) + gray_inverse(rev);
           }
-          W |= quant_nibble<CLIP>(v[k][i], r, q.c, q.lo, q.hi) << (4 * pos);
+          if (p.bits8) {
+            const uint32_t b = quant_byte<CLIP>(v[k][i], r, q.c, q.lo, q.hi);
+            if (pos < 4) B0 |= b << (8 * pos); else B1 |= b << (8 * (pos - 4));
+          } else {
+            W |= quant_nibble<CLIP>(v[k][i], r, q.c, q.lo, q.hi) << (4 * pos);
+          }
           if (p.rot_debug != nullptr) p.rot_debug[row * p.Kp + 8 * g + pos] = v[k][i] * p.inv_sqrt_block;
         }
-        *reinterpret_cast<uint32_t*>(crow + 4 * g) = W;
+        if (p.bits8)
+          *reinterpret_cast<uint2*>(crow + 8 * g) = make_uint2(B0, B1);
+        else
+          *reinterpret_cast<uint32_t*>(crow + 4 * g) = W;
       }
     }
     row_barrier(rg, nt);                   // red is reused by the next row
@@ -732,6 +808,7 @@ struct FewRowsParams {
   int32_t* zeros;             // asymmetric activations: zero points [rows] (null: symmetric)
   __half* out16;
   float* rot_debug;
+  int32_t bits8;              // 8-bit codes (one int8 per code) instead of nibbles
 };
 
 constexpr int kFewMaxChunks = 4;   // 8-column chunks per thread (K <= 32768 at 1024 threads)
@@ -922,12 +999,14 @@ __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsPara
     }
   }
   const bool lead = t == 0 && cr == 0;
-  const RowQ q = !ASYM
-                     ? sym_row_q(m0, p.clip_ratio, p.inv_sqrt_block, lead ? p.scales + row : nullptr)
-                     : asym_row_q(-m1, m0, p.clip_ratio, p.inv_sqrt_block,
-                                  lead ? p.scales + row : nullptr, p.zeros + row);
+  const RowQ q = ASYM ? asym_row_q(-m1, m0, p.clip_ratio, p.inv_sqrt_block,
+                                   lead ? p.scales + row : nullptr, p.zeros + row)
+                 : p.bits8 ? sym_row_q8(m0, p.clip_ratio, p.inv_sqrt_block,
+                                        lead ? p.scales + row : nullptr)
+                           : sym_row_q(m0, p.clip_ratio, p.inv_sqrt_block,
+                                       lead ? p.scales + row : nullptr);
   const float r = q.r;
-  uint8_t* crow = p.codes + row * (p.Kp >> 1);
+  uint8_t* crow = p.codes + row * (p.bits8 ? p.Kp : (p.Kp >> 1));
   const int bm = (1 << p.lb) - 1;
   for (int g = t; g < (nloc >> 3); g += nthr) {
     const int el = 8 * g;                          // local index of the group
@@ -946,7 +1025,10 @@ __global__ void __launch_bounds__(1024, 1) wht_few_rows_kernel(const FewRowsPara
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
       v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
-    *reinterpret_cast<uint32_t*>(crow + ((e_lo + el) >> 1)) = quant_word<CLIP>(v, r, q.c, q.lo, q.hi);
+    if (!ASYM && p.bits8)
+      *reinterpret_cast<uint2*>(crow + e_lo + el) = quant_bytes8<CLIP>(v, r, q.c, q.lo, q.hi);
+    else
+      *reinterpret_cast<uint32_t*>(crow + ((e_lo + el) >> 1)) = quant_word<CLIP>(v, r, q.c, q.lo, q.hi);
     if (p.rot_debug != nullptr)
 #pragma unroll
       for (int i = 0; i < 8; ++i) p.rot_debug[row * p.Kp + e_lo + el + i] = v[i] * p.inv_sqrt_block;
@@ -1233,6 +1315,7 @@ qr_status launch_wht_few_rows(const RowJob& job, cudaStream_t stream) {
   p.zeros = job.zeros;
   p.out16 = reinterpret_cast<__half*>(job.out16);
   p.rot_debug = job.rot_debug;
+  p.bits8 = job.bits == 8;
   // CTAs per row: up to 8 (and the SMs left per row), each a span of whole
   // blocks that is a multiple of 128 elements
   const int unit = std::max(1, 128 >> p.lb);                  // blocks per 128 elements
@@ -1297,6 +1380,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.zeros = job.zeros;
   p.out16 = reinterpret_cast<__half*>(job.out16);
   p.rot_debug = job.rot_debug;
+  p.bits8 = job.bits == 8;
   if (job.Kp > 32768) return QR_ERR_UNSUPPORTED;
 
   const bool small = lb <= 3;
@@ -1563,6 +1647,8 @@ qr_status launch_kv_group_quant(const uint16_t* src, int64_t groups, int group, 
 
 qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream) {
   if (job.rows == 0) return QR_OK;
+  if (job.bits == 8 && (job.rot->kind == QR_ROT_KRON || job.zeros != nullptr))
+    return QR_ERR_UNSUPPORTED;
   if (job.rot->kind == QR_ROT_KRON)
     return kron_tc_supported(job) ? launch_kron_tc(job, stream) : launch_kron_rows(job, stream);
   return few_rows(job) ? launch_wht_few_rows(job, stream) : launch_wht_rows(job, stream);

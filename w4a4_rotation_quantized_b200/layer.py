@@ -88,7 +88,8 @@ def packed_k(rot: Rotation, K: int, n_out: int = 0) -> int:
     return kp
 
 
-def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool, asym: bool = False):
+def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool, asym: bool = False,
+          bits: int = 4):
     _need_cuda(x, torch.float16, "input")
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("input must be a 2-D row-major tensor")
@@ -101,7 +102,8 @@ def _rows(fn, rot: Rotation, x: torch.Tensor, outlier_idx, debug: bool, asym: bo
     if kp < 0:
         raise ValueError("invalid rotation descriptor or sizes")
     dev = x.device
-    codes = torch.empty((rows, kp // 2), dtype=torch.uint8, device=dev)
+    codes = (torch.empty((rows, kp), dtype=torch.int8, device=dev) if bits == 8
+             else torch.empty((rows, kp // 2), dtype=torch.uint8, device=dev))
     scales = torch.empty(rows, dtype=torch.float32, device=dev)
     out16 = torch.empty((rows, n_out), dtype=torch.float16, device=dev) if n_out else None
     dbg = torch.empty((rows, kp), dtype=torch.float32, device=dev) if debug else None
@@ -125,6 +127,33 @@ def rotate_quant_asym(x, rot: Rotation, outlier_idx=None, debug: bool = False):
     """Online activation path with QUIK's asymmetric per-token quantizer:
     (codes, scales, zeros, x_out, x_rot or None); x ~= scale * (code - zero)."""
     return _rows(L.qr_rotate_quant_asym, rot, x, outlier_idx, debug, asym=True)
+
+
+def rotate_quant8(x, rot: Rotation, outlier_idx=None, debug: bool = False):
+    """Online activation path with 8-bit codes (QUIK's INT8 layers):
+    (codes int8 [rows x K_p], scales, x_out, x_rot or None)."""
+    return _rows(L.qr_rotate_quant8, rot, x, outlier_idx, debug, bits=8)
+
+
+def pack_weights8(w, rot_w: Rotation, outlier_idx=None, debug: bool = False):
+    """Offline weight path with 8-bit codes: (codes int8, scales, w_out, w_rot or None)."""
+    return _rows(L.qr_pack_weights8, rot_w, w, outlier_idx, debug, bits=8)
+
+
+def w8a8_linear(a_codes, a_scales, w_codes, w_scales, x_out=None, w_out=None,
+                out: Optional[torch.Tensor] = None, acc_debug: bool = False):
+    """The 8-bit linear: Y = fp16(acc * sa * sw + x_out w_out^T) for int8 codes;
+    returns (Y, acc or None)."""
+    M, kp = a_codes.shape
+    N = w_codes.shape[0]
+    n_out = 0 if x_out is None else x_out.shape[1]
+    dev = a_codes.device
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev) if acc_debug else None
+    L.qr_w8a8_linear(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(),
+                     w_scales.data_ptr(), M, N, kp, _ptr(x_out), _ptr(w_out), n_out,
+                     y.data_ptr(), y.stride(0), _ptr(acc), _stream())
+    return y, acc
 
 
 def weight_code_sums(w_codes: torch.Tensor) -> torch.Tensor:
@@ -217,19 +246,28 @@ def select_outliers(x_calib: torch.Tensor, k: int) -> torch.Tensor:
 
 
 class QuantizedLinear:
-    """A linear layer held as rotated 4-bit weights; forward() is the online path."""
+    """A linear layer held as rotated 4-bit (or, with bits=8, 8-bit) weights;
+    forward() is the online path."""
 
     def __init__(self, weight: torch.Tensor, rot: Rotation, outlier_idx=None,
-                 asym_activations: bool = False):
+                 asym_activations: bool = False, bits: int = 4):
+        if bits not in (4, 8) or (bits == 8 and asym_activations):
+            raise ValueError("bits must be 4, or 8 with symmetric activations")
         self.rot = rot
         self.rot_w = weight_rotation(rot)
         self.outlier_idx = outlier_idx
         self.asym = asym_activations
-        self.w_codes, self.w_scales, self.w_out, _ = pack_weights(weight, self.rot_w, outlier_idx)
+        self.bits = bits
+        pack = pack_weights8 if bits == 8 else pack_weights
+        self.w_codes, self.w_scales, self.w_out, _ = pack(weight, self.rot_w, outlier_idx)
         self.w_sums = weight_code_sums(self.w_codes) if asym_activations else None
         self.out_features, self.in_features = weight.shape
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
+        if self.bits == 8:
+            codes, scales, x_out, _ = rotate_quant8(x, self.rot, self.outlier_idx)
+            y, _ = w8a8_linear(codes, scales, self.w_codes, self.w_scales, x_out, self.w_out)
+            return y
         if self.asym:
             codes, scales, zeros, x_out, _ = rotate_quant_asym(x, self.rot, self.outlier_idx)
             y, _ = w4a4_linear_asym(codes, scales, zeros, self.w_codes, self.w_scales, self.w_sums,

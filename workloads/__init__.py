@@ -48,6 +48,7 @@ class Spec:
     n2: int = 0
     n_keep_fp16: int = 0        # QUIK fp16 outlier columns selected by calibration
     calib_tokens: int = 0
+    bits: int = 4               # code width of the layer (8: QUIK's INT8 layers)
     description: str = ""
 
 
@@ -90,6 +91,16 @@ SPECS = {
                     "256 outlier columns x50 kept fp16 (chosen on a 512-token "
                     "calibration batch), the other 7936 columns rotated by "
                     "4096-point Hadamard blocks"),
+    "down_proj_int8_11008": Spec(
+        "down_proj_int8_11008", M=2048, K=11008, N=4096, seed=20261209,
+        rotation=GSR, block=128, n_outlier_channels=32, outlier_scale=40.0,
+        x_dist="silu_gated", n_keep_fp16=688, calib_tokens=512, bits=8,
+        description="QUIK's INT8 LLaMA-2-7B down_proj: X[2048x11008] = "
+                    "SiLU(A)*B, 32 outlier channels x40; 688 fp16 outlier "
+                    "columns (256 per 4096 inputs) chosen on a 512-token "
+                    "calibration batch; the other 10320 columns GSR-rotated "
+                    "in 128-blocks; 8-bit activations and weights; "
+                    "W[4096x11008] N(0,0.02^2)"),
 }
 
 DECODE_TOKENS = (1, 4, 16, 64)
