@@ -778,6 +778,532 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
   }
 }
 
+// Three-input maximum / minimum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// ------------------------------------------------------------------ block-local rows
+// Blocks of 2^LB (6 <= LB <= 8): a block never leaves one warp's chunk of
+// four blocks, so the change of layout between the two butterfly passes goes
+// through a small per-warp shared-memory buffer with __syncwarp only.  A row
+// group of W warps holds one row in registers (chunk c of the row is item
+// c / W of warp c % W); its one row-wide step is the absmax (or min/max)
+// reduction.  Rows stream into a shared-memory ring by bulk copies from a
+// producer warp; with QUIK outliers the kept columns are gathered from the
+// ring copy through the kept-column table.
+//   layout A: lane l holds chunk elements [256 j + 8 l, +8) for each 256-element
+//             piece j (in-block bits 0-2 inside the thread);
+//   layout B: lane l = 8 b + t holds elements t + 8 m of block b of the chunk
+//             (in-block bits 3..LB-1 inside the thread).
+template <int LB>
+struct BlkGeom {
+  static constexpr int kBlock = 1 << LB;
+  static constexpr int kVB = 1 << (LB - 3);      // layout-B values per thread per chunk
+  static constexpr int kChunk = 4 << LB;         // elements per warp chunk
+  static constexpr int kPieces = 1 << (LB - 6);  // layout-A pieces of 8 per thread
+  static constexpr int kStride = kBlock + 8;     // floats per block in a warp buffer
+  static constexpr int kBufFloats = 4 * kStride;
+};
+
+// Warp-buffer position of in-block index q of chunk block b:
+// b * kStride + (q ^ (bit 5 of q) << 2).  The 8 floats of padding per block
+// put the four blocks of a layout-B read in different banks; swapping the
+// 4-float halves of every other 8-float group makes the layout-A 16-byte
+// stores conflict-free.  The kernel resolves it into per-lane base offsets.
+
+// Threads per CTA the kernel is compiled for, from its register budget: the
+// values one thread holds plus an overhead that grows with them (set where
+// the compiler stops spilling).
+template <int LB, int CPW>
+struct BlkBounds {
+  static constexpr int kVals = CPW * BlkGeom<LB>::kVB;
+  static constexpr int kRegs = 56 + kVals + (kVals >= 64 ? 24 : 0) + (LB == 6 ? 16 : 0);
+  static constexpr int value = ((65536 / kRegs) / 32) * 32 > 1024 ? 1024 : ((65536 / kRegs) / 32) * 32;
+};
+
+// Eight rotated-domain elements [e, e+8) of a ring row: straight 16-byte
+// loads without outliers, else gathered through the kept-column table; zero
+// at and beyond Kr.
+__device__ __forceinline__ void blk_load8(const WhtParams& p, const __half* rrow,
+                                          const uint16_t* kept, int e, float (&x)[8]) {
+  if (e + 8 <= p.Kr) {
+    if (p.n_out == 0) {
+      const uint4 u = *reinterpret_cast<const uint4*>(rrow + e);
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(h[q]);
+        x[2 * q] = f.x;
+        x[2 * q + 1] = f.y;
+      }
+    } else {
+      const uint4 k = *reinterpret_cast<const uint4*>(kept + e);
+      const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {     // (a malformed outlier list leaves 0xFFFF: read as 0)
+        const uint32_t c0 = kk[q] & 0xFFFFu, c1 = kk[q] >> 16;
+        x[2 * q] = c0 < static_cast<uint32_t>(p.K) ? __half2float(rrow[c0]) : 0.0f;
+        x[2 * q + 1] = c1 < static_cast<uint32_t>(p.K) ? __half2float(rrow[c1]) : 0.0f;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ei = e + i;
+      const int c = ei < p.Kr ? (p.n_out ? static_cast<int>(kept[ei]) : ei) : p.K;
+      x[i] = c < p.K ? __half2float(rrow[c]) : 0.0f;
+    }
+  }
+}
+
+// MODE: 0 = symmetric 4-bit, 1 = asymmetric 4-bit, 2 = symmetric 8-bit.
+template <int LB, int CPW, int MODE, bool CLIP>
+__global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(const WhtParams p) {
+  using G = BlkGeom<LB>;
+  constexpr int VB = G::kVB;
+  static_assert(LB >= 6 && LB <= 8, "block-local kernel: blocks of 64..256");
+  grid_dep_wait();
+  grid_dep_launch();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int W = p.nt >> 5;                       // warps per row group
+  const int groups = p.rows_per_cta;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = warp / W, wr = warp - rg * W;
+  uint64_t* ring_full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
+  uint64_t* ring_empty = ring_full + p.ring_slots;
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(ring_empty + p.ring_slots);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * p.rows_per_block;
+  const int64_t row1 = row0 + p.rows_per_block < p.rows ? row0 + p.rows_per_block : p.rows;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.ring_slots; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], W);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  uint8_t* sbits = smem + p.off_signs;
+  if (p.signs != nullptr) build_sign_bits(p.signs, p.Kp, sbits);
+  uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
+  const int32_t* sidx = reinterpret_cast<const int32_t*>(smem + p.off_idx);
+  if (p.n_out > 0)   // (synchronizes the CTA)
+    build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept, reinterpret_cast<int32_t*>(smem + p.off_idx));
+  __syncthreads();
+
+  if (warp == groups * W) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      const int n = static_cast<int>(row1 - row0);
+      int i = 0;
+      bool ok = true;
+      for (; i < n; ++i) {
+        const int s = i % p.ring_slots;
+        const uint32_t ph = (i / p.ring_slots) & 1;
+        if (!(ok = mbar_wait_bounded(&ring_empty[s], ph ^ 1, abort_flag, p.status,
+                                     kDevTimeoutProducer)))
+          break;
+        mbar_arrive_expect_tx(&ring_full[s], p.ring_row_bytes);
+        bulk_load(smem + p.off_ring + static_cast<size_t>(s) * p.ring_row_bytes,
+                  p.src + (row0 + i) * p.ld, p.ring_row_bytes, &ring_full[s]);
+      }
+      // every copy issued lands before the CTA may exit
+      for (int j = (i > p.ring_slots ? i - p.ring_slots : 0); j < i; ++j)
+        mbar_wait_bounded(&ring_full[j % p.ring_slots], (j / p.ring_slots) & 1, abort_flag,
+                          nullptr, 0, kDrainLimitNs);
+    }
+    return;
+  }
+
+  float* buf = reinterpret_cast<float*>(smem + p.off_buf) + warp * G::kBufFloats;
+  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 64;   // [2 rows][16 warps][2]
+  const int nchunks = (p.Kp + G::kChunk - 1) / G::kChunk;
+  const int nb = p.Kp >> LB;
+  const int b = lane >> 3, tl = lane & 7;
+  // Layout-A stores: piece j of this lane lands at a_pos + j * (256 >> LB) *
+  // kStride (its second half at a_pos2 + ...), the half swap resolved per lane.
+  const int qa = (8 * lane) & (G::kBlock - 1);
+  const int xa = ((qa >> 5) & 1) << 2;
+  const int a_pos = (lane >> (LB - 3)) * G::kStride + qa + xa;
+  const int a_pos2 = (lane >> (LB - 3)) * G::kStride + qa + 4 - xa;
+  // Layout-B loads: value m sits at b_pos[(m >> 2) & 1] + 8 m.
+  const int b_pos0 = b * G::kStride + tl, b_pos1 = b * G::kStride + (tl ^ 4);
+  int par = 0;
+  for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
+    const int i = static_cast<int>(row - row0);
+    const int slot = i % p.ring_slots;
+    if (!mbar_wait_bounded(&ring_full[slot], (i / p.ring_slots) & 1, abort_flag, p.status,
+                           kDevTimeoutWiden))
+      break;
+    const __half* rrow =
+        reinterpret_cast<const __half*>(smem + p.off_ring + static_cast<size_t>(slot) * p.ring_row_bytes);
+    if (p.n_out > 0 && p.out16 != nullptr)
+      for (int j = wr * 32 + lane; j < p.n_out; j += W * 32) {
+        const int c = sidx[j];
+        p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? rrow[c] : __float2half(0.0f);
+      }
+
+    // ---- both butterfly passes, one chunk at a time
+    float v[CPW][VB];
+    float am = 0.0f, mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < CPW; ++c) {
+      const int ch = wr + c * W;
+      if (ch < nchunks) {                         // warp-uniform
+        const int e0 = ch * G::kChunk;
+#pragma unroll
+        for (int j = 0; j < G::kPieces; ++j) {
+          const int o = 256 * j + 8 * lane;
+          float x[8];
+          blk_load8(p, rrow, kept, e0 + o, x);
+          if (p.signs != nullptr && e0 + o < p.Kp) apply_signs8(sbits, e0 + o, x);
+          wht_stages<0, 3>(x);
+          constexpr int kPieceStride = (256 >> LB) * G::kStride;
+          *reinterpret_cast<float4*>(buf + a_pos + j * kPieceStride) = make_float4(x[0], x[1], x[2], x[3]);
+          *reinterpret_cast<float4*>(buf + a_pos2 + j * kPieceStride) = make_float4(x[4], x[5], x[6], x[7]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int m = 0; m < VB; ++m) v[c][m] = buf[(((m >> 2) & 1) ? b_pos1 : b_pos0) + 8 * m];
+        __syncwarp();                             // before the next chunk's stores
+        wht_stages<0, LB - 3>(v[c]);
+        if constexpr (MODE == 1) {
+          if (ch * 4 + b < nb)
+#pragma unroll
+            for (int m = 0; m < VB; m += 2) {
+              mn = fmin3(mn, v[c][m], v[c][m + 1]);
+              mx = fmax3(mx, v[c][m], v[c][m + 1]);
+            }
+        } else {
+#pragma unroll
+          for (int m = 0; m < VB; m += 2) am = fmax3(am, fabsf(v[c][m]), fabsf(v[c][m + 1]));
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ring_empty[slot]);   // this warp is done with the ring row
+
+    // ---- the row's scale: warp reduction, then across the group's warps
+    float* rp = red + par * 32;
+    RowQ q;
+    if constexpr (MODE == 1) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      if (lane == 0) { rp[2 * wr] = mx; rp[2 * wr + 1] = mn; }
+      row_barrier(rg, p.nt);
+      mx = lane < W ? rp[2 * lane] : -INFINITY;
+      mn = lane < W ? rp[2 * lane + 1] : INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      const bool first = wr == 0 && lane == 0;
+      q = asym_row_q(mn, mx, p.clip_ratio, p.inv_sqrt_block, first ? p.scales + row : nullptr,
+                     p.zeros + row);
+    } else {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      if (lane == 0) rp[wr] = am;
+      row_barrier(rg, p.nt);
+      am = lane < W ? rp[lane] : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      float* so = (wr == 0 && lane == 0) ? p.scales + row : nullptr;
+      q = MODE == 2 ? sym_row_q8(am, p.clip_ratio, p.inv_sqrt_block, so)
+                    : sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, so);
+    }
+    const float r = q.r;
+
+    // ---- codes
+    uint8_t* crow = p.codes + row * (MODE == 2 ? p.Kp : (p.Kp >> 1));
+#pragma unroll
+    for (int c = 0; c < CPW; ++c) {
+      const int ch = wr + c * W;
+      if (ch >= nchunks) continue;                // warp-uniform
+      const int bg = ch * 4 + b;                  // block of the row
+      const bool ok = bg < nb;
+      if (p.rot_debug != nullptr && ok) {
+#pragma unroll
+        for (int m = 0; m < VB; ++m) {
+          int n = tl + 8 * m;
+          if (p.gsr) n = gray_inverse(static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - LB)));
+          p.rot_debug[row * p.Kp + (bg << LB) + n] = v[c][m] * p.inv_sqrt_block;
+        }
+      }
+      if (p.gsr) {
+        // sequency order: one thread owns each 8-position output word
+        const int a0 = tl & 1, a1 = (tl >> 1) & 1, a2 = (tl >> 2) & 1;
+        const int p1 = a0, p2 = a1 ^ a0, p3 = a2 ^ p2;
+#pragma unroll
+        for (int f = 0; f < (1 << (LB - 6)); ++f) {
+          const int kw = f | (p3 << (LB - 6)) | (p2 << (LB - 5)) | (p1 << (LB - 4));
+          float w8[8];
+#pragma unroll
+          for (int tt = 0; tt < 8; ++tt) {
+            const int js = gsr_j_static<LB>(tt, f);
+            w8[tt] = p3 ? v[c][js ^ 1] : v[c][js];
+          }
+          if (ok) {
+            if constexpr (MODE == 2)
+              *reinterpret_cast<uint2*>(crow + (bg << LB) + 8 * kw) = quant_bytes8<CLIP>(w8, r, q.c, q.lo, q.hi);
+            else
+              *reinterpret_cast<uint32_t*>(crow + (((bg << LB) + 8 * kw) >> 1)) =
+                  quant_word<CLIP>(w8, r, q.c, q.lo, q.hi);
+          }
+        }
+      } else if constexpr (MODE == 2) {
+        if (ok)
+#pragma unroll
+          for (int m = 0; m < VB; ++m)
+            crow[(bg << LB) + tl + 8 * m] = static_cast<uint8_t>(quant_byte<CLIP>(v[c][m], r, q.c, q.lo, q.hi));
+      } else {
+        // natural order: 8x8 nibble transposes across the 8 lanes of a block
+        const uint32_t sel4 = (tl & 4) ? 0x3276u : 0x5410u;
+        const uint32_t sel2 = (tl & 2) ? 0x3715u : 0x6240u;
+        const uint32_t rot1 = (tl & 1) ? 28u : 4u;
+        const uint32_t msk1 = (tl & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+        uint32_t wd[VB / 8];
+#pragma unroll
+        for (int wb = 0; wb < VB / 8; ++wb) {
+          float q8[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) q8[jj] = v[c][8 * wb + jj];
+          wd[wb] = quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
+        }
+#pragma unroll
+        for (int wb = 0; wb < VB / 8; ++wb) wd[wb] = prmt(wd[wb], __shfl_xor_sync(0xffffffffu, wd[wb], 4), sel4);
+#pragma unroll
+        for (int wb = 0; wb < VB / 8; ++wb) wd[wb] = prmt(wd[wb], __shfl_xor_sync(0xffffffffu, wd[wb], 2), sel2);
+#pragma unroll
+        for (int wb = 0; wb < VB / 8; ++wb) {
+          const uint32_t P = __shfl_xor_sync(0xffffffffu, wd[wb], 1);
+          const uint32_t s4 = __funnelshift_l(P, P, rot1);
+          uint32_t nw;
+          asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(nw) : "r"(wd[wb]), "r"(s4), "r"(msk1));
+          if (ok) *reinterpret_cast<uint32_t*>(crow + (((bg << LB) + 8 * (8 * wb + tl)) >> 1)) = nw;
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ 4096-point rows
+// Blocks of 4096, a row group of two warps per block, 64 values per thread:
+//   layout A: thread t of a block holds elements 8 t + 512 h + i (h, i < 8),
+//             in-block bits 0-2 and 9-11 inside the thread;
+//   layout B: thread t holds elements (t & 7) + 8 j + 512 (t >> 3) (j < 64),
+//             bits 3-8 inside the thread.
+// One pass through the group's fp32 row buffer moves the row from A to B.
+// In the buffer, element e of a block sits at (e + 8 (e >> 9)) with bit 2
+// flipped where bit 5 of e is set: the padding spreads a layout-B read over
+// all banks, the flip makes the layout-A 16-byte stores conflict-free.
+// Rows stream into a shared-memory ring by bulk copies (one producer warp).
+constexpr int kH12Floats = 4096 + 64;
+
+// MODE: 0 = symmetric, 1 = asymmetric (4-bit codes, natural order).
+template <int MODE, bool CLIP>
+__global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int nt = p.nt;                          // 64 x blocks per row
+  const int groups = p.rows_per_cta;
+  const int rg = threadIdx.x / nt, t = threadIdx.x - rg * nt;
+  const int lane = threadIdx.x & 31;
+  uint64_t* ring_full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
+  uint64_t* ring_empty = ring_full + p.ring_slots;
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(ring_empty + p.ring_slots);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * p.rows_per_block;
+  const int64_t row1 = row0 + p.rows_per_block < p.rows ? row0 + p.rows_per_block : p.rows;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.ring_slots; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], nt / 32);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  uint8_t* sbits = smem + p.off_signs;
+  if (p.signs != nullptr) build_sign_bits(p.signs, p.Kp, sbits);
+  __syncthreads();
+
+  if (rg == groups) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      const int n = static_cast<int>(row1 - row0);
+      int i = 0;
+      bool ok = true;
+      for (; i < n; ++i) {
+        const int s = i % p.ring_slots;
+        const uint32_t ph = (i / p.ring_slots) & 1;
+        if (!(ok = mbar_wait_bounded(&ring_empty[s], ph ^ 1, abort_flag, p.status,
+                                     kDevTimeoutProducer)))
+          break;
+        mbar_arrive_expect_tx(&ring_full[s], p.ring_row_bytes);
+        bulk_load(smem + p.off_ring + static_cast<size_t>(s) * p.ring_row_bytes,
+                  p.src + (row0 + i) * p.ld, p.ring_row_bytes, &ring_full[s]);
+      }
+      for (int j = (i > p.ring_slots ? i - p.ring_slots : 0); j < i; ++j)
+        mbar_wait_bounded(&ring_full[j % p.ring_slots], (j / p.ring_slots) & 1, abort_flag,
+                          nullptr, 0, kDrainLimitNs);
+    }
+    return;
+  }
+
+  const int blk = t >> 6, tb = t & 63;
+  float* buf = reinterpret_cast<float*>(smem + p.off_buf) +
+               (static_cast<size_t>(rg) * (nt >> 6) + blk) * kH12Floats;
+  float* red = reinterpret_cast<float*>(smem + p.off_red) + rg * 64;   // [2 rows][16 warps][2]
+  const int nw = nt >> 5, wr = t >> 5;
+  // layout-A stores of group h: a_pos + 520 h (first half), a_pos2 + 520 h
+  const int xa = ((tb >> 2) & 1) << 2;
+  const int a_pos = 8 * tb + xa, a_pos2 = 8 * tb + 4 - xa;
+  // layout-B loads: value j at (bit 2 of j ? b_pos1 : b_pos0) + 8 j
+  const int b_pos0 = (tb & 7) + 520 * (tb >> 3), b_pos1 = ((tb & 7) ^ 4) + 520 * (tb >> 3);
+  const int eA = blk * 4096 + 8 * tb;           // row element of layout-A group h = 0
+  int par = 0;
+  for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
+    const int i = static_cast<int>(row - row0);
+    const int slot = i % p.ring_slots;
+    if (!mbar_wait_bounded(&ring_full[slot], (i / p.ring_slots) & 1, abort_flag, p.status,
+                           kDevTimeoutWiden))
+      break;
+    const __half* rrow =
+        reinterpret_cast<const __half*>(smem + p.off_ring + static_cast<size_t>(slot) * p.ring_row_bytes);
+
+    // ---- phase A: bits 0-2 and 9-11
+    float v[64];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const int e = eA + 512 * h;
+      if (e + 8 <= p.K) {
+        const uint4 u = *reinterpret_cast<const uint4*>(rrow + e);
+        const __half2* hh = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(hh[q]);
+          v[8 * h + 2 * q] = f.x;
+          v[8 * h + 2 * q + 1] = f.y;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[8 * h + q] = 0.0f;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ring_empty[slot]);   // this warp is done with the ring row
+    if (p.signs != nullptr) {
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float x[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = v[8 * h + q];
+        apply_signs8(sbits, eA + 512 * h, x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[8 * h + q] = x[q];
+      }
+    }
+    wht_stages<0, 6>(v);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      *reinterpret_cast<float4*>(buf + a_pos + 520 * h) = make_float4(v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3]);
+      *reinterpret_cast<float4*>(buf + a_pos2 + 520 * h) = make_float4(v[8 * h + 4], v[8 * h + 5], v[8 * h + 6], v[8 * h + 7]);
+    }
+    row_barrier(rg, nt);
+
+    // ---- phase B: bits 3-8, then the row's scale
+#pragma unroll
+    for (int j = 0; j < 64; ++j) v[j] = buf[(((j >> 2) & 1) ? b_pos1 : b_pos0) + 8 * j];
+    wht_stages<0, 6>(v);
+    float* rp = red + par * 32;
+    RowQ q;
+    if constexpr (MODE == 1) {
+      float mn = fmin3(v[0], v[1], v[2]), mx = fmax3(v[0], v[1], v[2]);
+#pragma unroll
+      for (int j = 3; j < 63; j += 2) {
+        mn = fmin3(mn, v[j], v[j + 1]);
+        mx = fmax3(mx, v[j], v[j + 1]);
+      }
+      mn = fminf(mn, v[63]);
+      mx = fmaxf(mx, v[63]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      if (lane == 0) { rp[2 * wr] = mx; rp[2 * wr + 1] = mn; }
+      row_barrier(rg, nt);
+      mx = lane < nw ? rp[2 * lane] : -INFINITY;
+      mn = lane < nw ? rp[2 * lane + 1] : INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      q = asym_row_q(mn, mx, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr,
+                     p.zeros + row);
+    } else {
+      float am = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) am = fmax3(am, fabsf(v[j]), fabsf(v[j + 1]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      if (lane == 0) rp[wr] = am;
+      row_barrier(rg, nt);
+      am = lane < nw ? rp[lane] : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      q = sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
+    }
+    const float r = q.r;
+    uint8_t* crow = p.codes + row * (p.Kp >> 1);
+    const int eB = blk * 4096 + 512 * (tb >> 3);  // row element of this thread's layout-B group
+    if (p.rot_debug != nullptr)
+#pragma unroll
+      for (int j = 0; j < 64; ++j) p.rot_debug[row * p.Kp + eB + (tb & 7) + 8 * j] = v[j] * p.inv_sqrt_block;
+
+    // ---- codes in natural order: 8x8 nibble transposes across the 8 lanes
+    // holding one 512-element group
+    const int l = tb & 7;
+    const uint32_t sel4 = (l & 4) ? 0x3276u : 0x5410u;
+    const uint32_t sel2 = (l & 2) ? 0x3715u : 0x6240u;
+    const uint32_t rot1 = (l & 1) ? 28u : 4u;
+    const uint32_t msk1 = (l & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+    uint32_t wd[8];
+#pragma unroll
+    for (int wb = 0; wb < 8; ++wb) {
+      float q8[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) q8[jj] = v[8 * wb + jj];
+      wd[wb] = quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
+    }
+#pragma unroll
+    for (int wb = 0; wb < 8; ++wb) wd[wb] = prmt(wd[wb], __shfl_xor_sync(0xffffffffu, wd[wb], 4), sel4);
+#pragma unroll
+    for (int wb = 0; wb < 8; ++wb) wd[wb] = prmt(wd[wb], __shfl_xor_sync(0xffffffffu, wd[wb], 2), sel2);
+#pragma unroll
+    for (int wb = 0; wb < 8; ++wb) {
+      const uint32_t P = __shfl_xor_sync(0xffffffffu, wd[wb], 1);
+      const uint32_t s4 = __funnelshift_l(P, P, rot1);
+      uint32_t nw2;
+      asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(nw2) : "r"(wd[wb]), "r"(s4), "r"(msk1));
+      *reinterpret_cast<uint32_t*>(crow + ((eB + 64 * wb + 8 * l) >> 1)) = nw2;
+    }
+    row_barrier(rg, nt);                          // the row buffer is reused by the next row
+  }
+}
+
 // ------------------------------------------------------------------ few rows
 
 // Few rows (decode): a cluster of CL CTAs per row, each holding a span of
@@ -1220,6 +1746,148 @@ cudaError_t launch_ring_kernel(Kernel k, const WhtParams& p, int threads, size_t
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
+template <int LB, int CPW>
+cudaError_t dispatch_blk(int mode, bool clip, const WhtParams& p, int threads, size_t smem, int grid,
+                         cudaStream_t s) {
+  if (mode == 1) return launch_ring_kernel(wht_blk_kernel<LB, CPW, 1, true>, p, threads, smem, grid, s);
+  if (mode == 2)
+    return clip ? launch_ring_kernel(wht_blk_kernel<LB, CPW, 2, true>, p, threads, smem, grid, s)
+                : launch_ring_kernel(wht_blk_kernel<LB, CPW, 2, false>, p, threads, smem, grid, s);
+  return clip ? launch_ring_kernel(wht_blk_kernel<LB, CPW, 0, true>, p, threads, smem, grid, s)
+              : launch_ring_kernel(wht_blk_kernel<LB, CPW, 0, false>, p, threads, smem, grid, s);
+}
+
+// Thread budget of the block-local kernel instantiation for (lb, cpw).
+int blk_bound(int lb, int cpw) {
+  switch (lb * 16 + cpw) {
+    case 6 * 16 + 4: return BlkBounds<6, 4>::value;
+    case 7 * 16 + 2: return BlkBounds<7, 2>::value;
+    case 7 * 16 + 4: return BlkBounds<7, 4>::value;
+    case 8 * 16 + 1: return BlkBounds<8, 1>::value;
+    case 8 * 16 + 2: return BlkBounds<8, 2>::value;
+    default: return 0;
+  }
+}
+
+// Rows of blocks of 64..256 through wht_blk_kernel.  Returns false (nothing
+// launched) when the row shape does not fit it.
+bool launch_wht_blk(const RowJob& job, WhtParams p, int lb, cudaStream_t stream, qr_status* st) {
+  if (lb < 6 || lb > 8 || job.K <= 0 || job.Kp <= 0 || job.rows <= 0 || job.K % 8 != 0 || job.ld % 8 != 0 ||
+      reinterpret_cast<uintptr_t>(job.src) % 16 != 0)
+    return false;
+  p.status = device_status_word();
+  if (p.status == nullptr) return false;
+  const int chunk = 4 << lb;
+  const int nchunks = (job.Kp + chunk - 1) / chunk;
+  const int cpw_small = lb == 6 ? 4 : (lb == 7 ? 2 : 1);
+  int cpw = (nchunks + cpw_small - 1) / cpw_small <= 16 ? cpw_small : (lb == 6 ? 0 : 2 * cpw_small);
+  if (cpw == 0) return false;
+  const int W = (nchunks + cpw - 1) / cpw;
+  if (W < 1 || W > 16) return false;
+  const int bound = blk_bound(lb, cpw);
+  const int64_t blocks = std::min<int64_t>(job.rows, sm_count());
+  const int64_t per_block = (job.rows + blocks - 1) / blocks;
+  const int row_bytes = static_cast<int>(job.K * 2);
+  const size_t buf_floats = 4 * static_cast<size_t>((1 << lb) + 8);
+  const size_t sign_bytes = p.signs != nullptr ? static_cast<size_t>(job.Kp / 8) : 0;
+  int groups = static_cast<int>(std::min<int64_t>(std::min(8, (bound - 32) / (32 * W)), per_block));
+  for (; groups >= 1; --groups) {
+    size_t off = sizeof(float) * 64 * groups;                                   // red
+    p.off_red = 0;
+    p.off_buf = static_cast<int32_t>(align_up(off, 16));
+    off = p.off_buf + sizeof(float) * buf_floats * W * groups;
+    p.off_kept = static_cast<int32_t>(align_up(off, 16));
+    if (job.n_out > 0) off = p.off_kept + sizeof(uint16_t) * align_up(job.Kr, 8);
+    p.off_idx = static_cast<int32_t>(align_up(off, 16));
+    if (job.n_out > 0) off = p.off_idx + sizeof(int32_t) * job.n_out;
+    p.off_signs = static_cast<int32_t>(align_up(off, 16));
+    off = p.off_signs + sign_bytes;
+    p.off_ring = static_cast<int32_t>(align_up(off, 128));
+    const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - p.off_ring - 16 * per_block - 16 - 16) /
+                        row_bytes;
+    int slots = static_cast<int>(std::min<int64_t>(per_block, fit));
+    // reused slots each belong to one row group (no parity aliasing)
+    if (slots < per_block) slots = slots / groups * groups;
+    if (slots < 1) continue;
+    p.ring_slots = slots;
+    p.ring_row_bytes = row_bytes;
+    p.off_bars = static_cast<int32_t>(align_up(p.off_ring + static_cast<size_t>(slots) * row_bytes, 16));
+    const size_t smem = p.off_bars + 16 * static_cast<size_t>(slots) + 16;
+    p.rows_per_block = static_cast<int32_t>(per_block);
+    p.rows_per_cta = groups;
+    p.nt = 32 * W;
+    const int threads = groups * 32 * W + 32;
+    const int grid = static_cast<int>((job.rows + per_block - 1) / per_block);
+    const int mode = job.zeros != nullptr ? 1 : (job.bits == 8 ? 2 : 0);
+    const bool clip = p.clip_ratio < 1.0f;
+    cudaError_t e;
+    switch (lb * 16 + cpw) {
+      case 6 * 16 + 4: e = dispatch_blk<6, 4>(mode, clip, p, threads, smem, grid, stream); break;
+      case 7 * 16 + 2: e = dispatch_blk<7, 2>(mode, clip, p, threads, smem, grid, stream); break;
+      case 7 * 16 + 4: e = dispatch_blk<7, 4>(mode, clip, p, threads, smem, grid, stream); break;
+      case 8 * 16 + 1: e = dispatch_blk<8, 1>(mode, clip, p, threads, smem, grid, stream); break;
+      case 8 * 16 + 2: e = dispatch_blk<8, 2>(mode, clip, p, threads, smem, grid, stream); break;
+      default: return false;
+    }
+    *st = e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+    return true;
+  }
+  return false;
+}
+
+// Rows of 4096-point blocks through wht_h12_kernel (4-bit codes, no outlier
+// gather, aligned rows).  Returns false (nothing launched) when the shape
+// does not fit it.
+bool launch_wht_h12(const RowJob& job, WhtParams p, int lb, cudaStream_t stream, qr_status* st) {
+  if (lb != 12 || job.bits != 4 || job.n_out != 0 || job.K <= 0 || job.rows <= 0 || job.K % 8 != 0 ||
+      job.ld % 8 != 0 || reinterpret_cast<uintptr_t>(job.src) % 16 != 0 || job.Kp % 4096 != 0)
+    return false;
+  p.status = device_status_word();
+  if (p.status == nullptr) return false;
+  const int nblk = job.Kp / 4096;
+  const int nt = 64 * nblk;
+  if (nt + 32 > 512) return false;
+  const int64_t blocks = std::min<int64_t>(job.rows, sm_count());
+  const int64_t per_block = (job.rows + blocks - 1) / blocks;
+  const int row_bytes = static_cast<int>(job.K * 2);
+  const size_t sign_bytes = p.signs != nullptr ? static_cast<size_t>(job.Kp / 8) : 0;
+  int groups = static_cast<int>(std::min<int64_t>(std::min(8, (512 - 32) / nt), per_block));
+  for (; groups >= 1; --groups) {
+    p.off_red = 0;
+    size_t off = sizeof(float) * 64 * groups;
+    p.off_buf = static_cast<int32_t>(align_up(off, 16));
+    off = p.off_buf + sizeof(float) * static_cast<size_t>(kH12Floats) * nblk * groups;
+    p.off_signs = static_cast<int32_t>(align_up(off, 16));
+    off = p.off_signs + sign_bytes;
+    p.off_ring = static_cast<int32_t>(align_up(off, 128));
+    const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - p.off_ring - 16 * per_block - 16 - 16) /
+                        row_bytes;
+    int slots = static_cast<int>(std::min<int64_t>(per_block, fit));
+    if (slots < per_block) slots = slots / groups * groups;   // reused slots: one group each
+    if (slots < 1) continue;
+    p.ring_slots = slots;
+    p.ring_row_bytes = row_bytes;
+    p.off_bars = static_cast<int32_t>(align_up(p.off_ring + static_cast<size_t>(slots) * row_bytes, 16));
+    const size_t smem = p.off_bars + 16 * static_cast<size_t>(slots) + 16;
+    p.rows_per_block = static_cast<int32_t>(per_block);
+    p.rows_per_cta = groups;
+    p.nt = nt;
+    const int threads = groups * nt + 32;
+    const int grid = static_cast<int>((job.rows + per_block - 1) / per_block);
+    const bool clip = p.clip_ratio < 1.0f;
+    cudaError_t e;
+    if (job.zeros != nullptr)
+      e = launch_ring_kernel(wht_h12_kernel<1, true>, p, threads, smem, grid, stream);
+    else if (clip)
+      e = launch_ring_kernel(wht_h12_kernel<0, true>, p, threads, smem, grid, stream);
+    else
+      e = launch_ring_kernel(wht_h12_kernel<0, false>, p, threads, smem, grid, stream);
+    *st = e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+    return true;
+  }
+  return false;
+}
+
 template <int MB, int HA, int OUT, bool CLIP, bool RING>
 cudaError_t dispatch_items(int items, const WhtParams& p, int threads, size_t smem, int grid,
                            cudaStream_t s) {
@@ -1382,6 +2050,11 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
   p.rot_debug = job.rot_debug;
   p.bits8 = job.bits == 8;
   if (job.Kp > 32768) return QR_ERR_UNSUPPORTED;
+  {
+    qr_status st = QR_OK;
+    if (launch_wht_blk(job, p, lb, stream, &st)) return st;
+    if (launch_wht_h12(job, p, lb, stream, &st)) return st;
+  }
 
   const bool small = lb <= 3;
   int items_total, imax;
@@ -1441,13 +2114,22 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
     int groups = static_cast<int>(std::min<int64_t>(max_groups, per_block));
     while (groups > 1 && groups * nt + 32 > bound) --groups;
     // layout: red | row-group buffers | ring slots | barriers
-    size_t roff = align_up(sizeof(float) * 32 * groups, 16);
-    const size_t buf_off = roff;
-    roff = align_up(roff + static_cast<size_t>(p.buf_bytes) * groups, 128);
-    const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - static_cast<int64_t>(roff) -
-                         16 * per_block - 16 - 1024 - static_cast<int64_t>(sign_bytes)) / row_bytes;
-    const int slots = static_cast<int>(std::min<int64_t>(per_block, fit));
-    if (slots >= 1 && groups * nt + 32 <= bound) {
+    size_t roff = 0, buf_off = 0;
+    int slots = 0;
+    for (; groups >= 1; --groups) {
+      roff = align_up(sizeof(float) * 32 * groups, 16);
+      buf_off = roff;
+      roff = align_up(roff + static_cast<size_t>(p.buf_bytes) * groups, 128);
+      const int64_t fit = (static_cast<int64_t>(max_smem_optin()) - static_cast<int64_t>(roff) -
+                           16 * per_block - 16 - 1024 - static_cast<int64_t>(sign_bytes)) / row_bytes;
+      slots = static_cast<int>(std::min<int64_t>(per_block, fit));
+      // Reused slots must each belong to one row group (a slot count that is a
+      // multiple of the groups): a group then never waits on a slot more than
+      // one phase past its own last use of it, so parity waits cannot alias.
+      if (slots < per_block) slots = slots / groups * groups;
+      if (slots >= 1) break;
+    }
+    if (groups >= 1 && slots >= 1 && groups * nt + 32 <= bound) {
       p.off_red = 0;
       p.off_buf = static_cast<int32_t>(buf_off);
       p.off_kept = p.off_idx = 0;                                // no outlier gather here
