@@ -323,6 +323,37 @@ def dequant_fp4_rows(q: Fp4Quantized) -> np.ndarray:
     return np.asarray(q.scales, np.float64)[:, None] * e2m1_value(q.codes)
 
 
+def pack_fp4(codes: np.ndarray) -> np.ndarray:
+    """e2m1 nibbles two per byte, element 2j in the low nibble (R15)."""
+    c = np.asarray(codes, dtype=np.int64)
+    if c.shape[-1] % 2:
+        raise ValueError("packed rows need an even width")
+    return ((c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def unpack_fp4(b: np.ndarray) -> np.ndarray:
+    """Inverse of pack_fp4: uint8 nibble codes."""
+    b = np.asarray(b, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def fp4_gemm(ca: np.ndarray, cw: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k e2m1(ca[m, k]) e2m1(cw[n, k]) as float64, exact.
+
+    Every e2m1 value is a multiple of 1/2 of magnitude <= 6, so each product
+    is a multiple of 1/4 below 36 and every partial sum is an exact float64
+    (and float32, below 2^22 quarters) whatever the order (R15).
+    """
+    a = e2m1_value(ca)
+    w = e2m1_value(cw)
+    if a.shape[1] * 36 * 4 >= 2 ** 53:
+        raise ValueError("K too large for an exact float64 dot product")
+    return a @ w.T
+
+
 @dataclass
 class AsymQuantized:
     codes: np.ndarray        # int8 [rows x K_p]: q - 8, in [-8, 7]
@@ -539,6 +570,44 @@ def linear_forward(x, w, rot: Rotation, outlier_idx=None, bits: int = 4):
     a = quantize_activations(x, rot, outlier_idx, bits)
     ws = quantize_weights(w, rot, outlier_idx, bits)
     acc, y = linear(a, ws)
+    return a, ws, acc, y
+
+
+def quantize_activations_fp4(x: np.ndarray, rot: Rotation,
+                             outlier_idx: Optional[np.ndarray] = None) -> Side:
+    """The online activation path with e2m1 codes and a per-token scale (R15)."""
+    x_in, x_out = split_outliers(x, outlier_idx)
+    n_out = 0 if outlier_idx is None else len(outlier_idx)
+    k_p = packed_width(rot, np.asarray(x).shape[1], n_out)
+    xr = rotate_activations(pad_columns(np.asarray(x_in, np.float64), k_p), rot)
+    q = quantize_rows_fp4(xr, rot.clip_ratio)
+    return Side(xr, q, pack_fp4(q.codes), np.asarray(x_out, np.float16))
+
+
+def quantize_weights_fp4(w: np.ndarray, rot: Rotation,
+                         outlier_idx: Optional[np.ndarray] = None) -> Side:
+    """The offline weight path with e2m1 codes and a per-channel scale (R15)."""
+    w_in, w_out = split_outliers(w, outlier_idx)
+    n_out = 0 if outlier_idx is None else len(outlier_idx)
+    k_p = packed_width(rot, np.asarray(w).shape[1], n_out)
+    wr = rotate_weights(pad_columns(np.asarray(w_in, np.float64), k_p), rot)
+    q = quantize_rows_fp4(wr, rot.clip_ratio)
+    return Side(wr, q, pack_fp4(q.codes), np.asarray(w_out, np.float16))
+
+
+def linear_fp4(a: Side, w: Side):
+    """(acc, Y) of the FP4 layer: acc = sum e2m1(q_a) e2m1(q_w) (exact),
+    Y = fp16(acc s_a s_w + X_out W_out^T) as for the integer codes (R15)."""
+    acc = fp4_gemm(a.q.codes, w.q.codes)
+    y = dequant_epilogue(acc, a.q.scales, w.q.scales, a.fp16_part, w.fp16_part)
+    return acc, y
+
+
+def linear_forward_fp4(x, w, rot: Rotation, outlier_idx=None):
+    """The whole layer through rotated e2m1 codes (R15)."""
+    a = quantize_activations_fp4(x, rot, outlier_idx)
+    ws = quantize_weights_fp4(w, rot, outlier_idx)
+    acc, y = linear_fp4(a, ws)
     return a, ws, acc, y
 
 

@@ -674,3 +674,54 @@ def test_fp4_quantizer_error_bound():
     assert np.all(np.abs(xh - x) <= gap * s * (1 + 1e-5) + 1e-12)
     # each row's largest value lands on the top of the grid (6 s = absmax)
     np.testing.assert_allclose(np.abs(xh).max(axis=1), np.abs(x).max(axis=1), rtol=1e-6)
+
+
+def _e2m1_decode_bits(c: int) -> float:
+    """e2m1 decoded from its fields, independently of the oracle's table:
+    sign bit 3, exponent bits 2-1 (bias 1), mantissa bit 0; exponent 0 is
+    subnormal (m / 2)."""
+    sign = -1.0 if c & 8 else 1.0
+    e, m = (c >> 1) & 3, c & 1
+    return sign * (m * 0.5 if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1))
+
+
+def test_fp4_pack_layout():
+    # element 2j in the low nibble: codes (1, 9, 15, 0) -> bytes 0x91, 0x0F
+    b = O.pack_fp4(np.array([[1, 9, 15, 0]], np.uint8))
+    assert b.tolist() == [[0x91, 0x0F]]
+    rng = np.random.default_rng(5)
+    c = rng.integers(0, 16, size=(3, 64)).astype(np.uint8)
+    assert np.array_equal(O.unpack_fp4(O.pack_fp4(c)), c)
+
+
+def test_fp4_gemm_brute_force():
+    # the exact accumulator against a triple loop over field-decoded values
+    rng = np.random.default_rng(6)
+    ca = rng.integers(0, 16, size=(3, 40)).astype(np.uint8)
+    cw = rng.integers(0, 16, size=(4, 40)).astype(np.uint8)
+    acc = O.fp4_gemm(ca, cw)
+    for m in range(3):
+        for n in range(4):
+            want = sum(_e2m1_decode_bits(int(ca[m, k])) * _e2m1_decode_bits(int(cw[n, k]))
+                       for k in range(40))
+            assert acc[m, n] == want
+    # products are quarter-integers: the sum is exact, and equals it at the
+    # extremes (all +-6: 36 K)
+    full = np.full((1, 4096), 7, np.uint8)                  # +6
+    neg = np.full((1, 4096), 15, np.uint8)                  # -6
+    assert O.fp4_gemm(full, np.vstack([full, neg]))[0].tolist() == [36.0 * 4096, -36.0 * 4096]
+
+
+def test_fp4_layer_is_lossless_on_grid_inputs():
+    # rows that are (scale x e2m1 values) with absmax 6 x scale quantize
+    # without error, so with no rotation Y = fp16(X W^T) exactly (float64 sum)
+    rng = np.random.default_rng(8)
+    grid = np.concatenate([-O.E2M1, O.E2M1])
+    K = 64
+    x = rng.choice(grid, size=(4, K)) * 0.25
+    w = rng.choice(grid, size=(5, K)) * 0.125
+    x[:, 0] = 6 * 0.25
+    w[:, 0] = -6 * 0.125
+    a, ws, acc, y = O.linear_forward_fp4(x, w, O.Rotation(O.NONE))
+    assert np.array_equal(y, (x @ w.T).astype(np.float16))
+    np.testing.assert_array_equal(acc * 0.25 * 0.125, x @ w.T)
