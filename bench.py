@@ -52,6 +52,8 @@ KERNEL_SOURCES = {
     "w4a4_gemm_pair_kernel": ["w4a4_gemm_pair.cu", "qr_device.cuh"],
     "w4a4_gemm_decode_kernel": ["w4a4_gemm_decode.cu", "qr_device.cuh"],
     "wht_ab_kernel": ["rotate_quant.cu", "qr_device.cuh"],
+    "wht_blk_kernel": ["rotate_quant.cu", "qr_device.cuh"],
+    "wht_h12_kernel": ["rotate_quant.cu", "qr_device.cuh"],
     "wht_few_rows_kernel": ["rotate_quant.cu", "qr_device.cuh"],
     "kron_tc_kernel": ["kron_tc.cu", "qr_device.cuh"],
     "w8a8_gemm_kernel": ["w8a8_gemm.cu", "qr_device.cuh"],
@@ -88,9 +90,17 @@ def gemm_kernel_name(M: int, bits: int = 4) -> str:
 
 
 def rotate_kernel_name(spec, M: int, sms: int) -> str:
+    """The rotate kernel the library routes these (aligned) rows to."""
     if spec.rotation == "kron":
         return "kron_tc_kernel"
-    return "wht_few_rows_kernel" if M <= sms else "wht_ab_kernel"
+    if M <= sms:
+        return "wht_few_rows_kernel"
+    block = spec.block or spec.K
+    if block in (64, 128, 256):
+        return "wht_blk_kernel"
+    if block == 4096 and spec.bits == 4 and spec.n_keep_fp16 == 0:
+        return "wht_h12_kernel"
+    return "wht_ab_kernel"
 
 
 def load_peaks():
@@ -271,8 +281,9 @@ def run_ours(args, rank, world, local_rank):
     kp = Q.packed_k(rot, s.K, s.n_keep_fp16)
     asym = args.asym_activations
     bits = s.bits
-    if bits == 8 and asym:
-        raise SystemExit("the 8-bit layers take symmetric activations")
+    fp4 = s.fp4
+    if (bits == 8 or fp4) and asym:
+        raise SystemExit("the 8-bit and FP4 layers take symmetric activations")
     gemm_ops, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp, asym)
 
     # input sets: enough copies that one pass over them exceeds L2 twice
@@ -280,10 +291,10 @@ def run_ours(args, rank, world, local_rank):
     w0 = torch.from_numpy(wl.W).cuda()
     t_pack0 = torch.cuda.Event(enable_timing=True)
     t_pack1 = torch.cuda.Event(enable_timing=True)
-    Q.QuantizedLinear(w0, rot, idx, asym, bits)      # warm-up (module load, attributes)
+    Q.QuantizedLinear(w0, rot, idx, asym, bits, fp4)      # warm-up (module load, attributes)
     torch.cuda.synchronize()
     t_pack0.record()
-    layer0 = Q.QuantizedLinear(w0, rot, idx, asym, bits)
+    layer0 = Q.QuantizedLinear(w0, rot, idx, asym, bits, fp4)
     t_pack1.record()
     torch.cuda.synchronize()
     pack_ms = t_pack0.elapsed_time(t_pack1)
@@ -307,6 +318,9 @@ def run_ours(args, rank, world, local_rank):
         if bits == 8:
             codes, scales, x_out, _ = Q.rotate_quant8(x, rot, idx)
             return codes, scales, x_out, None
+        if fp4:
+            codes, scales, x_out, _ = Q.rotate_quant_fp4(x, rot, idx)
+            return codes, scales, x_out, None
         codes, scales, x_out, _ = Q.rotate_quant(x, rot, idx)
         return codes, scales, x_out, None
 
@@ -317,6 +331,8 @@ def run_ours(args, rank, world, local_rank):
             Q.w4a4_linear_asym(codes, scales, zeros, wc, wsc, wsum, x_out, wo, out=y)
         elif bits == 8:
             Q.w8a8_linear(codes, scales, wc, wsc, x_out, wo, out=y)
+        elif fp4:
+            Q.fp4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
         else:
             Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
 
@@ -429,7 +445,7 @@ def run_ours(args, rank, world, local_rank):
     hbm = peaks["hbm_gbs"]
     clocks = sampler.summary(t0, t1)
     sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
-    gemm_name = gemm_kernel_name(M, bits)
+    gemm_name = gemm_kernel_name(M, 8 if fp4 else bits)    # e2m1 runs the pair kernel of the 8-bit codes
     # the GEMM's bound: tensor cores above the ridge point, HBM below it.
     # The denominator is the burst figure (the timed region is well under a
     # second of GPU time); the sustained and datasheet fractions ride along.
@@ -460,8 +476,10 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "s8",
-        "precision": (f"int{bits} codes on s8 tensor-core MMA, s32 accumulate; fp32 rotation; "
+        "dtype": "e2m1" if fp4 else "s8",
+        "precision": ("e2m1 codes on the f8f6f4 tensor-core MMA, fp32 accumulate; fp32 rotation; "
+                      "fp16 in/out" if fp4 else
+                      f"int{bits} codes on s8 tensor-core MMA, s32 accumulate; fp32 rotation; "
                       "fp16 in/out"),
         "data": "synthetic",
         "config": {"workload": s.name, "M": M, "K": s.K, "N": s.N, "K_p": kp,
@@ -471,6 +489,7 @@ def run_ours(args, rank, world, local_rank):
                    "clip_ratio": s.clip_ratio,
                    "activations": "asymmetric per-token" if asym else "symmetric per-token",
                    "bits": bits,
+                   "codes": "e2m1" if fp4 else "int",
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
@@ -539,8 +558,10 @@ def aggregate_max(value_ms: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- oracle
 
-def oracle_step(O, asym: bool, bits: int = 4):
+def oracle_step(O, asym: bool, bits: int = 4, fp4: bool = False):
     """The oracle's online path: activation quantizer, then the linear."""
+    if fp4:
+        return lambda x, rot, idx, wside: O.linear_fp4(O.quantize_activations_fp4(x, rot, idx), wside)
     if asym:
         return lambda x, rot, idx, wside: O.linear_asym(
             O.quantize_activations_asym(x, rot, idx), wside)
@@ -562,7 +583,8 @@ def oracle_sample(workload: str, tokens: int, rows, M_total=None, random_signs: 
     s = wl.spec
     rot = oracle_rotation(wl, oracle_signs(wl, random_signs))
     idx = O.select_outliers(wl.X_calib, s.n_keep_fp16) if s.n_keep_fp16 else None
-    wside = O.quantize_weights(wl.W.astype(np.float64), rot, idx, s.bits)
+    wside = (O.quantize_weights_fp4(wl.W.astype(np.float64), rot, idx) if s.fp4 else
+             O.quantize_weights(wl.W.astype(np.float64), rot, idx, s.bits))
     x = wl.X[:tokens].astype(np.float64)
     return wl, rot, idx, wside, x
 
@@ -577,7 +599,7 @@ def oracle_baseline(workload: str, tokens: int, rows, repeats: int = 1, M_total=
 
     wl, rot, idx, wside, x = oracle_sample(workload, tokens, rows, M_total, random_signs)
     n_rows = wl.W.shape[0]
-    run = oracle_step(O, asym, wl.spec.bits)
+    run = oracle_step(O, asym, wl.spec.bits, wl.spec.fp4)
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
@@ -617,7 +639,7 @@ def run_reference(args, rank, world):
     wl, rot, idx, wside, x = oracle_sample(args.workload, tokens, rows, args.tokens,
                                            args.random_signs)
     s = wl.spec
-    run = oracle_step(O, args.asym_activations, s.bits)
+    run = oracle_step(O, args.asym_activations, s.bits, s.fp4)
 
     def step():
         run(x, rot, idx, wside)

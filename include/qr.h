@@ -112,8 +112,8 @@ typedef struct {
 } qr_rotation;
 
 /* ABI version of this header (bumped on any change to the entry points;
- * 3 added the 8-bit calls and qr_check_wait_timeout). */
-#define QR_ABI_VERSION 3
+ * 3 added the 8-bit calls and qr_check_wait_timeout, 4 the FP4 calls). */
+#define QR_ABI_VERSION 4
 QR_API int32_t qr_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -220,6 +220,42 @@ QR_API qr_status qr_w8a8_linear(const int8_t* a_codes, const float* a_scales,
                                 int64_t N, int64_t K_p, const uint16_t* x_out,
                                 const uint16_t* w_out, int32_t n_out, uint16_t* Y, int64_t ldy,
                                 int32_t* acc_debug, qr_stream stream);
+
+/* ----------------------------------------------------------------------
+ * FP4 layers (the W-fp4/A-fp4 benchmark on Blackwell's fp4 tensor cores
+ * that the "SpinQuant" review discussion, reviewer brBn W3/A3, names as
+ * planned work, with no format given).  Read as the e2m1 element type with
+ * a per-row fp32 scale, the analogue of the INT4 quantizer: per row,
+ * s = alpha * absmax / 6 and the code of x is the e2m1 value nearest x / s
+ * (ties to the even mantissa, saturating at +-6).  An e2m1 nibble is sign
+ * (bit 3), exponent (bits 2-1, bias 1), mantissa (bit 0); -0 may appear and
+ * decodes to 0.  Codes are packed two per byte, element 2j in the low
+ * nibble: uint8 [rows x K_p / 2], 32-byte aligned.
+ *
+ * qr_rotate_quant_fp4 / qr_pack_weights_fp4: arguments and errors as
+ * qr_rotate_quant / qr_pack_weights.  Supported rotations: HADAMARD or
+ * GSR with blocks of 64, 128 or 256 (outlier columns allowed), and
+ * 4096-point blocks without outliers; others, and KRON, are UNSUPPORTED.
+ * qr_fp4_linear: as qr_w4a4_linear for packed e2m1 codes
+ * (K_p % 128 == 0, K_p <= 65536, code pointers 32-byte aligned):
+ *   acc[m, n] = sum_k e2m1(qa[m, k]) e2m1(qw[n, k])   (fp32; every product
+ *               and partial sum is a multiple of 1/4 of magnitude at most
+ *               36 K_p < 2^22, exactly representable)
+ *   Y[m, n]   = fp16(acc * a_scales[m] * w_scales[n] + X_out[m] . W_out[n])
+ * acc_debug (optional, float [M x N]) receives acc. */
+QR_API qr_status qr_rotate_quant_fp4(const qr_rotation* rot, const uint16_t* X, int64_t M,
+                                     int64_t K, int64_t ldx, const int32_t* outlier_idx,
+                                     int32_t n_out, uint8_t* codes, float* scales,
+                                     uint16_t* x_out, float* x_rot_debug, qr_stream stream);
+QR_API qr_status qr_pack_weights_fp4(const qr_rotation* rot_w, const uint16_t* W, int64_t N,
+                                     int64_t K, int64_t ldw, const int32_t* outlier_idx,
+                                     int32_t n_out, uint8_t* w_codes, float* w_scales,
+                                     uint16_t* w_out, float* w_rot_debug, qr_stream stream);
+QR_API qr_status qr_fp4_linear(const uint8_t* a_codes, const float* a_scales,
+                               const uint8_t* w_codes, const float* w_scales, int64_t M,
+                               int64_t N, int64_t K_p, const uint16_t* x_out,
+                               const uint16_t* w_out, int32_t n_out, uint16_t* Y, int64_t ldy,
+                               float* acc_debug, qr_stream stream);
 
 /* ----------------------------------------------------------------------
  * Asymmetric per-token activations ("QUIK：LLM上的一种4-bit推理方法",

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.qr_abi_version() == 3
+    assert L.qr_abi_version() == 4
     for s in range(6):
         assert L.status_string(s) and L.status_string(s) != "unknown status"
     assert L.status_string(99) == "unknown status"
@@ -218,3 +218,24 @@ def test_int8_entry_points_argument_errors(lib):
     assert lin8(a=FAKE + 4) == L.QR_ERR_ALIGNMENT
     assert lin8(n_out=12, xo=FAKE, wo=FAKE) == L.QR_ERR_UNSUPPORTED
     assert lin8(M=0) == L.QR_OK
+
+
+def test_fp4_entry_points_argument_errors(lib):
+    # the e2m1 calls validate like the others, and want 32-byte aligned codes
+    h = _rot(L.QR_ROT_HADAMARD, 256)
+    def rq4(rot, codes=FAKE, M=4, K=512):
+        return L.qr_rotate_quant_fp4(rot, FAKE, M, K, K, None, 0, codes, FAKE, None, None, None,
+                                     check=False)
+    assert rq4(h, codes=FAKE + 16) == L.QR_ERR_ALIGNMENT
+    assert rq4(h, M=-1) == L.QR_ERR_INVALID_ARG
+    assert rq4(h, M=0) == L.QR_OK
+    assert rq4(_rot(L.QR_ROT_KRON, n1=16, n2=32), K=512) == L.QR_ERR_UNSUPPORTED
+    assert L.qr_pack_weights_fp4(h, FAKE, 4, 512, 512, None, 0, None, FAKE, None, None, None,
+                                 check=False) == L.QR_ERR_INVALID_ARG
+    def lin4(Kp=256, a=FAKE, w=FAKE, M=16):
+        return L.qr_fp4_linear(a, FAKE, w, FAKE, M, 16, Kp, None, None, 0, FAKE, 16, None, None,
+                               check=False)
+    assert lin4(Kp=200) == L.QR_ERR_INVALID_ARG
+    assert lin4(a=FAKE + 16) == L.QR_ERR_ALIGNMENT
+    assert lin4(w=FAKE + 16) == L.QR_ERR_ALIGNMENT
+    assert lin4(M=0) == L.QR_OK

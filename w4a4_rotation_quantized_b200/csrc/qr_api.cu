@@ -129,7 +129,9 @@ static qr_status rows_call(const qr_rotation* rot, const uint16_t* src, int64_t 
     if (reinterpret_cast<uintptr_t>(rot->signs) % 8 != 0) return QR_ERR_ALIGNMENT;
   }
   if (zeros != nullptr && rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
-  if (bits == 8 && rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
+  if ((bits == 8 || bits == kFp4Codes) && rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
+  if (bits == kFp4Codes && kp > 0 && reinterpret_cast<uintptr_t>(codes) % 32 != 0)
+    return QR_ERR_ALIGNMENT;
   RowJob job{};
   job.bits = bits;
   job.src = src;
@@ -257,6 +259,9 @@ static qr_status linear_call(const uint8_t* a_codes, const float* a_scales, cons
   if (K_p > 65536 || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
   if (n_out % 8 != 0) return QR_ERR_UNSUPPORTED;
   if (K_p > 0 && (!aligned16(a_codes) || !aligned16(w_codes))) return QR_ERR_ALIGNMENT;
+  if (bits == kFp4Codes && K_p > 0 &&     // the 4-bit tensor maps want 32-byte bases
+      (reinterpret_cast<uintptr_t>(a_codes) % 32 != 0 || reinterpret_cast<uintptr_t>(w_codes) % 32 != 0))
+    return QR_ERR_ALIGNMENT;
   if (n_out > 0 && (!aligned16(x_out) || !aligned16(w_out))) return QR_ERR_ALIGNMENT;
   GemmJob j{};
   j.a_codes = a_codes;
@@ -274,8 +279,9 @@ static qr_status linear_call(const uint8_t* a_codes, const float* a_scales, cons
   j.Y = Y;
   j.ldy = ldy;
   j.acc_debug = acc_debug;
-  return bits == 8 ? launch_w8a8_gemm(j, reinterpret_cast<cudaStream_t>(stream))
-                   : launch_w4a4_gemm(j, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return bits == 8 ? launch_w8a8_gemm(j, st) : bits == kFp4Codes ? launch_fp4_gemm(j, st)
+                                                                 : launch_w4a4_gemm(j, st);
 }
 
 }  // namespace qr
@@ -338,6 +344,31 @@ qr_status qr_w8a8_linear(const int8_t* a_codes, const float* a_scales, const int
   return linear_call(reinterpret_cast<const uint8_t*>(a_codes), a_scales, nullptr,
                      reinterpret_cast<const uint8_t*>(w_codes), w_scales, nullptr, M, N, K_p,
                      x_out, w_out, n_out, Y, ldy, acc_debug, stream, 8);
+}
+
+qr_status qr_rotate_quant_fp4(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                              int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
+                              uint8_t* codes, float* scales, uint16_t* x_out, float* x_rot_debug,
+                              qr_stream stream) {
+  return rows_call(rot, X, M, K, ldx, outlier_idx, n_out, codes, scales, nullptr, x_out,
+                   x_rot_debug, stream, kFp4Codes);
+}
+
+qr_status qr_pack_weights_fp4(const qr_rotation* rot_w, const uint16_t* W, int64_t N, int64_t K,
+                              int64_t ldw, const int32_t* outlier_idx, int32_t n_out,
+                              uint8_t* w_codes, float* w_scales, uint16_t* w_out,
+                              float* w_rot_debug, qr_stream stream) {
+  return rows_call(rot_w, W, N, K, ldw, outlier_idx, n_out, w_codes, w_scales, nullptr, w_out,
+                   w_rot_debug, stream, kFp4Codes);
+}
+
+qr_status qr_fp4_linear(const uint8_t* a_codes, const float* a_scales, const uint8_t* w_codes,
+                        const float* w_scales, int64_t M, int64_t N, int64_t K_p,
+                        const uint16_t* x_out, const uint16_t* w_out, int32_t n_out, uint16_t* Y,
+                        int64_t ldy, float* acc_debug, qr_stream stream) {
+  return linear_call(a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, M, N, K_p, x_out,
+                     w_out, n_out, Y, ldy, reinterpret_cast<int32_t*>(acc_debug), stream,
+                     kFp4Codes);
 }
 
 qr_status qr_check_wait_timeout(int64_t limit_ns, qr_stream stream) {

@@ -535,6 +535,25 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D(tmem of both CTAs, fp32) (+)= A(smem of both CTAs) x B(smem halves)^T
+// with the kind::f8f6f4 operand types of the instruction descriptor (e2m1
+// here), M = 256 across the pair.  Issued by one thread of the even CTA.
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// M=256 over a CTA pair, N=n: e2m1 x e2m1 -> fp32 (kind::f8f6f4, operand
+// format code 5 for A and B), K-major.
+__host__ __device__ constexpr uint32_t idesc_e2m1_m256(uint32_t n) {
+  return (1u << 4) | (5u << 7) | (5u << 10) | ((n >> 3) << 17) | ((256u >> 4) << 24);
+}
+
 // M=256 over a CTA pair, N=n: fp16 x fp16 -> fp32, K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_m256(uint32_t n) {
   return (1u << 4) | ((n >> 3) << 17) | ((256u >> 4) << 24);

@@ -64,8 +64,11 @@ struct RowJob {
   int32_t* zeros;             // [rows] zero points (asymmetric activations) or null
   uint16_t* out16;            // [rows x n_out] or null
   float* rot_debug;           // [rows x Kp] or null
-  int32_t bits;               // code width: 4 (packed nibbles) or 8 (one int8 per code)
+  int32_t bits;               // codes: 4 (int4 nibbles), 8 (one int8 each) or kFp4Codes
 };
+
+// RowJob::bits for e2m1 codes, packed two per byte like the int4 nibbles.
+constexpr int32_t kFp4Codes = 0xF4;
 
 qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream);
 
@@ -90,6 +93,10 @@ qr_status launch_w4a4_gemm(const GemmJob& job, cudaStream_t stream);
 // 8-bit codes (one int8 per code, rows of K_p bytes): TMA-fed tcgen05
 // kind::i8 MMAs with both operands in shared memory.
 qr_status launch_w8a8_gemm(const GemmJob& job, cudaStream_t stream);
+// Packed e2m1 codes (two per byte, rows of K_p / 2 bytes): the same pair
+// kernel with kind::f8f6f4 MMAs and an fp32 accumulator (acc_debug is then
+// a float array).
+qr_status launch_fp4_gemm(const GemmJob& job, cudaStream_t stream);
 
 // M > 64: 2-SM tcgen05 MMA with the activation operand in TMEM, fp16
 // outlier columns as a second MMA.

@@ -778,6 +778,33 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
   }
 }
 
+// FP4 (e2m1) codes with a per-row scale: s = alpha * absmax / 6; the codes
+// are the nearest e2m1 values of x / s (ties to the even mantissa,
+// saturating at +-6), the tensor core's own conversion.
+__device__ __forceinline__ RowQ sym_row_qf4(float am, float clip, float inv_sqrt, float* scale_out) {
+  if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 6.0f;
+  return RowQ{(am > 0.0f) ? 6.0f / (clip * am) : 0.0f, 0.0f, 0.0f, 0.0f};
+}
+
+// Two e2m1 codes of (lo * r, hi * r) in one byte, lo in the low nibble.
+__device__ __forceinline__ uint32_t e2m1_pair(float lo, float hi, float r) {
+  uint32_t b;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(b)
+      : "f"(hi * r), "f"(lo * r));
+  return b;
+}
+
+// Eight consecutive e2m1 codes of v[i] * r packed two per byte, v[0] in the
+// low nibble (the layout of quant_word).
+__device__ __forceinline__ uint32_t quant_word_fp4(const float (&v)[8], float r) {
+  const uint32_t b0 = e2m1_pair(v[0], v[1], r), b1 = e2m1_pair(v[2], v[3], r);
+  const uint32_t b2 = e2m1_pair(v[4], v[5], r), b3 = e2m1_pair(v[6], v[7], r);
+  return prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
+}
+
 // Three-input maximum / minimum (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -788,6 +815,24 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   float r;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// Stage-0 butterfly of a half2 (lo, hi) straight into fp32: (lo + hi, lo - hi),
+// each with one rounding (mixed-precision fma with an fp16 multiplicand).
+__device__ __forceinline__ void bfly_h2(uint32_t w, float& y0, float& y1) {
+  asm("{\n\t.reg .f16 l, h, one;\n\t.reg .f32 fh, nfh;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "mov.b16 one, 0x3C00;\n\t"
+      "cvt.f32.f16 fh, h;\n\t"
+      "neg.f32 nfh, fh;\n\t"
+      "fma.rn.f32.f16 %0, l, one, fh;\n\t"
+      "fma.rn.f32.f16 %1, l, one, nfh;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "r"(w));
+}
+// Sign flips of a half2 word for elements 2q, 2q+1 from a byte of sign bits.
+__device__ __forceinline__ uint32_t sign_mask_h2(uint32_t b, int q) {
+  return (((b >> (2 * q)) & 1u) << 15) | (((b >> (2 * q + 1)) & 1u) << 31);
 }
 
 // ------------------------------------------------------------------ block-local rows
@@ -864,7 +909,8 @@ __device__ __forceinline__ void blk_load8(const WhtParams& p, const __half* rrow
   }
 }
 
-// MODE: 0 = symmetric 4-bit, 1 = asymmetric 4-bit, 2 = symmetric 8-bit.
+// MODE: 0 = symmetric 4-bit, 1 = asymmetric 4-bit, 2 = symmetric 8-bit,
+// 3 = e2m1 (FP4).
 template <int LB, int CPW, int MODE, bool CLIP>
 __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(const WhtParams p) {
   using G = BlkGeom<LB>;
@@ -935,6 +981,7 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
   const int a_pos2 = (lane >> (LB - 3)) * G::kStride + qa + 4 - xa;
   // Layout-B loads: value m sits at b_pos[(m >> 2) & 1] + 8 m.
   const int b_pos0 = b * G::kStride + tl, b_pos1 = b * G::kStride + (tl ^ 4);
+  const bool plain = p.n_out == 0 && p.signs == nullptr;   // no gather, no sign flips
   int par = 0;
   for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
     const int i = static_cast<int>(row - row0);
@@ -958,16 +1005,42 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
       const int ch = wr + c * W;
       if (ch < nchunks) {                         // warp-uniform
         const int e0 = ch * G::kChunk;
+        constexpr int kPieceStride = (256 >> LB) * G::kStride;
+        if (plain && e0 + G::kChunk <= p.Kr) {
+          // whole chunk of a plain row: no per-piece checks
 #pragma unroll
-        for (int j = 0; j < G::kPieces; ++j) {
-          const int o = 256 * j + 8 * lane;
-          float x[8];
-          blk_load8(p, rrow, kept, e0 + o, x);
-          if (p.signs != nullptr && e0 + o < p.Kp) apply_signs8(sbits, e0 + o, x);
-          wht_stages<0, 3>(x);
-          constexpr int kPieceStride = (256 >> LB) * G::kStride;
-          *reinterpret_cast<float4*>(buf + a_pos + j * kPieceStride) = make_float4(x[0], x[1], x[2], x[3]);
-          *reinterpret_cast<float4*>(buf + a_pos2 + j * kPieceStride) = make_float4(x[4], x[5], x[6], x[7]);
+          for (int j = 0; j < G::kPieces; ++j) {
+            const uint4 u = *reinterpret_cast<const uint4*>(rrow + e0 + 256 * j + 8 * lane);
+            float x[8];
+            bfly_h2(u.x, x[0], x[1]); bfly_h2(u.y, x[2], x[3]);
+            bfly_h2(u.z, x[4], x[5]); bfly_h2(u.w, x[6], x[7]);
+            wht_stages<1, 3>(x);
+            *reinterpret_cast<float4*>(buf + a_pos + j * kPieceStride) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4*>(buf + a_pos2 + j * kPieceStride) = make_float4(x[4], x[5], x[6], x[7]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < G::kPieces; ++j) {
+            const int e = e0 + 256 * j + 8 * lane;
+            float x[8];
+            if (p.n_out == 0 && e + 8 <= p.Kr) {
+              uint4 u = *reinterpret_cast<const uint4*>(rrow + e);
+              if (p.signs != nullptr) {
+                const uint32_t sb = sbits[e >> 3];
+                u.x ^= sign_mask_h2(sb, 0); u.y ^= sign_mask_h2(sb, 1);
+                u.z ^= sign_mask_h2(sb, 2); u.w ^= sign_mask_h2(sb, 3);
+              }
+              bfly_h2(u.x, x[0], x[1]); bfly_h2(u.y, x[2], x[3]);
+              bfly_h2(u.z, x[4], x[5]); bfly_h2(u.w, x[6], x[7]);
+              wht_stages<1, 3>(x);
+            } else {
+              blk_load8(p, rrow, kept, e, x);
+              if (p.signs != nullptr && e < p.Kp) apply_signs8(sbits, e, x);
+              wht_stages<0, 3>(x);
+            }
+            *reinterpret_cast<float4*>(buf + a_pos + j * kPieceStride) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4*>(buf + a_pos2 + j * kPieceStride) = make_float4(x[4], x[5], x[6], x[7]);
+          }
         }
         __syncwarp();
 #pragma unroll
@@ -1020,8 +1093,9 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
       float* so = (wr == 0 && lane == 0) ? p.scales + row : nullptr;
-      q = MODE == 2 ? sym_row_q8(am, p.clip_ratio, p.inv_sqrt_block, so)
-                    : sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, so);
+      q = MODE == 2   ? sym_row_q8(am, p.clip_ratio, p.inv_sqrt_block, so)
+          : MODE == 3 ? sym_row_qf4(am, p.clip_ratio, p.inv_sqrt_block, so)
+                      : sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, so);
     }
     const float r = q.r;
 
@@ -1057,6 +1131,8 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
           if (ok) {
             if constexpr (MODE == 2)
               *reinterpret_cast<uint2*>(crow + (bg << LB) + 8 * kw) = quant_bytes8<CLIP>(w8, r, q.c, q.lo, q.hi);
+            else if constexpr (MODE == 3)
+              *reinterpret_cast<uint32_t*>(crow + (((bg << LB) + 8 * kw) >> 1)) = quant_word_fp4(w8, r);
             else
               *reinterpret_cast<uint32_t*>(crow + (((bg << LB) + 8 * kw) >> 1)) =
                   quant_word<CLIP>(w8, r, q.c, q.lo, q.hi);
@@ -1079,7 +1155,7 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
           float q8[8];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) q8[jj] = v[c][8 * wb + jj];
-          wd[wb] = quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
+          wd[wb] = MODE == 3 ? quant_word_fp4(q8, r) : quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
         }
 #pragma unroll
         for (int wb = 0; wb < VB / 8; ++wb) wd[wb] = prmt(wd[wb], __shfl_xor_sync(0xffffffffu, wd[wb], 4), sel4);
@@ -1111,7 +1187,8 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
 // Rows stream into a shared-memory ring by bulk copies (one producer warp).
 constexpr int kH12Floats = 4096 + 64;
 
-// MODE: 0 = symmetric, 1 = asymmetric (4-bit codes, natural order).
+// MODE: 0 = symmetric, 1 = asymmetric (4-bit codes), 2 = e2m1 (FP4);
+// natural order.
 template <int MODE, bool CLIP>
 __global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
   grid_dep_wait();
@@ -1172,6 +1249,7 @@ __global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
   // layout-B loads: value j at (bit 2 of j ? b_pos1 : b_pos0) + 8 j
   const int b_pos0 = (tb & 7) + 520 * (tb >> 3), b_pos1 = ((tb & 7) ^ 4) + 520 * (tb >> 3);
   const int eA = blk * 4096 + 8 * tb;           // row element of layout-A group h = 0
+  const bool full_plain = p.K == p.Kp && p.signs == nullptr;   // no zero tail, no sign flips
   int par = 0;
   for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
     const int i = static_cast<int>(row - row0);
@@ -1184,37 +1262,35 @@ __global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
 
     // ---- phase A: bits 0-2 and 9-11
     float v[64];
+    if (full_plain) {
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const uint4 u = *reinterpret_cast<const uint4*>(rrow + eA + 512 * h);
+        bfly_h2(u.x, v[8 * h], v[8 * h + 1]); bfly_h2(u.y, v[8 * h + 2], v[8 * h + 3]);
+        bfly_h2(u.z, v[8 * h + 4], v[8 * h + 5]); bfly_h2(u.w, v[8 * h + 6], v[8 * h + 7]);
+      }
+    } else {
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       const int e = eA + 512 * h;
       if (e + 8 <= p.K) {
-        const uint4 u = *reinterpret_cast<const uint4*>(rrow + e);
-        const __half2* hh = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __half22float2(hh[q]);
-          v[8 * h + 2 * q] = f.x;
-          v[8 * h + 2 * q + 1] = f.y;
+        uint4 u = *reinterpret_cast<const uint4*>(rrow + e);
+        if (p.signs != nullptr) {
+          const uint32_t sb = sbits[e >> 3];
+          u.x ^= sign_mask_h2(sb, 0); u.y ^= sign_mask_h2(sb, 1);
+          u.z ^= sign_mask_h2(sb, 2); u.w ^= sign_mask_h2(sb, 3);
         }
+        bfly_h2(u.x, v[8 * h], v[8 * h + 1]); bfly_h2(u.y, v[8 * h + 2], v[8 * h + 3]);
+        bfly_h2(u.z, v[8 * h + 4], v[8 * h + 5]); bfly_h2(u.w, v[8 * h + 6], v[8 * h + 7]);
       } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q) v[8 * h + q] = 0.0f;
       }
     }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&ring_empty[slot]);   // this warp is done with the ring row
-    if (p.signs != nullptr) {
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        float x[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] = v[8 * h + q];
-        apply_signs8(sbits, eA + 512 * h, x);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[8 * h + q] = x[q];
-      }
-    }
-    wht_stages<0, 6>(v);
+    wht_stages<1, 6>(v);
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       *reinterpret_cast<float4*>(buf + a_pos + 520 * h) = make_float4(v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3]);
@@ -1264,7 +1340,8 @@ __global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
       am = lane < nw ? rp[lane] : 0.0f;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      q = sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
+      q = MODE == 2 ? sym_row_qf4(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr)
+                    : sym_row_q(am, p.clip_ratio, p.inv_sqrt_block, t == 0 ? p.scales + row : nullptr);
     }
     const float r = q.r;
     uint8_t* crow = p.codes + row * (p.Kp >> 1);
@@ -1286,7 +1363,7 @@ __global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
       float q8[8];
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) q8[jj] = v[8 * wb + jj];
-      wd[wb] = quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
+      wd[wb] = MODE == 2 ? quant_word_fp4(q8, r) : quant_word<CLIP>(q8, r, q.c, q.lo, q.hi);
     }
 #pragma unroll
     for (int wb = 0; wb < 8; ++wb) wd[wb] = prmt(wd[wb], __shfl_xor_sync(0xffffffffu, wd[wb], 4), sel4);
@@ -1750,6 +1827,7 @@ template <int LB, int CPW>
 cudaError_t dispatch_blk(int mode, bool clip, const WhtParams& p, int threads, size_t smem, int grid,
                          cudaStream_t s) {
   if (mode == 1) return launch_ring_kernel(wht_blk_kernel<LB, CPW, 1, true>, p, threads, smem, grid, s);
+  if (mode == 3) return launch_ring_kernel(wht_blk_kernel<LB, CPW, 3, false>, p, threads, smem, grid, s);
   if (mode == 2)
     return clip ? launch_ring_kernel(wht_blk_kernel<LB, CPW, 2, true>, p, threads, smem, grid, s)
                 : launch_ring_kernel(wht_blk_kernel<LB, CPW, 2, false>, p, threads, smem, grid, s);
@@ -1818,7 +1896,7 @@ bool launch_wht_blk(const RowJob& job, WhtParams p, int lb, cudaStream_t stream,
     p.nt = 32 * W;
     const int threads = groups * 32 * W + 32;
     const int grid = static_cast<int>((job.rows + per_block - 1) / per_block);
-    const int mode = job.zeros != nullptr ? 1 : (job.bits == 8 ? 2 : 0);
+    const int mode = job.zeros != nullptr ? 1 : job.bits == 8 ? 2 : job.bits == kFp4Codes ? 3 : 0;
     const bool clip = p.clip_ratio < 1.0f;
     cudaError_t e;
     switch (lb * 16 + cpw) {
@@ -1839,7 +1917,7 @@ bool launch_wht_blk(const RowJob& job, WhtParams p, int lb, cudaStream_t stream,
 // gather, aligned rows).  Returns false (nothing launched) when the shape
 // does not fit it.
 bool launch_wht_h12(const RowJob& job, WhtParams p, int lb, cudaStream_t stream, qr_status* st) {
-  if (lb != 12 || job.bits != 4 || job.n_out != 0 || job.K <= 0 || job.rows <= 0 || job.K % 8 != 0 ||
+  if (lb != 12 || (job.bits != 4 && job.bits != kFp4Codes) || job.n_out != 0 || job.K <= 0 || job.rows <= 0 || job.K % 8 != 0 ||
       job.ld % 8 != 0 || reinterpret_cast<uintptr_t>(job.src) % 16 != 0 || job.Kp % 4096 != 0)
     return false;
   p.status = device_status_word();
@@ -1876,7 +1954,9 @@ bool launch_wht_h12(const RowJob& job, WhtParams p, int lb, cudaStream_t stream,
     const int grid = static_cast<int>((job.rows + per_block - 1) / per_block);
     const bool clip = p.clip_ratio < 1.0f;
     cudaError_t e;
-    if (job.zeros != nullptr)
+    if (job.bits == kFp4Codes)
+      e = launch_ring_kernel(wht_h12_kernel<2, false>, p, threads, smem, grid, stream);
+    else if (job.zeros != nullptr)
       e = launch_ring_kernel(wht_h12_kernel<1, true>, p, threads, smem, grid, stream);
     else if (clip)
       e = launch_ring_kernel(wht_h12_kernel<0, true>, p, threads, smem, grid, stream);
@@ -2054,6 +2134,7 @@ qr_status launch_wht_rows(const RowJob& job, cudaStream_t stream) {
     qr_status st = QR_OK;
     if (launch_wht_blk(job, p, lb, stream, &st)) return st;
     if (launch_wht_h12(job, p, lb, stream, &st)) return st;
+    if (job.bits == kFp4Codes) return QR_ERR_UNSUPPORTED;   // e2m1 codes: those two kernels only
   }
 
   const bool small = lb <= 3;
@@ -2331,6 +2412,9 @@ qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream) {
   if (job.rows == 0) return QR_OK;
   if (job.bits == 8 && (job.rot->kind == QR_ROT_KRON || job.zeros != nullptr))
     return QR_ERR_UNSUPPORTED;
+  if (job.bits == kFp4Codes)
+    return (job.rot->kind == QR_ROT_KRON || job.zeros != nullptr) ? QR_ERR_UNSUPPORTED
+                                                                   : launch_wht_rows(job, stream);
   if (job.rot->kind == QR_ROT_KRON)
     return kron_tc_supported(job) ? launch_kron_tc(job, stream) : launch_kron_rows(job, stream);
   return few_rows(job) ? launch_wht_few_rows(job, stream) : launch_wht_rows(job, stream);

@@ -70,7 +70,7 @@ struct W8Params {
   const float* w_scales;
   __half* Y;
   int64_t ldy;
-  int32_t* acc_debug;
+  void* acc_debug;                 // int32 (8-bit codes) or float (e2m1 codes) [M x N], or null
   int32_t M, N;
   int32_t kt, ot;                  // int8 K steps, outlier steps
   int32_t tiles_m, tiles_n;        // 256-row activation tiles, 256-row weight tiles
@@ -78,7 +78,9 @@ struct W8Params {
   int32_t* status;
 };
 
-template <bool OUT>
+// FP4: e2m1 codes (kind::f8f6f4, fp32 accumulator), else 8-bit integer codes
+// (kind::i8, int32 accumulator).  Both stage 128 codes per 128-byte row.
+template <bool OUT, bool FP4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads8, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const __grid_constant__ CUtensorMap map_oa,
@@ -147,7 +149,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         for (int st = 0; st < steps; ++st, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (!(ok = mbar_wait_cluster_bounded(&empty[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
-          mbar_arrive_expect_tx(&full[s], S::kStage);
+          // e2m1 tiles count the packed bytes read (half the 128-byte rows
+          // they fill in shared memory)
+          mbar_arrive_expect_tx(&full[s], (FP4 && st < p.kt) ? S::kStage / 2 : S::kStage);
           uint8_t* sa = smem + S::off_ring + s * S::kStage;
           if (st < p.kt) {
             tma_load_2d(sa, &map_a, &full[s], st * kRow, ya);
@@ -180,7 +184,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
     if (leader && lane == 0) {
       // ------------------------------------------------------------ MMA (even CTA)
-      constexpr uint32_t idesc = idesc_i8_m256(BN);
+      constexpr uint32_t idesc = FP4 ? idesc_e2m1_m256(BN) : idesc_i8_m256(BN);
       constexpr uint32_t idesc_o = idesc_f16_m256(BN);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
@@ -198,7 +202,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           if (st < p.kt) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)       // 4 x K32 (32 bytes each)
-              mma_i8_pair(d, da + 2 * k, db + 2 * k, idesc, (st | k) != 0);
+              if constexpr (FP4)
+                mma_f8f6f4_pair(d, da + 2 * k, db + 2 * k, idesc, (st | k) != 0);
+              else
+                mma_i8_pair(d, da + 2 * k, db + 2 * k, idesc, (st | k) != 0);
           } else {
 #pragma unroll
             for (int k = 0; k < 4; ++k)       // 4 x K16 fp16 (32 bytes each)
@@ -246,8 +253,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         uint32_t hp[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          float y0 = kz ? 0.0f : static_cast<float>(static_cast<int32_t>(acc[2 * j])) * sa * sb[32 * c + 2 * j];
-          float y1 = kz ? 0.0f : static_cast<float>(static_cast<int32_t>(acc[2 * j + 1])) * sa * sb[32 * c + 2 * j + 1];
+          const float a0 = FP4 ? __uint_as_float(acc[2 * j]) : static_cast<float>(static_cast<int32_t>(acc[2 * j]));
+          const float a1 = FP4 ? __uint_as_float(acc[2 * j + 1]) : static_cast<float>(static_cast<int32_t>(acc[2 * j + 1]));
+          float y0 = kz ? 0.0f : a0 * sa * sb[32 * c + 2 * j];
+          float y1 = kz ? 0.0f : a1 * sa * sb[32 * c + 2 * j + 1];
           if (OUT && !oz) {
             y0 += __uint_as_float(oacc[2 * j]);
             y1 += __uint_as_float(oacc[2 * j + 1]);
@@ -271,8 +280,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           if (p.acc_debug != nullptr)
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (n0 + j < p.N)
-                p.acc_debug[static_cast<int64_t>(m) * p.N + n0 + j] = kz ? 0 : static_cast<int32_t>(acc[j]);
+              if (n0 + j < p.N)          // raw accumulator bits: int32, or the fp32 sum
+                static_cast<uint32_t*>(p.acc_debug)[static_cast<int64_t>(m) * p.N + n0 + j] = kz ? 0u : acc[j];
         }
       }
       tc_fence_before();
@@ -290,10 +299,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   }
 }
 
-template <bool OUT>
+template <bool OUT, bool FP4>
 cudaError_t run_w8(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& moa,
                    const CUtensorMap& mob, const W8Params& p, cudaStream_t stream) {
-  auto k = w8a8_gemm_kernel<OUT>;
+  auto k = w8a8_gemm_kernel<OUT, FP4>;
   const int smem = W8Smem::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -304,7 +313,10 @@ cudaError_t run_w8(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorM
 
 }  // namespace
 
-qr_status launch_w8a8_gemm(const GemmJob& j, cudaStream_t stream) {
+// The pair kernel on 8-bit integer codes (one byte per code) or on packed
+// e2m1 codes (two per byte), which TMA unpacks into the tensor core's
+// 16-byte-aligned 4-bit layout (8 bytes of 16 codes, then 8 bytes of gap).
+qr_status launch_pair_gemm8(const GemmJob& j, bool fp4, cudaStream_t stream) {
   if (j.M == 0 || j.N == 0) return QR_OK;
   const bool out = j.n_out > 0;
   W8Params p{};
@@ -323,13 +335,14 @@ qr_status launch_w8a8_gemm(const GemmJob& j, cudaStream_t stream) {
   p.status = device_status_word();
   if (p.status == nullptr) return QR_ERR_CUDA;
   CUtensorMap ma{}, mb{}, moa{}, mob{};
-  const uint64_t kb = static_cast<uint64_t>(j.Kp);        // one byte per code
-  if (p.kt > 0 &&
-      (!make_tensor_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.a_codes, kb, j.M, kb, kRow, 128,
-                           CU_TENSOR_MAP_SWIZZLE_128B) ||
-       !make_tensor_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, j.w_codes, kb, j.N, kb, kRow, kHalf8,
-                           CU_TENSOR_MAP_SWIZZLE_128B)))
-    return QR_ERR_CUDA;
+  if (p.kt > 0) {
+    const uint64_t kc = static_cast<uint64_t>(j.Kp);                  // codes per row
+    const uint64_t pitch = fp4 ? kc / 2 : kc;                          // bytes per row
+    const CUtensorMapDataType dt = fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    if (!make_tensor_map_2d(&ma, dt, j.a_codes, kc, j.M, pitch, kRow, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tensor_map_2d(&mb, dt, j.w_codes, kc, j.N, pitch, kRow, kHalf8, CU_TENSOR_MAP_SWIZZLE_128B))
+      return QR_ERR_CUDA;
+  }
   if (out) {
     const uint64_t no = static_cast<uint64_t>(j.n_out);
     if (!make_tensor_map_2d(&moa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, j.x_out, no, j.M, no * 2,
@@ -338,9 +351,20 @@ qr_status launch_w8a8_gemm(const GemmJob& j, cudaStream_t stream) {
                             kRow / 2, kHalf8, CU_TENSOR_MAP_SWIZZLE_128B))
       return QR_ERR_CUDA;
   }
-  const cudaError_t e = out ? run_w8<true>(ma, mb, moa, mob, p, stream)
-                            : run_w8<false>(ma, mb, moa, mob, p, stream);
+  cudaError_t e;
+  if (fp4)
+    e = out ? run_w8<true, true>(ma, mb, moa, mob, p, stream) : run_w8<false, true>(ma, mb, moa, mob, p, stream);
+  else
+    e = out ? run_w8<true, false>(ma, mb, moa, mob, p, stream) : run_w8<false, false>(ma, mb, moa, mob, p, stream);
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
+}
+
+qr_status launch_w8a8_gemm(const GemmJob& j, cudaStream_t stream) {
+  return launch_pair_gemm8(j, false, stream);
+}
+
+qr_status launch_fp4_gemm(const GemmJob& j, cudaStream_t stream) {
+  return launch_pair_gemm8(j, true, stream);
 }
 
 }  // namespace qr

@@ -156,6 +156,33 @@ def w8a8_linear(a_codes, a_scales, w_codes, w_scales, x_out=None, w_out=None,
     return y, acc
 
 
+def rotate_quant_fp4(x, rot: Rotation, outlier_idx=None, debug: bool = False):
+    """Online activation path with e2m1 codes (two per byte, element 2j in
+    the low nibble): (codes uint8 [rows x K_p/2], scales, x_out, x_rot or None)."""
+    return _rows(L.qr_rotate_quant_fp4, rot, x, outlier_idx, debug)
+
+
+def pack_weights_fp4(w, rot_w: Rotation, outlier_idx=None, debug: bool = False):
+    """Offline weight path with e2m1 codes: (codes, scales, w_out, w_rot or None)."""
+    return _rows(L.qr_pack_weights_fp4, rot_w, w, outlier_idx, debug)
+
+
+def fp4_linear(a_codes, a_scales, w_codes, w_scales, x_out=None, w_out=None,
+               out: Optional[torch.Tensor] = None, acc_debug: bool = False):
+    """The FP4 linear: Y = fp16(acc * sa * sw + x_out w_out^T) for packed
+    e2m1 codes; returns (Y, acc float32 or None)."""
+    M, kp2 = a_codes.shape
+    N = w_codes.shape[0]
+    n_out = 0 if x_out is None else x_out.shape[1]
+    dev = a_codes.device
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=dev)
+    acc = torch.empty((M, N), dtype=torch.float32, device=dev) if acc_debug else None
+    L.qr_fp4_linear(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(),
+                    w_scales.data_ptr(), M, N, 2 * kp2, _ptr(x_out), _ptr(w_out), n_out,
+                    y.data_ptr(), y.stride(0), _ptr(acc), _stream())
+    return y, acc
+
+
 def weight_code_sums(w_codes: torch.Tensor) -> torch.Tensor:
     """Per weight row, the sum of its packed codes (int32 [N])."""
     N, kp2 = w_codes.shape
@@ -246,24 +273,31 @@ def select_outliers(x_calib: torch.Tensor, k: int) -> torch.Tensor:
 
 
 class QuantizedLinear:
-    """A linear layer held as rotated 4-bit (or, with bits=8, 8-bit) weights;
-    forward() is the online path."""
+    """A linear layer held as rotated 4-bit (or, with bits=8, 8-bit; with
+    fp4=True, e2m1) weights; forward() is the online path."""
 
     def __init__(self, weight: torch.Tensor, rot: Rotation, outlier_idx=None,
-                 asym_activations: bool = False, bits: int = 4):
+                 asym_activations: bool = False, bits: int = 4, fp4: bool = False):
         if bits not in (4, 8) or (bits == 8 and asym_activations):
             raise ValueError("bits must be 4, or 8 with symmetric activations")
+        if fp4 and (bits != 4 or asym_activations):
+            raise ValueError("fp4 codes are 4-bit with symmetric activations")
         self.rot = rot
         self.rot_w = weight_rotation(rot)
         self.outlier_idx = outlier_idx
         self.asym = asym_activations
         self.bits = bits
-        pack = pack_weights8 if bits == 8 else pack_weights
+        self.fp4 = fp4
+        pack = pack_weights_fp4 if fp4 else pack_weights8 if bits == 8 else pack_weights
         self.w_codes, self.w_scales, self.w_out, _ = pack(weight, self.rot_w, outlier_idx)
         self.w_sums = weight_code_sums(self.w_codes) if asym_activations else None
         self.out_features, self.in_features = weight.shape
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
+        if self.fp4:
+            codes, scales, x_out, _ = rotate_quant_fp4(x, self.rot, self.outlier_idx)
+            y, _ = fp4_linear(codes, scales, self.w_codes, self.w_scales, x_out, self.w_out)
+            return y
         if self.bits == 8:
             codes, scales, x_out, _ = rotate_quant8(x, self.rot, self.outlier_idx)
             y, _ = w8a8_linear(codes, scales, self.w_codes, self.w_scales, x_out, self.w_out)

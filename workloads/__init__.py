@@ -49,6 +49,7 @@ class Spec:
     n_keep_fp16: int = 0        # QUIK fp16 outlier columns selected by calibration
     calib_tokens: int = 0
     bits: int = 4               # code width of the layer (8: QUIK's INT8 layers)
+    fp4: bool = False           # 4-bit codes are e2m1 values (FP4) instead of integers
     description: str = ""
 
 
@@ -91,6 +92,13 @@ SPECS = {
                     "256 outlier columns x50 kept fp16 (chosen on a 512-token "
                     "calibration batch), the other 7936 columns rotated by "
                     "4096-point Hadamard blocks"),
+    "qkv_prefill_fp4_4096": Spec(
+        "qkv_prefill_fp4_4096", M=2048, K=4096, N=12288, seed=20261204,
+        rotation=HADAMARD, block=4096, n_outlier_channels=16,
+        outlier_scale=30.0, massive_token_scale=300.0, fp4=True,
+        description="the fused QKV prefill layer (same inputs as qkv_prefill_4096) "
+                    "with e2m1 (FP4) codes for activations and weights, per-token "
+                    "and per-channel fp32 scales, on the fp4 tensor-core operands"),
     "down_proj_int8_11008": Spec(
         "down_proj_int8_11008", M=2048, K=11008, N=4096, seed=20261209,
         rotation=GSR, block=128, n_outlier_channels=32, outlier_scale=40.0,
