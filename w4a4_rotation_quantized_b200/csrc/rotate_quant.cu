@@ -982,6 +982,12 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
   // Layout-B loads: value m sits at b_pos[(m >> 2) & 1] + 8 m.
   const int b_pos0 = b * G::kStride + tl, b_pos1 = b * G::kStride + (tl ^ 4);
   const bool plain = p.n_out == 0 && p.signs == nullptr;   // no gather, no sign flips
+  // GSR: the lanes whose sequency words take Hadamard outputs j ^ 1 (the
+  // parity of t, see gsr_j_static) get them in place: y[j ^ 1] is the
+  // transform of x with odd-j inputs negated, which the first layout-B
+  // butterfly absorbs as (x0 + s x1, x0 - s x1) with s = -1.
+  const int swap_par = p.gsr ? ((tl ^ (tl >> 1) ^ (tl >> 2)) & 1) : 0;
+  const float bsign = swap_par ? -1.0f : 1.0f;
   int par = 0;
   for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
     const int i = static_cast<int>(row - row0);
@@ -1046,7 +1052,13 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
 #pragma unroll
         for (int m = 0; m < VB; ++m) v[c][m] = buf[(((m >> 2) & 1) ? b_pos1 : b_pos0) + 8 * m];
         __syncwarp();                             // before the next chunk's stores
-        wht_stages<0, LB - 3>(v[c]);
+#pragma unroll
+        for (int m = 0; m < VB; m += 2) {
+          const float x0 = v[c][m], x1 = v[c][m + 1];
+          v[c][m] = fmaf(x1, bsign, x0);
+          v[c][m + 1] = fmaf(x1, -bsign, x0);
+        }
+        wht_stages<1, LB - 3>(v[c]);
         if constexpr (MODE == 1) {
           if (ch * 4 + b < nb)
 #pragma unroll
@@ -1110,7 +1122,7 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
       if (p.rot_debug != nullptr && ok) {
 #pragma unroll
         for (int m = 0; m < VB; ++m) {
-          int n = tl + 8 * m;
+          int n = tl + 8 * (m ^ swap_par);
           if (p.gsr) n = gray_inverse(static_cast<int>(__brev(static_cast<unsigned>(n)) >> (32 - LB)));
           p.rot_debug[row * p.Kp + (bg << LB) + n] = v[c][m] * p.inv_sqrt_block;
         }
@@ -1126,7 +1138,7 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
 #pragma unroll
           for (int tt = 0; tt < 8; ++tt) {
             const int js = gsr_j_static<LB>(tt, f);
-            w8[tt] = p3 ? v[c][js ^ 1] : v[c][js];
+            w8[tt] = v[c][js];                   // (odd-parity lanes hold j ^ 1 here)
           }
           if (ok) {
             if constexpr (MODE == 2)
@@ -1181,6 +1193,8 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
 //   layout B: thread t holds elements (t & 7) + 8 j + 512 (t >> 3) (j < 64),
 //             bits 3-8 inside the thread.
 // One pass through the group's fp32 row buffer moves the row from A to B.
+// Compiled for 608 threads (96 registers each): nine row groups per SM,
+// which hides more latency than eight at 128 registers.
 // In the buffer, element e of a block sits at (e + 8 (e >> 9)) with bit 2
 // flipped where bit 5 of e is set: the padding spreads a layout-B read over
 // all banks, the flip makes the layout-A 16-byte stores conflict-free.
@@ -1190,7 +1204,7 @@ constexpr int kH12Floats = 4096 + 64;
 // MODE: 0 = symmetric, 1 = asymmetric (4-bit codes), 2 = e2m1 (FP4);
 // natural order.
 template <int MODE, bool CLIP>
-__global__ void __launch_bounds__(512, 1) wht_h12_kernel(const WhtParams p) {
+__global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
   grid_dep_wait();
   grid_dep_launch();
   extern __shared__ __align__(128) uint8_t smem[];
@@ -1924,12 +1938,12 @@ bool launch_wht_h12(const RowJob& job, WhtParams p, int lb, cudaStream_t stream,
   if (p.status == nullptr) return false;
   const int nblk = job.Kp / 4096;
   const int nt = 64 * nblk;
-  if (nt + 32 > 512) return false;
+  if (nt + 32 > 608) return false;
   const int64_t blocks = std::min<int64_t>(job.rows, sm_count());
   const int64_t per_block = (job.rows + blocks - 1) / blocks;
   const int row_bytes = static_cast<int>(job.K * 2);
   const size_t sign_bytes = p.signs != nullptr ? static_cast<size_t>(job.Kp / 8) : 0;
-  int groups = static_cast<int>(std::min<int64_t>(std::min(8, (512 - 32) / nt), per_block));
+  int groups = static_cast<int>(std::min<int64_t>(std::min(9, (608 - 32) / nt), per_block));
   for (; groups >= 1; --groups) {
     p.off_red = 0;
     size_t off = sizeof(float) * 64 * groups;
