@@ -268,16 +268,16 @@ __device__ __forceinline__ int swz(int e) {
 struct RowQ { float r, c, lo, hi; };
 
 __device__ __forceinline__ RowQ sym_row_q(float am, float clip, float inv_sqrt, float* scale_out) {
-  if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 7.0f;
-  return RowQ{(am > 0.0f) ? 7.0f / (clip * am) : 0.0f, kRoundMagic, kRoundMagic - 7.0f,
+  if (scale_out != nullptr) *scale_out = __fdividef(clip * (am * inv_sqrt), 7.0f);
+  return RowQ{(am > 0.0f) ? __fdividef(7.0f, clip * am) : 0.0f, kRoundMagic, kRoundMagic - 7.0f,
               kRoundMagic + 7.0f};
 }
 
 // 8-bit symmetric codes (QUIK's INT8 layers): s = alpha * absmax / 127,
 // codes clamped to +-127.
 __device__ __forceinline__ RowQ sym_row_q8(float am, float clip, float inv_sqrt, float* scale_out) {
-  if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 127.0f;
-  return RowQ{(am > 0.0f) ? 127.0f / (clip * am) : 0.0f, kRoundMagic, kRoundMagic - 127.0f,
+  if (scale_out != nullptr) *scale_out = __fdividef(clip * (am * inv_sqrt), 127.0f);
+  return RowQ{(am > 0.0f) ? __fdividef(127.0f, clip * am) : 0.0f, kRoundMagic, kRoundMagic - 127.0f,
               kRoundMagic + 127.0f};
 }
 
@@ -782,8 +782,8 @@ __global__ void __launch_bounds__(512) wht_small_kernel(const WhtParams p) {
 // are the nearest e2m1 values of x / s (ties to the even mantissa,
 // saturating at +-6), the tensor core's own conversion.
 __device__ __forceinline__ RowQ sym_row_qf4(float am, float clip, float inv_sqrt, float* scale_out) {
-  if (scale_out != nullptr) *scale_out = (clip * (am * inv_sqrt)) / 6.0f;
-  return RowQ{(am > 0.0f) ? 6.0f / (clip * am) : 0.0f, 0.0f, 0.0f, 0.0f};
+  if (scale_out != nullptr) *scale_out = __fdividef(clip * (am * inv_sqrt), 6.0f);
+  return RowQ{(am > 0.0f) ? __fdividef(6.0f, clip * am) : 0.0f, 0.0f, 0.0f, 0.0f};
 }
 
 // Two e2m1 codes of (lo * r, hi * r) in one byte, lo in the low nibble.
@@ -989,11 +989,12 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
   const int swap_par = p.gsr ? ((tl ^ (tl >> 1) ^ (tl >> 2)) & 1) : 0;
   const float bsign = swap_par ? -1.0f : 1.0f;
   int par = 0;
+  // this group's rows are rg, rg + groups, ...: slot and parity advance by
+  // `groups` slots per row (groups <= ring_slots, so one wrap at most)
+  int slot = rg;
+  uint32_t rph = 0;
   for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
-    const int i = static_cast<int>(row - row0);
-    const int slot = i % p.ring_slots;
-    if (!mbar_wait_bounded(&ring_full[slot], (i / p.ring_slots) & 1, abort_flag, p.status,
-                           kDevTimeoutWiden))
+    if (!mbar_wait_bounded(&ring_full[slot], rph, abort_flag, p.status, kDevTimeoutWiden))
       break;
     const __half* rrow =
         reinterpret_cast<const __half*>(smem + p.off_ring + static_cast<size_t>(slot) * p.ring_row_bytes);
@@ -1183,6 +1184,8 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
         }
       }
     }
+    slot += groups;
+    if (slot >= p.ring_slots) { slot -= p.ring_slots; rph ^= 1; }
   }
 }
 
@@ -1265,11 +1268,12 @@ __global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
   const int eA = blk * 4096 + 8 * tb;           // row element of layout-A group h = 0
   const bool full_plain = p.K == p.Kp && p.signs == nullptr;   // no zero tail, no sign flips
   int par = 0;
+  // this group's rows are rg, rg + groups, ...: slot and parity advance by
+  // `groups` slots per row (groups <= ring_slots, so one wrap at most)
+  int slot = rg;
+  uint32_t rph = 0;
   for (int64_t row = row0 + rg; row < row1; row += groups, par ^= 1) {
-    const int i = static_cast<int>(row - row0);
-    const int slot = i % p.ring_slots;
-    if (!mbar_wait_bounded(&ring_full[slot], (i / p.ring_slots) & 1, abort_flag, p.status,
-                           kDevTimeoutWiden))
+    if (!mbar_wait_bounded(&ring_full[slot], rph, abort_flag, p.status, kDevTimeoutWiden))
       break;
     const __half* rrow =
         reinterpret_cast<const __half*>(smem + p.off_ring + static_cast<size_t>(slot) * p.ring_row_bytes);
@@ -1392,6 +1396,8 @@ __global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
       *reinterpret_cast<uint32_t*>(crow + ((eB + 64 * wb + 8 * l) >> 1)) = nw2;
     }
     row_barrier(rg, nt);                          // the row buffer is reused by the next row
+    slot += groups;
+    if (slot >= p.ring_slots) { slot -= p.ring_slots; rph ^= 1; }
   }
 }
 
