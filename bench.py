@@ -93,12 +93,12 @@ def rotate_kernel_name(spec, M: int, sms: int) -> str:
     """The rotate kernel the library routes these (aligned) rows to."""
     if spec.rotation == "kron":
         return "kron_tc_kernel"
-    if M <= sms:
-        return "wht_few_rows_kernel"
     block = spec.block or spec.K
+    if M <= sms and not spec.fp4:
+        return "wht_few_rows_kernel"
     if block in (64, 128, 256):
         return "wht_blk_kernel"
-    if block == 4096 and spec.bits == 4 and spec.n_keep_fp16 == 0:
+    if block == 4096 and spec.bits == 4:
         return "wht_h12_kernel"
     return "wht_ab_kernel"
 

@@ -234,8 +234,8 @@ QR_API qr_status qr_w8a8_linear(const int8_t* a_codes, const float* a_scales,
  *
  * qr_rotate_quant_fp4 / qr_pack_weights_fp4: arguments and errors as
  * qr_rotate_quant / qr_pack_weights.  Supported rotations: HADAMARD or
- * GSR with blocks of 64, 128 or 256 (outlier columns allowed), and
- * 4096-point blocks without outliers; others, and KRON, are UNSUPPORTED.
+ * GSR with blocks of 64, 128, 256 or 4096 (outlier columns allowed);
+ * others, and KRON, are UNSUPPORTED.
  * qr_fp4_linear: as qr_w4a4_linear for packed e2m1 codes
  * (K_p % 128 == 0, K_p <= 65536, code pointers 32-byte aligned):
  *   acc[m, n] = sum_k e2m1(qa[m, k]) e2m1(qw[n, k])   (fp32; every product

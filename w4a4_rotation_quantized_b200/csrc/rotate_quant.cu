@@ -141,22 +141,32 @@ __device__ __forceinline__ int gray_inverse(int g) {
 }
 
 // Builds, in shared memory, kept[e] = the source column of rotated column e
-// (0xFFFF = none), from the strictly ascending outlier index list.  Malformed
-// lists never write outside [0, Kr).
+// (0xFFFF = none), from the strictly ascending outlier index list.  Each
+// thread takes a contiguous range of source columns: one binary search for
+// the outliers before it, then a walk that skips the outliers it meets.
+// Malformed lists never write outside [0, Kr).
 __device__ void build_kept_table(const int32_t* __restrict__ outlier_idx, int n_out, int K,
                                  int Kr, uint16_t* kept, int32_t* sidx) {
   for (int i = threadIdx.x; i < n_out; i += blockDim.x) sidx[i] = outlier_idx[i];
   for (int e = threadIdx.x; e < Kr; e += blockDim.x) kept[e] = 0xFFFFu;
   __syncthreads();
-  for (int c = threadIdx.x; c < K; c += blockDim.x) {
-    int lo = 0, hi = n_out;            // lo = number of outliers < c
+  const int per = (K + blockDim.x - 1) / blockDim.x;
+  const int c0 = threadIdx.x * per;
+  const int c1 = c0 + per < K ? c0 + per : K;
+  if (c0 < c1) {
+    int lo = 0, hi = n_out;            // lo = number of outliers < c0
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (sidx[mid] < c) lo = mid + 1; else hi = mid;
+      if (sidx[mid] < c0) lo = mid + 1; else hi = mid;
     }
-    const bool is_out = lo < n_out && sidx[lo] == c;
-    const int pos = c - lo;
-    if (!is_out && pos >= 0 && pos < Kr) kept[pos] = static_cast<uint16_t>(c);
+    for (int c = c0; c < c1; ++c) {
+      if (lo < n_out && sidx[lo] == c) {
+        ++lo;
+        continue;
+      }
+      const int pos = c - lo;
+      if (pos >= 0 && pos < Kr) kept[pos] = static_cast<uint16_t>(c);
+    }
   }
   __syncthreads();
 }
@@ -1196,7 +1206,8 @@ __global__ void __launch_bounds__(BlkBounds<LB, CPW>::value, 1) wht_blk_kernel(c
 //   layout B: thread t holds elements (t & 7) + 8 j + 512 (t >> 3) (j < 64),
 //             bits 3-8 inside the thread.
 // One pass through the group's fp32 row buffer moves the row from A to B.
-// Compiled for 608 threads (96 registers each): nine row groups per SM,
+// With QUIK outliers the kept columns are gathered from the ring copy of the
+// row through the kept-column table.  Compiled for 608 threads (96 registers each): nine row groups per SM,
 // which hides more latency than eight at 128 registers.
 // In the buffer, element e of a block sits at (e + 8 (e >> 9)) with bit 2
 // flipped where bit 5 of e is set: the padding spreads a layout-B read over
@@ -1230,6 +1241,10 @@ __global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
   }
   uint8_t* sbits = smem + p.off_signs;
   if (p.signs != nullptr) build_sign_bits(p.signs, p.Kp, sbits);
+  uint16_t* kept = reinterpret_cast<uint16_t*>(smem + p.off_kept);
+  const int32_t* sidx = reinterpret_cast<const int32_t*>(smem + p.off_idx);
+  if (p.n_out > 0)   // (synchronizes the CTA)
+    build_kept_table(p.outlier_idx, p.n_out, p.K, p.Kr, kept, reinterpret_cast<int32_t*>(smem + p.off_idx));
   __syncthreads();
 
   if (rg == groups) {
@@ -1266,7 +1281,8 @@ __global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
   // layout-B loads: value j at (bit 2 of j ? b_pos1 : b_pos0) + 8 j
   const int b_pos0 = (tb & 7) + 520 * (tb >> 3), b_pos1 = ((tb & 7) ^ 4) + 520 * (tb >> 3);
   const int eA = blk * 4096 + 8 * tb;           // row element of layout-A group h = 0
-  const bool full_plain = p.K == p.Kp && p.signs == nullptr;   // no zero tail, no sign flips
+  // no outlier gather, no zero tail, no sign flips
+  const bool full_plain = p.n_out == 0 && p.K == p.Kp && p.signs == nullptr;
   int par = 0;
   // this group's rows are rg, rg + groups, ...: slot and parity advance by
   // `groups` slots per row (groups <= ring_slots, so one wrap at most)
@@ -1277,6 +1293,11 @@ __global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
       break;
     const __half* rrow =
         reinterpret_cast<const __half*>(smem + p.off_ring + static_cast<size_t>(slot) * p.ring_row_bytes);
+    if (p.n_out > 0 && p.out16 != nullptr)         // QUIK outlier columns, copied through
+      for (int j = t; j < p.n_out; j += nt) {
+        const int c = sidx[j];
+        p.out16[row * p.n_out + j] = (c >= 0 && c < p.K) ? rrow[c] : __float2half(0.0f);
+      }
 
     // ---- phase A: bits 0-2 and 9-11
     float v[64];
@@ -1286,6 +1307,18 @@ __global__ void __launch_bounds__(608, 1) wht_h12_kernel(const WhtParams p) {
         const uint4 u = *reinterpret_cast<const uint4*>(rrow + eA + 512 * h);
         bfly_h2(u.x, v[8 * h], v[8 * h + 1]); bfly_h2(u.y, v[8 * h + 2], v[8 * h + 3]);
         bfly_h2(u.z, v[8 * h + 4], v[8 * h + 5]); bfly_h2(u.w, v[8 * h + 6], v[8 * h + 7]);
+      }
+    } else if (p.n_out > 0) {
+      // kept columns gathered from the ring copy of the row (zero beyond K_r)
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const int e = eA + 512 * h;
+        float x[8];
+        blk_load8(p, rrow, kept, e, x);
+        if (p.signs != nullptr) apply_signs8(sbits, e, x);
+        wht_stages<0, 1>(x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[8 * h + q] = x[q];
       }
     } else {
 #pragma unroll
@@ -1933,11 +1966,11 @@ bool launch_wht_blk(const RowJob& job, WhtParams p, int lb, cudaStream_t stream,
   return false;
 }
 
-// Rows of 4096-point blocks through wht_h12_kernel (4-bit codes, no outlier
-// gather, aligned rows).  Returns false (nothing launched) when the shape
-// does not fit it.
+// Rows of 4096-point blocks through wht_h12_kernel (4-bit integer or e2m1
+// codes, aligned rows, any row count).  Returns false (nothing launched)
+// when the shape does not fit it.
 bool launch_wht_h12(const RowJob& job, WhtParams p, int lb, cudaStream_t stream, qr_status* st) {
-  if (lb != 12 || (job.bits != 4 && job.bits != kFp4Codes) || job.n_out != 0 || job.K <= 0 || job.rows <= 0 || job.K % 8 != 0 ||
+  if (lb != 12 || (job.bits != 4 && job.bits != kFp4Codes) || job.K <= 0 || job.rows <= 0 || job.K % 8 != 0 ||
       job.ld % 8 != 0 || reinterpret_cast<uintptr_t>(job.src) % 16 != 0 || job.Kp % 4096 != 0)
     return false;
   p.status = device_status_word();
@@ -1955,6 +1988,10 @@ bool launch_wht_h12(const RowJob& job, WhtParams p, int lb, cudaStream_t stream,
     size_t off = sizeof(float) * 64 * groups;
     p.off_buf = static_cast<int32_t>(align_up(off, 16));
     off = p.off_buf + sizeof(float) * static_cast<size_t>(kH12Floats) * nblk * groups;
+    p.off_kept = static_cast<int32_t>(align_up(off, 16));
+    if (job.n_out > 0) off = p.off_kept + sizeof(uint16_t) * align_up(job.Kr, 8);
+    p.off_idx = static_cast<int32_t>(align_up(off, 16));
+    if (job.n_out > 0) off = p.off_idx + sizeof(int32_t) * job.n_out;
     p.off_signs = static_cast<int32_t>(align_up(off, 16));
     off = p.off_signs + sign_bytes;
     p.off_ring = static_cast<int32_t>(align_up(off, 128));
@@ -2437,6 +2474,9 @@ qr_status launch_rotate_quant(const RowJob& job, cudaStream_t stream) {
                                                                    : launch_wht_rows(job, stream);
   if (job.rot->kind == QR_ROT_KRON)
     return kron_tc_supported(job) ? launch_kron_tc(job, stream) : launch_kron_rows(job, stream);
+  // (The row-group kernels at one row per CTA lose to the one-row-per-
+  // cluster kernel on decode-sized jobs: 28 us against 8 us for 64 QUIK
+  // rows, mostly the per-CTA outlier-table setup and the load latency.)
   return few_rows(job) ? launch_wht_few_rows(job, stream) : launch_wht_rows(job, stream);
 }
 
