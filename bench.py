@@ -51,10 +51,11 @@ DATASHEET_INT8_TOPS = 4500.0
 KERNEL_SOURCES = {
     "w4a4_gemm_pair_kernel": ["w4a4_gemm_pair.cu", "qr_device.cuh"],
     "w4a4_gemm_decode_kernel": ["w4a4_gemm_decode.cu", "qr_device.cuh"],
-    "wht_ab_kernel": ["rotate_quant.cu", "qr_device.cuh"],
-    "wht_blk_kernel": ["rotate_quant.cu", "qr_device.cuh"],
-    "wht_h12_kernel": ["rotate_quant.cu", "qr_device.cuh"],
-    "wht_few_rows_kernel": ["rotate_quant.cu", "qr_device.cuh"],
+    "w4a4_gemm_decode_kernel_fused": ["w4a4_gemm_decode.cu", "qr_device.cuh", "row_quant.cuh"],
+    "wht_ab_kernel": ["rotate_quant.cu", "qr_device.cuh", "row_quant.cuh"],
+    "wht_blk_kernel": ["rotate_quant.cu", "qr_device.cuh", "row_quant.cuh"],
+    "wht_h12_kernel": ["rotate_quant.cu", "qr_device.cuh", "row_quant.cuh"],
+    "wht_few_rows_kernel": ["rotate_quant.cu", "qr_device.cuh", "row_quant.cuh"],
     "kron_tc_kernel": ["kron_tc.cu", "qr_device.cuh"],
     "w8a8_gemm_kernel": ["w8a8_gemm.cu", "qr_device.cuh"],
 }
@@ -285,16 +286,19 @@ def run_ours(args, rank, world, local_rank):
     if (bits == 8 or fp4) and asym:
         raise SystemExit("the 8-bit and FP4 layers take symmetric activations")
     gemm_ops, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp, asym)
+    # --fused: decode batches run as one kernel (rotate + quantize + GEMM)
+    fused = M <= DECODE_MAX_TOKENS and bits == 4 and not fp4 and s.rotation != "kron" and \
+        args.fused
 
     # input sets: enough copies that one pass over them exceeds L2 twice
     x0 = torch.from_numpy(wl.X).cuda()
     w0 = torch.from_numpy(wl.W).cuda()
     t_pack0 = torch.cuda.Event(enable_timing=True)
     t_pack1 = torch.cuda.Event(enable_timing=True)
-    Q.QuantizedLinear(w0, rot, idx, asym, bits, fp4)      # warm-up (module load, attributes)
+    Q.QuantizedLinear(w0, rot, idx, asym, bits, fp4, fused)      # warm-up (module load, attributes)
     torch.cuda.synchronize()
     t_pack0.record()
-    layer0 = Q.QuantizedLinear(w0, rot, idx, asym, bits, fp4)
+    layer0 = Q.QuantizedLinear(w0, rot, idx, asym, bits, fp4, fused)
     t_pack1.record()
     torch.cuda.synchronize()
     pack_ms = t_pack0.elapsed_time(t_pack1)
@@ -336,8 +340,17 @@ def run_ours(args, rank, world, local_rank):
         else:
             Q.w4a4_linear(codes, scales, wc, wsc, x_out, wo, out=y)
 
+    sync = torch.zeros(2, dtype=torch.int32, device="cuda")
+
+    def fused_step(x, wset):
+        wc, wsc, wo, wsum = wset
+        Q.w4a4_linear_fused(x, rot, idx, wc, wsc, wo, wsum, asym, sync, out=y)
+
     def step(i):
-        linear(rq(xs[i % nsets]), wsets[i % nsets])
+        if fused:
+            fused_step(xs[i % nsets], wsets[i % nsets])
+        else:
+            linear(rq(xs[i % nsets]), wsets[i % nsets])
 
     for i in range(args.warmup):
         step(i)
@@ -348,14 +361,21 @@ def run_ours(args, rank, world, local_rank):
     # over the sets), another runs the G GEMMs on its outputs.  The timed
     # region replays them in turn; events between replays give each kernel's
     # device time.  A last pair of graphs takes the K mod G remaining steps.
+    # (fused: the rotate graph is empty and the second graph runs the fused
+    # steps, so its events time the one kernel)
     def rot_pass(n):
-        return [rq(xs[i]) for i in range(n)]
+        return [] if fused else [rq(xs[i]) for i in range(n)]
 
     def gemm_pass(outs, n):
         for i in range(n):
-            linear(outs[i], wsets[i])
+            if fused:
+                fused_step(xs[i], wsets[i])
+            else:
+                linear(outs[i], wsets[i])
 
     def capture(fn):
+        if fused and fn is not None and getattr(fn, "rot_side", False):
+            return None, fn()                         # nothing to rotate apart
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             r = fn()
@@ -364,16 +384,22 @@ def run_ours(args, rank, world, local_rank):
     G = nsets
     full, rem = divmod(args.steps, G)
     passes = []
+    def rot_fn(n):
+        f = lambda: rot_pass(n)
+        f.rot_side = True
+        return f
+
     if full:
-        g_rot, outs = capture(lambda: rot_pass(G))
+        g_rot, outs = capture(rot_fn(G))
         g_gemm, _ = capture(lambda: gemm_pass(outs, G))
         passes += [(g_rot, g_gemm)] * full
     if rem:
-        g_rot_r, outs_r = capture(lambda: rot_pass(rem))
+        g_rot_r, outs_r = capture(rot_fn(rem))
         g_gemm_r, _ = capture(lambda: gemm_pass(outs_r, rem))
         passes.append((g_rot_r, g_gemm_r))
     for gr, gg in set(passes):                        # upload + one untimed replay
-        gr.replay()
+        if gr is not None:
+            gr.replay()
         gg.replay()
     torch.cuda.synchronize()
 
@@ -391,7 +417,8 @@ def run_ours(args, rank, world, local_rank):
     start.record(stream)
     for (gr, gg), ev in zip(passes, evs):
         ev[0].record(stream)
-        gr.replay()
+        if gr is not None:
+            gr.replay()
         ev[1].record(stream)
         gg.replay()
         ev[2].record(stream)
@@ -432,13 +459,20 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = aggregate_max(e0.elapsed_time(e1), world) / e2e_steps
 
     peaks, peak_src = load_peaks()
+    if fused:
+        # one kernel: X read, codes, scales (zero points) and the outlier copy
+        # written (the GEMM phase reads them back while they sit in L2), the
+        # weight side read, Y written
+        k_int = s.K - s.n_keep_fp16
+        reread = M * k_int * 0.5 + M * 4 + M * s.n_keep_fp16 * 2 + (M * 4 if asym else 0)
+        gemm_bytes = rq_bytes + gemm_bytes - reread
     ms_per_step = elapsed_ms / args.steps
     value = world * gemm_ops / (ms_per_step * 1e-3) / 1e12
     gemm_avg = gemm_total / args.steps
     rq_avg = rq_total / args.steps
     gemm_tops = gemm_ops / (gemm_avg * 1e-3) / 1e12
     gemm_gbs = gemm_bytes / (gemm_avg * 1e-3) / 1e9
-    rq_gbs = rq_bytes / (rq_avg * 1e-3) / 1e9
+    rq_gbs = rq_bytes / (rq_avg * 1e-3) / 1e9 if rq_avg > 0 else 0.0
     int8_sust = peaks["bf16_tflops_sustained"] * INT8_PER_BF16
     int8_burst = peaks["bf16_tflops"] * INT8_PER_BF16
     timed_s = elapsed_ms * 1e-3
@@ -446,6 +480,7 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.summary(t0, t1)
     sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
     gemm_name = gemm_kernel_name(M, 8 if fp4 else bits)    # e2m1 runs the pair kernel of the 8-bit codes
+    traffic_name = "w4a4_gemm_decode_kernel_fused" if fused else gemm_name
     # the GEMM's bound: tensor cores above the ridge point, HBM below it.
     # The denominator is the burst figure (the timed region is well under a
     # second of GPU time); the sustained and datasheet fractions ride along.
@@ -464,7 +499,9 @@ def run_ours(args, rank, world, local_rank):
                     "peak_source": f"{peak_src} HBM copy bandwidth"}
     roofline.update({"ops_per_launch": gemm_ops, "ms_per_launch": round(gemm_avg, 5),
                      "algorithmic_bytes_per_launch": gemm_bytes,
-                     "traffic": dram_traffic(gemm_name, s.name) if M == s.M else None})
+                     "traffic": dram_traffic(traffic_name, s.name) if M == s.M else None})
+    if fused:
+        roofline["fused_rotate_quant"] = True
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -483,6 +520,8 @@ def run_ours(args, rank, world, local_rank):
                       "fp16 in/out"),
         "data": "synthetic",
         "config": {"workload": s.name, "M": M, "K": s.K, "N": s.N, "K_p": kp,
+                   "step": ("one fused kernel (rotate + quantize, grid barrier, GEMM)" if fused
+                            else "rotate + quantize kernel, then the GEMM kernel"),
                    "rotation": (("random-sign " if signs is not None else "") +
                                 f"{s.rotation}-{s.block}") if s.rotation != "kron"
                    else f"kron-{s.n1}x{s.n2}", "n_out": s.n_keep_fp16,
@@ -494,17 +533,21 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 1e6:.0f} MB "
                          f"> 126 MB L2)"},
         "roofline": roofline,
-        "rotate_quant": dict(rotate_quant_roofline(wl, M, rq_bytes, rq_avg, peaks, peak_src,
-                                                   rotate_kernel_name(s, M, sms)),
-                             traffic=dram_traffic(rotate_kernel_name(s, M, sms), s.name)
-                             if M == s.M else None),
+        "rotate_quant": ({"fused_into": gemm_name, "bytes_per_launch": rq_bytes,
+                          "note": "rotate + quantize run inside the decode kernel, before its "
+                                  "grid barrier; their time is part of roofline.ms_per_launch"}
+                         if fused else
+                         dict(rotate_quant_roofline(wl, M, rq_bytes, rq_avg, peaks, peak_src,
+                                                    rotate_kernel_name(s, M, sms)),
+                              traffic=dram_traffic(rotate_kernel_name(s, M, sms), s.name)
+                              if M == s.M else None)),
         "gemm_hbm_bytes_per_launch": gemm_bytes,
         "offline_weight_pack_ms": round(pack_ms, 3),
         "e2e": {"value": round(world * gemm_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 2), "steps": e2e_steps,
                 "api": "GraphedLinear"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 if fused else 2) * args.steps,
         "clocks": clocks,
     }
     return result
@@ -840,6 +883,9 @@ def main(argv=None):
                     help="weight rows in the reference arm's per-step sample (capped at N)")
     ap.add_argument("--random-signs", action="store_true",
                     help="randomized Hadamard: a seeded random-sign diagonal before the blocks")
+    ap.add_argument("--fused", action="store_true",
+                    help="decode batches (<= 64 tokens): time the fused decode kernel (rotate + "
+                         "quantize + GEMM in one launch) instead of the two launches")
     ap.add_argument("--asym-activations", action="store_true",
                     help="QUIK's asymmetric per-token activation quantizer (zero point per token)")
     args = ap.parse_args(argv)

@@ -112,8 +112,9 @@ typedef struct {
 } qr_rotation;
 
 /* ABI version of this header (bumped on any change to the entry points;
- * 3 added the 8-bit calls and qr_check_wait_timeout, 4 the FP4 calls). */
-#define QR_ABI_VERSION 4
+ * 3 added the 8-bit calls and qr_check_wait_timeout, 4 the FP4 calls, 5
+ * qr_w4a4_linear_fused). */
+#define QR_ABI_VERSION 5
 QR_API int32_t qr_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -190,6 +191,43 @@ QR_API qr_status qr_w4a4_linear(const uint8_t* a_codes, const float* a_scales,
                          const uint16_t* x_out, const uint16_t* w_out, int32_t n_out,
                          uint16_t* Y, int64_t ldy, int32_t* acc_debug,
                          qr_stream stream);
+
+/* The decode step in one kernel (FlatQuant "模型架构": the online transform
+ * and the quantization fused into the kernel that consumes them; QUIK
+ * "性能分析": the separate quantization and dequantization passes are why
+ * measured speedups trail the ideal).  Computes exactly what
+ * qr_rotate_quant (or qr_rotate_quant_asym when a_zeros != NULL) followed by
+ * qr_w4a4_linear (or qr_w4a4_linear_asym) computes, with the same codes,
+ * scales and outlier copy and the same Y bit for bit, in one launch: the
+ * kernel first rotates and quantizes the M token rows, writes a_codes,
+ * a_scales (a_zeros) and x_out, meets all of its CTAs at a grid-wide
+ * barrier, then runs the decode GEMM on them.
+ *  rot, X, M, K, ldx, outlier_idx, n_out: as qr_rotate_quant, with
+ *            1 <= M <= 64 and a NONE, HADAMARD or GSR rotation
+ *  w_codes, w_scales, w_out, N: the packed weights, as qr_w4a4_linear;
+ *            w_sums [N] (qr_weight_code_sums) with a_zeros, else ignored
+ *  a_codes, a_scales, a_zeros, x_out: outputs, as qr_rotate_quant(_asym);
+ *            the GEMM phase reads them back
+ *  Y         fp16 [M x ldy], ldy >= N
+ *  sync      two uint32 words of device memory, 8-byte aligned, that the
+ *            caller sets to zero once before the first call; every call
+ *            that completes leaves the first word zero again (the second
+ *            counts calls).  Calls that share `sync` must not run at the
+ *            same time (one stream, or ordered streams).
+ * The CTAs of the launch must all be resident at once; when the device
+ * cannot hold them (or K_p does not fit the kernel's row buffer) the call
+ * returns UNSUPPORTED without launching, and the two-call path applies.
+ * A barrier wait that runs out records QR_DEV_TIMEOUT_GRID_SYNC in the
+ * device status word.
+ * Errors: INVALID_ARG, UNSUPPORTED (M > 64, KRON, sizes), ALIGNMENT (as the
+ * two calls; sync not 8-byte aligned), CUDA. */
+QR_API qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_t M,
+                                      int64_t K, int64_t ldx, const int32_t* outlier_idx,
+                                      int32_t n_out, const uint8_t* w_codes, const float* w_scales,
+                                      const int32_t* w_sums, const uint16_t* w_out, int64_t N,
+                                      uint8_t* a_codes, float* a_scales, int32_t* a_zeros,
+                                      uint16_t* x_out, uint16_t* Y, int64_t ldy, uint32_t* sync,
+                                      qr_stream stream);
 
 /* ----------------------------------------------------------------------
  * 8-bit layers ("QUIK：LLM上的一种4-bit推理方法", QUIK量化, results: the
@@ -351,6 +389,7 @@ QR_API qr_status qr_kv_quantize(const uint16_t* Q, const uint16_t* K, const uint
 #define QR_DEV_TIMEOUT_MMA       0x103   /* the MMA-issuing thread */
 #define QR_DEV_TIMEOUT_EPILOGUE  0x104   /* an epilogue role */
 #define QR_DEV_TIMEOUT_DRAIN     0x105   /* draining in-flight work on abort */
+#define QR_DEV_TIMEOUT_GRID_SYNC 0x106   /* qr_w4a4_linear_fused's grid-wide barrier */
 #define QR_DEV_TIMEOUT_SELFCHECK 0x1FF   /* qr_check_wait_timeout */
 
 /* Reads, and clears, the current device's status word that kernels set when

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.qr_abi_version() == 4
+    assert L.qr_abi_version() == 5
     for s in range(6):
         assert L.status_string(s) and L.status_string(s) != "unknown status"
     assert L.status_string(99) == "unknown status"
@@ -239,3 +239,23 @@ def test_fp4_entry_points_argument_errors(lib):
     assert lin4(a=FAKE + 16) == L.QR_ERR_ALIGNMENT
     assert lin4(w=FAKE + 16) == L.QR_ERR_ALIGNMENT
     assert lin4(M=0) == L.QR_OK
+
+
+def test_fused_decode_argument_errors(lib):
+    # the one-kernel decode step validates both halves' arguments, takes at
+    # most 64 tokens and no Kronecker rotation, and wants its barrier words
+    h = _rot(L.QR_ROT_HADAMARD, 256)
+    def fused(rot=h, M=4, K=512, sync=FAKE, a=FAKE, n_out=0, idx=None, xo=None, wo=None,
+              zeros=None, sums=None):
+        return L.qr_w4a4_linear_fused(rot, FAKE, M, K, K, idx, n_out, FAKE, FAKE, sums, wo, 16, a,
+                                      FAKE, zeros, xo, FAKE, 16, sync, None, check=False)
+    assert fused(M=0) == L.QR_OK
+    assert fused(M=-1) == L.QR_ERR_INVALID_ARG
+    assert fused(M=65) == L.QR_ERR_UNSUPPORTED
+    assert fused(sync=None) == L.QR_ERR_INVALID_ARG
+    assert fused(sync=FAKE + 4) == L.QR_ERR_ALIGNMENT
+    assert fused(a=FAKE + 8) == L.QR_ERR_ALIGNMENT
+    assert fused(n_out=8) == L.QR_ERR_INVALID_ARG                 # no outlier list or copies
+    assert fused(n_out=4, idx=FAKE, xo=FAKE, wo=FAKE) == L.QR_ERR_UNSUPPORTED   # n_out % 8
+    assert fused(zeros=FAKE) == L.QR_ERR_INVALID_ARG              # asymmetric without w_sums
+    assert fused(rot=_rot(L.QR_ROT_KRON, n1=16, n2=32)) == L.QR_ERR_UNSUPPORTED

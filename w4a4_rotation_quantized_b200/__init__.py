@@ -13,5 +13,6 @@ from .layer import (GSR, HADAMARD, KRON, NONE, GraphedLinear, QuantizedLinear,  
                     invert_transpose, kv_quantize, pack_weights, packed_k, rotate_quant,
                     pack_weights8, rotate_quant8, rotate_quant_asym, w8a8_linear,
                     fp4_linear, pack_weights_fp4, rotate_quant_fp4,
-                    select_outliers, w4a4_linear, w4a4_linear_asym, weight_code_sums,
+                    select_outliers, w4a4_linear, w4a4_linear_asym, w4a4_linear_fused,
+                    weight_code_sums,
                     weight_rotation)

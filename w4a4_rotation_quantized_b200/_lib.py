@@ -19,9 +19,11 @@ EXPORTED = ("qr_abi_version", "qr_status_string", "qr_packed_k", "qr_rotate_quan
             "qr_invert_transpose", "qr_device_status", "qr_rotate_quant_asym",
             "qr_weight_code_sums", "qr_w4a4_linear_asym", "qr_kv_quantize",
             "qr_check_wait_timeout", "qr_rotate_quant8", "qr_pack_weights8", "qr_w8a8_linear",
-            "qr_rotate_quant_fp4", "qr_pack_weights_fp4", "qr_fp4_linear")
+            "qr_rotate_quant_fp4", "qr_pack_weights_fp4", "qr_fp4_linear",
+            "qr_w4a4_linear_fused")
 
 # codes of the device status word (qr_device_status)
+QR_DEV_TIMEOUT_GRID_SYNC = 0x106
 QR_DEV_TIMEOUT_SELFCHECK = 0x1FF
 
 
@@ -90,6 +92,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                vp]),
         "qr_fp4_linear": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, i32, vp, i64, vp,
                                          vp]),
+        "qr_w4a4_linear_fused": (ctypes.c_int, [rot_p, vp, i64, i64, i64, vp, i32, vp, vp, vp, vp,
+                                                i64, vp, vp, vp, vp, vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -262,4 +266,15 @@ def qr_fp4_linear(a_codes, a_scales, w_codes, w_scales, M, N, K_p, x_out, w_out,
                               n_out, Y, ldy, acc_debug, stream)
     if check:
         _check("qr_fp4_linear", st)
+    return st
+
+
+def qr_w4a4_linear_fused(rot, X, M, K, ldx, outlier_idx, n_out, w_codes, w_scales, w_sums, w_out,
+                         N, a_codes, a_scales, a_zeros, x_out, Y, ldy, sync, stream, *,
+                         check=True):
+    st = load().qr_w4a4_linear_fused(ctypes.byref(rot), X, M, K, ldx, outlier_idx, n_out, w_codes, w_scales,
+                                     w_sums, w_out, N, a_codes, a_scales, a_zeros, x_out, Y, ldy,
+                                     sync, stream)
+    if check:
+        _check("qr_w4a4_linear_fused", st)
     return st

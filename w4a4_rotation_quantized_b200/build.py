@@ -4,6 +4,7 @@ Usage: python -m w4a4_rotation_quantized_b200.build [--verbose]
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -49,13 +50,20 @@ def build(verbose: bool = False, force: bool = False) -> str:
         return LIB_PATH
     os.makedirs(BUILD_DIR, exist_ok=True)
     nvcc = nvcc_path()
-    objs = []
-    for src in sources():
+
+    def compile_one(src):
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
         cmd = [nvcc, *ARCH_FLAGS, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
-        res = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, subprocess.run(cmd, capture_output=True, text=True)
+
+    # the translation units are independent: compile them side by side
+    workers = max(1, min(len(sources()), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+        results = list(pool.map(compile_one, sources()))
+    objs = []
+    for src, obj, res in results:
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{res.stderr}")
         if verbose and res.stderr:

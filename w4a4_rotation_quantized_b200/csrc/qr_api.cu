@@ -307,6 +307,70 @@ qr_status qr_w4a4_linear_asym(const uint8_t* a_codes, const float* a_scales,
                      w_out, n_out, Y, ldy, acc_debug, stream);
 }
 
+qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                               int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
+                               const uint8_t* w_codes, const float* w_scales, const int32_t* w_sums,
+                               const uint16_t* w_out, int64_t N, uint8_t* a_codes, float* a_scales,
+                               int32_t* a_zeros, uint16_t* x_out, uint16_t* Y, int64_t ldy,
+                               uint32_t* sync, qr_stream stream) {
+  if (rot == nullptr || M < 0 || N < 0 || K < 0 || n_out < 0 || n_out > K) return QR_ERR_INVALID_ARG;
+  const int64_t kp = packed_k(rot, K, n_out);
+  if (kp < 0) {
+    if (rot->kind < QR_ROT_NONE || rot->kind > QR_ROT_KRON) return QR_ERR_INVALID_ARG;
+    return (rot->clip_ratio > 0.0f && rot->clip_ratio <= 1.0f) ? QR_ERR_UNSUPPORTED
+                                                               : QR_ERR_INVALID_ARG;
+  }
+  if (M == 0 || N == 0) return QR_OK;
+  if (X == nullptr || ldx < K || a_scales == nullptr || w_scales == nullptr || Y == nullptr ||
+      ldy < N || sync == nullptr)
+    return QR_ERR_INVALID_ARG;
+  if (kp > 0 && (a_codes == nullptr || w_codes == nullptr)) return QR_ERR_INVALID_ARG;
+  if (n_out > 0 && (outlier_idx == nullptr || x_out == nullptr || w_out == nullptr))
+    return QR_ERR_INVALID_ARG;
+  if (a_zeros != nullptr && w_sums == nullptr) return QR_ERR_INVALID_ARG;
+  if (rot->signs != nullptr) {
+    if (rot->kind != QR_ROT_HADAMARD && rot->kind != QR_ROT_GSR) return QR_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(rot->signs) % 8 != 0) return QR_ERR_ALIGNMENT;
+  }
+  if (M > 64 || rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
+  if (kp > 32768 || K > 32768 || n_out > 8192 || N > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
+  if (n_out % 8 != 0) return QR_ERR_UNSUPPORTED;
+  if (kp > 0 && (!aligned16(a_codes) || !aligned16(w_codes))) return QR_ERR_ALIGNMENT;
+  if (n_out > 0 && (!aligned16(x_out) || !aligned16(w_out))) return QR_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(sync) % 8 != 0) return QR_ERR_ALIGNMENT;
+  RowJob r{};
+  r.bits = 4;
+  r.src = X;
+  r.rows = M;
+  r.K = K;
+  r.ld = ldx;
+  r.outlier_idx = n_out > 0 ? outlier_idx : nullptr;
+  r.n_out = n_out;
+  r.Kp = static_cast<int32_t>(kp);
+  r.Kr = static_cast<int32_t>(K - n_out);
+  r.rot = rot;
+  r.codes = a_codes;
+  r.scales = a_scales;
+  r.zeros = a_zeros;
+  r.out16 = n_out > 0 ? x_out : nullptr;
+  GemmJob j{};
+  j.a_codes = a_codes;
+  j.a_scales = a_scales;
+  j.a_zeros = a_zeros;
+  j.w_codes = w_codes;
+  j.w_scales = w_scales;
+  j.w_sums = a_zeros != nullptr ? w_sums : nullptr;
+  j.M = M;
+  j.N = N;
+  j.Kp = kp;
+  j.x_out = n_out > 0 ? x_out : nullptr;
+  j.w_out = n_out > 0 ? w_out : nullptr;
+  j.n_out = n_out;
+  j.Y = Y;
+  j.ldy = ldy;
+  return launch_w4a4_decode_fused(j, r, sync, reinterpret_cast<cudaStream_t>(stream));
+}
+
 qr_status qr_select_outliers(const uint16_t* X_calib, int64_t T, int64_t K, int64_t ldx,
                              int32_t k, int32_t* idx_out, qr_stream stream) {
   if (T < 0 || K < 1 || k < 0 || k > K || ldx < K) return QR_ERR_INVALID_ARG;

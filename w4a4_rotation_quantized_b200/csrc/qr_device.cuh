@@ -17,6 +17,7 @@ enum DeviceCode : int32_t {
   kDevTimeoutMma = 0x103,
   kDevTimeoutEpilogue = 0x104,
   kDevTimeoutDrain = 0x105,
+  kDevTimeoutGridSync = 0x106,
   kDevTimeoutSelfCheck = 0x1FF,
 };
 
@@ -441,6 +442,58 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* s
           dst),
       "r"(smem_u32(src)), "r"(bytes), "r"(dst_bar)
       : "memory");
+}
+
+// ----------------------------------------------------------------- grid sync
+
+// Orders this thread's generic-proxy global-memory accesses with its later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// One arrival per CTA on a grid-wide barrier of `n` CTAs, then a bounded
+// wait for the other n - 1.  sync[0] counts arrivals and sync[1] is the
+// generation: the last CTA to arrive resets the count and advances the
+// generation, which the others watch, so the words are ready for the next
+// launch without a reset (both start at zero).  The CTAs must be resident
+// together; a wait that outlasts `limit_ns` records kDevTimeoutGridSync and
+// returns false, and since its CTA has arrived the count still completes
+// and resets when the late CTAs run.  Called by one thread of each CTA,
+// after its CTA's stores are fenced.
+__device__ __forceinline__ bool grid_sync_bounded(uint32_t* sync, uint32_t n, int32_t* status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  uint32_t gen;                              // (ordered before the arrival by its release)
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(sync + 1) : "memory");
+  if (atom_add_acq_rel_gpu(sync, 1u) == n - 1) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(sync), "r"(0u) : "memory");
+    st_release_gpu(sync + 1, gen + 1);
+    return true;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_gpu(sync + 1) != gen) return true;
+    if ((it & 15u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+      if (status) atomicCAS(status, 0, static_cast<int32_t>(kDevTimeoutGridSync));
+      return false;
+    }
+  }
 }
 
 // Named barrier over `count` threads (a multiple of 32) of the CTA.

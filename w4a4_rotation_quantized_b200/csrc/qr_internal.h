@@ -104,6 +104,12 @@ qr_status launch_w4a4_gemm_pair(const GemmJob& job, cudaStream_t stream);
 // M <= 64: weights in TMEM, K split over a cluster.
 qr_status launch_w4a4_gemm_decode(const GemmJob& job, cudaStream_t stream);
 int decode_k_split(int64_t tiles, int64_t steps, int sms);
+// The decode step in one kernel: the token rows of `rows` (M <= 64, a
+// Hadamard, GSR or identity rotation) rotated and quantized into its codes,
+// scales and outlier copy, then the decode GEMM on them, the two phases
+// separated by a grid-wide barrier on the two words at `sync`.
+qr_status launch_w4a4_decode_fused(const GemmJob& job, const RowJob& rows, uint32_t* sync,
+                                   cudaStream_t stream);
 int pair_tile_width(int64_t M, int64_t N, int sms);
 
 // Row-major 2-D tensor map: `rows` rows of `cols` elements, row pitch

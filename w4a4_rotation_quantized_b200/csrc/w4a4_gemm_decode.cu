@@ -29,14 +29,24 @@
 //               the fp16 outlier ring, whose steps the MMA thread interleaves
 //               with the int steps
 //   warp  13    TMEM allocation and the MMA-issuing thread
+//
+// Fused variant (ROT): the kernel first rotates and quantizes the token rows
+// itself (warps 0-11, whole rows per CTA, in the wide-B area of shared
+// memory before the ring starts), writes their codes, scales and outlier
+// columns to global memory, and meets the other CTAs at a grid-wide barrier;
+// meanwhile the producer has already put the weight halves of the first ring
+// slots in flight.  The token halves of the ring and the token scales are
+// read after the barrier.  One launch per decode step instead of two.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "qr_device.cuh"
 #include "qr_internal.h"
+#include "row_quant.cuh"
 
 namespace qr {
 
@@ -52,6 +62,29 @@ constexpr int kMmaWarp = 13;
 constexpr int kThreads = 32 * 14;
 constexpr int kSmemBudget = 227 * 1024;
 
+// The token rows of a decode step as the fused kernel takes them: the same
+// steps as the row kernels (FlatQuant "模型架构": the online transform and
+// the quantization fused into the kernel that consumes them; QUIK "性能分析":
+// the separate quantization pass is what keeps the measured speedup below
+// the ideal one).  Kept columns of QUIK §1 gathered in order, the optional
+// random-sign diagonal, Walsh-Hadamard butterflies per block in fp32 (QuaRot
+// §2), the row absmax (or min and max) and its scale, round-half-to-even
+// codes packed two per byte, the GSR sequency order by a gather at packing.
+struct FusedRows {
+  const __half* src;               // tokens [M x ld] fp16
+  int64_t ld;
+  int32_t K, Kr, Kp, n_out;        // Kr = K - n_out rotated columns, Kp packed width
+  const int32_t* outlier_idx;      // ascending [n_out], or null
+  const int8_t* signs;             // random-sign diagonal [Kp], or null
+  int32_t lb, gsr, aligned;        // log2 block, sequency order, 16-byte rows
+  float clip_ratio, inv_sqrt_block;
+  uint8_t* codes;                  // [M x Kp/2]: written here, read back by the ring
+  float* scales;                   // [M]
+  int32_t* zeros;                  // [M] zero points (asymmetric) or null
+  __half* out16;                   // [M x n_out] or null
+  uint32_t* sync;                  // grid barrier words [2]
+};
+
 struct DecodeParams {
   const float* w_scales;           // [N]
   const float* a_scales;           // [M]
@@ -65,6 +98,7 @@ struct DecodeParams {
   int32_t ks;                      // CTAs splitting K in a cluster
   int32_t y_tma;                   // Y leaves through tensor stores (map_y is valid)
   int32_t* status;
+  FusedRows rows;                  // the fused kernel's token rows
 };
 
 template <int BN, bool OUT>
@@ -103,10 +137,15 @@ struct DecodeLayout {
   static constexpr int kSendBytes = (128 - 128 / kMaxKS) * kRowWords * 4;
   static constexpr int off_ybox = (kSendBytes + 1023) / 1024 * 1024;
   static_assert(off_ybox + BN * 128 * 2 <= kNW * kWideB, "epilogue staging");
-  // full_p, empty_p, full_w, empty_w, full_o, empty_o, tmem_full, recv, drain
-  static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 * kNO + 3;
+  // full_p, empty_p, full_w, empty_w, full_o, empty_o, tmem_full, recv, drain,
+  // rows_ready (fused kernel: the token rows of every CTA are in memory),
+  // xbar[2] (fused kernel: the cluster's span maxima of a row landed)
+  static constexpr int kNumBars = 2 * kNP + 2 * kNW + 2 * kNO + 6;
   static constexpr int off_misc = off_bar + 8 * kNumBars;
-  static constexpr int kBytes = off_misc + 16 + 1024;
+  // misc: TMEM base, abort flag, 8 spare bytes, then the fused kernel's
+  // span maxima [2 row parities][max, -min][4 CTAs]
+  static constexpr int off_xmax = off_misc + 16;
+  static constexpr int kBytes = off_xmax + 64 + 1024;
   static_assert(kNW >= 3, "stage ring");
   static_assert(kBytes <= kSmemBudget, "shared memory");
   static_assert(BN == 32 || BN == 64, "token tile");
@@ -134,7 +173,195 @@ __device__ __forceinline__ StepRange step_range(int r, int ks, int kt, int ot) {
   return StepRange{i0, min(kt, i0 + q), 0, 0};
 }
 
-template <int BN, bool OUT, bool ASYM>
+// ------------------------------------------------------------ fused rotate
+
+constexpr int kRotThreads = 384;          // warps 0-11 rotate before their GEMM roles
+constexpr uint32_t kRotBar = 3;           // their named barrier
+
+__device__ __forceinline__ void rot_sync() { named_barrier(kRotBar, kRotThreads); }
+
+// Maximum over the rotating warps; `red` holds one float per warp.
+__device__ __forceinline__ float rot_max(float v, float* red, int t) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((t & 31) == 0) red[t >> 5] = v;
+  rot_sync();
+  float m = red[0];
+#pragma unroll
+  for (int w = 1; w < kRotThreads / 32; ++w) m = fmaxf(m, red[w]);
+  rot_sync();                              // red is reused
+  return m;
+}
+
+// Span of rotated positions [e_lo, e_hi) that CTA `rank` of a cluster of
+// `ks` takes in every row: whole blocks (at least 128 positions), split as
+// evenly as they go.  The host sizes the row buffer with the same rule.
+__host__ __device__ __forceinline__ int fused_span(int Kp, int lb, int ks) {
+  const int unit = (1 << lb) > 128 ? (1 << lb) : 128;
+  return (Kp / unit + ks - 1) / ks * unit;
+}
+
+// Rotates and quantizes the token rows of this CTA's cluster (rows c, c + Q,
+// ... below M for cluster c of Q) with the kRotThreads threads t.  Each row
+// is split over the cluster's ks CTAs by fused_span; a CTA reads the source
+// columns that can land in its span, keeps the non-outlier ones (one binary
+// search of the ascending outlier list per thread, then a walk over its
+// contiguous chunks), runs the butterflies on its span in shared memory
+// (`buf`, few_swz order), and takes its span's absmax (or max and -max of
+// -x).  The CTAs' maxima meet through distributed shared memory: each sends
+// its maxima to every CTA of the cluster (`xmax`, two sets by row parity)
+// and arrives on that CTA's `xbar`.  Codes always clamp to the quantizer's
+// range (a no-op for codes in range).
+template <bool ASYM>
+__device__ void fused_rotate_rows(const FusedRows& f, int M, int rank, int ks, float* buf,
+                                  int* sidx, float* red, float* xmax, uint64_t* xbar,
+                                  volatile int32_t* abort_flag, int32_t* status, int t) {
+  const int cluster = static_cast<int>(blockIdx.x) / ks;
+  const int nclusters = static_cast<int>(gridDim.x) / ks;
+  if (cluster >= M) return;
+  const int span = fused_span(f.Kp, f.lb, ks);
+  const int e_lo = min(f.Kp, rank * span), e_hi = min(f.Kp, e_lo + span);
+  const int nloc = e_hi - e_lo;
+  // the source columns of [e_lo, e_hi) lie in [e_lo, e_hi + n_out)
+  const int col_hi = min(f.K, e_hi + f.n_out);
+  const int nch = nloc > 0 ? (col_hi - e_lo + 7) >> 3 : 0;
+  const int cpt = (nch + kRotThreads - 1) / kRotThreads;     // contiguous chunks per thread
+  for (int j = t; j < f.n_out; j += kRotThreads) sidx[j] = __ldg(f.outlier_idx + j);
+  const int bm = (1 << f.lb) - 1;
+  int it = 0;
+  for (int row = cluster; row < M; row += nclusters, ++it) {
+    const __half* srow = f.src + static_cast<int64_t>(row) * f.ld;
+    uint4 raw[4];
+    auto issue = [&](int q0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col0 = e_lo + 8 * (t * cpt + q0 + q);
+        raw[q] = make_uint4(0u, 0u, 0u, 0u);
+        if (q0 + q < cpt && f.aligned && col0 + 8 <= f.K) raw[q] = ld_stream_v4(srow + col0);
+      }
+    };
+    issue(0);                                // the loads' latency overlaps the work below
+    rot_sync();                              // sidx staged; the last row's buf reads done
+    if (rank == 0 && f.out16 != nullptr)
+      for (int j = t; j < f.n_out; j += kRotThreads) {
+        const int c = sidx[j];
+        f.out16[static_cast<int64_t>(row) * f.n_out + j] =
+            (c >= 0 && c < f.K) ? srow[c] : __float2half(0.0f);
+      }
+    for (int e = max(f.Kr, e_lo) + t; e < e_hi; e += kRotThreads) buf[few_swz(e - e_lo)] = 0.0f;
+    for (int q0 = 0; q0 < cpt; q0 += 4) {
+      if (q0 > 0) issue(q0);
+      // outlier columns left of this batch's first column
+      const int col_first = e_lo + 8 * (t * cpt + q0);
+      int before = 0, hi = f.n_out;
+      while (before < hi) {
+        const int mid = (before + hi) >> 1;
+        if (sidx[mid] < col_first) before = mid + 1;
+        else hi = mid;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col0 = col_first + 8 * q;
+        if (q0 + q >= cpt || col0 >= col_hi) break;
+        float x[8];
+        if (f.aligned && col0 + 8 <= f.K) {
+          const __half2* h = reinterpret_cast<const __half2*>(&raw[q]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 v = __half22float2(h[i]);
+            x[2 * i] = v.x;
+            x[2 * i + 1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = (col0 + i < f.K) ? __half2float(srow[col0 + i]) : 0.0f;
+        }
+        uint32_t m8 = 0u;
+        for (int k = before; k < f.n_out && k < before + 8; ++k) {
+          const int d = sidx[k] - col0;
+          if (d >= 8) break;
+          if (d >= 0) m8 |= 1u << d;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = col0 + i - before;
+          if ((m8 >> i) & 1u) {
+            ++before;
+          } else if (col0 + i < f.K && e < f.Kr && e >= e_lo && e < e_hi) {
+            float xv = x[i];
+            if (f.signs != nullptr && __ldg(f.signs + e) < 0) xv = -xv;
+            buf[few_swz(e - e_lo)] = xv;
+          }
+        }
+      }
+    }
+    rot_sync();
+    float am = 0.0f;
+    for (int s = 0; s < f.lb; s += 3) {
+      const int r = min(3, f.lb - s);
+      if (r == 3) am = wht_smem_pass<3>(buf, nloc, s, t, kRotThreads);
+      else if (r == 2) am = wht_smem_pass<2>(buf, nloc, s, t, kRotThreads);
+      else am = wht_smem_pass<1>(buf, nloc, s, t, kRotThreads);
+      rot_sync();
+    }
+    if (f.lb == 0)
+      for (int e = t; e < nloc; e += kRotThreads) am = fmaxf(am, fabsf(buf[e]));
+    float m0 = am, m1 = 0.0f;
+    if (ASYM) {
+      m0 = -INFINITY;
+      m1 = -INFINITY;
+      for (int e = t; e < nloc; e += kRotThreads) {
+        m0 = fmaxf(m0, buf[e]);
+        m1 = fmaxf(m1, -buf[e]);
+      }
+      m1 = rot_max(m1, red, t);
+    }
+    m0 = rot_max(m0, red, t);
+    if (ks > 1) {
+      // every CTA's maxima into every CTA of the cluster, then wait for all
+      const int par = it & 1;
+      if (t < ks) {
+        const uint32_t dst = mapa_shared(smem_u32(xmax + 8 * par + rank), static_cast<uint32_t>(t));
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst), "f"(m0) : "memory");
+        if (ASYM) asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst + 16u), "f"(m1) : "memory");
+        mbar_arrive_cluster(mapa_shared(smem_u32(xbar + par), static_cast<uint32_t>(t)));
+      }
+      mbar_wait_cluster_bounded(xbar + par, static_cast<uint32_t>((it >> 1) & 1), abort_flag, status,
+                                kDevTimeoutGridSync);
+      for (int i = 0; i < ks; ++i) {
+        m0 = fmaxf(m0, xmax[8 * par + i]);
+        if (ASYM) m1 = fmaxf(m1, xmax[8 * par + 4 + i]);
+      }
+    }
+    const bool lead = t == 0 && rank == 0;
+    const RowQ q = ASYM ? asym_row_q(-m1, m0, f.clip_ratio, f.inv_sqrt_block,
+                                     lead ? f.scales + row : nullptr, f.zeros + row)
+                        : sym_row_q(m0, f.clip_ratio, f.inv_sqrt_block,
+                                    lead ? f.scales + row : nullptr);
+    uint8_t* crow = f.codes + static_cast<int64_t>(row) * (f.Kp >> 1) + (e_lo >> 1);
+    for (int g = t; g < (nloc >> 3); g += kRotThreads) {
+      const int el = 8 * g;
+      float v[8];
+      if (f.gsr) {
+        // sequency position j of a block takes Hadamard output bitrev(gray(j))
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = (el + i) & bm;
+          const int nat = static_cast<int>(__brev(static_cast<unsigned>(j ^ (j >> 1))) >> (32 - f.lb));
+          v[i] = buf[few_swz(((el + i) & ~bm) + nat)];
+        }
+      } else {
+        const float4 a = *reinterpret_cast<const float4*>(buf + few_swz(el));
+        const float4 b = *reinterpret_cast<const float4*>(buf + few_swz(el) + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      }
+      *reinterpret_cast<uint32_t*>(crow + (el >> 1)) = quant_word<true>(v, q.r, q.c, q.lo, q.hi);
+    }
+  }
+}
+
+template <int BN, bool OUT, bool ASYM, bool ROT>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
                         const __grid_constant__ CUtensorMap map_x,
@@ -157,6 +384,9 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   uint64_t* tmem_full = empty_o + kNO;       // accumulators final
   uint64_t* recv = tmem_full + 1;            // the other CTAs' partials of my rows landed
   uint64_t* drain = recv + 1;
+  uint64_t* rows_ready = drain + 1;          // fused: every CTA's token rows are in memory
+  uint64_t* xbar = rows_ready + 1;           // fused: [2] the cluster's row maxima landed
+  float* xmax = reinterpret_cast<float*>(smem + L::off_xmax);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_misc);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + L::off_misc + 4);
   uint32_t* slots = reinterpret_cast<uint32_t*>(smem + L::off_red);
@@ -177,6 +407,9 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     mbar_init(tmem_full, 1);
     mbar_init(recv, 1);
     mbar_init(drain, 1);
+    mbar_init(rows_ready, 1);
+    mbar_init(&xbar[0], static_cast<uint32_t>(p.ks));
+    mbar_init(&xbar[1], static_cast<uint32_t>(p.ks));
     *abort_flag = 0;
     fence_mbar_init();
     // the other CTAs' partials of my rows arrive by bulk copies
@@ -200,11 +433,45 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   grid_dep_launch();
   const int y_w = tile * 128;                // first weight row of the tile
 
+  if (ROT && warp < kRotThreads / 32) {
+    // ------------------------------------------------------------ fused rotate
+    // the wide-B area is free until these warps start widening
+    float* rbuf = reinterpret_cast<float*>(smem + L::off_wide_b);
+    int* ridx = reinterpret_cast<int*>(rbuf + fused_span(p.rows.Kp, p.rows.lb, p.ks));
+    float* rred = reinterpret_cast<float*>(ridx + p.rows.n_out);
+    fused_rotate_rows<ASYM>(p.rows, p.M, rank, p.ks, rbuf, ridx, rred, xmax, xbar, abort_flag,
+                            p.status, static_cast<int>(threadIdx.x));
+    __threadfence();                         // this CTA's rows, visible GPU-wide
+    fence_proxy_async_global();
+    rot_sync();
+    if (threadIdx.x == 0) {
+      grid_sync_bounded(p.rows.sync, gridDim.x, p.status);
+      mbar_arrive(rows_ready);
+    }
+  }
+
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
       uint32_t it = 0;
+      if (ROT) {
+        // the weight halves of the first slots go out before the token rows
+        // exist; their token halves follow the grid barrier
+        const uint32_t pre = static_cast<uint32_t>(min(kNP, n_slots));
+        for (uint32_t i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full_p[i], L::kPackA + L::kPackB);
+          tma_load_2d(smem + L::off_pack_a + i * L::kPackA, &map_w, &full_p[i],
+                      (sr.i0 + 2 * static_cast<int>(i)) * kStep, y_w);
+        }
+        ok = mbar_wait_bounded(rows_ready, 0, abort_flag, p.status, kDevTimeoutProducer);
+        fence_proxy_async_global();
+        // (issued even after a timeout, so that every slot completes)
+        for (uint32_t i = 0; i < pre; ++i)
+          tma_load_2d(smem + L::off_pack_b + i * L::kPackB, &map_x, &full_p[i],
+                      (sr.i0 + 2 * static_cast<int>(i)) * kStep, 0);
+        it = pre;
+      }
       for (; static_cast<int>(it) < n_slots; ++it) {
         const uint32_t s = it % kNP, ph = (it / kNP) & 1;
         const int x = (sr.i0 + 2 * static_cast<int>(it)) * kStep;
@@ -220,6 +487,10 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
       // the outlier ring, beside the int ring, so that its loads overlap it
       bool ok = true;
       uint32_t ot = 0;
+      if (ROT) {
+        ok = mbar_wait_bounded(rows_ready, 0, abort_flag, p.status, kDevTimeoutProducer);
+        fence_proxy_async_global();
+      }
       for (int os = sr.o0; os < sr.o1; ++os, ++ot) {
         const uint32_t s = ot % kNO, ph = (ot / kNO) & 1;
         if (!(ok = mbar_wait_bounded(&empty_o[s], ph ^ 1, abort_flag, p.status, kDevTimeoutProducer))) break;
@@ -352,11 +623,22 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     const bool has_out = OUT && p.ot > 0;
     const int n = y_w + lrow;                      // output column = weight row
     float* tok = reinterpret_cast<float*>(smem + L::off_tok);   // [BN] scales, [BN] 256 x zeros
-    if (warp == 0)
-      for (int i = lane; i < BN; i += 32) {
-        tok[i] = i < p.M ? __ldg(p.a_scales + i) : 0.0f;
-        if (ASYM) tok[BN + i] = i < p.M ? 256.0f * static_cast<float>(__ldg(p.a_zeros + i)) : 0.0f;
+    if (warp == 0) {
+      if (ROT) {
+        // written in this launch by other CTAs: after the grid barrier, and
+        // through L2 (not the read-only path)
+        mbar_wait_bounded(rows_ready, 0, abort_flag, p.status, kDevTimeoutEpilogue);
+        for (int i = lane; i < BN; i += 32) {
+          tok[i] = i < p.M ? __ldcg(p.a_scales + i) : 0.0f;
+          if (ASYM) tok[BN + i] = i < p.M ? 256.0f * static_cast<float>(__ldcg(p.a_zeros + i)) : 0.0f;
+        }
+      } else {
+        for (int i = lane; i < BN; i += 32) {
+          tok[i] = i < p.M ? __ldg(p.a_scales + i) : 0.0f;
+          if (ASYM) tok[BN + i] = i < p.M ? 256.0f * static_cast<float>(__ldg(p.a_zeros + i)) : 0.0f;
+        }
       }
+    }
     named_barrier(1, 128);                         // the four epilogue warps
     // asymmetric activations: acc - 256 * zero[m] * w_sum[n] (the accumulator is 256 x)
     float s_row = 0.0f, wsum = 0.0f;
@@ -510,16 +792,60 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
   }
 }
 
-template <int BN, bool OUT, bool ASYM>
+template <int BN, bool OUT, bool ASYM, bool ROT>
 cudaError_t run_decode(const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& mwo,
                        const CUtensorMap& mxo, const CUtensorMap& my, const DecodeParams& p,
                        int tiles, cudaStream_t stream) {
-  auto k = w4a4_gemm_decode_kernel<BN, OUT, ASYM>;
+  auto k = w4a4_gemm_decode_kernel<BN, OUT, ASYM, ROT>;
   const int smem = DecodeLayout<BN, OUT>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(k, dim3(static_cast<unsigned>(tiles * p.ks)), dim3(kThreads), smem, stream,
-                 static_cast<unsigned>(p.ks), mw, mx, mwo, mxo, my, p);
+  const unsigned grid = static_cast<unsigned>(tiles * p.ks);
+  if (!ROT) {
+    e = launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, static_cast<unsigned>(p.ks), mw, mx,
+                   mwo, mxo, my, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  // The fused kernel's CTAs meet at a grid-wide barrier, so all of them must
+  // be resident at once: the launch goes ahead only when every cluster fits
+  // on the device together.  It keeps programmatic dependent launch: CTAs
+  // that start early wait in grid_dep_wait until the previous kernel has
+  // finished, and the rest start as that kernel's CTAs leave, so all of them
+  // become resident; the barrier's bounded wait guards the rest (another
+  // process holding SMs).
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  int64_t resident = 0;
+  if (p.ks > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(p.ks);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, k, &cfg);
+    if (e != cudaSuccess) return e;
+    resident = static_cast<int64_t>(clusters) * p.ks;
+  } else {
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    resident = static_cast<int64_t>(per_sm) * sm_count();
+  }
+  if (resident < static_cast<int64_t>(grid)) return cudaErrorCooperativeLaunchTooLarge;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = n + 1;
+  e = cudaLaunchKernelEx(&cfg, k, mw, mx, mwo, mxo, my, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -534,7 +860,9 @@ int decode_k_split(int64_t tiles, int64_t steps, int sms) {
   return ks;
 }
 
-qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
+namespace {
+
+qr_status decode_common(const GemmJob& j, const FusedRows* fr, cudaStream_t stream) {
   const bool out = j.n_out > 0;
   const int bn = j.M <= 32 ? 32 : 64;
   const int64_t tiles = (j.N + 127) / 128;
@@ -579,13 +907,70 @@ qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
   const int t = static_cast<int>(tiles);
   cudaError_t e;
   const bool asym = p.a_zeros != nullptr;
-#define QR_RUN_DECODE(B, O)                                                        \
-  (asym ? run_decode<B, O, true>(mw, mx, mwo, mxo, my, p, t, stream)               \
-        : run_decode<B, O, false>(mw, mx, mwo, mxo, my, p, t, stream))
+  if (fr != nullptr) {
+    p.rows = *fr;
+    // the row buffer, the outlier list and the warp maxima live in the
+    // wide-B area until the ring starts
+    const int64_t need = 4ll * (fused_span(fr->Kp, fr->lb, p.ks) + fr->n_out + kRotThreads / 32);
+    const int64_t room = bn == 32 ? (out ? DecodeLayout<32, true>::kNW * DecodeLayout<32, true>::kWideB
+                                         : DecodeLayout<32, false>::kNW * DecodeLayout<32, false>::kWideB)
+                                  : (out ? DecodeLayout<64, true>::kNW * DecodeLayout<64, true>::kWideB
+                                         : DecodeLayout<64, false>::kNW * DecodeLayout<64, false>::kWideB);
+    if (need > room) return QR_ERR_UNSUPPORTED;
+  }
+  const bool rot = fr != nullptr;
+#define QR_RUN_DECODE(B, O)                                                                  \
+  (rot ? (asym ? run_decode<B, O, true, true>(mw, mx, mwo, mxo, my, p, t, stream)            \
+               : run_decode<B, O, false, true>(mw, mx, mwo, mxo, my, p, t, stream))          \
+       : (asym ? run_decode<B, O, true, false>(mw, mx, mwo, mxo, my, p, t, stream)           \
+               : run_decode<B, O, false, false>(mw, mx, mwo, mxo, my, p, t, stream)))
   if (bn == 32) e = out ? QR_RUN_DECODE(32, true) : QR_RUN_DECODE(32, false);
   else e = out ? QR_RUN_DECODE(64, true) : QR_RUN_DECODE(64, false);
 #undef QR_RUN_DECODE
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return QR_ERR_UNSUPPORTED;
+  }
   return e == cudaSuccess ? QR_OK : QR_ERR_CUDA;
 }
+
+}  // namespace
+
+qr_status launch_w4a4_gemm_decode(const GemmJob& j, cudaStream_t stream) {
+  return decode_common(j, nullptr, stream);
+}
+
+qr_status launch_w4a4_decode_fused(const GemmJob& j, const RowJob& r, uint32_t* sync,
+                                   cudaStream_t stream) {
+  const qr_rotation& rot = *r.rot;
+  if (rot.kind != QR_ROT_NONE && rot.kind != QR_ROT_HADAMARD && rot.kind != QR_ROT_GSR)
+    return QR_ERR_UNSUPPORTED;
+  if (j.M > 64 || r.rows != j.M || r.Kp != j.Kp || r.n_out != j.n_out) return QR_ERR_INVALID_ARG;
+  FusedRows f{};
+  f.src = reinterpret_cast<const __half*>(r.src);
+  f.ld = r.ld;
+  f.K = static_cast<int32_t>(r.K);
+  f.Kr = r.Kr;
+  f.Kp = r.Kp;
+  f.n_out = r.n_out;
+  f.outlier_idx = r.outlier_idx;
+  f.signs = rot.kind == QR_ROT_NONE ? nullptr : rot.signs;
+  const int block = rot.kind == QR_ROT_NONE ? 1 : rot.block;
+  int lb = 0;
+  while ((1 << lb) < block) ++lb;
+  f.lb = lb;
+  f.gsr = rot.kind == QR_ROT_GSR;
+  f.aligned = (reinterpret_cast<uintptr_t>(r.src) % 16 == 0) && (r.ld % 8 == 0);
+  f.clip_ratio = rot.clip_ratio;
+  f.inv_sqrt_block = static_cast<float>(1.0 / std::sqrt(static_cast<double>(block)));
+  f.codes = r.codes;
+  f.scales = r.scales;
+  f.zeros = r.zeros;
+  f.out16 = reinterpret_cast<__half*>(r.out16);
+  f.sync = sync;
+  return decode_common(j, &f, stream);
+}
+
+
 
 }  // namespace qr

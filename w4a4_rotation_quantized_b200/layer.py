@@ -228,6 +228,47 @@ def w4a4_linear_asym(a_codes, a_scales, a_zeros, w_codes, w_scales, w_sums, x_ou
     return y, acc
 
 
+def w4a4_linear_fused(x, rot: Rotation, outlier_idx, w_codes, w_scales, w_out=None, w_sums=None,
+                      asym: bool = False, sync: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None, check: bool = True):
+    """The decode step in one kernel: rotate + quantize the M <= 64 rows of x
+    and multiply them with the packed weights.  Same results as rotate_quant
+    (rotate_quant_asym) followed by w4a4_linear (w4a4_linear_asym).  Returns
+    (Y, codes, scales, zeros or None, x_out or None), or None when check is
+    False and the library answers UNSUPPORTED (the caller then takes the
+    two-call path).  `sync` is two int32 words, zero before the first call,
+    that calls sharing it must not overlap; a fresh zeroed pair when None."""
+    _need_cuda(x, torch.float16, "input")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("input must be a 2-D row-major tensor")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    n_out = 0 if outlier_idx is None else int(outlier_idx.numel())
+    crot = rot.c()
+    kp = L.qr_packed_k(crot, K, n_out)
+    if kp < 0:
+        raise ValueError("invalid rotation descriptor or sizes")
+    dev = x.device
+    codes = torch.empty((M, kp // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(M, dtype=torch.float32, device=dev)
+    zeros = torch.empty(M, dtype=torch.int32, device=dev) if asym else None
+    x_out = torch.empty((M, n_out), dtype=torch.float16, device=dev) if n_out else None
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=dev)
+    if sync is None:
+        sync = torch.zeros(2, dtype=torch.int32, device=dev)
+    st = L.qr_w4a4_linear_fused(crot, x.data_ptr(), M, K, x.stride(0),
+                                _ptr(outlier_idx) if n_out else None, n_out, w_codes.data_ptr(),
+                                w_scales.data_ptr(), _ptr(w_sums) if asym else None,
+                                _ptr(w_out) if n_out else None, N, codes.data_ptr(),
+                                scales.data_ptr(), _ptr(zeros), _ptr(x_out), y.data_ptr(),
+                                y.stride(0), sync.data_ptr(), _stream(), check=check)
+    if st == L.QR_ERR_UNSUPPORTED and not check:
+        return None
+    if st != L.QR_OK:
+        raise L.QrError("qr_w4a4_linear_fused", st)
+    return y, codes, scales, zeros, x_out
+
+
 def kv_quantize(q: Optional[torch.Tensor], k: Optional[torch.Tensor], v: Optional[torch.Tensor],
                 head_dim: int, group: int = 128):
     """The KV-cache step after RoPE: R3 (H_d / sqrt(d) per head) on q and k,
@@ -277,7 +318,8 @@ class QuantizedLinear:
     fp4=True, e2m1) weights; forward() is the online path."""
 
     def __init__(self, weight: torch.Tensor, rot: Rotation, outlier_idx=None,
-                 asym_activations: bool = False, bits: int = 4, fp4: bool = False):
+                 asym_activations: bool = False, bits: int = 4, fp4: bool = False,
+                 fused_decode: bool = False):
         if bits not in (4, 8) or (bits == 8 and asym_activations):
             raise ValueError("bits must be 4, or 8 with symmetric activations")
         if fp4 and (bits != 4 or asym_activations):
@@ -292,6 +334,12 @@ class QuantizedLinear:
         self.w_codes, self.w_scales, self.w_out, _ = pack(weight, self.rot_w, outlier_idx)
         self.w_sums = weight_code_sums(self.w_codes) if asym_activations else None
         self.out_features, self.in_features = weight.shape
+        # with fused_decode, decode steps (M <= 64 tokens) run as one fused
+        # kernel when the library takes the shape; its grid barrier words
+        # live here, so forward calls of one layer must not overlap (one
+        # stream)
+        self.fused_decode = fused_decode and bits == 4 and not fp4 and rot.kind != L.QR_ROT_KRON
+        self._sync = torch.zeros(2, dtype=torch.int32, device=weight.device)
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         if self.fp4:
@@ -302,6 +350,11 @@ class QuantizedLinear:
             codes, scales, x_out, _ = rotate_quant8(x, self.rot, self.outlier_idx)
             y, _ = w8a8_linear(codes, scales, self.w_codes, self.w_scales, x_out, self.w_out)
             return y
+        if self.fused_decode and x.dim() == 2 and 0 < x.shape[0] <= 64:
+            r = w4a4_linear_fused(x, self.rot, self.outlier_idx, self.w_codes, self.w_scales,
+                                  self.w_out, self.w_sums, self.asym, self._sync, check=False)
+            if r is not None:
+                return r[0]
         if self.asym:
             codes, scales, zeros, x_out, _ = rotate_quant_asym(x, self.rot, self.outlier_idx)
             y, _ = w4a4_linear_asym(codes, scales, zeros, self.w_codes, self.w_scales, self.w_sums,
