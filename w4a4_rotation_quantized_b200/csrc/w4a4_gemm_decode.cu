@@ -77,6 +77,7 @@ struct FusedRows {
   const int32_t* outlier_idx;      // ascending [n_out], or null
   const int8_t* signs;             // random-sign diagonal [Kp], or null
   int32_t lb, gsr, aligned;        // log2 block, sequency order, 16-byte rows
+  int32_t padded;                  // scatter through the padded buffer (room permitting)
   float clip_ratio, inv_sqrt_block;
   uint8_t* codes;                  // [M x Kp/2]: written here, read back by the ring
   float* scales;                   // [M]
@@ -193,6 +194,39 @@ __device__ __forceinline__ float rot_max(float v, float* red, int t) {
   return m;
 }
 
+// Position of span element e in the scatter buffer: one float of padding
+// after every 16, so that threads writing 16 consecutive elements each hit
+// distinct banks (17 is odd).
+__device__ __forceinline__ int pad16(int e) { return e + (e >> 4); }
+
+// The first butterfly pass of a span: groups of 8 consecutive elements read
+// from the padded scatter buffer `pbuf`, R (<= 3) stages on index bits
+// [0, R) in registers, written to `buf` in few_swz order with two 16-byte
+// stores.  Returns the largest |value| this thread wrote.
+template <int R>
+__device__ __forceinline__ float wht_first_pass(const float* pbuf, float* buf, int nloc, int t) {
+  float am = 0.0f;
+  for (int g = t; g < (nloc >> 3); g += kRotThreads) {
+    float x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = pbuf[pad16(8 * g + k)];
+#pragma unroll
+    for (int st = 0; st < R; ++st)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (!(k & (1 << st))) {
+          const float a = x[k], b = x[k | (1 << st)];
+          x[k] = a + b;
+          x[k | (1 << st)] = a - b;
+        }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) am = fmaxf(am, fabsf(x[k]));
+    *reinterpret_cast<float4*>(buf + few_swz(8 * g)) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(buf + few_swz(8 * g) + 4) = make_float4(x[4], x[5], x[6], x[7]);
+  }
+  return am;
+}
+
 // Span of rotated positions [e_lo, e_hi) that CTA `rank` of a cluster of
 // `ks` takes in every row: whole blocks (at least 128 positions), split as
 // evenly as they go.  The host sizes the row buffer with the same rule.
@@ -214,7 +248,7 @@ __host__ __device__ __forceinline__ int fused_span(int Kp, int lb, int ks) {
 // range (a no-op for codes in range).
 template <bool ASYM>
 __device__ void fused_rotate_rows(const FusedRows& f, int M, int rank, int ks, float* buf,
-                                  int* sidx, float* red, float* xmax, uint64_t* xbar,
+                                  float* pbuf, int* sidx, float* red, float* xmax, uint64_t* xbar,
                                   volatile int32_t* abort_flag, int32_t* status, int t) {
   const int cluster = static_cast<int>(blockIdx.x) / ks;
   const int nclusters = static_cast<int>(gridDim.x) / ks;
@@ -248,7 +282,10 @@ __device__ void fused_rotate_rows(const FusedRows& f, int M, int rank, int ks, f
         f.out16[static_cast<int64_t>(row) * f.n_out + j] =
             (c >= 0 && c < f.K) ? srow[c] : __float2half(0.0f);
       }
-    for (int e = max(f.Kr, e_lo) + t; e < e_hi; e += kRotThreads) buf[few_swz(e - e_lo)] = 0.0f;
+    for (int e = max(f.Kr, e_lo) + t; e < e_hi; e += kRotThreads) {
+      if (f.padded) pbuf[pad16(e - e_lo)] = 0.0f;
+      else buf[few_swz(e - e_lo)] = 0.0f;
+    }
     for (int q0 = 0; q0 < cpt; q0 += 4) {
       if (q0 > 0) issue(q0);
       // outlier columns left of this batch's first column
@@ -290,22 +327,39 @@ __device__ void fused_rotate_rows(const FusedRows& f, int M, int rank, int ks, f
           } else if (col0 + i < f.K && e < f.Kr && e >= e_lo && e < e_hi) {
             float xv = x[i];
             if (f.signs != nullptr && __ldg(f.signs + e) < 0) xv = -xv;
-            buf[few_swz(e - e_lo)] = xv;
+            if (f.padded) pbuf[pad16(e - e_lo)] = xv;
+            else buf[few_swz(e - e_lo)] = xv;
           }
         }
       }
     }
     rot_sync();
+    // stages [0, 3) (or all of a smaller block) on the way out of the
+    // scatter buffer, the rest three at a time in place
+    const int r0 = min(3, f.lb);
     float am = 0.0f;
-    for (int s = 0; s < f.lb; s += 3) {
+    if (f.padded) {
+      am = r0 == 3 ? wht_first_pass<3>(pbuf, buf, nloc, t)
+         : r0 == 2 ? wht_first_pass<2>(pbuf, buf, nloc, t)
+         : r0 == 1 ? wht_first_pass<1>(pbuf, buf, nloc, t)
+                   : wht_first_pass<0>(pbuf, buf, nloc, t);
+    } else {
+      // (rows too long for both buffers: scattered straight into buf)
+      am = r0 == 3 ? wht_smem_pass<3>(buf, nloc, 0, t, kRotThreads)
+         : r0 == 2 ? wht_smem_pass<2>(buf, nloc, 0, t, kRotThreads)
+         : r0 == 1 ? wht_smem_pass<1>(buf, nloc, 0, t, kRotThreads)
+                   : 0.0f;
+      if (r0 == 0)
+        for (int e = t; e < nloc; e += kRotThreads) am = fmaxf(am, fabsf(buf[e]));
+    }
+    rot_sync();
+    for (int s = 3; s < f.lb; s += 3) {
       const int r = min(3, f.lb - s);
       if (r == 3) am = wht_smem_pass<3>(buf, nloc, s, t, kRotThreads);
       else if (r == 2) am = wht_smem_pass<2>(buf, nloc, s, t, kRotThreads);
       else am = wht_smem_pass<1>(buf, nloc, s, t, kRotThreads);
       rot_sync();
     }
-    if (f.lb == 0)
-      for (int e = t; e < nloc; e += kRotThreads) am = fmaxf(am, fabsf(buf[e]));
     float m0 = am, m1 = 0.0f;
     if (ASYM) {
       m0 = -INFINITY;
@@ -437,10 +491,12 @@ w4a4_gemm_decode_kernel(const __grid_constant__ CUtensorMap map_w,
     // ------------------------------------------------------------ fused rotate
     // the wide-B area is free until these warps start widening
     float* rbuf = reinterpret_cast<float*>(smem + L::off_wide_b);
-    int* ridx = reinterpret_cast<int*>(rbuf + fused_span(p.rows.Kp, p.rows.lb, p.ks));
+    const int span = fused_span(p.rows.Kp, p.rows.lb, p.ks);
+    float* pbuf = rbuf + span;
+    int* ridx = reinterpret_cast<int*>(p.rows.padded ? pbuf + pad16(span) : pbuf);
     float* rred = reinterpret_cast<float*>(ridx + p.rows.n_out);
-    fused_rotate_rows<ASYM>(p.rows, p.M, rank, p.ks, rbuf, ridx, rred, xmax, xbar, abort_flag,
-                            p.status, static_cast<int>(threadIdx.x));
+    fused_rotate_rows<ASYM>(p.rows, p.M, rank, p.ks, rbuf, pbuf, ridx, rred, xmax, xbar,
+                            abort_flag, p.status, static_cast<int>(threadIdx.x));
     __threadfence();                         // this CTA's rows, visible GPU-wide
     fence_proxy_async_global();
     rot_sync();
@@ -909,14 +965,18 @@ qr_status decode_common(const GemmJob& j, const FusedRows* fr, cudaStream_t stre
   const bool asym = p.a_zeros != nullptr;
   if (fr != nullptr) {
     p.rows = *fr;
-    // the row buffer, the outlier list and the warp maxima live in the
-    // wide-B area until the ring starts
-    const int64_t need = 4ll * (fused_span(fr->Kp, fr->lb, p.ks) + fr->n_out + kRotThreads / 32);
+    // the row buffer, the padded scatter buffer (when there is room), the
+    // outlier list and the warp maxima live in the wide-B area until the
+    // ring starts
+    const int span = fused_span(fr->Kp, fr->lb, p.ks);
+    const int64_t need = 4ll * (span + fr->n_out + kRotThreads / 32);
+    const int64_t pad_need = need + 4ll * (span + span / 16);
     const int64_t room = bn == 32 ? (out ? DecodeLayout<32, true>::kNW * DecodeLayout<32, true>::kWideB
                                          : DecodeLayout<32, false>::kNW * DecodeLayout<32, false>::kWideB)
                                   : (out ? DecodeLayout<64, true>::kNW * DecodeLayout<64, true>::kWideB
                                          : DecodeLayout<64, false>::kNW * DecodeLayout<64, false>::kWideB);
     if (need > room) return QR_ERR_UNSUPPORTED;
+    p.rows.padded = pad_need <= room;
   }
   const bool rot = fr != nullptr;
 #define QR_RUN_DECODE(B, O)                                                                  \
