@@ -113,8 +113,8 @@ typedef struct {
 
 /* ABI version of this header (bumped on any change to the entry points;
  * 3 added the 8-bit calls and qr_check_wait_timeout, 4 the FP4 calls, 5
- * qr_w4a4_linear_fused). */
-#define QR_ABI_VERSION 5
+ * qr_w4a4_linear_fused, 6 qr_w4a4_linear_fused_noalloc). */
+#define QR_ABI_VERSION 6
 QR_API int32_t qr_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -228,6 +228,29 @@ QR_API qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X,
                                       uint8_t* a_codes, float* a_scales, int32_t* a_zeros,
                                       uint16_t* x_out, uint16_t* Y, int64_t ldy, uint32_t* sync,
                                       qr_stream stream);
+
+/* qr_w4a4_linear_fused without caller scratch.  The pages have no
+ * counterpart: this is a convenience form of the call above for callers
+ * that want only Y.  The token rows' codes, scales, zero points and outlier
+ * copy and the two grid-barrier words live in a scratch array of the
+ * library itself, one per device (a __device__ array found with
+ * cudaGetSymbolAddress; no memory is allocated).  The barrier words start at
+ * zero when the library loads and every completed call leaves the count at
+ * zero again.  All calls on one device share this scratch, so two calls
+ * that may run at the same time (different streams, or different host
+ * threads) race: order them on one stream.
+ *  arguments as qr_w4a4_linear_fused, without a_codes, a_scales, a_zeros,
+ *  x_out and sync; asym != 0 selects asymmetric activations (w_sums then
+ *  required)
+ * Errors: as qr_w4a4_linear_fused; UNSUPPORTED also for sizes above the
+ * scratch's capacity: M > 64, K_p > 32768 or n_out > 8192. */
+QR_API qr_status qr_w4a4_linear_fused_noalloc(const qr_rotation* rot, const uint16_t* X,
+                                              int64_t M, int64_t K, int64_t ldx,
+                                              const int32_t* outlier_idx, int32_t n_out,
+                                              const uint8_t* w_codes, const float* w_scales,
+                                              const int32_t* w_sums, const uint16_t* w_out,
+                                              int64_t N, int32_t asym, uint16_t* Y, int64_t ldy,
+                                              qr_stream stream);
 
 /* ----------------------------------------------------------------------
  * 8-bit layers ("QUIK：LLM上的一种4-bit推理方法", QUIK量化, results: the

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.qr_abi_version() == 5
+    assert L.qr_abi_version() == 6
     for s in range(6):
         assert L.status_string(s) and L.status_string(s) != "unknown status"
     assert L.status_string(99) == "unknown status"
@@ -259,3 +259,12 @@ def test_fused_decode_argument_errors(lib):
     assert fused(n_out=4, idx=FAKE, xo=FAKE, wo=FAKE) == L.QR_ERR_UNSUPPORTED   # n_out % 8
     assert fused(zeros=FAKE) == L.QR_ERR_INVALID_ARG              # asymmetric without w_sums
     assert fused(rot=_rot(L.QR_ROT_KRON, n1=16, n2=32)) == L.QR_ERR_UNSUPPORTED
+    # the no-alloc form: the same checks, and the scratch's capacity
+    def noalloc(rot=h, M=4, K=512, n_out=0, idx=None, wo=None, asym=0, sums=None):
+        return L.qr_w4a4_linear_fused_noalloc(rot, FAKE, M, K, K, idx, n_out, FAKE, FAKE, sums, wo,
+                                              16, asym, FAKE, 16, None, check=False)
+    assert noalloc(M=0) == L.QR_OK
+    assert noalloc(M=65) == L.QR_ERR_UNSUPPORTED
+    assert noalloc(n_out=8) == L.QR_ERR_INVALID_ARG
+    assert noalloc(asym=1) == L.QR_ERR_INVALID_ARG                # asymmetric without w_sums
+    assert noalloc(rot=_rot(L.QR_ROT_KRON, n1=16, n2=32)) == L.QR_ERR_UNSUPPORTED

@@ -14,5 +14,6 @@ from .layer import (GSR, HADAMARD, KRON, NONE, GraphedLinear, QuantizedLinear,  
                     pack_weights8, rotate_quant8, rotate_quant_asym, w8a8_linear,
                     fp4_linear, pack_weights_fp4, rotate_quant_fp4,
                     select_outliers, w4a4_linear, w4a4_linear_asym, w4a4_linear_fused,
+                    w4a4_linear_fused_noalloc,
                     weight_code_sums,
                     weight_rotation)

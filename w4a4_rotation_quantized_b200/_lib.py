@@ -20,7 +20,7 @@ EXPORTED = ("qr_abi_version", "qr_status_string", "qr_packed_k", "qr_rotate_quan
             "qr_weight_code_sums", "qr_w4a4_linear_asym", "qr_kv_quantize",
             "qr_check_wait_timeout", "qr_rotate_quant8", "qr_pack_weights8", "qr_w8a8_linear",
             "qr_rotate_quant_fp4", "qr_pack_weights_fp4", "qr_fp4_linear",
-            "qr_w4a4_linear_fused")
+            "qr_w4a4_linear_fused", "qr_w4a4_linear_fused_noalloc")
 
 # codes of the device status word (qr_device_status)
 QR_DEV_TIMEOUT_GRID_SYNC = 0x106
@@ -94,6 +94,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                          vp]),
         "qr_w4a4_linear_fused": (ctypes.c_int, [rot_p, vp, i64, i64, i64, vp, i32, vp, vp, vp, vp,
                                                 i64, vp, vp, vp, vp, vp, i64, vp, vp]),
+        "qr_w4a4_linear_fused_noalloc": (ctypes.c_int, [rot_p, vp, i64, i64, i64, vp, i32, vp, vp,
+                                                        vp, vp, i64, i32, vp, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -277,4 +279,14 @@ def qr_w4a4_linear_fused(rot, X, M, K, ldx, outlier_idx, n_out, w_codes, w_scale
                                      sync, stream)
     if check:
         _check("qr_w4a4_linear_fused", st)
+    return st
+
+
+def qr_w4a4_linear_fused_noalloc(rot, X, M, K, ldx, outlier_idx, n_out, w_codes, w_scales, w_sums,
+                                 w_out, N, asym, Y, ldy, stream, *, check=True):
+    st = load().qr_w4a4_linear_fused_noalloc(ctypes.byref(rot), X, M, K, ldx, outlier_idx, n_out,
+                                             w_codes, w_scales, w_sums, w_out, N, asym, Y, ldy,
+                                             stream)
+    if check:
+        _check("qr_w4a4_linear_fused_noalloc", st)
     return st

@@ -21,9 +21,21 @@ namespace {
 
 __device__ int32_t g_status_word;   // see qr_device_status()
 
+// Scratch of qr_w4a4_linear_fused_noalloc, one copy per device (a __device__
+// array of this library's module, zero when the module loads): the two
+// grid-barrier words, then the token rows' scales, zero points, codes and
+// outlier copy at their largest sizes.  The barrier count is back at zero
+// after every completed call; calls on one device share all of it.
+constexpr int64_t kScratchMaxM = 64, kScratchMaxKp = 32768, kScratchMaxOut = 8192;
+constexpr size_t kScratchOffScales = 256, kScratchOffZeros = 512, kScratchOffCodes = 1024;
+constexpr size_t kScratchOffOut = kScratchOffCodes + kScratchMaxM * kScratchMaxKp / 2;
+constexpr size_t kScratchBytes = kScratchOffOut + kScratchMaxM * kScratchMaxOut * 2;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
+
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int32_t* g_status_ptr[kMaxDevices] = {};
+uint8_t* g_scratch_ptr[kMaxDevices] = {};
 int g_sms[kMaxDevices] = {};
 int g_smem[kMaxDevices] = {};
 
@@ -48,6 +60,19 @@ int32_t* device_status_word() {
     g_status_ptr[d] = static_cast<int32_t*>(p);
   }
   return g_status_ptr[d];
+}
+
+// Device address of this device's copy of the no-alloc scratch, or null.
+uint8_t* noalloc_scratch() {
+  const int d = current_device();
+  if (d < 0) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_ptr[d] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[d] = static_cast<uint8_t*>(p);
+  }
+  return g_scratch_ptr[d];
 }
 
 int sm_count() {
@@ -307,12 +332,20 @@ qr_status qr_w4a4_linear_asym(const uint8_t* a_codes, const float* a_scales,
                      w_out, n_out, Y, ldy, acc_debug, stream);
 }
 
-qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
-                               int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
-                               const uint8_t* w_codes, const float* w_scales, const int32_t* w_sums,
-                               const uint16_t* w_out, int64_t N, uint8_t* a_codes, float* a_scales,
-                               int32_t* a_zeros, uint16_t* x_out, uint16_t* Y, int64_t ldy,
-                               uint32_t* sync, qr_stream stream) {
+}  // extern "C"
+
+namespace qr {
+
+// Shared by qr_w4a4_linear_fused and its no-alloc form: with `noalloc`, the
+// token rows' codes, scales, zero points and outlier copy and the barrier
+// words live in this device's scratch (resolved after the arguments pass;
+// a_zeros is then only a flag: non-null for asymmetric activations).
+static qr_status fused_call(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                            int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
+                            const uint8_t* w_codes, const float* w_scales, const int32_t* w_sums,
+                            const uint16_t* w_out, int64_t N, uint8_t* a_codes, float* a_scales,
+                            int32_t* a_zeros, uint16_t* x_out, uint16_t* Y, int64_t ldy,
+                            uint32_t* sync, qr_stream stream, bool noalloc) {
   if (rot == nullptr || M < 0 || N < 0 || K < 0 || n_out < 0 || n_out > K) return QR_ERR_INVALID_ARG;
   const int64_t kp = packed_k(rot, K, n_out);
   if (kp < 0) {
@@ -321,11 +354,11 @@ qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_
                                                                : QR_ERR_INVALID_ARG;
   }
   if (M == 0 || N == 0) return QR_OK;
-  if (X == nullptr || ldx < K || a_scales == nullptr || w_scales == nullptr || Y == nullptr ||
-      ldy < N || sync == nullptr)
+  if (X == nullptr || ldx < K || (!noalloc && a_scales == nullptr) || w_scales == nullptr ||
+      Y == nullptr || ldy < N || (!noalloc && sync == nullptr))
     return QR_ERR_INVALID_ARG;
-  if (kp > 0 && (a_codes == nullptr || w_codes == nullptr)) return QR_ERR_INVALID_ARG;
-  if (n_out > 0 && (outlier_idx == nullptr || x_out == nullptr || w_out == nullptr))
+  if (kp > 0 && ((!noalloc && a_codes == nullptr) || w_codes == nullptr)) return QR_ERR_INVALID_ARG;
+  if (n_out > 0 && (outlier_idx == nullptr || (!noalloc && x_out == nullptr) || w_out == nullptr))
     return QR_ERR_INVALID_ARG;
   if (a_zeros != nullptr && w_sums == nullptr) return QR_ERR_INVALID_ARG;
   if (rot->signs != nullptr) {
@@ -335,6 +368,16 @@ qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_
   if (M > 64 || rot->kind == QR_ROT_KRON) return QR_ERR_UNSUPPORTED;
   if (kp > 32768 || K > 32768 || n_out > 8192 || N > 0x7FFFFFFF) return QR_ERR_UNSUPPORTED;
   if (n_out % 8 != 0) return QR_ERR_UNSUPPORTED;
+  if (noalloc) {
+    if (M > kScratchMaxM || kp > kScratchMaxKp || n_out > kScratchMaxOut) return QR_ERR_UNSUPPORTED;
+    uint8_t* sc = noalloc_scratch();
+    if (sc == nullptr) return QR_ERR_CUDA;
+    sync = reinterpret_cast<uint32_t*>(sc);
+    a_scales = reinterpret_cast<float*>(sc + kScratchOffScales);
+    a_zeros = a_zeros != nullptr ? reinterpret_cast<int32_t*>(sc + kScratchOffZeros) : nullptr;
+    a_codes = sc + kScratchOffCodes;
+    x_out = reinterpret_cast<uint16_t*>(sc + kScratchOffOut);
+  }
   if (kp > 0 && (!aligned16(a_codes) || !aligned16(w_codes))) return QR_ERR_ALIGNMENT;
   if (n_out > 0 && (!aligned16(x_out) || !aligned16(w_out))) return QR_ERR_ALIGNMENT;
   if (reinterpret_cast<uintptr_t>(sync) % 8 != 0) return QR_ERR_ALIGNMENT;
@@ -369,6 +412,32 @@ qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_
   j.Y = Y;
   j.ldy = ldy;
   return launch_w4a4_decode_fused(j, r, sync, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace qr
+
+extern "C" {
+
+qr_status qr_w4a4_linear_fused(const qr_rotation* rot, const uint16_t* X, int64_t M, int64_t K,
+                               int64_t ldx, const int32_t* outlier_idx, int32_t n_out,
+                               const uint8_t* w_codes, const float* w_scales, const int32_t* w_sums,
+                               const uint16_t* w_out, int64_t N, uint8_t* a_codes, float* a_scales,
+                               int32_t* a_zeros, uint16_t* x_out, uint16_t* Y, int64_t ldy,
+                               uint32_t* sync, qr_stream stream) {
+  return fused_call(rot, X, M, K, ldx, outlier_idx, n_out, w_codes, w_scales, w_sums, w_out, N,
+                    a_codes, a_scales, a_zeros, x_out, Y, ldy, sync, stream, false);
+}
+
+qr_status qr_w4a4_linear_fused_noalloc(const qr_rotation* rot, const uint16_t* X, int64_t M,
+                                       int64_t K, int64_t ldx, const int32_t* outlier_idx,
+                                       int32_t n_out, const uint8_t* w_codes,
+                                       const float* w_scales, const int32_t* w_sums,
+                                       const uint16_t* w_out, int64_t N, int32_t asym,
+                                       uint16_t* Y, int64_t ldy, qr_stream stream) {
+  static int32_t flag = 1;                  // any non-null pointer selects zero points
+  return fused_call(rot, X, M, K, ldx, outlier_idx, n_out, w_codes, w_scales, w_sums, w_out, N,
+                    nullptr, nullptr, asym ? &flag : nullptr, nullptr, Y, ldy, nullptr, stream,
+                    true);
 }
 
 qr_status qr_select_outliers(const uint16_t* X_calib, int64_t T, int64_t K, int64_t ldx,

@@ -269,6 +269,26 @@ def w4a4_linear_fused(x, rot: Rotation, outlier_idx, w_codes, w_scales, w_out=No
     return y, codes, scales, zeros, x_out
 
 
+def w4a4_linear_fused_noalloc(x, rot: Rotation, outlier_idx, w_codes, w_scales, w_out=None,
+                              w_sums=None, asym: bool = False, out: Optional[torch.Tensor] = None):
+    """w4a4_linear_fused with its intermediate arrays and barrier words in the
+    library's own per-device scratch; returns Y only.  Calls on one device
+    share that scratch, so they must not overlap (one stream)."""
+    _need_cuda(x, torch.float16, "input")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("input must be a 2-D row-major tensor")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    n_out = 0 if outlier_idx is None else int(outlier_idx.numel())
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    L.qr_w4a4_linear_fused_noalloc(rot.c(), x.data_ptr(), M, K, x.stride(0),
+                                   _ptr(outlier_idx) if n_out else None, n_out, w_codes.data_ptr(),
+                                   w_scales.data_ptr(), _ptr(w_sums) if asym else None,
+                                   _ptr(w_out) if n_out else None, N, 1 if asym else 0,
+                                   y.data_ptr(), y.stride(0), _stream())
+    return y
+
+
 def kv_quantize(q: Optional[torch.Tensor], k: Optional[torch.Tensor], v: Optional[torch.Tensor],
                 head_dim: int, group: int = 128):
     """The KV-cache step after RoPE: R3 (H_d / sqrt(d) per head) on q and k,
