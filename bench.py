@@ -248,6 +248,19 @@ def algorithmic_counts(wl, M, kp, asym=False, N=None):
     return gemm_ops, rq_bytes, gemm_bytes
 
 
+def fused_step_bytes(wl, M, kp, asym=False):
+    """Algorithmic bytes of one fused decode step (rotate + quantize + GEMM
+    in one kernel): the rotate's bytes plus the GEMM's, less the codes,
+    scales (zero points) and outlier copy that the GEMM phase reads back
+    while they sit in L2 -- X read; codes, scales and the outlier copy
+    written; the weight side read; Y written."""
+    s = wl.spec
+    _, rq_bytes, gemm_bytes = algorithmic_counts(wl, M, kp, asym)
+    k_int = s.K - s.n_keep_fp16
+    reread = M * k_int * 0.5 + M * 4 + M * s.n_keep_fp16 * 2 + (M * 4 if asym else 0)
+    return rq_bytes + gemm_bytes - reread
+
+
 def kron_split_flops(wl, M):
     """Tensor-core FLOPs of the Kronecker transform of M rows: the two small
     products vec(P1^T mat(x) P2), 2 M K (n1 + n2) FLOPs, three times over for
@@ -460,12 +473,7 @@ def run_ours(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     if fused:
-        # one kernel: X read, codes, scales (zero points) and the outlier copy
-        # written (the GEMM phase reads them back while they sit in L2), the
-        # weight side read, Y written
-        k_int = s.K - s.n_keep_fp16
-        reread = M * k_int * 0.5 + M * 4 + M * s.n_keep_fp16 * 2 + (M * 4 if asym else 0)
-        gemm_bytes = rq_bytes + gemm_bytes - reread
+        gemm_bytes = fused_step_bytes(wl, M, kp, asym)
     ms_per_step = elapsed_ms / args.steps
     value = world * gemm_ops / (ms_per_step * 1e-3) / 1e12
     gemm_avg = gemm_total / args.steps

@@ -70,6 +70,22 @@ def test_algorithmic_counts_of_the_qkv_workload():
     assert rq == 2048 * 4096 * 2 + 2048 * 4096 / 2 + 2048 * 4
 
 
+def test_fused_decode_step_bytes():
+    # the fused step moves X in, the codes, scales and outlier copy out, the
+    # weight side in and Y out, counted by hand for the QUIK decode layer
+    import workloads
+    wl = workloads.make_workload("quik_decode_8192", M=4, N=8, with_weights=False)
+    M, K, N, n_out = 64, 8192, 8192, 256
+    kp = 8192
+    x_in = M * K * 2
+    a_out = M * (K - n_out) // 2 + M * 4 + M * n_out * 2
+    w_in = N * (K - n_out) // 2 + N * 4 + N * n_out * 2
+    y_out = M * N * 2
+    assert bench.fused_step_bytes(wl, M, kp) == x_in + a_out + w_in + y_out
+    # asymmetric activations add a zero point per token and a code sum per weight row
+    assert bench.fused_step_bytes(wl, M, kp, asym=True) == x_in + a_out + w_in + y_out + M * 4 + N * 4
+
+
 def test_reference_arm_with_random_signs(capsys):
     # the oracle arm takes the same randomized rotation as the GPU arm
     assert bench.main(["--impl", "reference", "--workload", "tiny_256", "--random-signs",
@@ -89,7 +105,8 @@ def test_gpu_arm_never_reaches_the_oracle():
     # calls nothing from the oracle; only the CPU-baseline and reference legs do
     import inspect
     for fn in (bench.run_ours, bench.workload_signs, bench.rotation_for, bench.run_kv,
-               bench.rotate_quant_roofline, bench.algorithmic_counts, bench.kron_split_flops):
+               bench.rotate_quant_roofline, bench.algorithmic_counts, bench.kron_split_flops,
+               bench.fused_step_bytes):
         src = inspect.getsource(fn)
         assert "import oracle" not in src and "O." not in src, fn.__name__
         assert "oracle_signs" not in src and "oracle_rotation" not in src, fn.__name__
